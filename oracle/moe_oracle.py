@@ -1,0 +1,342 @@
+"""CPU oracle for the fused Mixture-of-Experts layer.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or
+execute this module: only the tests, the smoke check of the graft entry point
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.
+It shares no code, table or helper with the CUDA library and imports nothing
+from it.
+
+What it computes
+----------------
+The layer the pages describe: "a token usually activates only a selected
+subset" of the experts, and the work is "routing tokens to experts, moving data
+and combining expert outputs" (toolboxkart.tech, "AWS SageMaker MoE kernel
+optimizations H200", section "Why MoE inference needs specialized kernels").
+The pages do not spell the arithmetic out; this module takes the plain reading
+of a top-k softmax MoE layer with SwiGLU experts:
+
+1. route   - per token, the k largest logits (ties to the lower expert id),
+             weights = full softmax restricted to those k and renormalised;
+2. permute - pair ids p = t*k + j grouped by expert, ascending p inside each
+             expert, optionally padded to a tile of BT rows;
+3. FP8     - per-tensor e4m3 quantisation of weights (one scale per expert and
+             tensor), of x and of the intermediate h ("FP8 tensor-quantized
+             fused MoE", same page, section "2. FP8 backend routing changes
+             which kernel path runs"; E4M3 = 4 exponent and 3 mantissa bits,
+             kongchang.com, "MoE Kernel Engineering Optimization Practices on
+             Amazon SageMaker AI", section "Triton Backend Routing");
+4. experts - h = silu(W_gate x) * (W_up x), y = W_down h;
+5. combine - out_t = sum_j w_tj * y_(t,j), the routing-weight scale applied
+             after the down projection ("fuses scaling, matrix multiplication,
+             and expert aggregation into one GPU pass", aib.vote, "AWS
+             SageMaker MoE kernel optimizations", third paragraph).
+
+Swap-AB (computing C^T = B^T A^T, kongchang.com page, section "Swap-AB:
+Making WGMMA Run at Full Utilization") changes no arithmetic, so the oracle has
+a single GEMM orientation.
+
+Precision: fp64 throughout, except that every step that turns a float into an
+integer code (the e4m3 quantisation of weights, x and h) is taken in IEEE fp32,
+the precision in which the kernels take it.
+
+Every function here is pinned by the CPU tests in ``tests/test_oracle_*.py``
+against brute force, closed forms, invariants or an independent library
+routine; no function is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+E4M3_MAX = 448.0          # largest finite e4m3 magnitude (exponent 1111, mantissa 110)
+E4M3_MIN_NORMAL_EXP = -6  # 2^-6 is the smallest normal e4m3 magnitude
+E4M3_SUBNORMAL_STEP = 2.0 ** -9
+
+
+# --------------------------------------------------------------------------- routing
+def route(logits: np.ndarray, k: int):
+    """Top-k selection on the logits and the renormalised softmax weights.
+
+    Selection is on the logits themselves (exp is monotone, so this is the
+    same set as selection on probabilities, and it keeps ties exact). Order
+    within a token: descending logit, equal logits by ascending expert id;
+    -0.0 and +0.0 compare equal. The weights are the literal definition: a
+    softmax over all E logits in fp64 (max subtracted), restricted to the
+    selected experts and divided by their sum.
+
+    Returns (ids [M,k] int32, w [M,k] float64).
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    M, E = logits.shape
+    if not (1 <= k <= E):
+        raise ValueError("need 1 <= k <= E")
+    # a stable sort of -logit keeps equal logits in ascending id order
+    order = np.argsort(-logits.astype(np.float64), axis=1, kind="stable")
+    ids = order[:, :k].astype(np.int32)
+    l64 = logits.astype(np.float64)
+    mx = l64.max(axis=1, keepdims=True)
+    p = np.exp(l64 - mx)
+    p /= p.sum(axis=1, keepdims=True)
+    sel = np.take_along_axis(p, ids.astype(np.int64), axis=1)
+    w = sel / sel.sum(axis=1, keepdims=True)
+    return ids, w
+
+
+# --------------------------------------------------------------------------- permutation
+def permute(ids: np.ndarray, E: int):
+    """Group (token, slot) pairs by expert.
+
+    Pair id p = t*k + j. For e = 0..E-1 in order, list the pairs routed to e in
+    ascending p. Returns (counts [E], offsets [E+1], sorted_pairs [P]) with
+    offsets the exclusive prefix sum of counts.
+    """
+    flat = np.asarray(ids, dtype=np.int64).ravel()
+    groups = [np.nonzero(flat == e)[0] for e in range(E)]
+    counts = np.array([g.size for g in groups], dtype=np.int64)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    sorted_pairs = (np.concatenate(groups) if groups else np.zeros(0, np.int64))
+    return counts, offsets, sorted_pairs.astype(np.int64)
+
+
+def pad_permutation(counts: np.ndarray, sorted_pairs: np.ndarray, BT: int, sentinel: int):
+    """Pad every expert's group of pairs up to a multiple of BT rows.
+
+    Pad slots hold ``sentinel`` (the pair count P). Returns
+    (padded_offsets [E+1], padded_pairs [sum ceil(n_e/BT)*BT]).
+    """
+    counts = np.asarray(counts, dtype=np.int64)
+    E = counts.size
+    padded = ((counts + BT - 1) // BT) * BT
+    poff = np.zeros(E + 1, dtype=np.int64)
+    poff[1:] = np.cumsum(padded)
+    out = np.full(int(poff[-1]), sentinel, dtype=np.int64)
+    src = 0
+    for e in range(E):
+        n = int(counts[e])
+        out[poff[e]:poff[e] + n] = sorted_pairs[src:src + n]
+        src += n
+    return poff, out
+
+
+# --------------------------------------------------------------------------- e4m3 codec
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each e4m3 code: 1 sign, 4 exponent (bias 7), 3 mantissa bits.
+
+    Exponent field 0 is subnormal (m * 2^-9); S.1111.111 is NaN; there is no
+    infinity. Returns float64.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    ex = (c >> 3) & 0xF
+    man = c & 0x7
+    normal = (1.0 + man / 8.0) * np.exp2(ex - 7.0)
+    sub = man * E4M3_SUBNORMAL_STEP
+    mag = np.where(ex == 0, sub, normal)
+    mag = np.where((ex == 15) & (man == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Round fp32 values to e4m3: round to nearest, ties to even, saturating.
+
+    Magnitudes above 448 (infinity included) become 448; NaN becomes the NaN
+    code with the input's sign bit. Works on the exact value of each fp32
+    input (held in fp64, which represents every fp32 exactly).
+    """
+    f = np.asarray(v, dtype=np.float32)
+    neg = np.signbit(f)
+    nan = np.isnan(f)
+    a = np.abs(f.astype(np.float64))
+    a = np.where(nan, 0.0, np.minimum(a, E4M3_MAX))
+    # binade of a: a = m * 2^ex with m in [0.5, 1)  =>  floor(log2 a) = ex - 1
+    _, ex = np.frexp(a)
+    e = ex.astype(np.int64) - 1
+    subnormal = (a < 2.0 ** E4M3_MIN_NORMAL_EXP)
+    # quantum of the grid at a: 2^-9 below the normal range, 2^(e-3) above
+    step = np.where(subnormal, E4M3_SUBNORMAL_STEP, np.exp2((e - 3).astype(np.float64)))
+    q = np.rint(a / step).astype(np.int64)  # np.rint rounds half to even
+    # subnormal: the code is q itself (q == 8 lands exactly on 2^-6, code 0x08)
+    code_sub = q
+    # normal: q in [8, 16]; 16 carries into the next binade
+    carry = q == 16
+    e_n = np.where(carry, e + 1, e)
+    q_n = np.where(carry, 8, q)
+    code_norm = ((e_n + 7) << 3) | (q_n - 8)
+    code = np.where(subnormal, code_sub, code_norm)
+    code = np.where(a == 0.0, 0, code)
+    code = np.where(nan, 0x7F, code)
+    code = code | np.where(neg, 0x80, 0)
+    return code.astype(np.uint8)
+
+
+def per_tensor_scale(t: np.ndarray) -> np.float32:
+    """s = amax(|t|) / 448 in fp32; an all-zero tensor takes s = 1."""
+    a = np.float32(np.max(np.abs(np.asarray(t, dtype=np.float32)))) if np.size(t) else np.float32(0)
+    if a == 0:
+        return np.float32(1.0)
+    return np.float32(a) / np.float32(E4M3_MAX)
+
+
+def quantize(t: np.ndarray, s: np.float32) -> np.ndarray:
+    """e4m3 codes of t / s, the division in IEEE fp32."""
+    q = np.asarray(t, dtype=np.float32) / np.float32(s)
+    return e4m3_encode(q.astype(np.float32))
+
+
+def dequantize(codes: np.ndarray, s) -> np.ndarray:
+    return e4m3_decode(codes) * float(s)
+
+
+def quantize_expert_weights(W: np.ndarray):
+    """One scale per expert for a stacked weight tensor W [E, rows, cols].
+
+    Returns (scales [E] float32, codes [E, rows, cols] uint8).
+    """
+    W = np.asarray(W, dtype=np.float32)
+    E = W.shape[0]
+    scales = np.zeros(E, dtype=np.float32)
+    codes = np.zeros(W.shape, dtype=np.uint8)
+    for e in range(E):
+        s = per_tensor_scale(W[e])
+        scales[e] = s
+        codes[e] = quantize(W[e], s)
+    return scales, codes
+
+
+# --------------------------------------------------------------------------- experts
+def silu(z: np.ndarray) -> np.ndarray:
+    """silu(z) = z / (1 + e^-z), in fp64."""
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+class _Weights:
+    """Per-expert weight access in fp64: plain arrays or a callable e -> (Wg, Wu, Wd)."""
+
+    def __init__(self, w_gate=None, w_up=None, w_down=None, provider=None):
+        self.provider = provider
+        self.wg, self.wu, self.wd = w_gate, w_up, w_down
+
+    def get(self, e: int):
+        if self.provider is not None:
+            g, u, d = self.provider(e)
+        else:
+            g, u, d = self.wg[e], self.wu[e], self.wd[e]
+        return (np.asarray(g, dtype=np.float32), np.asarray(u, dtype=np.float32),
+                np.asarray(d, dtype=np.float32))
+
+
+def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
+                provider=None, tokens=None, return_intermediates=False):
+    """The layer's output in fp64.
+
+    x       [M, H]  bf16 values (any float array holding them)
+    logits  [M, E]  fp32
+    w_gate  [E, I, H], w_up [E, I, H], w_down [E, H, I] (bf16 values), or
+    provider(e) -> (w_gate[e], w_up[e], w_down[e]) for weights too large to
+            hold on the host at once.
+    fp8     emulate the per-tensor e4m3 path: each weight tensor of each
+            expert quantised with its own scale, x quantised with one scale
+            over all M*H elements, h quantised with one scale over all valid
+            (token, slot) rows; dequantised values feed the fp64 arithmetic.
+    tokens  optional list of token indices whose output rows are wanted; the
+            other rows come back as NaN. Routing, the permutation, s_x and
+            (FP8) s_h are still computed over the whole batch, as defined.
+
+    Returns out [M, H] float64, or (out, dict of intermediates).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    logits = np.asarray(logits, dtype=np.float32)
+    M, H = x.shape
+    E = logits.shape[1]
+    W = _Weights(w_gate, w_up, w_down, provider)
+    ids, w = route(logits, k)
+    counts, offsets, sorted_pairs = permute(ids, E)
+    P = M * k
+
+    inter = {"ids": ids, "w": w, "counts": counts, "offsets": offsets,
+             "sorted_pairs": sorted_pairs}
+
+    if fp8:
+        s_x = per_tensor_scale(x)
+        x_codes = quantize(x, s_x)
+        xin = dequantize(x_codes, s_x)
+        inter["s_x"] = s_x
+        inter["x_codes"] = x_codes
+        inter["w_scales"] = np.zeros((E, 3), dtype=np.float32)
+    else:
+        xin = x.astype(np.float64)
+
+    want = np.ones(M, dtype=bool) if tokens is None else np.zeros(M, dtype=bool)
+    if tokens is not None:
+        want[np.asarray(tokens, dtype=np.int64)] = True
+
+    def expert_weights(e):
+        g_w, u_w, d_w = W.get(e)
+        if not fp8:
+            return g_w.astype(np.float64), u_w.astype(np.float64), d_w.astype(np.float64)
+        s_g, s_u, s_d = per_tensor_scale(g_w), per_tensor_scale(u_w), per_tensor_scale(d_w)
+        inter["w_scales"][e] = (s_g, s_u, s_d)
+        return (dequantize(quantize(g_w, s_g), s_g), dequantize(quantize(u_w, s_u), s_u),
+                dequantize(quantize(d_w, s_d), s_d))
+
+    # pass 1: gate/up projections and SwiGLU. FP8 needs every valid h row for
+    # the amax behind s_h; the bf16 path only needs the wanted tokens' pairs.
+    h_rows = {}
+    h_amax = np.float32(0.0)
+    Y = {}
+    for e in range(E):
+        n = int(counts[e])
+        if n == 0:
+            continue
+        pairs = sorted_pairs[offsets[e]:offsets[e] + n]
+        sel = want[pairs // k]
+        if not fp8 and not sel.any():
+            continue
+        g_w, u_w, d_w = expert_weights(e)
+        rows = pairs if fp8 else pairs[sel]
+        X = xin[rows // k]
+        Hh = silu(X @ g_w.T) * (X @ u_w.T)
+        if fp8:
+            h_amax = max(h_amax, np.float32(np.max(np.abs(Hh.astype(np.float32)))))
+            for i, p in enumerate(rows):
+                if want[p // k]:
+                    h_rows[int(p)] = Hh[i]
+        else:
+            # bf16 path: down projection right away
+            Ym = Hh @ d_w.T
+            for i, p in enumerate(rows):
+                h_rows[int(p)] = Hh[i]
+                Y[int(p)] = Ym[i]
+
+    if fp8:
+        s_h = np.float32(1.0) if h_amax == 0 else np.float32(h_amax) / np.float32(E4M3_MAX)
+        inter["s_h"] = s_h
+        # pass 2: quantised h through the dequantised down projection
+        for e in range(E):
+            n = int(counts[e])
+            if n == 0:
+                continue
+            pairs = [int(p) for p in sorted_pairs[offsets[e]:offsets[e] + n] if want[int(p) // k]]
+            if not pairs:
+                continue
+            d_w = expert_weights(e)[2]
+            Hm = np.stack([h_rows[p] for p in pairs])
+            Hm = dequantize(quantize(Hm.astype(np.float32), s_h), s_h)
+            Ym = Hm @ d_w.T
+            for i, p in enumerate(pairs):
+                Y[p] = Ym[i]
+
+    out = np.full((M, H), np.nan, dtype=np.float64)
+    for t in range(M):
+        if not want[t]:
+            continue
+        acc = np.zeros(H, dtype=np.float64)
+        for j in range(k):            # combine in slot order
+            acc += w[t, j] * Y[t * k + j]
+        out[t] = acc
+    if return_intermediates:
+        inter["h_rows"] = h_rows
+        return out, inter
+    return out
