@@ -1,0 +1,154 @@
+/*
+ * moe_b200.h - C ABI of the B200-native (sm_100a) fused Mixture-of-Experts layer.
+ *
+ * The layer, per token t of a batch of M tokens:
+ *   1. route:   the k largest router logits pick k experts (equal logits go to the
+ *               lower expert id); their softmax weights are renormalised to sum to 1
+ *               ("a token usually activates only a selected subset" of the experts;
+ *               toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200",
+ *               section "Why MoE inference needs specialized kernels");
+ *   2. align:   (token, slot) pairs are grouped by expert and padded to tile size
+ *               ("routing tokens to experts, moving data", same section);
+ *   3. gate_up: h = silu(W_gate[e] x_t) * (W_up[e] x_t), a grouped GEMM with the
+ *               SwiGLU activation fused into its epilogue;
+ *   4. down:    out_t = sum_j w_tj * (W_down[e_j] h_(t,j)), a grouped GEMM whose
+ *               epilogue applies the routing weight and scatter-adds into token
+ *               order ("fuses scaling, matrix multiplication, and expert aggregation
+ *               into one GPU pass", aib.vote, "AWS SageMaker MoE kernel
+ *               optimizations", third paragraph).
+ * The FP8 variant stores weights as e4m3 with one fp32 scale per expert tensor and
+ * quantises x and h per tensor on the fly ("FP8 tensor-quantized fused MoE",
+ * toolboxkart.tech page, section "2. FP8 backend routing changes which kernel path
+ * runs"; E4M3 format: kongchang.com, "MoE Kernel Engineering Optimization Practices
+ * on Amazon SageMaker AI", section "Triton Backend Routing").
+ *
+ * The token count M is a runtime argument of every call: no kernel is compiled,
+ * specialised or re-encoded per M ("Removing repeat compilation can reduce
+ * first-token delay", toolboxkart.tech page, section 3).
+ *
+ * Conventions for every entry point:
+ *   - Every call returns a moe_status; nothing aborts or throws across the ABI.
+ *   - Tensor pointers are DEVICE pointers on the layer's device unless a parameter
+ *     says "host"; they must be 16-byte aligned, contiguous and row-major.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - The caller keeps ownership of every pointer it passes; the library owns the
+ *     handle, its weights and its workspace, and frees them in moe_destroy.
+ *   - Calls on one handle must not run concurrently from several host threads.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_layer moe_layer;   /* opaque handle */
+
+typedef enum {
+  MOE_DTYPE_BF16 = 0,       /* bf16 weights and activations, fp32 accumulation        */
+  MOE_DTYPE_FP8_E4M3 = 1    /* e4m3 weights (per expert-tensor scale), e4m3 activations
+                               (per-tensor dynamic scale), fp32 accumulation           */
+} moe_dtype;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,    /* bad size, null or misaligned pointer, bad dtype      */
+  MOE_ERR_NOT_LOADED = -2,     /* forward before moe_load_weights                      */
+  MOE_ERR_OOM = -3,            /* device allocation failed                             */
+  MOE_ERR_CUDA = -4,           /* a CUDA runtime or driver call failed                 */
+  MOE_ERR_UNSUPPORTED = -5,    /* device is not sm_100, or the shape is not supported  */
+  MOE_ERR_DEVICE_TIMEOUT = -6  /* a kernel's bounded wait expired (see device error)   */
+} moe_status;
+
+/* Create a layer with E experts, top-k routing, hidden size H and expert
+ * intermediate size I, on the current CUDA device.
+ * Limits (checked): 1 <= E <= 512, 1 <= topk <= min(E, 16), H and I multiples of
+ * 128 with 128 <= H, I <= 16384. On success *out receives the handle. */
+MOE_API int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out);
+
+/* Release the handle, its weights and its workspace. Synchronises the device. */
+MOE_API int moe_destroy(moe_layer* layer);
+
+/* Copy bf16 expert weights into library-owned memory (device pointers):
+ *   w_gate [E, I, H], w_up [E, I, H], w_down [E, H, I], each row-major bf16.
+ * For an FP8 layer the library quantises them: one fp32 scale per (expert, tensor)
+ * s = amax|W| / 448 (s = 1 for an all-zero tensor), codes = e4m3(W / s) with an IEEE
+ * fp32 division, round-to-nearest-even, saturating to +-448.
+ * Runs on `stream` and synchronises it before returning; the caller may free the
+ * sources afterwards. Calling it again replaces the weights. */
+MOE_API int moe_load_weights(moe_layer* layer, const void* w_gate, const void* w_up,
+                     const void* w_down, void* stream);
+
+/* Load already-quantised e4m3 weights into an FP8 layer (device pointers):
+ *   q_gate [E, I, H], q_up [E, I, H], q_down [E, H, I] (uint8 e4m3 codes) and
+ *   scales [E, 3] fp32 (gate, up, down scale of each expert; host pointer).
+ * Weight value = decode(code) * scale. Synchronises `stream`. */
+MOE_API int moe_load_weights_fp8(moe_layer* layer, const void* q_gate, const void* q_up,
+                         const void* q_down, const float* scales_host, void* stream);
+
+/* Pre-size the workspace for batches of up to M_max tokens. moe_forward grows the
+ * workspace itself when a batch is larger (synchronising the device to do so), so
+ * call this once before capturing moe_forward into a CUDA graph. */
+MOE_API int moe_reserve(moe_layer* layer, int M_max, void* stream);
+
+/* The layer's forward pass, asynchronous on `stream`:
+ *   x             [M, H] bf16 (device)
+ *   router_logits [M, E] fp32 (device)
+ *   out           [M, H] bf16 (device), overwritten
+ * M = 0 is a no-op. No host-device synchronisation happens inside (unless the
+ * workspace must grow). Calls on one handle must be stream-ordered: the handle's
+ * workspace is shared by its calls. */
+MOE_API int moe_forward(moe_layer* layer, const void* x, const float* router_logits, int M,
+                void* out, void* stream);
+
+/* Host-buffer convenience: copies x_host [M,H] bf16 and logits_host [M,E] fp32 to
+ * the device, runs moe_forward and copies out [M,H] bf16 back to out_host, all on
+ * `stream`, and synchronises it. Pinned host memory gives asynchronous copies. */
+MOE_API int moe_forward_host(moe_layer* layer, const void* x_host, const float* logits_host,
+                     int M, void* out_host, void* stream);
+
+/* Text of a status code (static storage). */
+MOE_API const char* moe_status_string(int status);
+
+/* Synchronise the device and read (then clear) the handle's device error word:
+ * 0 when no kernel reported an error; otherwise a code whose low byte names the
+ * kernel and wait that gave up (bounded waits never spin forever). */
+MOE_API int moe_get_device_error(moe_layer* layer, int* code);
+
+/* Number of kernels the last moe_forward launched (0 for M = 0). */
+MOE_API int moe_last_launch_count(moe_layer* layer);
+
+/* Test access: copy the routing of the last forward to caller device buffers
+ * (any pointer may be NULL to skip it), after synchronising the device:
+ *   topk_ids [M, k] int32, topk_w [M, k] fp32, counts [E] int32,
+ *   padded_offsets [E+1] int32, padded_pairs [padded_offsets[E]] int32 (pad = M*k),
+ *   scales_host [2] fp32: s_x and s_h of the last FP8 forward (1 for bf16 layers).
+ * `tile_rows` (host, may be NULL) receives the pad tile (rows per expert group). */
+MOE_API int moe_debug_routing(moe_layer* layer, int* topk_ids, float* topk_w, int* counts,
+                      int* padded_offsets, int* padded_pairs, float* scales_host,
+                      int* tile_rows);
+
+/* Test access: copy the permuted activations of the last forward (device buffer of
+ * padded_offsets[E] rows of H elements: bf16, or e4m3 codes for FP8 layers), and
+ * the intermediate h (rows of I bf16 values) when h_out is not NULL. */
+MOE_API int moe_debug_activations(moe_layer* layer, void* x_perm_out, void* h_out);
+
+/* Test access: copy the stored weights (device buffers): FP8 layers give e4m3 codes
+ * q_gate/q_up [E,I,H], q_down [E,H,I] and scales_host [E,3]; bf16 layers give the
+ * bf16 copies and leave scales_host untouched. Any pointer may be NULL. */
+MOE_API int moe_debug_weights(moe_layer* layer, void* gate_out, void* up_out, void* down_out,
+                      float* scales_host);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,184 @@
+// kernels_align.cu - moe_align: group the (token, slot) pairs by expert, pad each
+// group to 16 rows, and build the tile lists and split-K factors of both grouped
+// GEMMs, all in one thread block.
+//
+// "Routing tokens to experts, moving data and combining expert outputs can add
+// work around the matrix multiplications" (toolboxkart.tech, "AWS SageMaker MoE
+// kernel optimizations H200", section "Why MoE inference needs specialized
+// kernels"); the permutation below is that data movement's index map. Pair
+// p = t*k + j goes to expert topk_ids[p]; inside an expert pairs keep ascending p.
+// The tile list is the "dynamic scheduling" of thin, variable token batches the
+// aib.vote page describes ("AWS SageMaker MoE kernel optimizations", third
+// paragraph): it is built on the device from the counts, so the host never
+// learns the routing and no kernel depends on the token count at compile time.
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kAlignThreads = 1024;
+constexpr int kAlignWarps = kAlignThreads / 32;
+constexpr int kSplitOverhead = 2;   // per-unit fixed cost, in K-block equivalents
+
+__device__ int choose_splits(int tiles, int kblocks, int sms, bool allow) {
+  if (tiles <= 0) return 1;
+  int best = 1;
+  long long best_cost = (static_cast<long long>(tiles) + sms - 1) / sms * (kblocks + kSplitOverhead);
+  if (!allow) return 1;
+  const int smax = kblocks < kMaxSplits ? kblocks : kMaxSplits;
+  for (int s = 2; s <= smax; ++s) {
+    const long long units = static_cast<long long>(tiles) * s;
+    const long long waves = (units + sms - 1) / sms;
+    const long long cost = waves * ((kblocks + s - 1) / s + kSplitOverhead);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+// Exclusive scan of v[0..n) (n <= 32*chunk) by one warp; total written to v_out[n].
+__device__ void warp_exclusive_scan(const int* in, int* out, int n, int lane) {
+  const int chunk = (n + 31) / 32;
+  const int lo = lane * chunk;
+  const int hi = min(n, lo + chunk);
+  int local = 0;
+  for (int i = lo; i < hi; ++i) local += in[i];
+  int incl = local;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - local;
+  for (int i = lo; i < hi; ++i) {
+    out[i] = run;
+    run += in[i];
+  }
+  if (lane == 31) out[n] = incl;
+}
+
+__global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
+  extern __shared__ int sm[];
+  const int E = a.E;
+  int* s_count = sm;                    // [E]
+  int* s_padded = s_count + E;          // [E]   count rounded up to 16
+  int* s_poff = s_padded + E;           // [E+1] padded offsets
+  int* s_base = s_poff + E + 1;         // [E]   pairs of e placed by earlier chunks
+  int* s_nb = s_base + E;               // [E]   token blocks of e
+  int* s_nboff = s_nb + E;              // [E+1]
+  int* s_wc = s_nboff + E + 1;          // [32][E] per-warp counts of the current chunk
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  for (int e = tid; e < E; e += kAlignThreads) {
+    s_count[e] = 0;
+    s_base[e] = 0;
+  }
+  __syncthreads();
+  for (int p = tid; p < a.P; p += kAlignThreads) atomicAdd(&s_count[__ldg(a.topk_ids + p)], 1);
+  __syncthreads();
+  for (int e = tid; e < E; e += kAlignThreads) {
+    const int n = s_count[e];
+    s_padded[e] = (n + kPadRows - 1) / kPadRows * kPadRows;
+    s_nb[e] = (n + a.BN - 1) / a.BN;
+  }
+  __syncthreads();
+  if (warp == 0) warp_exclusive_scan(s_padded, s_poff, E, lane);
+  if (warp == 1) warp_exclusive_scan(s_nb, s_nboff, E, lane);
+  __syncthreads();
+
+  // Stable scatter, 1024 pairs per chunk: rank inside the warp from the match
+  // mask, plus the counts of earlier warps in this chunk, plus earlier chunks.
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int c0 = 0; c0 < a.P; c0 += kAlignThreads) {
+    for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) s_wc[i] = 0;
+    __syncthreads();
+    const int p = c0 + tid;
+    const bool valid = p < a.P;
+    const int e = valid ? __ldg(a.topk_ids + p) : 0x7FFFFFFF;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (valid && rank == 0) s_wc[warp * E + e] = __popc(peers);
+    __syncthreads();
+    if (valid) {
+      int pos = s_base[e] + rank;
+      for (int w = 0; w < warp; ++w) pos += s_wc[w * E + e];
+      a.padded_pairs[s_poff[e] + pos] = p;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += kAlignThreads) {
+      int tot = 0;
+      for (int w = 0; w < kAlignWarps; ++w) tot += s_wc[w * E + ee];
+      s_base[ee] += tot;
+    }
+    __syncthreads();
+  }
+
+  for (int e = tid; e < E; e += kAlignThreads) {
+    for (int r = s_poff[e] + s_count[e]; r < s_poff[e + 1]; ++r) a.padded_pairs[r] = a.P;
+    a.counts[e] = s_count[e];
+    a.padded_offsets[e] = s_poff[e];
+  }
+  if (tid == 0) a.padded_offsets[E] = s_poff[E];
+
+  // Tiles: for expert e, its token blocks b and weight row blocks f, in the
+  // order (e, f, b) so that tiles sharing a weight tile are neighbours.
+  for (int e = warp; e < E; e += kAlignWarps) {
+    const int n = s_count[e];
+    const int nb = s_nb[e];
+    if (nb == 0) continue;
+    const int base = s_nboff[e];
+    for (int idx = lane; idx < nb * a.fblocks1; idx += 32) {
+      const int f = idx / nb, b = idx - f * nb;
+      Tile t;
+      t.expert = e;
+      t.fblock = f;
+      t.row_start = s_poff[e] + b * a.BN;
+      t.n_valid = min(a.BN, n - b * a.BN);
+      a.tiles1[static_cast<size_t>(base) * a.fblocks1 + idx] = t;
+    }
+    for (int idx = lane; idx < nb * a.fblocks2; idx += 32) {
+      const int f = idx / nb, b = idx - f * nb;
+      Tile t;
+      t.expert = e;
+      t.fblock = f;
+      t.row_start = s_poff[e] + b * a.BN;
+      t.n_valid = min(a.BN, n - b * a.BN);
+      a.tiles2[static_cast<size_t>(base) * a.fblocks2 + idx] = t;
+    }
+  }
+
+  if (tid == 0) {
+    const int nblocks = s_nboff[E];
+    const int rows_used = s_poff[E];
+    const int t1 = nblocks * a.fblocks1;
+    const int t2 = nblocks * a.fblocks2;
+    a.header[kHdrRowsUsed] = rows_used;
+    a.header[kHdrTiles1] = t1;
+    a.header[kHdrSplits1] = choose_splits(t1, a.kblocks1, a.num_sms, rows_used <= a.ws1_rows_cap);
+    a.header[kHdrTiles2] = t2;
+    a.header[kHdrSplits2] = choose_splits(t2, a.kblocks2, a.num_sms, true);
+    a.header[kHdrTokenBlocks] = nblocks;
+  }
+}
+
+}  // namespace
+
+size_t align_smem_bytes(int E) { return static_cast<size_t>(6 * E + 2 + kAlignWarps * E) * sizeof(int); }
+
+cudaError_t align_configure() {
+  return cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(align_smem_bytes(512)));
+}
+
+cudaError_t launch_align(const AlignArgs& a, cudaStream_t s) {
+  align_kernel<<<1, kAlignThreads, align_smem_bytes(a.E), s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,441 @@
+// kernels_gemm.cu - the two grouped GEMMs of the MoE layer on 5th-generation
+// tensor cores (tcgen05, accumulators in TMEM, operands staged by TMA).
+//
+// Orientation: every tile is "swap-AB". The expert's weight rows fill the MMA's
+// M = 128 slot and the expert's few tokens are the N dimension (16..BN), i.e.
+// the kernel computes D^T = W * X^T instead of X * W^T. The identity
+// (A B)^T = B^T A^T changes no arithmetic (kongchang.com, "MoE Kernel
+// Engineering Optimization Practices on Amazon SageMaker AI", section "Swap-AB:
+// Making WGMMA Run at Full Utilization"); it keeps the tensor-core rows busy
+// when decode gives an expert only a handful of tokens (toolboxkart.tech, "AWS
+// SageMaker MoE kernel optimizations H200", section "1. Swap-AB makes better use
+// of the WGMMA tile"; aib.vote, "AWS SageMaker MoE kernel optimizations", second
+// paragraph). On sm_100 the N dimension reaches 256, so the same orientation also
+// covers prefill, where an expert holds ~128-256 tokens.
+//
+// gate_up (GEMM1): per tile, 128 rows of W_gate and the same 128 rows of W_up go
+// to two TMEM accumulators [128 x N]; the epilogue forms h = silu(g) * u and
+// stores it as bf16 ("fuses scaling, matrix multiplication ... into one GPU pass",
+// aib.vote page, third paragraph). down (GEMM2): 128 rows of W_down times h; the
+// epilogue multiplies by the routing weight (and the FP8 scales) and
+// scatter-adds into the fp32 token accumulator with red.global.add ("expert
+// aggregation").
+//
+// Work units: the tiles from the align kernel, each optionally split along K
+// (split-K) so that small decode batches still stream weights through all SMs.
+// A persistent grid of one CTA per SM walks units blockIdx.x, +gridDim.x, ...
+// Warp roles: warp 0 = TMA producer, warp 1 = TMEM owner + MMA issuer,
+// warps 2-5 = epilogue (TMEM lanes 32*(warp%4) .. +31).
+#include <cuda_fp8.h>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+
+template <bool kGateUp, bool kFP8, int BN, int STAGES>
+struct Cfg {
+  static constexpr int kATiles = kGateUp ? 2 : 1;
+  static constexpr int kABytes = kTileRows * kRowBytes;            // 16 KB per weight tile
+  static constexpr int kBBytes = BN * kRowBytes;
+  static constexpr int kStageBytes = kATiles * kABytes + kBBytes;
+  static constexpr int kAccCols = kGateUp ? 2 * BN : BN;
+  static constexpr int kTmemCols = kAccCols <= 32 ? 32 : kAccCols <= 64 ? 64 : kAccCols <= 128 ? 128
+                                   : kAccCols <= 256 ? 256 : 512;
+  static constexpr int kBarrierBytes = 256;
+  static constexpr int kSmemBytes = STAGES * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
+  static constexpr int kKPerBlock = kFP8 ? 128 : 64;                // elements in one 128-byte row
+  static constexpr int kMmaKBytes = 32;                             // K of one MMA = 32 bytes
+  static constexpr int kMmasPerBlock = kRowBytes / kMmaKBytes;
+  static_assert(kAccCols <= 512, "TMEM holds 512 columns");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N of an M=128 MMA");
+  static_assert(2 * STAGES * 8 + 16 + 4 + 16 <= kBarrierBytes, "barrier area");
+};
+
+struct Unit {
+  Tile t;
+  int kb0, kb1;
+  bool ok;
+};
+
+__device__ __forceinline__ Unit load_unit(const GemmArgs& a, int u, int S, int BN) {
+  Unit x;
+  x.t = a.tiles[u / S];
+  const int s = u - (u / S) * S;
+  x.kb0 = s * a.kblocks / S;
+  x.kb1 = (s + 1) * a.kblocks / S;
+  x.ok = x.t.n_valid >= 1 && x.t.n_valid <= BN && x.kb1 > x.kb0;
+  return x;
+}
+
+__device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
+
+__device__ __forceinline__ float scale_from_amax(unsigned bits) {
+  const float amax = __uint_as_float(bits);
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+}
+
+template <bool kGateUp, bool kFP8, int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmArgs a, const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_b) {
+  using C = Cfg<kGateUp, kFP8, BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  int* flags = reinterpret_cast<int*>(tmem_slot + 1);   // [0] abort, [1] last arriver, [2..3] wait outcome
+  volatile int* abort_flag = flags;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiThreads / 32);
+    for (int i = 0; i < 4; ++i) flags[i] = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int T = a.header[a.hdr_tiles];
+  const int S = a.header[a.hdr_splits];
+  const int units = T * S;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();   // weights stream through once
+      const uint64_t pol_b = l2_policy_evict_last();    // activations are re-read per tile
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool failed = false;
+      for (int u = blockIdx.x; u < units && !failed; u += gridDim.x) {
+        const Unit un = load_unit(a, u, S, BN);
+        if (!un.ok) continue;
+        const int nb16 = (un.t.n_valid + 15) >> 4;
+        const int wrow = un.t.expert * a.w_rows_per_expert + un.t.fblock * kTileRows;
+        const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+            report_error(a.err, kErrWaitEmpty);
+            *abort_flag = 1;
+            failed = true;
+            break;
+          }
+          uint8_t* st = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], tx);
+          const int kc = kb * C::kKPerBlock;
+          tma_load_2d(st, &tm_w, &full[stage], kc, wrow, pol_w);
+          if constexpr (kGateUp) tma_load_2d(st + C::kABytes, &tm_w, &full[stage], kc, wrow + a.up_offset, pol_w);
+          uint8_t* bdst = st + C::kATiles * C::kABytes;
+          for (int j = 0; j < nb16; ++j)
+            tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[stage], kc, un.t.row_start + 16 * j, pol_b);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (failed) {
+        // let the copies already in flight land before the CTA's shared memory goes away
+        int zero = 0;
+        int st = stage, ph = static_cast<int>(phase);
+        const int pending = issued < STAGES ? issued : STAGES;
+        for (int i = 0; i < pending; ++i) {
+          if (--st < 0) {
+            st = STAGES - 1;
+            ph ^= 1;
+          }
+          mbar_wait_bounded(&full[st], static_cast<uint32_t>(ph), &zero, 1ll << 26);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase = 0;
+      for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        const Unit un = load_unit(a, u, S, BN);
+        if (!un.ok) continue;
+        const uint32_t n_pad = static_cast<uint32_t>((un.t.n_valid + 15) & ~15);
+        const uint32_t idesc = idesc_make(kFP8 ? 0u : 1u, 128u, n_pad);
+        if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag)) {
+          report_error(a.err, kErrWaitAccEmpty);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        bool failed = false;
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+            report_error(a.err, kErrWaitFull);
+            *abort_flag = 1;
+            failed = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b0 = a0 + C::kATiles * C::kABytes;
+          #pragma unroll
+          for (int kk = 0; kk < C::kMmasPerBlock; ++kk) {
+            const uint32_t koff = kk * C::kMmaKBytes;
+            const uint32_t accum = (kb > un.kb0 || kk > 0) ? 1u : 0u;
+            const uint64_t bd = sdesc_k_sw128(b0 + koff);
+            if constexpr (kFP8) mma_e4m3(tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
+            else mma_bf16(tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
+            if constexpr (kGateUp) {
+              const uint64_t ad1 = sdesc_k_sw128(a0 + C::kABytes + koff);
+              if constexpr (kFP8) mma_e4m3(tmem + BN, ad1, bd, idesc, accum);
+              else mma_bf16(tmem + BN, ad1, bd, idesc, accum);
+            }
+          }
+          mma_commit(&empty[stage]);   // frees the stage once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (failed) break;
+        mma_commit(acc_full);          // accumulator complete
+        acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                       // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;                // weight row inside the tile
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int epi_tid = threadIdx.x - 64;
+    uint32_t acc_phase = 0;
+    int iter = 0;
+    float lmax = 0.f;
+    float sx = 1.f, sh = 1.f;
+    if constexpr (kFP8) {
+      sx = scale_from_amax(*a.amax_x);
+      if constexpr (!kGateUp) sh = scale_from_amax(*a.amax_h);
+    }
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const Unit un = load_unit(a, u, S, BN);
+      if (!un.ok) {
+        if (epi_tid == 0) report_error(a.err, kErrBadTile);
+        continue;
+      }
+      // One thread waits; the named barrier hands the outcome to the other 127,
+      // so that all of them leave together if the wait gives up. The flag slot
+      // alternates per unit: no thread can be two units ahead of another.
+      volatile int* okf = flags + 2 + (iter & 1);
+      ++iter;
+      if (epi_tid == 0) *okf = mbar_wait_bounded(acc_full, acc_phase, abort_flag) ? 1 : 0;
+      named_bar_sync(1, kEpiThreads);
+      if (*okf == 0) {
+        if (epi_tid == 0) {
+          report_error(a.err, kErrWaitAccFull);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      acc_phase ^= 1u;
+      const int n_valid = un.t.n_valid;
+      const int e = un.t.expert;
+      const int col = un.t.fblock * kTileRows + row;
+
+      if constexpr (kGateUp) {
+        float sg = 1.f, su = 1.f;
+        if constexpr (kFP8) {
+          sg = __ldg(a.w_scales + e * 3 + 0) * sx;
+          su = __ldg(a.w_scales + e * 3 + 1) * sx;
+        }
+        const bool split = S > 1;
+        const size_t ld_ws = static_cast<size_t>(2) * a.I;
+        for (int c0 = 0; c0 < n_valid; c0 += 16) {
+          float g[16], v[16];
+          __syncwarp();
+          tmem_ld16(t_lane + c0, g);
+          tmem_ld16(t_lane + BN + c0, v);
+          tmem_ld_wait();
+          if (c0 + 16 >= n_valid) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          #pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < n_valid) {
+              const size_t r = static_cast<size_t>(un.t.row_start + n);
+              if (split) {
+                red_add_f32(a.ws1 + r * ld_ws + col, g[j]);
+                red_add_f32(a.ws1 + r * ld_ws + a.I + col, v[j]);
+              } else {
+                const float hv = silu(g[j] * sg) * (v[j] * su);
+                const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+                a.h[r * a.I + col] = hb;
+                if constexpr (kFP8) lmax = fmaxf(lmax, fabsf(__bfloat162float(hb)));
+              }
+            }
+          }
+        }
+        if (split) {
+          // the last of the S units of this tile finishes it from the partial sums
+          __threadfence();
+          named_bar_sync(1, kEpiThreads);
+          if (epi_tid == 0) {
+            const int tile = u / S;
+            const int old = atomicAdd(a.tile_counters + tile, 1);
+            const int last = (old == S - 1) ? 1 : 0;
+            if (last) a.tile_counters[tile] = 0;
+            flags[1] = last;
+          }
+          named_bar_sync(1, kEpiThreads);
+          if (flags[1]) {
+            __threadfence();
+            for (int n = 0; n < n_valid; ++n) {
+              const size_t r = static_cast<size_t>(un.t.row_start + n);
+              float* pg = a.ws1 + r * ld_ws + col;
+              float* pu = pg + a.I;
+              const float gs = ld_cg_f32(pg), us = ld_cg_f32(pu);
+              *pg = 0.f;
+              *pu = 0.f;
+              const float hv = silu(gs * sg) * (us * su);
+              const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+              a.h[r * a.I + col] = hb;
+              if constexpr (kFP8) lmax = fmaxf(lmax, fabsf(__bfloat162float(hb)));
+            }
+          }
+        }
+      } else {
+        float scale = 1.f;
+        if constexpr (kFP8) scale = __ldg(a.w_scales + e * 3 + 2) * sh;
+        for (int c0 = 0; c0 < n_valid; c0 += 16) {
+          float y[16];
+          __syncwarp();
+          tmem_ld16(t_lane + c0, y);
+          tmem_ld_wait();
+          if (c0 + 16 >= n_valid) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          int tok = 0;
+          float wt = 0.f;
+          if (lane < 16 && c0 + lane < n_valid) {
+            const int p = __ldg(a.padded_pairs + un.t.row_start + c0 + lane);
+            tok = p / a.k;
+            wt = __ldg(a.topk_w + p) * scale;
+          }
+          #pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int tj = __shfl_sync(0xFFFFFFFFu, tok, j);
+            const float wj = __shfl_sync(0xFFFFFFFFu, wt, j);
+            if (c0 + j < n_valid) red_add_f32(a.acc + static_cast<size_t>(tj) * a.H + col, y[j] * wj);
+          }
+        }
+      }
+    }
+    if constexpr (kGateUp && kFP8) {
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
+      if (lane == 0 && lmax > 0.f) atomicMax(a.amax_h, __float_as_uint(lmax));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Variant table. Small: decode with a few tokens per expert; medium: up to a few
+// thousand (token, expert) pairs; large: prefill.
+constexpr int kBnSmall = 32, kBnMedium = 128, kBnLarge = 256;
+constexpr int kSt1Small = 6, kSt1Medium = 4, kSt1Large = 3;    // gate_up stages
+constexpr int kSt2Small = 10, kSt2Medium = 6, kSt2Large = 4;   // down stages
+
+template <bool kGateUp, bool kFP8, int BN, int ST>
+cudaError_t launch_one(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int grid, cudaStream_t s) {
+  using C = Cfg<kGateUp, kFP8, BN, ST>;
+  grouped_gemm_kernel<kGateUp, kFP8, BN, ST><<<grid, kThreads, C::kSmemBytes, s>>>(a, w, b);
+  return cudaGetLastError();
+}
+
+template <bool kGateUp, bool kFP8, int BN, int ST>
+cudaError_t configure_one() {
+  using C = Cfg<kGateUp, kFP8, BN, ST>;
+  static_assert(C::kSmemBytes <= 232448, "shared memory per CTA");
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kFP8, BN, ST>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+}
+
+template <bool kGateUp, bool kFP8>
+cudaError_t launch_variant(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int variant, int grid,
+                           cudaStream_t s) {
+  if (variant == kVariantSmall)
+    return launch_one<kGateUp, kFP8, kBnSmall, kGateUp ? kSt1Small : kSt2Small>(a, w, b, grid, s);
+  if (variant == kVariantMedium)
+    return launch_one<kGateUp, kFP8, kBnMedium, kGateUp ? kSt1Medium : kSt2Medium>(a, w, b, grid, s);
+  return launch_one<kGateUp, kFP8, kBnLarge, kGateUp ? kSt1Large : kSt2Large>(a, w, b, grid, s);
+}
+
+template <bool kGateUp, bool kFP8>
+cudaError_t configure_all() {
+  cudaError_t e;
+  if ((e = configure_one<kGateUp, kFP8, kBnSmall, kGateUp ? kSt1Small : kSt2Small>()) != cudaSuccess) return e;
+  if ((e = configure_one<kGateUp, kFP8, kBnMedium, kGateUp ? kSt1Medium : kSt2Medium>()) != cudaSuccess) return e;
+  return configure_one<kGateUp, kFP8, kBnLarge, kGateUp ? kSt1Large : kSt2Large>();
+}
+
+}  // namespace
+
+int variant_bn(int v) { return v == kVariantSmall ? kBnSmall : v == kVariantMedium ? kBnMedium : kBnLarge; }
+
+cudaError_t gemm_configure() {
+  cudaError_t e;
+  if ((e = configure_all<true, false>()) != cudaSuccess) return e;
+  if ((e = configure_all<true, true>()) != cudaSuccess) return e;
+  if ((e = configure_all<false, false>()) != cudaSuccess) return e;
+  return configure_all<false, true>();
+}
+
+cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8, int variant,
+                         int grid, cudaStream_t s) {
+  return fp8 ? launch_variant<true, true>(a, w, x, variant, grid, s)
+             : launch_variant<true, false>(a, w, x, variant, grid, s);
+}
+
+cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int variant,
+                         int grid, cudaStream_t s) {
+  return fp8 ? launch_variant<false, true>(a, w, h, variant, grid, s)
+             : launch_variant<false, false>(a, w, h, variant, grid, s);
+}
+
+}  // namespace moe

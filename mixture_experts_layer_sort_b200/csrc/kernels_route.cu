@@ -1,0 +1,295 @@
+// kernels_route.cu - router top-k, activation gather/quantise, h quantise,
+// finalise, and the load-time weight quantiser.
+//
+// Router: "a token usually activates only a selected subset" of the experts
+// (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section
+// "Why MoE inference needs specialized kernels"). Each token keeps its k largest
+// logits, equal logits going to the lower expert id, and weights the selected
+// experts by their softmax renormalised over the selection.
+//
+// FP8: per-tensor ("tensor-quantized", same page, section "2. FP8 backend routing
+// changes which kernel path runs") e4m3 codes, s = amax/448, codes = RNE(v / s)
+// saturated to +-448, the division in IEEE fp32.
+#include <cuda_fp8.h>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouteWarps = 8;
+constexpr int kRouteMaxPerLane = 16;   // E <= 512 logits = 16 per lane
+
+// Orderable key of (logit, expert id): larger key = better. Higher logits first,
+// equal logits by ascending id, -0.0 equal to +0.0, NaN below -inf. Key 0 means
+// "no candidate".
+__device__ __forceinline__ unsigned long long route_key(float v, int e) {
+  unsigned b = __float_as_uint(v);
+  if (v == 0.0f) b = 0u;
+  unsigned ord;
+  if (v != v) ord = 0u;
+  else ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<unsigned long long>(ord) << 32) | (0xFFFFFFFFu - static_cast<unsigned>(e));
+}
+
+__device__ __forceinline__ float key_logit(unsigned long long key) {
+  const unsigned ord = static_cast<unsigned>(key >> 32);
+  const unsigned b = (ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord;
+  return __uint_as_float(b);
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    v = other > v ? other : v;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
+  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= a.M) return;
+
+  const float* row = a.logits + static_cast<size_t>(t) * a.E;
+  unsigned long long key[kRouteMaxPerLane];
+  #pragma unroll
+  for (int i = 0; i < kRouteMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = (e < a.E) ? route_key(__ldg(row + e), e) : 0ull;
+  }
+
+  int my_id = 0;
+  float my_logit = 0.f;
+  for (int j = 0; j < a.k; ++j) {
+    unsigned long long best = 0ull;
+    #pragma unroll
+    for (int i = 0; i < kRouteMaxPerLane; ++i) best = key[i] > best ? key[i] : best;
+    best = warp_max_u64(best);
+    const int id = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFu));
+    #pragma unroll
+    for (int i = 0; i < kRouteMaxPerLane; ++i)
+      if (lane + 32 * i == id) key[i] = 0ull;
+    if (lane == j) {
+      my_id = id;
+      my_logit = key_logit(best);
+    }
+  }
+  // slot 0 holds the largest selected logit
+  const float lmax = __shfl_sync(0xFFFFFFFFu, my_logit, 0);
+  float ex = (lane < a.k) ? expf(my_logit - lmax) : 0.f;
+  float sum = ex;
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  if (lane < a.k) {
+    a.topk_ids[static_cast<size_t>(t) * a.k + lane] = my_id;
+    a.topk_w[static_cast<size_t>(t) * a.k + lane] = ex / sum;
+  }
+
+  if (a.amax_x != nullptr) {
+    // FP8: this token's contribution to max |x|
+    const uint4* xr = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
+    float m = 0.f;
+    for (int i = lane; i < a.H / 8; i += 32) {
+      const uint4 v = __ldg(xr + i);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+      #pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(p[q]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) atomicMax(a.amax_x, __float_as_uint(m));
+  }
+}
+
+__device__ __forceinline__ float scale_from_amax(unsigned amax_bits) {
+  const float amax = __uint_as_float(amax_bits);
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+}
+
+// 8 fp32 values -> 8 e4m3 codes (RNE, saturating), v[i] / s with IEEE division.
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
+  uint2 r;
+  unsigned short c[4];
+  #pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float2 f = make_float2(__fdiv_rn(v[2 * q], s), __fdiv_rn(v[2 * q + 1], s));
+    c[q] = static_cast<unsigned short>(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3));
+  }
+  r.x = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
+  r.y = static_cast<unsigned>(c[2]) | (static_cast<unsigned>(c[3]) << 16);
+  return r;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&v)[8]) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+  #pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(p[q]);
+    v[2 * q] = f.x;
+    v[2 * q + 1] = f.y;
+  }
+}
+
+// One warp per padded row: copy (or quantise) the token's x row into x_perm.
+template <bool kFP8>
+__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= a.rows_bound || r >= __ldg(a.header + kHdrRowsUsed)) return;
+  const int p = __ldg(a.padded_pairs + r);
+  if (p >= a.P) return;   // pad row: never read by an output column
+  const int t = p / a.k;
+  const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
+  const int nvec = a.H / 8;
+  if constexpr (!kFP8) {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.x_perm) +
+                                          static_cast<size_t>(r) * a.H);
+    for (int i = lane; i < nvec; i += 32) dst[i] = __ldg(src + i);
+  } else {
+    const float s = scale_from_amax(*a.amax_x);
+    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.x_perm) +
+                                          static_cast<size_t>(r) * a.H);
+    for (int i = lane; i < nvec; i += 32) {
+      float v[8];
+      bf16x8_to_f32(__ldg(src + i), v);
+      dst[i] = quant8(v, s);
+    }
+  }
+}
+
+// FP8: h (bf16) -> e4m3 codes with s_h = amax(h)/448 over the valid rows.
+__global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= a.rows_bound || r >= __ldg(a.header + kHdrRowsUsed)) return;
+  if (__ldg(a.padded_pairs + r) >= a.P) return;
+  const float s = scale_from_amax(*a.amax_h);
+  const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(r) * a.I);
+  uint2* dst = reinterpret_cast<uint2*>(a.h_q + static_cast<size_t>(r) * a.I);
+  for (int i = lane; i < a.I / 8; i += 32) {
+    float v[8];
+    bf16x8_to_f32(src[i], v);
+    dst[i] = quant8(v, s);
+  }
+}
+
+// out = bf16(acc); acc = 0 for the next forward; reset the FP8 amax words.
+__global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.amax != nullptr) {
+    if (a.last_scales != nullptr) {
+      a.last_scales[0] = scale_from_amax(a.amax[0]);
+      a.last_scales[1] = scale_from_amax(a.amax[1]);
+    }
+    a.amax[0] = 0u;
+    a.amax[1] = 0u;
+  }
+  const long long n4 = a.n / 4;
+  float4* acc4 = reinterpret_cast<float4*>(a.acc);
+  uint2* out4 = reinterpret_cast<uint2*>(a.out);
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += static_cast<long long>(gridDim.x) * 256) {
+    const float4 v = acc4[i];
+    acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const unsigned*>(&lo);
+    o.y = *reinterpret_cast<const unsigned*>(&hi);
+    out4[i] = o;
+  }
+}
+
+// Load time: scale of one expert's tensor = amax/448 (1 for an all-zero tensor).
+__global__ void __launch_bounds__(1024) weight_amax_kernel(const __nv_bfloat16* w, long long per_expert,
+                                                           float* scales, int stride) {
+  const int e = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * per_expert);
+  float m = 0.f;
+  for (long long i = threadIdx.x; i < per_expert / 8; i += blockDim.x) {
+    float v[8];
+    bf16x8_to_f32(__ldg(src + i), v);
+    #pragma unroll
+    for (int q = 0; q < 8; ++q) m = fmaxf(m, fabsf(v[q]));
+  }
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ float red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (threadIdx.x == 0) scales[static_cast<size_t>(e) * stride] = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
+  }
+}
+
+__global__ void __launch_bounds__(256) weight_quant_kernel(const __nv_bfloat16* w, long long per_expert,
+                                                           int E, const float* scales, int stride,
+                                                           uint8_t* q, long long q_expert_stride) {
+  const long long vec_per_expert = per_expert / 8;
+  const long long total = vec_per_expert * E;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
+    const long long e = i / vec_per_expert;
+    const long long j = i - e * vec_per_expert;
+    const float s = __ldg(scales + e * stride);
+    float v[8];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(w) + i), v);
+    reinterpret_cast<uint2*>(q + e * q_expert_stride)[j] = quant8(v, s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
+  const int grid = (a.M + kRouteWarps - 1) / kRouteWarps;
+  route_kernel<<<grid, kRouteWarps * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s) {
+  const int grid = (a.rows_bound + 7) / 8;
+  if (fp8) gather_kernel<true><<<grid, 256, 0, s>>>(a);
+  else gather_kernel<false><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s) {
+  const int grid = (a.rows_bound + 7) / 8;
+  quant_h_kernel<<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s) {
+  long long n4 = a.n / 4;
+  long long blocks = (n4 + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  finalize_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_amax(const __nv_bfloat16* w, long long per_expert, int E, float* scales,
+                               int stride, cudaStream_t s) {
+  weight_amax_kernel<<<E, 1024, 0, s>>>(w, per_expert, scales, stride);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_quant(const __nv_bfloat16* w, long long per_expert, int E,
+                                const float* scales, int stride, uint8_t* q, long long q_expert_stride,
+                                cudaStream_t s) {
+  const long long total = per_expert / 8 * E;
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  weight_quant_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(w, per_expert, E, scales, stride, q,
+                                                                q_expert_stride);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

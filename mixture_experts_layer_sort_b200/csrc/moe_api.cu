@@ -1,0 +1,578 @@
+// moe_api.cu - the C ABI (include/moe_b200.h) and the host dispatcher: argument
+// checks, weight storage, workspace sizing, TMA descriptor encoding, the variant
+// table and the launch chain of one forward pass.
+//
+// The forward pass is a fixed chain of precompiled kernels; the token count M is
+// a runtime argument of each, and the variant (tile width BN) comes from a fixed
+// table keyed by M*k. Nothing is compiled, specialised or re-encoded per M (the
+// pages' third change removes exactly such per-token-count recompiles:
+// toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "3.
+// Removing repeat compilation can reduce first-token delay"). Tensor maps are
+// encoded once per weight load and once per workspace allocation.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/moe_b200.h"
+#include "moe_internal.h"
+
+using moe::Tile;
+
+struct moe_layer {
+  int E = 0, k = 0, H = 0, I = 0, dtype = 0, device = 0, num_sms = 0;
+  bool loaded = false;
+  // weights (library owned)
+  void* w13 = nullptr;          // [E, 2I, H] gate rows then up rows of each expert (bf16 or e4m3)
+  void* wd = nullptr;           // [E, H, I]
+  float* wscales = nullptr;     // [E, 3] FP8 scales (device)
+  CUtensorMap tm_w13{}, tm_wd{};
+  // workspace, sized for M_cap tokens
+  int M_cap = 0;
+  long long P_cap = 0, rows_cap = 0, nblocks_cap = 0, t1_cap = 0, t2_cap = 0, ws1_rows_cap = 0;
+  std::vector<void*> ws_allocs;
+  int* topk_ids = nullptr;
+  float* topk_w = nullptr;
+  int* counts = nullptr;
+  int* poff = nullptr;
+  int* pairs = nullptr;
+  Tile* tiles1 = nullptr;
+  Tile* tiles2 = nullptr;
+  int* header = nullptr;
+  void* x_perm = nullptr;
+  __nv_bfloat16* h = nullptr;
+  uint8_t* h_q = nullptr;
+  float* ws1 = nullptr;
+  int* counters = nullptr;
+  float* acc = nullptr;
+  unsigned* amax = nullptr;     // [2] max|x|, max|h| (float bits)
+  float* last_scales = nullptr; // [2]
+  int* err = nullptr;
+  CUtensorMap tm_x{}, tm_h{};
+  // staging for moe_forward_host
+  void* hx = nullptr;
+  float* hl = nullptr;
+  void* hout = nullptr;
+  int host_cap = 0;
+  // bookkeeping
+  int last_M = 0, last_launches = 0, last_variant = 0;
+};
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+unsigned long long g_configured = 0;   // bit per device index whose kernels are configured
+
+#define MOE_CUDA(call)                                                                           \
+  do {                                                                                           \
+    cudaError_t e_ = (call);                                                                     \
+    if (e_ != cudaSuccess) {                                                                     \
+      std::fprintf(stderr, "moe_b200: %s failed: %s (%s:%d)\n", #call, cudaGetErrorString(e_),   \
+                   __FILE__, __LINE__);                                                          \
+      return e_ == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA;                       \
+    }                                                                                            \
+  } while (0)
+
+#define MOE_TRY(call)              \
+  do {                             \
+    int s_ = (call);               \
+    if (s_ != MOE_OK) return s_;   \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return MOE_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr) return MOE_ERR_CUDA;
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return MOE_OK;
+}
+
+// 2-D row-major tensor [rows, inner] of 1- or 2-byte elements, box [box_rows, 128 bytes], 128B swizzle.
+int encode_map(CUtensorMap* m, const void* base, bool fp8, long long inner, long long rows, int box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner * (fp8 ? 1 : 2))};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::fprintf(stderr, "moe_b200: cuTensorMapEncodeTiled failed (%d)\n", static_cast<int>(r));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int configure_device(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (dev < 64 && (g_configured >> dev) & 1ull) return MOE_OK;
+  MOE_CUDA(moe::gemm_configure());
+  MOE_CUDA(moe::align_configure());
+  if (dev < 64) g_configured |= 1ull << dev;
+  return MOE_OK;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = (prev == dev) || cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (ok && prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+void free_workspace(moe_layer* L) {
+  for (void* p : L->ws_allocs) cudaFree(p);
+  L->ws_allocs.clear();
+  L->M_cap = 0;
+}
+
+template <class T>
+int ws_alloc(moe_layer* L, T** p, size_t bytes, bool zero) {
+  void* q = nullptr;
+  bytes = std::max<size_t>(bytes, 256);
+  MOE_CUDA(cudaMalloc(&q, bytes));
+  L->ws_allocs.push_back(q);
+  if (zero) MOE_CUDA(cudaMemset(q, 0, bytes));
+  *p = static_cast<T*>(q);
+  return MOE_OK;
+}
+
+bool is_fp8(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E4M3; }
+
+int choose_variant(long long P) {
+  if (P <= 128) return moe::kVariantSmall;
+  if (P <= 4096) return moe::kVariantMedium;
+  return moe::kVariantLarge;
+}
+
+int ensure_workspace(moe_layer* L, int M) {
+  if (M <= L->M_cap) return MOE_OK;
+  int cap = 64;
+  while (cap < M) cap *= 2;
+  MOE_CUDA(cudaDeviceSynchronize());   // the old workspace may still be in use
+  free_workspace(L);
+  const long long P = static_cast<long long>(cap) * L->k;
+  const long long Emin = std::min<long long>(L->E, P);
+  L->P_cap = P;
+  L->rows_cap = P + Emin * (moe::kPadRows - 1);
+  L->nblocks_cap = (P + moe::variant_bn(moe::kVariantSmall) - 1) / moe::variant_bn(moe::kVariantSmall) + Emin;
+  L->t1_cap = L->nblocks_cap * (L->I / moe::kTileRows);
+  L->t2_cap = L->nblocks_cap * (L->H / moe::kTileRows);
+  const long long ws1_limit = (128ll << 20) / (8ll * L->I);
+  L->ws1_rows_cap = std::min(L->rows_cap, ws1_limit);
+  const size_t el = is_fp8(L) ? 1 : 2;
+  MOE_TRY(ws_alloc(L, &L->topk_ids, P * 4, false));
+  MOE_TRY(ws_alloc(L, &L->topk_w, P * 4, false));
+  MOE_TRY(ws_alloc(L, &L->counts, (L->E + 1) * 4, true));
+  MOE_TRY(ws_alloc(L, &L->poff, (L->E + 1) * 4, true));
+  MOE_TRY(ws_alloc(L, &L->pairs, L->rows_cap * 4, true));
+  MOE_TRY(ws_alloc(L, &L->tiles1, L->t1_cap * sizeof(Tile), false));
+  MOE_TRY(ws_alloc(L, &L->tiles2, L->t2_cap * sizeof(Tile), false));
+  MOE_TRY(ws_alloc(L, &L->header, moe::kHdrSlots * 4, true));
+  MOE_TRY(ws_alloc(L, &L->x_perm, L->rows_cap * L->H * el, true));
+  MOE_TRY(ws_alloc(L, &L->h, L->rows_cap * L->I * 2, true));
+  if (is_fp8(L)) MOE_TRY(ws_alloc(L, &L->h_q, L->rows_cap * L->I, true));
+  MOE_TRY(ws_alloc(L, &L->ws1, L->ws1_rows_cap * 2 * L->I * 4, true));
+  MOE_TRY(ws_alloc(L, &L->counters, L->t1_cap * 4, true));
+  MOE_TRY(ws_alloc(L, &L->acc, static_cast<size_t>(cap) * L->H * 4, true));
+  MOE_TRY(ws_alloc(L, &L->amax, 2 * 4, true));
+  MOE_TRY(ws_alloc(L, &L->last_scales, 2 * 4, false));
+  MOE_TRY(ws_alloc(L, &L->err, 4, true));
+  const float ones[2] = {1.f, 1.f};
+  MOE_CUDA(cudaMemcpy(L->last_scales, ones, sizeof(ones), cudaMemcpyHostToDevice));
+  MOE_TRY(encode_map(&L->tm_x, L->x_perm, is_fp8(L), L->H, L->rows_cap, 16));
+  MOE_TRY(encode_map(&L->tm_h, is_fp8(L) ? static_cast<void*>(L->h_q) : static_cast<void*>(L->h), is_fp8(L),
+                     L->I, L->rows_cap, 16));
+  L->M_cap = cap;
+  return MOE_OK;
+}
+
+int encode_weight_maps(moe_layer* L) {
+  MOE_TRY(encode_map(&L->tm_w13, L->w13, is_fp8(L), L->H, 2ll * L->E * L->I, moe::kTileRows));
+  MOE_TRY(encode_map(&L->tm_wd, L->wd, is_fp8(L), L->I, 1ll * L->E * L->H, moe::kTileRows));
+  return MOE_OK;
+}
+
+int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
+  MOE_TRY(ensure_workspace(L, M));
+  const bool fp8 = is_fp8(L);
+  const long long P = static_cast<long long>(M) * L->k;
+  const int variant = choose_variant(P);
+  const int BN = moe::variant_bn(variant);
+  const int rows_bound = static_cast<int>(P + std::min<long long>(L->E, P) * (moe::kPadRows - 1));
+  int launches = 0;
+
+  moe::RouteArgs ra{};
+  ra.logits = logits;
+  ra.x = static_cast<const __nv_bfloat16*>(x);
+  ra.M = M;
+  ra.E = L->E;
+  ra.k = L->k;
+  ra.H = L->H;
+  ra.topk_ids = L->topk_ids;
+  ra.topk_w = L->topk_w;
+  ra.amax_x = fp8 ? L->amax : nullptr;
+  MOE_CUDA(moe::launch_route(ra, st));
+  ++launches;
+
+  moe::AlignArgs aa{};
+  aa.topk_ids = L->topk_ids;
+  aa.P = static_cast<int>(P);
+  aa.E = L->E;
+  aa.k = L->k;
+  aa.BN = BN;
+  aa.fblocks1 = L->I / moe::kTileRows;
+  aa.fblocks2 = L->H / moe::kTileRows;
+  const int kper = fp8 ? 128 : 64;
+  aa.kblocks1 = L->H / kper;
+  aa.kblocks2 = L->I / kper;
+  aa.num_sms = L->num_sms;
+  aa.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
+  aa.counts = L->counts;
+  aa.padded_offsets = L->poff;
+  aa.padded_pairs = L->pairs;
+  aa.tiles1 = L->tiles1;
+  aa.tiles2 = L->tiles2;
+  aa.header = L->header;
+  MOE_CUDA(moe::launch_align(aa, st));
+  ++launches;
+
+  moe::GatherArgs ga{};
+  ga.x = static_cast<const __nv_bfloat16*>(x);
+  ga.padded_pairs = L->pairs;
+  ga.header = L->header;
+  ga.rows_bound = rows_bound;
+  ga.P = static_cast<int>(P);
+  ga.k = L->k;
+  ga.H = L->H;
+  ga.x_perm = L->x_perm;
+  ga.amax_x = L->amax;
+  MOE_CUDA(moe::launch_gather(ga, fp8, st));
+  ++launches;
+
+  moe::GemmArgs g{};
+  g.header = L->header;
+  g.h = L->h;
+  g.I = L->I;
+  g.ws1 = L->ws1;
+  g.tile_counters = L->counters;
+  g.amax_h = L->amax + 1;
+  g.amax_x = L->amax;
+  g.w_scales = L->wscales;
+  g.acc = L->acc;
+  g.H = L->H;
+  g.padded_pairs = L->pairs;
+  g.topk_w = L->topk_w;
+  g.k = L->k;
+  g.P = static_cast<int>(P);
+  g.err = L->err;
+
+  moe::GemmArgs g1 = g;
+  g1.tiles = L->tiles1;
+  g1.hdr_tiles = moe::kHdrTiles1;
+  g1.hdr_splits = moe::kHdrSplits1;
+  g1.kblocks = aa.kblocks1;
+  g1.w_rows_per_expert = 2 * L->I;
+  g1.up_offset = L->I;
+  MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, L->tm_x, fp8, variant, L->num_sms, st));
+  ++launches;
+
+  if (fp8) {
+    moe::QuantHArgs qa{};
+    qa.h = L->h;
+    qa.h_q = L->h_q;
+    qa.padded_pairs = L->pairs;
+    qa.header = L->header;
+    qa.rows_bound = rows_bound;
+    qa.P = static_cast<int>(P);
+    qa.I = L->I;
+    qa.amax_h = L->amax + 1;
+    MOE_CUDA(moe::launch_quant_h(qa, st));
+    ++launches;
+  }
+
+  moe::GemmArgs g2 = g;
+  g2.tiles = L->tiles2;
+  g2.hdr_tiles = moe::kHdrTiles2;
+  g2.hdr_splits = moe::kHdrSplits2;
+  g2.kblocks = aa.kblocks2;
+  g2.w_rows_per_expert = L->H;
+  g2.up_offset = 0;
+  MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, variant, L->num_sms, st));
+  ++launches;
+
+  moe::FinalizeArgs fa{};
+  fa.acc = L->acc;
+  fa.out = static_cast<__nv_bfloat16*>(out);
+  fa.n = static_cast<long long>(M) * L->H;
+  fa.amax = fp8 ? L->amax : nullptr;
+  fa.last_scales = fp8 ? L->last_scales : nullptr;
+  MOE_CUDA(moe::launch_finalize(fa, st));
+  ++launches;
+
+  L->last_M = M;
+  L->last_launches = launches;
+  L->last_variant = variant;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_NOT_LOADED: return "weights not loaded";
+    case MOE_ERR_OOM: return "device out of memory";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_UNSUPPORTED: return "unsupported device or shape";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (E < 1 || E > 512 || topk < 1 || topk > 16 || topk > E) return MOE_ERR_INVALID_ARG;
+  if (H < 128 || I < 128 || H > 16384 || I > 16384 || H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  MOE_CUDA(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(get_encoder());
+  MOE_TRY(configure_device(dev));
+  moe_layer* L = new (std::nothrow) moe_layer();
+  if (!L) return MOE_ERR_OOM;
+  L->E = E;
+  L->k = topk;
+  L->H = H;
+  L->I = I;
+  L->dtype = dtype;
+  L->device = dev;
+  L->num_sms = prop.multiProcessorCount;
+  const size_t el = dtype == MOE_DTYPE_FP8_E4M3 ? 1 : 2;
+  if (cudaMalloc(&L->w13, static_cast<size_t>(E) * 2 * I * H * el) != cudaSuccess ||
+      cudaMalloc(&L->wd, static_cast<size_t>(E) * H * I * el) != cudaSuccess ||
+      cudaMalloc(&L->wscales, static_cast<size_t>(E) * 3 * sizeof(float)) != cudaSuccess) {
+    cudaFree(L->w13);
+    cudaFree(L->wd);
+    cudaFree(L->wscales);
+    delete L;
+    return MOE_ERR_OOM;
+  }
+  std::vector<float> ones(static_cast<size_t>(E) * 3, 1.f);
+  cudaMemcpy(L->wscales, ones.data(), ones.size() * sizeof(float), cudaMemcpyHostToDevice);
+  *out = L;
+  return MOE_OK;
+}
+
+int moe_destroy(moe_layer* L) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  cudaDeviceSynchronize();
+  free_workspace(L);
+  cudaFree(L->w13);
+  cudaFree(L->wd);
+  cudaFree(L->wscales);
+  cudaFree(L->hx);
+  cudaFree(L->hl);
+  cudaFree(L->hout);
+  delete L;
+  return MOE_OK;
+}
+
+int moe_load_weights(moe_layer* L, const void* w_gate, const void* w_up, const void* w_down, void* stream) {
+  if (!L || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t IH = static_cast<size_t>(L->I) * L->H;
+  L->loaded = false;
+  if (!is_fp8(L)) {
+    uint8_t* w13 = static_cast<uint8_t*>(L->w13);
+    MOE_CUDA(cudaMemcpy2DAsync(w13, 2 * IH * 2, w_gate, IH * 2, IH * 2, L->E, cudaMemcpyDeviceToDevice, st));
+    MOE_CUDA(cudaMemcpy2DAsync(w13 + IH * 2, 2 * IH * 2, w_up, IH * 2, IH * 2, L->E, cudaMemcpyDeviceToDevice, st));
+    MOE_CUDA(cudaMemcpyAsync(L->wd, w_down, IH * 2 * L->E, cudaMemcpyDeviceToDevice, st));
+  } else {
+    const __nv_bfloat16* src[3] = {static_cast<const __nv_bfloat16*>(w_gate),
+                                   static_cast<const __nv_bfloat16*>(w_up),
+                                   static_cast<const __nv_bfloat16*>(w_down)};
+    for (int j = 0; j < 3; ++j)
+      MOE_CUDA(moe::launch_weight_amax(src[j], static_cast<long long>(IH), L->E, L->wscales + j, 3, st));
+    uint8_t* w13 = static_cast<uint8_t*>(L->w13);
+    MOE_CUDA(moe::launch_weight_quant(src[0], IH, L->E, L->wscales + 0, 3, w13, 2 * IH, st));
+    MOE_CUDA(moe::launch_weight_quant(src[1], IH, L->E, L->wscales + 1, 3, w13 + IH, 2 * IH, st));
+    MOE_CUDA(moe::launch_weight_quant(src[2], IH, L->E, L->wscales + 2, 3, static_cast<uint8_t*>(L->wd), IH, st));
+  }
+  MOE_CUDA(cudaStreamSynchronize(st));
+  MOE_TRY(encode_weight_maps(L));
+  L->loaded = true;
+  return MOE_OK;
+}
+
+int moe_load_weights_fp8(moe_layer* L, const void* q_gate, const void* q_up, const void* q_down,
+                         const float* scales_host, void* stream) {
+  if (!L || !q_gate || !q_up || !q_down || !scales_host) return MOE_ERR_INVALID_ARG;
+  if (!is_fp8(L)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(q_gate) || !aligned16(q_up) || !aligned16(q_down)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t IH = static_cast<size_t>(L->I) * L->H;
+  L->loaded = false;
+  uint8_t* w13 = static_cast<uint8_t*>(L->w13);
+  MOE_CUDA(cudaMemcpy2DAsync(w13, 2 * IH, q_gate, IH, IH, L->E, cudaMemcpyDeviceToDevice, st));
+  MOE_CUDA(cudaMemcpy2DAsync(w13 + IH, 2 * IH, q_up, IH, IH, L->E, cudaMemcpyDeviceToDevice, st));
+  MOE_CUDA(cudaMemcpyAsync(L->wd, q_down, IH * L->E, cudaMemcpyDeviceToDevice, st));
+  MOE_CUDA(cudaMemcpyAsync(L->wscales, scales_host, static_cast<size_t>(L->E) * 3 * sizeof(float),
+                           cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  MOE_TRY(encode_weight_maps(L));
+  L->loaded = true;
+  return MOE_OK;
+}
+
+int moe_reserve(moe_layer* L, int M_max, void* stream) {
+  (void)stream;
+  if (!L || M_max < 0) return MOE_ERR_INVALID_ARG;
+  if (M_max == 0) return MOE_OK;
+  DeviceGuard g(L->device);
+  return ensure_workspace(L, M_max);
+}
+
+int moe_forward(moe_layer* L, const void* x, const float* logits, int M, void* out, void* stream) {
+  if (!L || M < 0) return MOE_ERR_INVALID_ARG;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  if (M == 0) {
+    L->last_launches = 0;
+    L->last_M = 0;
+    return MOE_OK;
+  }
+  if (M > (1 << 22) / L->k) return MOE_ERR_INVALID_ARG;
+  if (!x || !logits || !out || !aligned16(x) || !aligned16(logits) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  return forward_impl(L, x, logits, M, out, static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_host(moe_layer* L, const void* x_host, const float* logits_host, int M, void* out_host,
+                     void* stream) {
+  if (!L || M < 0) return MOE_ERR_INVALID_ARG;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  if (M == 0) {
+    L->last_launches = 0;
+    return MOE_OK;
+  }
+  if (!x_host || !logits_host || !out_host) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M > L->host_cap) {
+    MOE_CUDA(cudaDeviceSynchronize());
+    cudaFree(L->hx);
+    cudaFree(L->hl);
+    cudaFree(L->hout);
+    L->hx = L->hout = nullptr;
+    L->hl = nullptr;
+    L->host_cap = 0;
+    MOE_CUDA(cudaMalloc(&L->hx, static_cast<size_t>(M) * L->H * 2));
+    MOE_CUDA(cudaMalloc(&L->hl, static_cast<size_t>(M) * L->E * 4));
+    MOE_CUDA(cudaMalloc(&L->hout, static_cast<size_t>(M) * L->H * 2));
+    L->host_cap = M;
+  }
+  MOE_CUDA(cudaMemcpyAsync(L->hx, x_host, static_cast<size_t>(M) * L->H * 2, cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaMemcpyAsync(L->hl, logits_host, static_cast<size_t>(M) * L->E * 4, cudaMemcpyHostToDevice, st));
+  MOE_TRY(forward_impl(L, L->hx, L->hl, M, L->hout, st));
+  MOE_CUDA(cudaMemcpyAsync(out_host, L->hout, static_cast<size_t>(M) * L->H * 2, cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  return MOE_OK;
+}
+
+int moe_get_device_error(moe_layer* L, int* code) {
+  if (!L || !code) return MOE_ERR_INVALID_ARG;
+  *code = 0;
+  DeviceGuard g(L->device);
+  MOE_CUDA(cudaDeviceSynchronize());
+  if (!L->err) return MOE_OK;
+  MOE_CUDA(cudaMemcpy(code, L->err, 4, cudaMemcpyDeviceToHost));
+  MOE_CUDA(cudaMemset(L->err, 0, 4));
+  return MOE_OK;
+}
+
+int moe_last_launch_count(moe_layer* L) { return L ? L->last_launches : 0; }
+
+int moe_debug_routing(moe_layer* L, int* topk_ids, float* topk_w, int* counts, int* padded_offsets,
+                      int* padded_pairs, float* scales_host, int* tile_rows) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  MOE_CUDA(cudaDeviceSynchronize());
+  if (tile_rows) *tile_rows = moe::kPadRows;
+  if (L->M_cap == 0 || L->last_M == 0) return MOE_OK;
+  const size_t P = static_cast<size_t>(L->last_M) * L->k;
+  if (topk_ids) MOE_CUDA(cudaMemcpy(topk_ids, L->topk_ids, P * 4, cudaMemcpyDeviceToDevice));
+  if (topk_w) MOE_CUDA(cudaMemcpy(topk_w, L->topk_w, P * 4, cudaMemcpyDeviceToDevice));
+  if (counts) MOE_CUDA(cudaMemcpy(counts, L->counts, L->E * 4, cudaMemcpyDeviceToDevice));
+  if (padded_offsets) MOE_CUDA(cudaMemcpy(padded_offsets, L->poff, (L->E + 1) * 4, cudaMemcpyDeviceToDevice));
+  if (padded_pairs) {
+    int rows = 0;
+    MOE_CUDA(cudaMemcpy(&rows, L->header + moe::kHdrRowsUsed, 4, cudaMemcpyDeviceToHost));
+    MOE_CUDA(cudaMemcpy(padded_pairs, L->pairs, static_cast<size_t>(rows) * 4, cudaMemcpyDeviceToDevice));
+  }
+  if (scales_host) MOE_CUDA(cudaMemcpy(scales_host, L->last_scales, 8, cudaMemcpyDeviceToHost));
+  return MOE_OK;
+}
+
+int moe_debug_activations(moe_layer* L, void* x_perm_out, void* h_out) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  MOE_CUDA(cudaDeviceSynchronize());
+  if (L->M_cap == 0 || L->last_M == 0) return MOE_OK;
+  int rows = 0;
+  MOE_CUDA(cudaMemcpy(&rows, L->header + moe::kHdrRowsUsed, 4, cudaMemcpyDeviceToHost));
+  const size_t el = is_fp8(L) ? 1 : 2;
+  if (x_perm_out)
+    MOE_CUDA(cudaMemcpy(x_perm_out, L->x_perm, static_cast<size_t>(rows) * L->H * el, cudaMemcpyDeviceToDevice));
+  if (h_out) MOE_CUDA(cudaMemcpy(h_out, L->h, static_cast<size_t>(rows) * L->I * 2, cudaMemcpyDeviceToDevice));
+  return MOE_OK;
+}
+
+int moe_debug_weights(moe_layer* L, void* gate_out, void* up_out, void* down_out, float* scales_host) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  DeviceGuard g(L->device);
+  MOE_CUDA(cudaDeviceSynchronize());
+  const size_t el = is_fp8(L) ? 1 : 2;
+  const size_t IH = static_cast<size_t>(L->I) * L->H * el;
+  const uint8_t* w13 = static_cast<const uint8_t*>(L->w13);
+  if (gate_out) MOE_CUDA(cudaMemcpy2D(gate_out, IH, w13, 2 * IH, IH, L->E, cudaMemcpyDeviceToDevice));
+  if (up_out) MOE_CUDA(cudaMemcpy2D(up_out, IH, w13 + IH, 2 * IH, IH, L->E, cudaMemcpyDeviceToDevice));
+  if (down_out) MOE_CUDA(cudaMemcpy(down_out, L->wd, IH * L->E, cudaMemcpyDeviceToDevice));
+  if (scales_host && is_fp8(L))
+    MOE_CUDA(cudaMemcpy(scales_host, L->wscales, static_cast<size_t>(L->E) * 3 * 4, cudaMemcpyDeviceToHost));
+  return MOE_OK;
+}
+
+}  // extern "C"

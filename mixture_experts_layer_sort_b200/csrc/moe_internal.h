@@ -1,0 +1,137 @@
+// moe_internal.h - structures shared by the host dispatcher and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kPadRows = 16;        // every expert's group of rows is padded to 16 (B tile granule)
+constexpr int kTileRows = 128;      // weight rows per GEMM tile (the MMA's M slot)
+constexpr int kRowBytes = 128;      // bytes per K block row (one 128-byte swizzle atom)
+constexpr int kMaxSplits = 16;      // largest split-K factor the scheduler picks
+
+// Layout of the scheduler header written by the align kernel (int32 slots).
+enum HeaderSlot : int {
+  kHdrRowsUsed = 0,     // padded rows in use (= padded_offsets[E])
+  kHdrTiles1 = 1,       // gate_up tiles
+  kHdrSplits1 = 2,      // gate_up split-K factor
+  kHdrTiles2 = 3,       // down tiles
+  kHdrSplits2 = 4,      // down split-K factor
+  kHdrTokenBlocks = 5,  // (expert, token block) pairs
+  kHdrSlots = 8
+};
+
+// One output tile of a grouped GEMM: weight rows [fblock*128, +128) of expert
+// `expert` times the token rows [row_start, row_start + n_valid) of the permuted
+// activations (row_start is a multiple of 16; n_valid in 1..BN).
+struct __align__(16) Tile {
+  int expert;
+  int fblock;
+  int row_start;
+  int n_valid;
+};
+
+struct RouteArgs {
+  const float* logits;     // [M, E]
+  const __nv_bfloat16* x;  // [M, H], read only for the FP8 amax
+  int M, E, k, H;
+  int* topk_ids;           // [M, k]
+  float* topk_w;           // [M, k]
+  unsigned* amax_x;        // FP8 only (else nullptr): running max |x| as float bits
+};
+
+struct AlignArgs {
+  const int* topk_ids;     // [P]
+  int P, E, k;
+  int BN;                  // token rows per tile (the variant's N)
+  int fblocks1, fblocks2;  // I/128 and H/128
+  int kblocks1, kblocks2;  // K blocks of gate_up (H) and down (I)
+  int num_sms;
+  int ws1_rows_cap;        // split-K of gate_up needs rows_used <= this
+  int* counts;             // [E]
+  int* padded_offsets;     // [E+1]
+  int* padded_pairs;       // [rows_cap]
+  Tile* tiles1;
+  Tile* tiles2;
+  int* header;             // [kHdrSlots]
+};
+
+struct GatherArgs {
+  const __nv_bfloat16* x;  // [M, H]
+  const int* padded_pairs;
+  const int* header;
+  int rows_bound;          // grid covers this many rows; rows >= rows_used exit
+  int P, k, H;
+  void* x_perm;            // [rows_cap, H] bf16 or e4m3
+  const unsigned* amax_x;  // FP8 only
+};
+
+struct GemmArgs {
+  const Tile* tiles;
+  const int* header;
+  int hdr_tiles, hdr_splits;
+  int kblocks;             // K blocks over the whole reduction
+  int w_rows_per_expert;   // rows of one expert in the 2-D weight map (2I or H)
+  int up_offset;           // gate_up: row offset of W_up inside an expert (I); else 0
+  // gate_up epilogue
+  __nv_bfloat16* h;        // [rows_cap, I]
+  int I;
+  float* ws1;              // [ws1_rows_cap, 2I] split-K partial sums (zero between uses)
+  int* tile_counters;      // [tiles1_cap] (zero between uses)
+  unsigned* amax_h;        // FP8: running max |h| as float bits
+  const unsigned* amax_x;  // FP8: max |x| (for s_x)
+  const float* w_scales;   // FP8: [E, 3]
+  // down epilogue
+  float* acc;              // [M, H] fp32 accumulator (zero between uses)
+  int H;
+  const int* padded_pairs;
+  const float* topk_w;
+  int k, P;
+  int* err;
+};
+
+struct QuantHArgs {
+  const __nv_bfloat16* h;
+  uint8_t* h_q;
+  const int* padded_pairs;
+  const int* header;
+  int rows_bound, P, I;
+  const unsigned* amax_h;
+};
+
+struct FinalizeArgs {
+  float* acc;              // [M, H]
+  __nv_bfloat16* out;      // [M, H]
+  long long n;             // M*H
+  unsigned* amax;          // [2] reset to 0 (may be nullptr)
+  float* last_scales;      // [2] s_x, s_h of this forward (may be nullptr)
+};
+
+// Variant table: precompiled (BN, stages) choices; picked on the host by M*k.
+enum Variant : int { kVariantSmall = 0, kVariantMedium = 1, kVariantLarge = 2, kNumVariants = 3 };
+int variant_bn(int v);
+
+// Kernel launchers (each returns the cudaError_t of its launch).
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_align(const AlignArgs& a, cudaStream_t s);
+cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s);
+cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8,
+                         int variant, int grid, cudaStream_t s);
+cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8,
+                         int variant, int grid, cudaStream_t s);
+cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s);
+cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
+cudaError_t gemm_configure();    // opt-in dynamic shared memory sizes (current device)
+cudaError_t align_configure();
+
+// Weight preparation (load time, not on the forward path).
+cudaError_t launch_weight_amax(const __nv_bfloat16* w, long long per_expert, int E,
+                               float* scales, int stride, cudaStream_t s);
+cudaError_t launch_weight_quant(const __nv_bfloat16* w, long long per_expert, int E,
+                                const float* scales, int stride, uint8_t* q, long long q_expert_stride,
+                                cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,153 @@
+"""Thin Python binding of the fused MoE layer: argument marshalling only.
+
+Every step of the forward pass runs in libmoe_b200.so; torch supplies device
+memory and streams.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import load_library, status_string
+
+BF16, FP8 = 0, 1
+_DTYPES = {"bf16": BF16, "fp8": FP8, "e4m3": FP8, BF16: BF16, FP8: FP8}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+        self.code = code
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class MoELayer:
+    """One fused MoE layer: E experts, top-k routing, hidden H, expert intermediate I."""
+
+    def __init__(self, E: int, topk: int, H: int, I: int, dtype="bf16"):
+        self.lib = load_library()
+        self.E, self.k, self.H, self.I = E, topk, H, I
+        self.dtype = _DTYPES[dtype]
+        h = ctypes.c_void_p()
+        self._check("moe_create", self.lib.moe_create(E, topk, H, I, self.dtype, ctypes.byref(h)))
+        self.handle = h.value
+
+    def _check(self, fn, code):
+        if code != 0:
+            raise MoEError(fn, code)
+
+    @property
+    def is_fp8(self) -> bool:
+        return self.dtype == FP8
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------------ weights
+    def load_weights(self, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, stream=None):
+        """bf16 device tensors W_gate [E,I,H], W_up [E,I,H], W_down [E,H,I]."""
+        for t, shape in ((w_gate, (self.E, self.I, self.H)), (w_up, (self.E, self.I, self.H)),
+                         (w_down, (self.E, self.H, self.I))):
+            assert t.is_cuda and t.dtype == torch.bfloat16 and tuple(t.shape) == shape and t.is_contiguous()
+        self._check("moe_load_weights", self.lib.moe_load_weights(
+            self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), _stream(stream)))
+
+    def load_weights_fp8(self, q_gate, q_up, q_down, scales, stream=None):
+        """uint8 e4m3 codes (device) and scales [E,3] fp32 (host)."""
+        sc = torch.as_tensor(scales, dtype=torch.float32).contiguous().cpu()
+        self._check("moe_load_weights_fp8", self.lib.moe_load_weights_fp8(
+            self.handle, _ptr(q_gate), _ptr(q_up), _ptr(q_down), sc.data_ptr(), _stream(stream)))
+
+    def reserve(self, M_max: int, stream=None):
+        self._check("moe_reserve", self.lib.moe_reserve(self.handle, M_max, _stream(stream)))
+
+    # ------------------------------------------------------------------ forward
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        M = x.shape[0]
+        if out is None:
+            out = torch.empty((M, self.H), dtype=torch.bfloat16, device=x.device)
+        self._check("moe_forward", self.lib.moe_forward(
+            self.handle, _ptr(x), _ptr(logits), M, _ptr(out), _stream(stream)))
+        return out
+
+    __call__ = forward
+
+    def forward_raw(self, x_ptr: int, logits_ptr: int, M: int, out_ptr: int, stream_handle: int):
+        self._check("moe_forward", self.lib.moe_forward(self.handle, x_ptr, logits_ptr, M, out_ptr, stream_handle))
+
+    def forward_host(self, x_cpu: torch.Tensor, logits_cpu: torch.Tensor, out_cpu: torch.Tensor, stream=None):
+        M = x_cpu.shape[0]
+        self._check("moe_forward_host", self.lib.moe_forward_host(
+            self.handle, _ptr(x_cpu), _ptr(logits_cpu), M, _ptr(out_cpu), _stream(stream)))
+        return out_cpu
+
+    @property
+    def last_launch_count(self) -> int:
+        return self.lib.moe_last_launch_count(self.handle)
+
+    def device_error(self) -> int:
+        c = ctypes.c_int(0)
+        self._check("moe_get_device_error", self.lib.moe_get_device_error(self.handle, ctypes.byref(c)))
+        return c.value
+
+    # ------------------------------------------------------------------ test access
+    def debug_routing(self, M: int):
+        dev = torch.device("cuda")
+        P = M * self.k
+        ids = torch.empty((M, self.k), dtype=torch.int32, device=dev)
+        w = torch.empty((M, self.k), dtype=torch.float32, device=dev)
+        counts = torch.empty(self.E, dtype=torch.int32, device=dev)
+        poff = torch.empty(self.E + 1, dtype=torch.int32, device=dev)
+        cap = P + min(self.E, P) * 15 + 16
+        pairs = torch.empty(cap, dtype=torch.int32, device=dev)
+        scales = torch.empty(2, dtype=torch.float32)
+        tile = ctypes.c_int(0)
+        self._check("moe_debug_routing", self.lib.moe_debug_routing(
+            self.handle, _ptr(ids), _ptr(w), _ptr(counts), _ptr(poff), _ptr(pairs), scales.data_ptr(),
+            ctypes.byref(tile)))
+        rows = int(poff[-1].item())
+        return {"ids": ids, "w": w, "counts": counts, "padded_offsets": poff, "padded_pairs": pairs[:rows],
+                "s_x": float(scales[0]), "s_h": float(scales[1]), "tile_rows": tile.value}
+
+    def debug_activations(self, rows: int):
+        dev = torch.device("cuda")
+        xp = torch.empty((rows, self.H), dtype=torch.uint8 if self.is_fp8 else torch.bfloat16, device=dev)
+        h = torch.empty((rows, self.I), dtype=torch.bfloat16, device=dev)
+        self._check("moe_debug_activations", self.lib.moe_debug_activations(self.handle, _ptr(xp), _ptr(h)))
+        return xp, h
+
+    def debug_weights(self):
+        dev = torch.device("cuda")
+        dt = torch.uint8 if self.is_fp8 else torch.bfloat16
+        g = torch.empty((self.E, self.I, self.H), dtype=dt, device=dev)
+        u = torch.empty((self.E, self.I, self.H), dtype=dt, device=dev)
+        d = torch.empty((self.E, self.H, self.I), dtype=dt, device=dev)
+        sc = torch.ones((self.E, 3), dtype=torch.float32)
+        self._check("moe_debug_weights", self.lib.moe_debug_weights(
+            self.handle, _ptr(g), _ptr(u), _ptr(d), sc.data_ptr()))
+        return g, u, d, sc
