@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 fused MoE layer.
+
+Default workload (N=1): the decode layer E=128 experts, top-8, H=2048, I=768,
+bf16 weights (1.2 GB), at the four decode batch sizes M = 1, 4, 16, 64. One
+step = one forward at each of the four M (85 tokens); the L2 cache (126 MB) is
+flushed before every forward by writing a 252 MB buffer, outside the timed
+events. Each forward is replayed from a CUDA graph captured once per M (the
+forward is a fixed launch chain with no host synchronisation).
+
+Reported (one JSON line, rank 0):
+  value      tokens/s over all ranks = N * 85 / (device time of one step)
+  roofline   gate_up GEMM (the kernel with the largest share): active-expert
+             W_gate+W_up bytes per launch / its CUDA-event duration, against
+             the measured HBM copy bandwidth
+  e2e        the same metric through moe_forward_host: host->device copies of
+             x and logits and the device->host copy of out inside the timing
+  cpu_baseline  the CPU oracle timed on the same decode sweep on the host cores
+
+--impl reference times the CPU oracle itself on the same workload (the
+reference arm); --gpus N runs N independent replicas (the layer needs no
+collective), max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused-MoE tokens/s and HBM GB/s vs roofline (decode M=1-64, prefill), 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 252 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["tiny", "decode", "decode_fp8", "large_decode", "prefill", "prefill_fp8"])
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying graphs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--only-M", type=int, default=None, help="run a single batch size of the workload")
+    return ap.parse_args()
+
+
+def workload_spec(name):
+    from mixture_experts_layer_sort_b200 import synth
+    if name == "prefill_fp8":
+        wl = synth.WORKLOADS["prefill"]
+        return wl, "fp8"
+    wl = synth.WORKLOADS[name]
+    return wl, wl.dtypes[0]
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def weight_bytes(wl, dtype):
+    return 1 if dtype == "fp8" else 2
+
+
+def alg_bytes_layer(wl, dtype, M, A):
+    """Algorithmic bytes of one forward: active-expert weights, FP8 scales, x, out, logits."""
+    bw = weight_bytes(wl, dtype)
+    b = A * 3 * wl.H * wl.I * bw + M * wl.H * 2 * 2 + M * wl.E * 4
+    if dtype == "fp8":
+        b += 3 * wl.E * 4
+    return b
+
+
+def alg_flops_layer(wl, M):
+    return 6 * M * wl.k * wl.H * wl.I
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = max((num(r[2]) for r in rows if num(r[2]) is not None), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        under_load = [v for v in sm if smax and v >= 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(under_load) if under_load else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, ws):
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    on_gpu = dist.get_backend() == "nccl"
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def time_oracle_sweep(wl, dtype, host_weights, tokens_per_M, budget_s=30.0, max_reps=50):
+    """Seconds per decode sweep of the CPU oracle (bounded: at least one sweep)."""
+    from oracle import moe_oracle as O
+    cache = {}
+    times = []
+    t_start = time.time()
+    for _ in range(max_reps):
+        t0 = time.time()
+        for M, (x, l) in tokens_per_M.items():
+            O.moe_forward(x, l, wl.k, *host_weights, fp8=(dtype == "fp8"), weight_cache=cache)
+        times.append(time.time() - t0)
+        if time.time() - t_start > budget_s:
+            break
+    return statistics.median(times), len(times)
+
+
+def reference_arm(args, ws, rank):
+    """The CPU oracle as the reference arm: rank 0 times it, the others exit."""
+    if rank != 0:
+        return 0
+    import torch
+    from mixture_experts_layer_sort_b200 import synth
+    wl, dtype = workload_spec(args.workload)
+    Ms = list(wl.Ms)
+    if args.workload in ("prefill", "prefill_fp8", "large_decode"):
+        print(json.dumps({"impl": "reference", "unavailable": "the CPU oracle needs the 22.5 GB weight set "
+                          "on the host; the reference arm runs on the decode workloads"}))
+        return 0
+    wg, wu, wd = synth.make_weights(wl.E, wl.H, wl.I, wl.w_std, seed=args.seed, device="cpu")
+    host = [w.float().numpy() for w in (wg, wu, wd)]
+    toks = {}
+    for M in Ms:
+        x, l = synth.make_tokens(wl.E, wl.H, M, seed=args.seed, zipf_s=wl.zipf_s)
+        toks[M] = (x.float().numpy(), l.numpy())
+    tokens = sum(Ms)
+    from oracle import moe_oracle as O
+    cache = {}
+    for _ in range(max(args.warmup, 0)):
+        for M, (x, l) in toks.items():
+            O.moe_forward(x, l, wl.k, *host, fp8=(dtype == "fp8"), weight_cache=cache)
+        break   # one warm-up sweep is enough for the CPU path (fills the FP8 weight cache)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.time()
+        for M, (x, l) in toks.items():
+            O.moe_forward(x, l, wl.k, *host, fp8=(dtype == "fp8"), weight_cache=cache)
+        times.append(time.time() - t0)
+    sec = statistics.mean(times)
+    value = tokens / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.description + f", M in {Ms} per step", "Ms": Ms, "global_batch": tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"full decode sweep M={Ms} ({tokens} tokens) per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------- main arm
+def traffic_from_profile(kernel_src_hash):
+    """Per-launch DRAM bytes of the gate_up GEMM from the committed ncu summary, or None
+    when the kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "gate_up_gemm_decode_traffic.txt")
+    try:
+        d = {}
+        with open(p) as f:
+            for line in f:
+                if "=" in line and not line.startswith("#"):
+                    k, v = line.split("=", 1)
+                    d[k.strip()] = v.strip()
+        if d.get("kernel_source_sha256") != kernel_src_hash:
+            return None
+        return {int(k.split("_")[-1]): float(v) for k, v in d.items() if k.startswith("dram_bytes_per_launch_M_")}
+    except Exception:
+        return None
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("kernels_gemm.cu", "sm100.cuh", "moe_internal.h"):
+        with open(os.path.join(ROOT, "mixture_experts_layer_sort_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def main():
+    args = parse_args()
+    ws, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        rc = reference_arm(args, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+
+    import numpy as np
+    import torch
+
+    from mixture_experts_layer_sort_b200 import MoELayer, synth
+
+    wl, dtype = workload_spec(args.workload)
+    Ms = [args.only_M] if args.only_M else list(wl.Ms)
+    dev = torch.device("cuda", local)
+    seed = args.seed + 1000 * rank
+    wg, wu, wd = synth.make_weights(wl.E, wl.H, wl.I, wl.w_std, seed=args.seed, device=dev)
+    layer = MoELayer(wl.E, wl.k, wl.H, wl.I, dtype)
+    layer.load_weights(wg, wu, wd)
+    layer.reserve(max(Ms))
+    toks = {M: synth.make_tokens(wl.E, wl.H, M, seed=seed, device=dev, zipf_s=wl.zipf_s) for M in Ms}
+    outs = {M: torch.empty((M, wl.H), dtype=torch.bfloat16, device=dev) for M in Ms}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    tokens_per_step = sum(Ms)
+
+    # active experts per M (from this forward's own routing counts)
+    A = {}
+    with torch.cuda.stream(stream):
+        for M in Ms:
+            layer.forward(*toks[M], out=outs[M])
+            A[M] = int(torch.count_nonzero(layer.debug_routing(M)["counts"]).item())
+    launches_per_M = {}
+    for M in Ms:
+        with torch.cuda.stream(stream):
+            layer.forward(*toks[M], out=outs[M])
+        launches_per_M[M] = layer.last_launch_count
+    torch.cuda.synchronize()
+
+    graphs = {}
+    if not args.no_graph:
+        for M in Ms:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                layer.forward(*toks[M], out=outs[M])
+            graphs[M] = g
+        torch.cuda.synchronize()
+
+    def run_forward(M):
+        if graphs:
+            graphs[M].replay()
+        else:
+            layer.forward(*toks[M], out=outs[M])
+
+    def step(events=None):
+        for i, M in enumerate(Ms):
+            flush.zero_()
+            if events is not None:
+                events[i][0].record(stream)
+            run_forward(M)
+            if events is not None:
+                events[i][1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------------------------- timed region
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in Ms]
+          for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for s in range(args.steps):
+            step(ev[s])
+    torch.cuda.synchronize()
+    wall = time.time() - t0
+    barrier(ws)
+    per_M_ms = {M: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i, M in enumerate(Ms)}
+    step_ms = [sum(per_M_ms[M][s] for M in Ms) for s in range(args.steps)]
+    ms_per_step = max_over_ranks(statistics.mean(step_ms), ws)
+
+    # ---------------------------------------------------------------- per-kernel events (same workload, eager)
+    layer.profile_enable(True)
+    prof_steps = max(3, min(args.steps, 20))
+    gate_bytes = 0.0
+    with torch.cuda.stream(stream):
+        for s in range(prof_steps):
+            for M in Ms:
+                flush.zero_()
+                layer.forward(*toks[M], out=outs[M])
+                gate_bytes += A[M] * 2 * wl.H * wl.I * weight_bytes(wl, dtype)
+    prof = layer.profile_read()
+    layer.profile_enable(False)
+    clk = clocks.stop()
+
+    hbm_gbs, bf16_tf, peak_src = read_peaks()
+    g_ms, g_n = prof["gate_up"]
+    achieved = gate_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else None
+    traffic_tbl = traffic_from_profile(kernel_source_hash())
+    traffic = None
+    if traffic_tbl and all(M in traffic_tbl for M in Ms):
+        traffic = statistics.mean(traffic_tbl[M] for M in Ms)
+    total_prof = sum(v[0] for v in prof.values())
+
+    # ---------------------------------------------------------------- e2e through host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {M: (toks[M][0].cpu().pin_memory(), toks[M][1].cpu().pin_memory(),
+                    torch.empty((M, wl.H), dtype=torch.bfloat16).pin_memory()) for M in Ms}
+        h2d = sum(M * wl.H * 2 + M * wl.E * 4 for M in Ms)
+        d2h = sum(M * wl.H * 2 for M in Ms)
+        for _ in range(2):
+            for M in Ms:
+                layer.forward_host(*host[M], stream=stream)
+        e_times = []
+        for s in range(args.steps):
+            tot = 0.0
+            for M in Ms:
+                flush.zero_()
+                torch.cuda.synchronize()
+                a = time.perf_counter()
+                layer.forward_host(*host[M], stream=stream)
+                tot += time.perf_counter() - a
+            e_times.append(tot)
+        e_sec = max_over_ranks(statistics.mean(e_times), ws)
+        e2e = {"value": ws * tokens_per_step / e_sec, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_sec * 1e3}
+
+    # ---------------------------------------------------------------- CPU oracle on the same sweep
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and args.workload in ("tiny", "decode", "decode_fp8"):
+        host_w = [synth.bf16_to_f32_numpy(w) for w in (wg, wu, wd)]
+        tpm = {M: (toks[M][0].float().cpu().numpy(), toks[M][1].cpu().numpy()) for M in Ms}
+        sec, reps = time_oracle_sweep(wl, dtype, host_w, tpm)
+        cpu = {"value": tokens_per_step / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{reps} full decode sweep(s) M={Ms} ({tokens_per_step} tokens), median"}
+
+    per_M = {}
+    for M in Ms:
+        t = statistics.mean(per_M_ms[M])
+        b = alg_bytes_layer(wl, dtype, M, A[M])
+        per_M[str(M)] = {"ms": t, "tokens_per_s": M / (t / 1e3), "active_experts": A[M],
+                         "alg_GB": b / 1e9, "alg_GBps": b / (t / 1e3) / 1e9,
+                         "roofline_frac": (b / (hbm_gbs * 1e9)) / (t / 1e3), "launches": launches_per_M[M]}
+
+    line = {
+        "metric": METRIC,
+        "value": ws * tokens_per_step / (ms_per_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if dtype == "bf16" else "e4m3",
+        "data": "synthetic",
+        "config": {"workload": wl.description + f", one step = one forward at each M in {Ms}",
+                   "E": wl.E, "topk": wl.k, "H": wl.H, "I": wl.I, "Ms": Ms, "global_batch": tokens_per_step * ws,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": "flushed (252 MB write) before every forward, outside the timed events",
+                   "launch": "CUDA graph replay per M" if graphs else "eager"},
+        "roofline": {"bound": "hbm", "kernel": "gate_up grouped GEMM", "achieved": achieved, "peak": hbm_gbs,
+                     "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None, "traffic": traffic,
+                     "peak_source": f"{peak_src} HBM copy bandwidth",
+                     "alg_bytes_per_launch": gate_bytes / max(g_n, 1),
+                     "avg_launch_ms": g_ms / max(g_n, 1)},
+        "kernel_share": {k: round(v[0] / total_prof, 4) for k, v in prof.items() if v[1] > 0} if total_prof else {},
+        "per_M": per_M,
+        "e2e": e2e,
+        "gpu_launches": sum(launches_per_M[M] for M in Ms) * args.steps,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "wall_s_timed": wall,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    for g in graphs.values():
+        del g
+    layer.close()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

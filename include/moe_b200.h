@@ -126,6 +126,19 @@ MOE_API int moe_get_device_error(moe_layer* layer, int* code);
 /* Number of kernels the last moe_forward launched (0 for M = 0). */
 MOE_API int moe_last_launch_count(moe_layer* layer);
 
+/* Per-kernel timing. While enabled, every moe_forward records a CUDA event
+ * before and after each kernel it launches, on the forward's stream. Kernel
+ * slots: 0 route, 1 align, 2 gather, 3 gate_up GEMM, 4 h quantise (FP8 only),
+ * 5 down GEMM, 6 finalise (MOE_PROFILE_SLOTS in all). Enabling clears the totals.
+ * Do not enable it while capturing moe_forward into a CUDA graph. */
+#define MOE_PROFILE_SLOTS 7
+MOE_API int moe_profile_enable(moe_layer* layer, int enable);
+
+/* Synchronise the device, then write per slot the summed kernel time in ms
+ * (ms_sum[MOE_PROFILE_SLOTS], host) and the number of timed launches
+ * (launches[MOE_PROFILE_SLOTS], host) since profiling was enabled. */
+MOE_API int moe_profile_read(moe_layer* layer, double* ms_sum, int* launches);
+
 /* Test access: copy the routing of the last forward to caller device buffers
  * (any pointer may be NULL to skip it), after synchronising the device:
  *   topk_ids [M, k] int32, topk_w [M, k] fp32, counts [E] int32,

@@ -62,6 +62,16 @@ struct moe_layer {
   int host_cap = 0;
   // bookkeeping
   int last_M = 0, last_launches = 0, last_variant = 0;
+  // per-kernel event timing
+  bool profiling = false;
+  struct Timed {
+    int slot;
+    cudaEvent_t a, b;
+  };
+  std::vector<Timed> pending;
+  std::vector<cudaEvent_t> event_pool;
+  double prof_ms[MOE_PROFILE_SLOTS] = {0};
+  int prof_n[MOE_PROFILE_SLOTS] = {0};
 };
 
 namespace {
@@ -214,6 +224,53 @@ int encode_weight_maps(moe_layer* L) {
   return MOE_OK;
 }
 
+cudaEvent_t pool_event(moe_layer* L) {
+  if (!L->event_pool.empty()) {
+    cudaEvent_t e = L->event_pool.back();
+    L->event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Records an event pair around one kernel launch when profiling is on.
+struct KernelTimer {
+  moe_layer* L;
+  int slot;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  KernelTimer(moe_layer* l, int s, cudaStream_t stream) : L(l), slot(s), st(stream) {
+    if (L->profiling && (a = pool_event(L)) != nullptr) cudaEventRecord(a, st);
+  }
+  ~KernelTimer() {
+    if (!a) return;
+    cudaEvent_t b = pool_event(L);
+    if (!b) {
+      L->event_pool.push_back(a);
+      return;
+    }
+    cudaEventRecord(b, st);
+    L->pending.push_back({slot, a, b});
+  }
+};
+
+int drain_profile(moe_layer* L) {
+  MOE_CUDA(cudaDeviceSynchronize());
+  for (auto& t : L->pending) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, t.a, t.b) == cudaSuccess) {
+      L->prof_ms[t.slot] += ms;
+      L->prof_n[t.slot] += 1;
+    }
+    L->event_pool.push_back(t.a);
+    L->event_pool.push_back(t.b);
+  }
+  L->pending.clear();
+  return MOE_OK;
+}
+
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
   const bool fp8 = is_fp8(L);
@@ -233,7 +290,10 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   ra.topk_ids = L->topk_ids;
   ra.topk_w = L->topk_w;
   ra.amax_x = fp8 ? L->amax : nullptr;
-  MOE_CUDA(moe::launch_route(ra, st));
+  {
+    KernelTimer kt(L, 0, st);
+    MOE_CUDA(moe::launch_route(ra, st));
+  }
   ++launches;
 
   moe::AlignArgs aa{};
@@ -255,7 +315,10 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   aa.tiles1 = L->tiles1;
   aa.tiles2 = L->tiles2;
   aa.header = L->header;
-  MOE_CUDA(moe::launch_align(aa, st));
+  {
+    KernelTimer kt(L, 1, st);
+    MOE_CUDA(moe::launch_align(aa, st));
+  }
   ++launches;
 
   moe::GatherArgs ga{};
@@ -268,7 +331,10 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   ga.H = L->H;
   ga.x_perm = L->x_perm;
   ga.amax_x = L->amax;
-  MOE_CUDA(moe::launch_gather(ga, fp8, st));
+  {
+    KernelTimer kt(L, 2, st);
+    MOE_CUDA(moe::launch_gather(ga, fp8, st));
+  }
   ++launches;
 
   moe::GemmArgs g{};
@@ -295,7 +361,10 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g1.kblocks = aa.kblocks1;
   g1.w_rows_per_expert = 2 * L->I;
   g1.up_offset = L->I;
-  MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, L->tm_x, fp8, variant, L->num_sms, st));
+  {
+    KernelTimer kt(L, 3, st);
+    MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, L->tm_x, fp8, variant, L->num_sms, st));
+  }
   ++launches;
 
   if (fp8) {
@@ -308,7 +377,10 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
     qa.P = static_cast<int>(P);
     qa.I = L->I;
     qa.amax_h = L->amax + 1;
-    MOE_CUDA(moe::launch_quant_h(qa, st));
+    {
+      KernelTimer kt(L, 4, st);
+      MOE_CUDA(moe::launch_quant_h(qa, st));
+    }
     ++launches;
   }
 
@@ -319,7 +391,10 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g2.kblocks = aa.kblocks2;
   g2.w_rows_per_expert = L->H;
   g2.up_offset = 0;
-  MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, variant, L->num_sms, st));
+  {
+    KernelTimer kt(L, 5, st);
+    MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, variant, L->num_sms, st));
+  }
   ++launches;
 
   moe::FinalizeArgs fa{};
@@ -328,7 +403,10 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   fa.n = static_cast<long long>(M) * L->H;
   fa.amax = fp8 ? L->amax : nullptr;
   fa.last_scales = fp8 ? L->last_scales : nullptr;
-  MOE_CUDA(moe::launch_finalize(fa, st));
+  {
+    KernelTimer kt(L, 6, st);
+    MOE_CUDA(moe::launch_finalize(fa, st));
+  }
   ++launches;
 
   L->last_M = M;
@@ -403,6 +481,11 @@ int moe_destroy(moe_layer* L) {
   cudaFree(L->hx);
   cudaFree(L->hl);
   cudaFree(L->hout);
+  for (auto& t : L->pending) {
+    cudaEventDestroy(t.a);
+    cudaEventDestroy(t.b);
+  }
+  for (auto e : L->event_pool) cudaEventDestroy(e);
   delete L;
   return MOE_OK;
 }
@@ -523,6 +606,29 @@ int moe_get_device_error(moe_layer* L, int* code) {
 }
 
 int moe_last_launch_count(moe_layer* L) { return L ? L->last_launches : 0; }
+
+int moe_profile_enable(moe_layer* L, int enable) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  MOE_TRY(drain_profile(L));
+  for (int i = 0; i < MOE_PROFILE_SLOTS; ++i) {
+    L->prof_ms[i] = 0.0;
+    L->prof_n[i] = 0;
+  }
+  L->profiling = enable != 0;
+  return MOE_OK;
+}
+
+int moe_profile_read(moe_layer* L, double* ms_sum, int* launches) {
+  if (!L || !ms_sum || !launches) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  MOE_TRY(drain_profile(L));
+  for (int i = 0; i < MOE_PROFILE_SLOTS; ++i) {
+    ms_sum[i] = L->prof_ms[i];
+    launches[i] = L->prof_n[i];
+  }
+  return MOE_OK;
+}
 
 int moe_debug_routing(moe_layer* L, int* topk_ids, float* topk_w, int* counts, int* padded_offsets,
                       int* padded_pairs, float* scales_host, int* tile_rows) {

@@ -110,6 +110,19 @@ class MoELayer:
     def last_launch_count(self) -> int:
         return self.lib.moe_last_launch_count(self.handle)
 
+    KERNEL_SLOTS = ("route", "align", "gather", "gate_up", "quant_h", "down", "finalize")
+
+    def profile_enable(self, enable: bool = True):
+        self._check("moe_profile_enable", self.lib.moe_profile_enable(self.handle, 1 if enable else 0))
+
+    def profile_read(self):
+        """{kernel: (total ms, launches)} since profiling was enabled."""
+        ms = (ctypes.c_double * 7)()
+        n = (ctypes.c_int * 7)()
+        self._check("moe_profile_read", self.lib.moe_profile_read(self.handle, ctypes.addressof(ms),
+                                                                  ctypes.addressof(n)))
+        return {k: (ms[i], n[i]) for i, k in enumerate(self.KERNEL_SLOTS)}
+
     def device_error(self) -> int:
         c = ctypes.c_int(0)
         self._check("moe_get_device_error", self.lib.moe_get_device_error(self.handle, ctypes.byref(c)))

@@ -184,8 +184,16 @@ def quantize(t: np.ndarray, s: np.float32) -> np.ndarray:
     return e4m3_encode(q.astype(np.float32))
 
 
+_E4M3_TABLE = None
+
+
 def dequantize(codes: np.ndarray, s) -> np.ndarray:
-    return e4m3_decode(codes) * float(s)
+    """decode(code) * s in fp64; the decode goes through a 256-entry table of
+    e4m3_decode, which is the same function evaluated once per code."""
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        _E4M3_TABLE = e4m3_decode(np.arange(256, dtype=np.uint8))
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)] * float(s)
 
 
 def quantize_expert_weights(W: np.ndarray):
@@ -227,8 +235,18 @@ class _Weights:
                 np.asarray(d, dtype=np.float32))
 
 
+def _map_experts(fn, experts, threads):
+    """fn(e) for every e, in expert order; threads only overlap independent experts."""
+    if threads <= 1 or len(experts) <= 1:
+        return [fn(e) for e in experts]
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return list(ex.map(fn, experts))
+
+
 def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
-                provider=None, tokens=None, return_intermediates=False):
+                provider=None, tokens=None, return_intermediates=False, threads=None,
+                weight_cache=None):
     """The layer's output in fp64.
 
     x       [M, H]  bf16 values (any float array holding them)
@@ -243,6 +261,11 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
     tokens  optional list of token indices whose output rows are wanted; the
             other rows come back as NaN. Routing, the permutation, s_x and
             (FP8) s_h are still computed over the whole batch, as defined.
+    threads experts are independent, so they may be evaluated on several
+            threads (default: the CPU count); no result depends on it.
+    weight_cache  optional dict reused across calls with the same weights: it
+            keeps each expert's FP8 scales and codes so that they are not
+            recomputed (the values are identical either way).
 
     Returns out [M, H] float64, or (out, dict of intermediates).
     """
@@ -272,61 +295,79 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
     if tokens is not None:
         want[np.asarray(tokens, dtype=np.int64)] = True
 
+    if threads is None:
+        import os
+        threads = os.cpu_count() or 1
+
     def expert_weights(e):
-        g_w, u_w, d_w = W.get(e)
         if not fp8:
+            g_w, u_w, d_w = W.get(e)
             return g_w.astype(np.float64), u_w.astype(np.float64), d_w.astype(np.float64)
-        s_g, s_u, s_d = per_tensor_scale(g_w), per_tensor_scale(u_w), per_tensor_scale(d_w)
-        inter["w_scales"][e] = (s_g, s_u, s_d)
-        return (dequantize(quantize(g_w, s_g), s_g), dequantize(quantize(u_w, s_u), s_u),
-                dequantize(quantize(d_w, s_d), s_d))
+        q = weight_cache.get(e) if weight_cache is not None else None
+        if q is None:
+            q = []
+            for t in W.get(e):
+                st = per_tensor_scale(t)
+                q.append((st, quantize(t, st)))
+            if weight_cache is not None:
+                weight_cache[e] = q
+        return tuple(dequantize(c, st) for st, c in q), tuple(st for st, _ in q)
+
+    active = [e for e in range(E) if counts[e] > 0]
 
     # pass 1: gate/up projections and SwiGLU. FP8 needs every valid h row for
     # the amax behind s_h; the bf16 path only needs the wanted tokens' pairs.
-    h_rows = {}
-    h_amax = np.float32(0.0)
-    Y = {}
-    for e in range(E):
+    def pass1(e):
         n = int(counts[e])
-        if n == 0:
-            continue
         pairs = sorted_pairs[offsets[e]:offsets[e] + n]
         sel = want[pairs // k]
         if not fp8 and not sel.any():
-            continue
-        g_w, u_w, d_w = expert_weights(e)
+            return e, None
+        if fp8:
+            (g_w, u_w, d_w), sc = expert_weights(e)
+            inter["w_scales"][e] = sc
+        else:
+            g_w, u_w, d_w = expert_weights(e)
         rows = pairs if fp8 else pairs[sel]
         X = xin[rows // k]
         Hh = silu(X @ g_w.T) * (X @ u_w.T)
+        amax = np.float32(np.max(np.abs(Hh.astype(np.float32)))) if fp8 else None
+        keep = {int(p): Hh[i] for i, p in enumerate(rows) if want[p // k]}
+        Ym = None if fp8 else Hh @ d_w.T      # bf16 path: down projection right away
+        return e, (rows, keep, amax, Ym)
+
+    h_rows, Y = {}, {}
+    h_amax = np.float32(0.0)
+    for e, res in _map_experts(pass1, active, threads):
+        if res is None:
+            continue
+        rows, keep, amax, Ym = res
+        h_rows.update(keep)
         if fp8:
-            h_amax = max(h_amax, np.float32(np.max(np.abs(Hh.astype(np.float32)))))
-            for i, p in enumerate(rows):
-                if want[p // k]:
-                    h_rows[int(p)] = Hh[i]
+            h_amax = max(h_amax, amax)
         else:
-            # bf16 path: down projection right away
-            Ym = Hh @ d_w.T
             for i, p in enumerate(rows):
-                h_rows[int(p)] = Hh[i]
                 Y[int(p)] = Ym[i]
 
     if fp8:
         s_h = np.float32(1.0) if h_amax == 0 else np.float32(h_amax) / np.float32(E4M3_MAX)
         inter["s_h"] = s_h
+
         # pass 2: quantised h through the dequantised down projection
-        for e in range(E):
+        def pass2(e):
             n = int(counts[e])
-            if n == 0:
-                continue
             pairs = [int(p) for p in sorted_pairs[offsets[e]:offsets[e] + n] if want[int(p) // k]]
             if not pairs:
-                continue
-            d_w = expert_weights(e)[2]
+                return []
+            d_w = expert_weights(e)[0][2]
             Hm = np.stack([h_rows[p] for p in pairs])
             Hm = dequantize(quantize(Hm.astype(np.float32), s_h), s_h)
             Ym = Hm @ d_w.T
-            for i, p in enumerate(pairs):
-                Y[p] = Ym[i]
+            return [(p, Ym[i]) for i, p in enumerate(pairs)]
+
+        for res in _map_experts(pass2, active, threads):
+            for p, y in res:
+                Y[p] = y
 
     out = np.full((M, H), np.nan, dtype=np.float64)
     for t in range(M):

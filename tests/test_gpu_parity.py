@@ -119,3 +119,13 @@ def test_repeated_calls_are_stable(tiny):
     # scatter-add order may differ between calls: compare within bf16 rounding
     assert torch.max(torch.abs(a - b)).item() <= 1e-2 * torch.max(torch.abs(a)).item()
     assert tiny.layer.device_error() == 0
+
+
+def test_tiny_large_variant(tiny):
+    # M*k > 4096 selects the widest tile variant (256 token rows per tile)
+    M = 2500
+    x, logits = tokens(tiny.E, tiny.H, M, seed=2500)
+    out = tiny.run(x, logits)
+    check_routing(tiny, logits, M)
+    ref, _ = oracle_full(tiny, x, logits, fp8=False)
+    check_output(out, ref, "bf16")
