@@ -115,6 +115,32 @@ MOE_API int moe_forward(moe_layer* layer, const void* x, const float* router_log
 MOE_API int moe_forward_host(moe_layer* layer, const void* x_host, const float* logits_host,
                      int M, void* out_host, void* stream);
 
+/* The forward pass for callers that cannot allocate device memory. (The pages have no
+ * counterpart to this entry point; it exists for how the library is deployed.)
+ * moe_forward allocates its per-call scratch on first use and grows it with cudaMalloc
+ * when a larger batch arrives. A caller whose runtime owns all of HBM and forbids later
+ * allocations, a caller that is capturing a stream into a CUDA graph, or a caller that
+ * cannot afford the device-wide synchronisation of cudaMalloc/cudaFree, uses this entry
+ * point instead: same arguments and same result as moe_forward, but every byte of
+ * per-call scratch comes from one fixed 32 MiB array in device memory that the library
+ * defines statically. Nothing is allocated or freed by the call.
+ *   - Limit: a batch whose scratch exceeds 32 MiB is rejected with MOE_ERR_INVALID_ARG and a
+ *     message on stderr (for the bf16 layer E=128, top-8, H=2048, I=768 that is a batch of
+ *     more than 307 tokens; for E=256, top-8, H=7168, I=2048, more than 7); use
+ *     moe_forward for those. Every GPU that loads the library holds the 32 MiB until the
+ *     process exits.
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current). Make that first call before any
+ *     stream capture.
+ *   - Sharing: all calls on a device, from every handle, use the same array and leave
+ *     their data in it; each call clears the parts that must start at zero. Two calls
+ *     whose work overlaps on the GPU (different streams, or different host threads) race
+ *     on the array: keep them stream-ordered.
+ *   - Kernel waits are bounded as in moe_forward, but this path does not write the
+ *     handle's device error word. */
+MOE_API int moe_forward_noalloc(moe_layer* layer, const void* x, const float* router_logits, int M,
+                                void* out, void* stream);
+
 /* Text of a status code (static storage). */
 MOE_API const char* moe_status_string(int status);
 

@@ -21,6 +21,7 @@ SIGNATURES = {
     "moe_load_weights_fp8": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "moe_reserve": (_c_int, [_c_void_p, _c_int, _c_void_p]),
     "moe_forward": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p]),
+    "moe_forward_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "moe_forward_host": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "moe_status_string": (ctypes.c_char_p, [_c_int]),
     "moe_get_device_error": (_c_int, [_c_void_p, ctypes.POINTER(ctypes.c_int)]),

@@ -417,6 +417,27 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
 
 }  // namespace
 
+int moe_layer_view(const moe_layer* L, moe::LayerView* v) {
+  if (!L || !v) return MOE_ERR_INVALID_ARG;
+  v->E = L->E;
+  v->k = L->k;
+  v->H = L->H;
+  v->I = L->I;
+  v->device = L->device;
+  v->num_sms = L->num_sms;
+  v->fp8 = is_fp8(L);
+  v->loaded = L->loaded;
+  v->wscales = L->wscales;
+  v->tm_w13 = L->tm_w13;
+  v->tm_wd = L->tm_wd;
+  return MOE_OK;
+}
+
+int moe_encode_tile_map(CUtensorMap* m, const void* base, bool fp8, long long inner, long long rows, int box_rows) {
+  MOE_TRY(get_encoder());
+  return encode_map(m, base, fp8, inner, rows, box_rows);
+}
+
 extern "C" {
 
 const char* moe_status_string(int status) {

@@ -134,4 +134,18 @@ cudaError_t launch_weight_quant(const __nv_bfloat16* w, long long per_expert, in
                                 const float* scales, int stride, uint8_t* q, long long q_expert_stride,
                                 cudaStream_t s);
 
+// Read-only view of a layer handle's shape, weights and weight tensor maps, for
+// entry points that live outside moe_api.cu.
+struct LayerView {
+  int E, k, H, I, device, num_sms;
+  bool fp8, loaded;
+  const float* wscales;
+  CUtensorMap tm_w13, tm_wd;
+};
+
 }  // namespace moe
+
+struct moe_layer;
+int moe_layer_view(const moe_layer* L, moe::LayerView* v);
+// 2-D tensor map [rows, inner] of bf16 (or e4m3 when fp8), 128-byte rows per box, box_rows rows.
+int moe_encode_tile_map(CUtensorMap* m, const void* base, bool fp8, long long inner, long long rows, int box_rows);

@@ -97,6 +97,13 @@ class MoELayer:
 
     __call__ = forward
 
+    def forward_noalloc(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor, stream=None):
+        """moe_forward_noalloc: the same forward with all per-call scratch taken from the
+        library's fixed 32 MiB device array (no allocation inside the call)."""
+        self._check("moe_forward_noalloc", self.lib.moe_forward_noalloc(
+            self.handle, _ptr(x), _ptr(logits), x.shape[0], _ptr(out), _stream(stream)))
+        return out
+
     def forward_raw(self, x_ptr: int, logits_ptr: int, M: int, out_ptr: int, stream_handle: int):
         self._check("moe_forward", self.lib.moe_forward(self.handle, x_ptr, logits_ptr, M, out_ptr, stream_handle))
 
