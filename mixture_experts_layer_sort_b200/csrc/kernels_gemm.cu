@@ -136,7 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit un = load_unit(a, u, S, BN);
         if (!un.ok) continue;
         const int nb16 = (un.t.n_valid + 15) >> 4;
-        const int wrow = un.t.expert * a.w_rows_per_expert + un.t.fblock * kTileRows;
+        // first tiled-weight block of this unit's row block (W_gate / W_down) and of W_up
+        const int wtile = (un.t.expert * a.w_rblocks + un.t.fblock) * a.kblocks;
+        const int wtile_up = (un.t.expert * a.w_rblocks + a.up_rblock + un.t.fblock) * a.kblocks;
         const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -148,8 +150,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], tx);
           const int kc = kb * C::kKPerBlock;
-          tma_load_2d(st, &tm_w, &full[stage], kc, wrow, pol_w);
-          if constexpr (kGateUp) tma_load_2d(st + C::kABytes, &tm_w, &full[stage], kc, wrow + a.up_offset, pol_w);
+          tma_load_2d(st, &tm_w, &full[stage], 0, (wtile + kb) * kTileRows, pol_w);
+          if constexpr (kGateUp)
+            tma_load_2d(st + C::kABytes, &tm_w, &full[stage], 0, (wtile_up + kb) * kTileRows, pol_w);
           uint8_t* bdst = st + C::kATiles * C::kABytes;
           for (int j = 0; j < nb16; ++j)
             tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[stage], kc, un.t.row_start + 16 * j, pol_b);

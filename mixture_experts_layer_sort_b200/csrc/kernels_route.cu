@@ -1,5 +1,5 @@
-// kernels_route.cu - router top-k, activation gather/quantise, h quantise,
-// finalise, and the load-time weight quantiser.
+// kernels_route.cu - router top-k, activation gather/quantise, h quantise and
+// finalise.
 //
 // Router: "a token usually activates only a selected subset" of the experts
 // (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section
@@ -205,46 +205,6 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
   }
 }
 
-// Load time: scale of one expert's tensor = amax/448 (1 for an all-zero tensor).
-__global__ void __launch_bounds__(1024) weight_amax_kernel(const __nv_bfloat16* w, long long per_expert,
-                                                           float* scales, int stride) {
-  const int e = blockIdx.x;
-  const uint4* src = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * per_expert);
-  float m = 0.f;
-  for (long long i = threadIdx.x; i < per_expert / 8; i += blockDim.x) {
-    float v[8];
-    bf16x8_to_f32(__ldg(src + i), v);
-    #pragma unroll
-    for (int q = 0; q < 8; ++q) m = fmaxf(m, fabsf(v[q]));
-  }
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  __shared__ float red[32];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (threadIdx.x == 0) scales[static_cast<size_t>(e) * stride] = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
-  }
-}
-
-__global__ void __launch_bounds__(256) weight_quant_kernel(const __nv_bfloat16* w, long long per_expert,
-                                                           int E, const float* scales, int stride,
-                                                           uint8_t* q, long long q_expert_stride) {
-  const long long vec_per_expert = per_expert / 8;
-  const long long total = vec_per_expert * E;
-  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
-    const long long e = i / vec_per_expert;
-    const long long j = i - e * vec_per_expert;
-    const float s = __ldg(scales + e * stride);
-    float v[8];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(w) + i), v);
-    reinterpret_cast<uint2*>(q + e * q_expert_stride)[j] = quant8(v, s);
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
@@ -272,23 +232,6 @@ cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s) {
   if (blocks < 1) blocks = 1;
   if (blocks > 148 * 8) blocks = 148 * 8;
   finalize_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_weight_amax(const __nv_bfloat16* w, long long per_expert, int E, float* scales,
-                               int stride, cudaStream_t s) {
-  weight_amax_kernel<<<E, 1024, 0, s>>>(w, per_expert, scales, stride);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_weight_quant(const __nv_bfloat16* w, long long per_expert, int E,
-                                const float* scales, int stride, uint8_t* q, long long q_expert_stride,
-                                cudaStream_t s) {
-  const long long total = per_expert / 8 * E;
-  long long blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  weight_quant_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(w, per_expert, E, scales, stride, q,
-                                                                q_expert_stride);
   return cudaGetLastError();
 }
 

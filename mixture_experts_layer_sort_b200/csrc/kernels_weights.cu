@@ -1,0 +1,131 @@
+// kernels_weights.cu - load-time weight preparation (not on the forward path):
+// per (expert, tensor) FP8 scales, e4m3 quantisation, and the tiled storage layout.
+//
+// Stored layout: tile (e, rb, kb) holds rows [rb*128, rb*128+128) and bytes
+// [kb*128, kb*128+128) of expert e's row-major matrix, as 128 rows of 128 bytes,
+// 16 KB contiguous; tiles are ordered by e, then rb, then kb. A GEMM stage's weight
+// tile is then one contiguous 16 KB read, which spreads over every HBM channel,
+// where a row-major tile would be 128 pieces of 128 bytes one row pitch apart.
+//
+// FP8 ("tensor-quantized", toolboxkart.tech, "AWS SageMaker MoE kernel
+// optimizations H200", section "2. FP8 backend routing changes which kernel path
+// runs"): one scale per expert tensor s = amax/448 (1 for an all-zero tensor),
+// codes = RNE(w / s) saturated to +-448, the division in IEEE fp32.
+#include <cuda_fp8.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ long long tiled_offset(const TileGeom& g, long long e, long long r, long long byte) {
+  const long long kbn = g.row_bytes / 128;
+  const long long tile = (e * g.rb_total + g.rb_offset + r / 128) * kbn + byte / 128;
+  return (tile * 128 + (r & 127)) * 128 + (byte & 127);
+}
+
+__global__ void __launch_bounds__(1024) weight_amax_kernel(const __nv_bfloat16* w, long long per_expert,
+                                                           float* scales, int stride) {
+  const int e = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * per_expert);
+  float m = 0.f;
+  for (long long i = threadIdx.x; i < per_expert / 8; i += blockDim.x) {
+    const uint4 u = __ldg(src + i);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(p[q]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ float red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (threadIdx.x == 0) scales[static_cast<size_t>(e) * stride] = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
+  }
+}
+
+// 8 bf16 -> 8 e4m3 codes (8 bytes) per thread, written at their tiled position.
+__global__ void __launch_bounds__(256) weight_quant_tiled_kernel(const __nv_bfloat16* w, TileGeom g,
+                                                                 const float* scales, int stride, uint8_t* dst) {
+  const long long K = g.row_bytes;                 // e4m3: one byte per element
+  const long long per_row = K / 8;
+  const long long total = static_cast<long long>(g.E) * g.rows * per_row;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
+    const long long row = i / per_row;              // e * rows + r
+    const long long c = (i - row * per_row) * 8;
+    const long long e = row / g.rows;
+    const long long r = row - e * g.rows;
+    const float s = __ldg(scales + e * stride);
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(w) + i);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+    unsigned short c2[4];
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(p[q]);
+      const float2 d = make_float2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s));
+      c2[q] = static_cast<unsigned short>(__nv_cvt_float2_to_fp8x2(d, __NV_SATFINITE, __NV_E4M3));
+    }
+    uint2 o;
+    o.x = static_cast<unsigned>(c2[0]) | (static_cast<unsigned>(c2[1]) << 16);
+    o.y = static_cast<unsigned>(c2[2]) | (static_cast<unsigned>(c2[3]) << 16);
+    *reinterpret_cast<uint2*>(dst + tiled_offset(g, e, r, c)) = o;
+  }
+}
+
+// 16-byte vectors between the row-major [E, rows, row_bytes] and the tiled layout.
+template <bool kToTiled>
+__global__ void __launch_bounds__(256) retile_kernel(const uint8_t* src, TileGeom g, uint8_t* dst) {
+  const long long per_row = g.row_bytes / 16;
+  const long long total = static_cast<long long>(g.E) * g.rows * per_row;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
+    const long long row = i / per_row;
+    const long long b = (i - row * per_row) * 16;
+    const long long e = row / g.rows;
+    const long long r = row - e * g.rows;
+    const long long t = tiled_offset(g, e, r, b);
+    if constexpr (kToTiled) *reinterpret_cast<uint4*>(dst + t) = __ldg(reinterpret_cast<const uint4*>(src) + i);
+    else reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(src + t);
+  }
+}
+
+int grid_for(long long work) {
+  long long b = (work + 255) / 256;
+  if (b > 148 * 32) b = 148 * 32;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
+}  // namespace
+
+cudaError_t launch_weight_amax(const __nv_bfloat16* w, long long per_expert, int E, float* scales,
+                               int stride, cudaStream_t s) {
+  weight_amax_kernel<<<E, 1024, 0, s>>>(w, per_expert, scales, stride);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_quant_tiled(const __nv_bfloat16* w, const TileGeom& g, const float* scales, int stride,
+                                      uint8_t* dst, cudaStream_t s) {
+  weight_quant_tiled_kernel<<<grid_for(g.E * g.rows * (g.row_bytes / 8)), 256, 0, s>>>(w, g, scales, stride, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_weights(const void* src, const TileGeom& g, void* dst, cudaStream_t s) {
+  retile_kernel<true><<<grid_for(g.E * g.rows * (g.row_bytes / 16)), 256, 0, s>>>(
+      static_cast<const uint8_t*>(src), g, static_cast<uint8_t*>(dst));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_untile_weights(const void* src, const TileGeom& g, void* dst, cudaStream_t s) {
+  retile_kernel<false><<<grid_for(g.E * g.rows * (g.row_bytes / 16)), 256, 0, s>>>(
+      static_cast<const uint8_t*>(src), g, static_cast<uint8_t*>(dst));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -219,9 +219,31 @@ int ensure_workspace(moe_layer* L, int M) {
 }
 
 int encode_weight_maps(moe_layer* L) {
-  MOE_TRY(encode_map(&L->tm_w13, L->w13, is_fp8(L), L->H, 2ll * L->E * L->I, moe::kTileRows));
-  MOE_TRY(encode_map(&L->tm_wd, L->wd, is_fp8(L), L->I, 1ll * L->E * L->H, moe::kTileRows));
+  // tiled storage: rows of 128 bytes, one 128-row box = one contiguous 16 KB tile
+  const long long el = is_fp8(L) ? 1 : 2;
+  const long long inner = 128 / el;
+  MOE_TRY(encode_map(&L->tm_w13, L->w13, is_fp8(L), inner, 2ll * L->E * L->I * L->H * el / 128, moe::kTileRows));
+  MOE_TRY(encode_map(&L->tm_wd, L->wd, is_fp8(L), inner, 1ll * L->E * L->H * L->I * el / 128, moe::kTileRows));
   return MOE_OK;
+}
+
+// Tile geometry of the three stored tensors: W_gate and W_up share w13 (up rows after gate rows).
+moe::TileGeom geom(const moe_layer* L, int which) {
+  const long long el = is_fp8(L) ? 1 : 2;
+  moe::TileGeom g{};
+  g.E = L->E;
+  if (which < 2) {
+    g.rows = L->I;
+    g.row_bytes = L->H * el;
+    g.rb_total = 2 * L->I / moe::kTileRows;
+    g.rb_offset = which == 0 ? 0 : L->I / moe::kTileRows;
+  } else {
+    g.rows = L->H;
+    g.row_bytes = L->I * el;
+    g.rb_total = L->H / moe::kTileRows;
+    g.rb_offset = 0;
+  }
+  return g;
 }
 
 cudaEvent_t pool_event(moe_layer* L) {
@@ -359,8 +381,8 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g1.hdr_tiles = moe::kHdrTiles1;
   g1.hdr_splits = moe::kHdrSplits1;
   g1.kblocks = aa.kblocks1;
-  g1.w_rows_per_expert = 2 * L->I;
-  g1.up_offset = L->I;
+  g1.w_rblocks = 2 * L->I / moe::kTileRows;
+  g1.up_rblock = L->I / moe::kTileRows;
   {
     KernelTimer kt(L, 3, st);
     MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, L->tm_x, fp8, variant, L->num_sms, st));
@@ -389,8 +411,8 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g2.hdr_tiles = moe::kHdrTiles2;
   g2.hdr_splits = moe::kHdrSplits2;
   g2.kblocks = aa.kblocks2;
-  g2.w_rows_per_expert = L->H;
-  g2.up_offset = 0;
+  g2.w_rblocks = L->H / moe::kTileRows;
+  g2.up_rblock = 0;
   {
     KernelTimer kt(L, 5, st);
     MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, variant, L->num_sms, st));
@@ -518,21 +540,16 @@ int moe_load_weights(moe_layer* L, const void* w_gate, const void* w_up, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t IH = static_cast<size_t>(L->I) * L->H;
   L->loaded = false;
+  const void* src[3] = {w_gate, w_up, w_down};
+  void* dst[3] = {L->w13, L->w13, L->wd};
   if (!is_fp8(L)) {
-    uint8_t* w13 = static_cast<uint8_t*>(L->w13);
-    MOE_CUDA(cudaMemcpy2DAsync(w13, 2 * IH * 2, w_gate, IH * 2, IH * 2, L->E, cudaMemcpyDeviceToDevice, st));
-    MOE_CUDA(cudaMemcpy2DAsync(w13 + IH * 2, 2 * IH * 2, w_up, IH * 2, IH * 2, L->E, cudaMemcpyDeviceToDevice, st));
-    MOE_CUDA(cudaMemcpyAsync(L->wd, w_down, IH * 2 * L->E, cudaMemcpyDeviceToDevice, st));
+    for (int j = 0; j < 3; ++j) MOE_CUDA(moe::launch_tile_weights(src[j], geom(L, j), dst[j], st));
   } else {
-    const __nv_bfloat16* src[3] = {static_cast<const __nv_bfloat16*>(w_gate),
-                                   static_cast<const __nv_bfloat16*>(w_up),
-                                   static_cast<const __nv_bfloat16*>(w_down)};
-    for (int j = 0; j < 3; ++j)
-      MOE_CUDA(moe::launch_weight_amax(src[j], static_cast<long long>(IH), L->E, L->wscales + j, 3, st));
-    uint8_t* w13 = static_cast<uint8_t*>(L->w13);
-    MOE_CUDA(moe::launch_weight_quant(src[0], IH, L->E, L->wscales + 0, 3, w13, 2 * IH, st));
-    MOE_CUDA(moe::launch_weight_quant(src[1], IH, L->E, L->wscales + 1, 3, w13 + IH, 2 * IH, st));
-    MOE_CUDA(moe::launch_weight_quant(src[2], IH, L->E, L->wscales + 2, 3, static_cast<uint8_t*>(L->wd), IH, st));
+    for (int j = 0; j < 3; ++j) {
+      const auto* w = static_cast<const __nv_bfloat16*>(src[j]);
+      MOE_CUDA(moe::launch_weight_amax(w, static_cast<long long>(IH), L->E, L->wscales + j, 3, st));
+      MOE_CUDA(moe::launch_weight_quant_tiled(w, geom(L, j), L->wscales + j, 3, static_cast<uint8_t*>(dst[j]), st));
+    }
   }
   MOE_CUDA(cudaStreamSynchronize(st));
   MOE_TRY(encode_weight_maps(L));
@@ -549,10 +566,10 @@ int moe_load_weights_fp8(moe_layer* L, const void* q_gate, const void* q_up, con
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t IH = static_cast<size_t>(L->I) * L->H;
   L->loaded = false;
-  uint8_t* w13 = static_cast<uint8_t*>(L->w13);
-  MOE_CUDA(cudaMemcpy2DAsync(w13, 2 * IH, q_gate, IH, IH, L->E, cudaMemcpyDeviceToDevice, st));
-  MOE_CUDA(cudaMemcpy2DAsync(w13 + IH, 2 * IH, q_up, IH, IH, L->E, cudaMemcpyDeviceToDevice, st));
-  MOE_CUDA(cudaMemcpyAsync(L->wd, q_down, IH * L->E, cudaMemcpyDeviceToDevice, st));
+  (void)IH;
+  const void* src[3] = {q_gate, q_up, q_down};
+  void* dst[3] = {L->w13, L->w13, L->wd};
+  for (int j = 0; j < 3; ++j) MOE_CUDA(moe::launch_tile_weights(src[j], geom(L, j), dst[j], st));
   MOE_CUDA(cudaMemcpyAsync(L->wscales, scales_host, static_cast<size_t>(L->E) * 3 * sizeof(float),
                            cudaMemcpyHostToDevice, st));
   MOE_CUDA(cudaStreamSynchronize(st));
@@ -691,12 +708,11 @@ int moe_debug_weights(moe_layer* L, void* gate_out, void* up_out, void* down_out
   if (!L->loaded) return MOE_ERR_NOT_LOADED;
   DeviceGuard g(L->device);
   MOE_CUDA(cudaDeviceSynchronize());
-  const size_t el = is_fp8(L) ? 1 : 2;
-  const size_t IH = static_cast<size_t>(L->I) * L->H * el;
-  const uint8_t* w13 = static_cast<const uint8_t*>(L->w13);
-  if (gate_out) MOE_CUDA(cudaMemcpy2D(gate_out, IH, w13, 2 * IH, IH, L->E, cudaMemcpyDeviceToDevice));
-  if (up_out) MOE_CUDA(cudaMemcpy2D(up_out, IH, w13 + IH, 2 * IH, IH, L->E, cudaMemcpyDeviceToDevice));
-  if (down_out) MOE_CUDA(cudaMemcpy(down_out, L->wd, IH * L->E, cudaMemcpyDeviceToDevice));
+  void* outs[3] = {gate_out, up_out, down_out};
+  const void* srcs[3] = {L->w13, L->w13, L->wd};
+  for (int j = 0; j < 3; ++j)
+    if (outs[j]) MOE_CUDA(moe::launch_untile_weights(srcs[j], geom(L, j), outs[j], nullptr));
+  MOE_CUDA(cudaDeviceSynchronize());
   if (scales_host && is_fp8(L))
     MOE_CUDA(cudaMemcpy(scales_host, L->wscales, static_cast<size_t>(L->E) * 3 * 4, cudaMemcpyDeviceToHost));
   return MOE_OK;

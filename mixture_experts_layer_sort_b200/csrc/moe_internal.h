@@ -74,8 +74,8 @@ struct GemmArgs {
   const int* header;
   int hdr_tiles, hdr_splits;
   int kblocks;             // K blocks over the whole reduction
-  int w_rows_per_expert;   // rows of one expert in the 2-D weight map (2I or H)
-  int up_offset;           // gate_up: row offset of W_up inside an expert (I); else 0
+  int w_rblocks;           // 128-row blocks of one expert's weights (2I/128 or H/128)
+  int up_rblock;           // gate_up: first row block of W_up inside an expert (I/128); else 0
   // gate_up epilogue
   __nv_bfloat16* h;        // [rows_cap, I]
   int I;
@@ -127,12 +127,25 @@ cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
 cudaError_t gemm_configure();    // opt-in dynamic shared memory sizes (current device)
 cudaError_t align_configure();
 
-// Weight preparation (load time, not on the forward path).
+// Weight preparation (load time, not on the forward path). Stored weights are
+// tiled: tile (e, rb, kb) = rows [rb*128, +128) x bytes [kb*128, +128) of expert e,
+// 16 KB contiguous (rows in order), tiles ordered e, then rb, then kb. This is the
+// exact byte block one TMA load of a GEMM stage fetches.
+struct TileGeom {
+  int E;
+  long long rows;       // rows of the source tensor per expert (I for gate/up, H for down)
+  long long row_bytes;  // bytes of one stored row (K * element size)
+  int rb_total;         // row blocks per expert in the destination (2I/128 or H/128)
+  int rb_offset;        // first destination row block of this source (I/128 for up)
+};
 cudaError_t launch_weight_amax(const __nv_bfloat16* w, long long per_expert, int E,
                                float* scales, int stride, cudaStream_t s);
-cudaError_t launch_weight_quant(const __nv_bfloat16* w, long long per_expert, int E,
-                                const float* scales, int stride, uint8_t* q, long long q_expert_stride,
-                                cudaStream_t s);
+// bf16 source [E, rows, K] -> e4m3 codes in the tiled layout, per-expert scale scales[e*stride].
+cudaError_t launch_weight_quant_tiled(const __nv_bfloat16* w, const TileGeom& g, const float* scales,
+                                      int stride, uint8_t* dst, cudaStream_t s);
+// row-major [E, rows, row_bytes] bytes -> tiled layout, and back.
+cudaError_t launch_tile_weights(const void* src, const TileGeom& g, void* dst, cudaStream_t s);
+cudaError_t launch_untile_weights(const void* src, const TileGeom& g, void* dst, cudaStream_t s);
 
 // Read-only view of a layer handle's shape, weights and weight tensor maps, for
 // entry points that live outside moe_api.cu.

@@ -199,8 +199,8 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g1.hdr_tiles = moe::kHdrTiles1;
   g1.hdr_splits = moe::kHdrSplits1;
   g1.kblocks = aa.kblocks1;
-  g1.w_rows_per_expert = 2 * v.I;
-  g1.up_offset = v.I;
+  g1.w_rblocks = 2 * v.I / moe::kTileRows;
+  g1.up_rblock = v.I / moe::kTileRows;
   NA_CUDA(moe::launch_gemm1(g1, v.tm_w13, tm_x, v.fp8, variant, v.num_sms, st));
 
   if (v.fp8) {
@@ -221,8 +221,8 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g2.hdr_tiles = moe::kHdrTiles2;
   g2.hdr_splits = moe::kHdrSplits2;
   g2.kblocks = aa.kblocks2;
-  g2.w_rows_per_expert = v.H;
-  g2.up_offset = 0;
+  g2.w_rblocks = v.H / moe::kTileRows;
+  g2.up_rblock = 0;
   NA_CUDA(moe::launch_gemm2(g2, v.tm_wd, tm_h, v.fp8, variant, v.num_sms, st));
 
   moe::FinalizeArgs fa{};
