@@ -463,6 +463,7 @@ def main():
                      "alg_bytes_per_launch": gate_bytes / max(g_n, 1),
                      "avg_launch_ms": g_ms / max(g_n, 1)},
         "kernel_share": {k: round(v[0] / total_prof, 4) for k, v in prof.items() if v[1] > 0} if total_prof else {},
+        "kernel_us_per_step": {k: round(v[0] * 1e3 / prof_steps, 2) for k, v in prof.items() if v[1] > 0},
         "per_M": per_M,
         "e2e": e2e,
         "gpu_launches": sum(launches_per_M[M] for M in Ms) * args.steps,

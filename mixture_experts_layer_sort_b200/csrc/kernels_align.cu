@@ -12,6 +12,7 @@
 // paragraph): it is built on the device from the counts, so the host never
 // learns the routing and no kernel depends on the token count at compile time.
 #include "moe_internal.h"
+#include "sm100.cuh"
 
 namespace moe {
 
@@ -79,8 +80,10 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     s_count[e] = 0;
     s_base[e] = 0;
   }
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
-  for (int p = tid; p < a.P; p += kAlignThreads) atomicAdd(&s_count[__ldg(a.topk_ids + p)], 1);
+  for (int p = tid; p < a.P; p += kAlignThreads) atomicAdd(&s_count[a.topk_ids[p]], 1);
   __syncthreads();
   for (int e = tid; e < E; e += kAlignThreads) {
     const int n = s_count[e];
@@ -100,7 +103,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     __syncthreads();
     const int p = c0 + tid;
     const bool valid = p < a.P;
-    const int e = valid ? __ldg(a.topk_ids + p) : 0x7FFFFFFF;
+    const int e = valid ? a.topk_ids[p] : 0x7FFFFFFF;
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
     const int rank = __popc(peers & lt_mask);
     if (valid && rank == 0) s_wc[warp * E + e] = __popc(peers);
@@ -153,6 +156,15 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     }
   }
 
+  // widest token tile: the GEMMs size their stage ring from it
+  __syncthreads();
+  if (warp == 0) {
+    int m = 0;
+    for (int e = lane; e < E; e += 32) m = max(m, min(a.BN, s_count[e]));
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) a.header[kHdrMaxRows] = (m + kPadRows - 1) / kPadRows * kPadRows;
+  }
   if (tid == 0) {
     const int nblocks = s_nboff[E];
     const int rows_used = s_poff[E];
@@ -177,8 +189,7 @@ cudaError_t align_configure() {
 }
 
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t s) {
-  align_kernel<<<1, kAlignThreads, align_smem_bytes(a.E), s>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(align_kernel, dim3(1), dim3(kAlignThreads), align_smem_bytes(a.E), s, a);
 }
 
 }  // namespace moe

@@ -38,24 +38,39 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 
-template <bool kGateUp, bool kFP8, int BN, int STAGES>
+template <bool kGateUp, bool kFP8, int BN>
 struct Cfg {
   static constexpr int kATiles = kGateUp ? 2 : 1;
   static constexpr int kABytes = kTileRows * kRowBytes;            // 16 KB per weight tile
-  static constexpr int kBBytes = BN * kRowBytes;
-  static constexpr int kStageBytes = kATiles * kABytes + kBBytes;
   static constexpr int kAccCols = kGateUp ? 2 * BN : BN;
-  static constexpr int kTmemCols = kAccCols <= 32 ? 32 : kAccCols <= 64 ? 64 : kAccCols <= 128 ? 128
-                                   : kAccCols <= 256 ? 256 : 512;
-  static constexpr int kBarrierBytes = 256;
-  static constexpr int kSmemBytes = STAGES * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
+  static constexpr int kTmemCols = 512;   // two accumulator buffers of up to 256 columns
+  // shared memory: [alignment slack][1 KB barriers and flags][stage ring]
+  static constexpr int kSmemBytes = 232448;                         // the sm_100 opt-in maximum
+  static constexpr int kBarrierBytes = 1024;
+  static constexpr int kRingBytes = kSmemBytes - 1024 - kBarrierBytes;
+  static constexpr int kMaxStages = 16;
   static constexpr int kKPerBlock = kFP8 ? 128 : 64;                // elements in one 128-byte row
   static constexpr int kMmaKBytes = 32;                             // K of one MMA = 32 bytes
   static constexpr int kMmasPerBlock = kRowBytes / kMmaKBytes;
   static_assert(kAccCols <= 512, "TMEM holds 512 columns");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N of an M=128 MMA");
-  static_assert(2 * STAGES * 8 + 16 + 4 + 16 <= kBarrierBytes, "barrier area");
+  static_assert(2 * kMaxStages * 8 + 32 + 4 + 16 <= kBarrierBytes, "barrier area");
+  static_assert(kATiles * kABytes + BN * kRowBytes <= kRingBytes / 2, "at least two stages");
 };
+
+// Stage size from the widest token tile of this forward (the align kernel writes it
+// to the header): a stage holds the weight tile(s) plus n_max rows of activations,
+// so thin decode batches get a deeper ring than prefill.
+template <class C>
+__device__ __forceinline__ void ring_geometry(int n_max, int BN, int max_stages, int& n_cap, int& stage_bytes,
+                                              int& stages) {
+  const int n = n_max < 16 ? 16 : (n_max > BN ? BN : ((n_max + 15) & ~15));
+  n_cap = n;
+  stage_bytes = (C::kATiles * C::kABytes + n * kRowBytes + 1023) & ~1023;
+  stages = C::kRingBytes / stage_bytes;
+  if (stages > C::kMaxStages) stages = C::kMaxStages;
+  if (max_stages >= 2 && stages > max_stages) stages = max_stages;
+}
 
 struct Unit {
   Tile t;
@@ -63,13 +78,15 @@ struct Unit {
   bool ok;
 };
 
-__device__ __forceinline__ Unit load_unit(const GemmArgs& a, int u, int S, int BN) {
+// A unit whose token tile does not fit the stage (n_cap rows) or the accumulator is
+// rejected identically by every role, so no role waits for work another skipped.
+__device__ __forceinline__ Unit load_unit(const GemmArgs& a, int u, int S, int n_cap) {
   Unit x;
   x.t = a.tiles[u / S];
   const int s = u - (u / S) * S;
   x.kb0 = s * a.kblocks / S;
   x.kb1 = (s + 1) * a.kblocks / S;
-  x.ok = x.t.n_valid >= 1 && x.t.n_valid <= BN && x.kb1 > x.kb0;
+  x.ok = x.t.n_valid >= 1 && x.t.n_valid <= n_cap && x.kb1 > x.kb0;
   return x;
 }
 
@@ -80,31 +97,42 @@ __device__ __forceinline__ float scale_from_amax(unsigned bits) {
   return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
 }
 
-template <bool kGateUp, bool kFP8, int BN, int STAGES>
+template <bool kGateUp, bool kFP8, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs a, const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_b) {
-  using C = Cfg<kGateUp, kFP8, BN, STAGES>;
+  using C = Cfg<kGateUp, kFP8, BN>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
-  uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = base + C::kBarrierBytes;                         // stage ring, 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(base);
+  uint64_t* empty = full + C::kMaxStages;
+  uint64_t* acc_full = empty + C::kMaxStages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;           // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   int* flags = reinterpret_cast<int*>(tmem_slot + 1);   // [0] abort, [1] last arriver, [2..3] wait outcome
   volatile int* abort_flag = flags;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  int n_cap, stage_bytes, STAGES;
+  ring_geometry<C>(a.header[kHdrMaxRows], BN, a.max_stages, n_cap, stage_bytes, STAGES);
+  // TMEM accumulators: buffer b starts at column 256*b. Two buffers let the MMA of
+  // the next unit run while the epilogue drains this one; gate_up needs two
+  // accumulators (gate, up) per buffer, so it double-buffers only up to 128 tokens.
+  const int nbuf = kGateUp ? (n_cap <= 128 ? 2 : 1) : 2;
+  const uint32_t up_col = kGateUp ? (nbuf == 2 ? 128u : 256u) : 0u;
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kEpiThreads / 32);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiThreads / 32);
+    }
     for (int i = 0; i < 4; ++i) flags[i] = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_w);
@@ -123,6 +151,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int S = a.header[a.hdr_splits];
   const int units = T * S;
 
+  // Everyone but the producer waits for the previous kernel here. The tile list and
+  // header come from the align kernel, at least two launches back, so they are
+  // complete already (see pdl_wait in sm100.cuh).
+  if (threadIdx.x != 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -132,8 +168,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool failed = false;
+      // Weights never depend on the previous kernel, activations do: the first
+      // STAGES weight loads go out before waiting for it, their activation loads after.
+      bool waited = false;
+      int npend = 0;
+      int pend_stage[C::kMaxStages], pend_kc[C::kMaxStages], pend_row[C::kMaxStages], pend_nb[C::kMaxStages];
+      auto release_pending = [&]() {
+        pdl_wait();
+        pdl_trigger();
+        waited = true;
+        for (int i = 0; i < npend; ++i) {
+          uint8_t* bdst = smem + pend_stage[i] * stage_bytes + C::kATiles * C::kABytes;
+          for (int j = 0; j < pend_nb[i]; ++j)
+            tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[pend_stage[i]], pend_kc[i], pend_row[i] + 16 * j,
+                        pol_b);
+        }
+        npend = 0;
+      };
       for (int u = blockIdx.x; u < units && !failed; u += gridDim.x) {
-        const Unit un = load_unit(a, u, S, BN);
+        const Unit un = load_unit(a, u, S, n_cap);
         if (!un.ok) continue;
         const int nb16 = (un.t.n_valid + 15) >> 4;
         // first tiled-weight block of this unit's row block (W_gate / W_down) and of W_up
@@ -147,15 +200,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             failed = true;
             break;
           }
-          uint8_t* st = smem + stage * C::kStageBytes;
+          uint8_t* st = smem + stage * stage_bytes;
           mbar_arrive_expect_tx(&full[stage], tx);
           const int kc = kb * C::kKPerBlock;
           tma_load_2d(st, &tm_w, &full[stage], 0, (wtile + kb) * kTileRows, pol_w);
           if constexpr (kGateUp)
             tma_load_2d(st + C::kABytes, &tm_w, &full[stage], 0, (wtile_up + kb) * kTileRows, pol_w);
-          uint8_t* bdst = st + C::kATiles * C::kABytes;
-          for (int j = 0; j < nb16; ++j)
-            tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[stage], kc, un.t.row_start + 16 * j, pol_b);
+          if (waited) {
+            uint8_t* bdst = st + C::kATiles * C::kABytes;
+            for (int j = 0; j < nb16; ++j)
+              tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[stage], kc, un.t.row_start + 16 * j, pol_b);
+          } else {
+            pend_stage[npend] = stage;
+            pend_kc[npend] = kc;
+            pend_row[npend] = un.t.row_start;
+            pend_nb[npend] = nb16;
+            if (++npend == STAGES) release_pending();
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -163,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (!waited) release_pending();
       if (failed) {
         // let the copies already in flight land before the CTA's shared memory goes away
         int zero = 0;
@@ -182,13 +244,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t acc_phase = 0;
+      int it = 0;
       for (int u = blockIdx.x; u < units; u += gridDim.x) {
-        const Unit un = load_unit(a, u, S, BN);
+        const Unit un = load_unit(a, u, S, n_cap);
         if (!un.ok) continue;
         const uint32_t n_pad = static_cast<uint32_t>((un.t.n_valid + 15) & ~15);
         const uint32_t idesc = idesc_make(kFP8 ? 0u : 1u, 128u, n_pad);
-        if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag)) {
+        const int buf = nbuf == 2 ? (it & 1) : 0;
+        const uint32_t acc_phase = nbuf == 2 ? ((it >> 1) & 1) : (it & 1);
+        const uint32_t d_tmem = tmem + 256u * buf;
+        ++it;
+        if (!mbar_wait_bounded(&acc_empty[buf], acc_phase ^ 1u, abort_flag)) {
           report_error(a.err, kErrWaitAccEmpty);
           *abort_flag = 1;
           break;
@@ -203,19 +269,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
           const uint32_t b0 = a0 + C::kATiles * C::kABytes;
           #pragma unroll
           for (int kk = 0; kk < C::kMmasPerBlock; ++kk) {
             const uint32_t koff = kk * C::kMmaKBytes;
             const uint32_t accum = (kb > un.kb0 || kk > 0) ? 1u : 0u;
             const uint64_t bd = sdesc_k_sw128(b0 + koff);
-            if constexpr (kFP8) mma_e4m3(tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
-            else mma_bf16(tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
+            if constexpr (kFP8) mma_e4m3(d_tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
+            else mma_bf16(d_tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
             if constexpr (kGateUp) {
               const uint64_t ad1 = sdesc_k_sw128(a0 + C::kABytes + koff);
-              if constexpr (kFP8) mma_e4m3(tmem + BN, ad1, bd, idesc, accum);
-              else mma_bf16(tmem + BN, ad1, bd, idesc, accum);
+              if constexpr (kFP8) mma_e4m3(d_tmem + up_col, ad1, bd, idesc, accum);
+              else mma_bf16(d_tmem + up_col, ad1, bd, idesc, accum);
             }
           }
           mma_commit(&empty[stage]);   // frees the stage once these MMAs have read it
@@ -225,17 +291,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (failed) break;
-        mma_commit(acc_full);          // accumulator complete
-        acc_phase ^= 1u;
+        mma_commit(&acc_full[buf]);    // accumulator complete
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                       // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;                // weight row inside the tile
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t t_lane0 = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int epi_tid = threadIdx.x - 64;
-    uint32_t acc_phase = 0;
     int iter = 0;
     float lmax = 0.f;
     float sx = 1.f, sh = 1.f;
@@ -244,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (!kGateUp) sh = scale_from_amax(*a.amax_h);
     }
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      const Unit un = load_unit(a, u, S, BN);
+      const Unit un = load_unit(a, u, S, n_cap);
       if (!un.ok) {
         if (epi_tid == 0) report_error(a.err, kErrBadTile);
         continue;
@@ -253,8 +317,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // so that all of them leave together if the wait gives up. The flag slot
       // alternates per unit: no thread can be two units ahead of another.
       volatile int* okf = flags + 2 + (iter & 1);
+      const int buf = nbuf == 2 ? (iter & 1) : 0;
+      const uint32_t acc_phase = nbuf == 2 ? ((iter >> 1) & 1) : (iter & 1);
+      const uint32_t t_lane = t_lane0 + 256u * buf;
       ++iter;
-      if (epi_tid == 0) *okf = mbar_wait_bounded(acc_full, acc_phase, abort_flag) ? 1 : 0;
+      if (epi_tid == 0) *okf = mbar_wait_bounded(&acc_full[buf], acc_phase, abort_flag) ? 1 : 0;
       named_bar_sync(1, kEpiThreads);
       if (*okf == 0) {
         if (epi_tid == 0) {
@@ -264,7 +331,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      acc_phase ^= 1u;
       const int n_valid = un.t.n_valid;
       const int e = un.t.expert;
       const int col = un.t.fblock * kTileRows + row;
@@ -281,12 +347,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           float g[16], v[16];
           __syncwarp();
           tmem_ld16(t_lane + c0, g);
-          tmem_ld16(t_lane + BN + c0, v);
+          tmem_ld16(t_lane + up_col + c0, v);
           tmem_ld_wait();
           if (c0 + 16 >= n_valid) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
           }
           #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -344,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c0 + 16 >= n_valid) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
           }
           int tok = 0;
           float wt = 0.f;
@@ -378,43 +444,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Variant table. Small: decode with a few tokens per expert; medium: up to a few
-// thousand (token, expert) pairs; large: prefill.
+// Variant table: the widest token tile BN (TMEM columns, epilogue range). The stage
+// ring depth follows the actual widest tile at run time (ring_geometry).
 constexpr int kBnSmall = 32, kBnMedium = 128, kBnLarge = 256;
-constexpr int kSt1Small = 6, kSt1Medium = 4, kSt1Large = 3;    // gate_up stages
-constexpr int kSt2Small = 10, kSt2Medium = 6, kSt2Large = 4;   // down stages
 
-template <bool kGateUp, bool kFP8, int BN, int ST>
+template <bool kGateUp, bool kFP8, int BN>
 cudaError_t launch_one(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int grid, cudaStream_t s) {
-  using C = Cfg<kGateUp, kFP8, BN, ST>;
-  grouped_gemm_kernel<kGateUp, kFP8, BN, ST><<<grid, kThreads, C::kSmemBytes, s>>>(a, w, b);
-  return cudaGetLastError();
+  using C = Cfg<kGateUp, kFP8, BN>;
+  return launch_kernel(grouped_gemm_kernel<kGateUp, kFP8, BN>, dim3(grid), dim3(kThreads),
+                       static_cast<size_t>(C::kSmemBytes), s, a, w, b);
 }
 
-template <bool kGateUp, bool kFP8, int BN, int ST>
+template <bool kGateUp, bool kFP8, int BN>
 cudaError_t configure_one() {
-  using C = Cfg<kGateUp, kFP8, BN, ST>;
-  static_assert(C::kSmemBytes <= 232448, "shared memory per CTA");
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kFP8, BN, ST>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  using C = Cfg<kGateUp, kFP8, BN>;
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kFP8, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              C::kSmemBytes);
 }
 
 template <bool kGateUp, bool kFP8>
 cudaError_t launch_variant(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int variant, int grid,
                            cudaStream_t s) {
-  if (variant == kVariantSmall)
-    return launch_one<kGateUp, kFP8, kBnSmall, kGateUp ? kSt1Small : kSt2Small>(a, w, b, grid, s);
-  if (variant == kVariantMedium)
-    return launch_one<kGateUp, kFP8, kBnMedium, kGateUp ? kSt1Medium : kSt2Medium>(a, w, b, grid, s);
-  return launch_one<kGateUp, kFP8, kBnLarge, kGateUp ? kSt1Large : kSt2Large>(a, w, b, grid, s);
+  if (variant == kVariantSmall) return launch_one<kGateUp, kFP8, kBnSmall>(a, w, b, grid, s);
+  if (variant == kVariantMedium) return launch_one<kGateUp, kFP8, kBnMedium>(a, w, b, grid, s);
+  return launch_one<kGateUp, kFP8, kBnLarge>(a, w, b, grid, s);
 }
 
 template <bool kGateUp, bool kFP8>
 cudaError_t configure_all() {
   cudaError_t e;
-  if ((e = configure_one<kGateUp, kFP8, kBnSmall, kGateUp ? kSt1Small : kSt2Small>()) != cudaSuccess) return e;
-  if ((e = configure_one<kGateUp, kFP8, kBnMedium, kGateUp ? kSt1Medium : kSt2Medium>()) != cudaSuccess) return e;
-  return configure_one<kGateUp, kFP8, kBnLarge, kGateUp ? kSt1Large : kSt2Large>();
+  if ((e = configure_one<kGateUp, kFP8, kBnSmall>()) != cudaSuccess) return e;
+  if ((e = configure_one<kGateUp, kFP8, kBnMedium>()) != cudaSuccess) return e;
+  return configure_one<kGateUp, kFP8, kBnLarge>();
 }
 
 }  // namespace

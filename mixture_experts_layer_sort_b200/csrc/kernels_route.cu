@@ -52,6 +52,8 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   if (t >= a.M) return;
 
   const float* row = a.logits + static_cast<size_t>(t) * a.E;
@@ -142,8 +144,10 @@ template <bool kFP8>
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (r >= a.rows_bound || r >= __ldg(a.header + kHdrRowsUsed)) return;
-  const int p = __ldg(a.padded_pairs + r);
+  pdl_wait();
+  pdl_trigger();
+  if (r >= a.rows_bound || r >= a.header[kHdrRowsUsed]) return;
+  const int p = a.padded_pairs[r];
   if (p >= a.P) return;   // pad row: never read by an output column
   const int t = p / a.k;
   const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
@@ -168,8 +172,10 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
 __global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (r >= a.rows_bound || r >= __ldg(a.header + kHdrRowsUsed)) return;
-  if (__ldg(a.padded_pairs + r) >= a.P) return;
+  pdl_wait();
+  pdl_trigger();
+  if (r >= a.rows_bound || r >= a.header[kHdrRowsUsed]) return;
+  if (a.padded_pairs[r] >= a.P) return;
   const float s = scale_from_amax(*a.amax_h);
   const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(r) * a.I);
   uint2* dst = reinterpret_cast<uint2*>(a.h_q + static_cast<size_t>(r) * a.I);
@@ -182,6 +188,8 @@ __global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
 
 // out = bf16(acc); acc = 0 for the next forward; reset the FP8 amax words.
 __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
+  pdl_wait();
+  pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.amax != nullptr) {
     if (a.last_scales != nullptr) {
       a.last_scales[0] = scale_from_amax(a.amax[0]);
@@ -209,21 +217,18 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   const int grid = (a.M + kRouteWarps - 1) / kRouteWarps;
-  route_kernel<<<grid, kRouteWarps * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(route_kernel, dim3(grid), dim3(kRouteWarps * 32), 0, s, a);
 }
 
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s) {
   const int grid = (a.rows_bound + 7) / 8;
-  if (fp8) gather_kernel<true><<<grid, 256, 0, s>>>(a);
-  else gather_kernel<false><<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  if (fp8) return launch_kernel(gather_kernel<true>, dim3(grid), dim3(256), 0, s, a);
+  return launch_kernel(gather_kernel<false>, dim3(grid), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s) {
   const int grid = (a.rows_bound + 7) / 8;
-  quant_h_kernel<<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(quant_h_kernel, dim3(grid), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s) {
@@ -231,8 +236,7 @@ cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s) {
   long long blocks = (n4 + 255) / 256;
   if (blocks < 1) blocks = 1;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  finalize_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(finalize_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, s, a);
 }
 
 }  // namespace moe

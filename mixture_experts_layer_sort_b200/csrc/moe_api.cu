@@ -15,6 +15,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -383,6 +384,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g1.kblocks = aa.kblocks1;
   g1.w_rblocks = 2 * L->I / moe::kTileRows;
   g1.up_rblock = L->I / moe::kTileRows;
+  g1.max_stages = moe::gemm_max_stages(true);
   {
     KernelTimer kt(L, 3, st);
     MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, L->tm_x, fp8, variant, L->num_sms, st));
@@ -413,6 +415,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g2.kblocks = aa.kblocks2;
   g2.w_rblocks = L->H / moe::kTileRows;
   g2.up_rblock = 0;
+  g2.max_stages = moe::gemm_max_stages(false);
   {
     KernelTimer kt(L, 5, st);
     MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, variant, L->num_sms, st));
@@ -438,6 +441,26 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
 }
 
 }  // namespace
+
+bool moe::pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("MOE_DISABLE_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+int moe::gemm_max_stages(bool gate_up) {
+  static const int caps[2] = {[] {
+                                const char* e = std::getenv("MOE_MAX_STAGES2");
+                                return e ? std::atoi(e) : 6;   // measured best for the down GEMM
+                              }(),
+                              [] {
+                                const char* e = std::getenv("MOE_MAX_STAGES1");
+                                return e ? std::atoi(e) : 4;   // measured best for gate_up
+                              }()};
+  return caps[gate_up ? 1 : 0];
+}
 
 int moe_layer_view(const moe_layer* L, moe::LayerView* v) {
   if (!L || !v) return MOE_ERR_INVALID_ARG;

@@ -21,6 +21,7 @@ enum HeaderSlot : int {
   kHdrTiles2 = 3,       // down tiles
   kHdrSplits2 = 4,      // down split-K factor
   kHdrTokenBlocks = 5,  // (expert, token block) pairs
+  kHdrMaxRows = 6,      // widest token tile (rows of activations a stage must hold), <= BN
   kHdrSlots = 8
 };
 
@@ -90,6 +91,7 @@ struct GemmArgs {
   const int* padded_pairs;
   const float* topk_w;
   int k, P;
+  int max_stages;          // upper bound of the stage ring depth (<= the kernel's own maximum)
   int* err;
 };
 
@@ -109,6 +111,27 @@ struct FinalizeArgs {
   unsigned* amax;          // [2] reset to 0 (may be nullptr)
   float* last_scales;      // [2] s_x, s_h of this forward (may be nullptr)
 };
+
+// Launch with programmatic stream serialisation (PDL) unless MOE_DISABLE_PDL=1 is set
+// in the environment: the kernel may be scheduled before its predecessor in the stream
+// finishes, and orders itself with griddepcontrol (see sm100.cuh).
+bool pdl_enabled();
+int gemm_max_stages(bool gate_up);   // ring depth cap (MOE_MAX_STAGES1/2 override, for tuning)
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Variant table: precompiled (BN, stages) choices; picked on the host by M*k.
 enum Variant : int { kVariantSmall = 0, kVariantMedium = 1, kVariantLarge = 2, kNumVariants = 3 };

@@ -201,6 +201,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g1.kblocks = aa.kblocks1;
   g1.w_rblocks = 2 * v.I / moe::kTileRows;
   g1.up_rblock = v.I / moe::kTileRows;
+  g1.max_stages = moe::gemm_max_stages(true);
   NA_CUDA(moe::launch_gemm1(g1, v.tm_w13, tm_x, v.fp8, variant, v.num_sms, st));
 
   if (v.fp8) {
@@ -223,6 +224,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g2.kblocks = aa.kblocks2;
   g2.w_rblocks = v.H / moe::kTileRows;
   g2.up_rblock = 0;
+  g2.max_stages = moe::gemm_max_stages(false);
   NA_CUDA(moe::launch_gemm2(g2, v.tm_wd, tm_h, v.fp8, variant, v.num_sms, st));
 
   moe::FinalizeArgs fa{};

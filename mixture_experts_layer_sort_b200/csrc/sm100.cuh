@@ -200,6 +200,15 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the forward chain runs its prologue, then pdl_wait() (returns once
+// the previous kernel of the stream has completed and its writes are visible), then
+// pdl_trigger() (lets the next kernel of the stream be scheduled). Because the trigger
+// follows the wait, a kernel that starts early can rely on every kernel two or more
+// launches back having completed. Both are no-ops for a launch without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
