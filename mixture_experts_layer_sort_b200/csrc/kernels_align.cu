@@ -22,22 +22,21 @@ constexpr int kAlignThreads = 1024;
 constexpr int kAlignWarps = kAlignThreads / 32;
 constexpr int kSplitOverhead = 2;   // per-unit fixed cost, in K-block equivalents
 
-__device__ int choose_splits(int tiles, int kblocks, int sms, bool allow) {
-  if (tiles <= 0) return 1;
-  int best = 1;
-  long long best_cost = (static_cast<long long>(tiles) + sms - 1) / sms * (kblocks + kSplitOverhead);
-  if (!allow) return 1;
-  const int smax = kblocks < kMaxSplits ? kblocks : kMaxSplits;
-  for (int s = 2; s <= smax; ++s) {
-    const long long units = static_cast<long long>(tiles) * s;
-    const long long waves = (units + sms - 1) / sms;
-    const long long cost = waves * ((kblocks + s - 1) / s + kSplitOverhead);
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = s;
-    }
+// Split-K factor of one GEMM, chosen by a whole warp: lane l prices s = l + 1 as
+// waves(tiles * s over the SMs) * (K blocks per split + fixed per-unit cost), and
+// the cheapest (smallest s on ties) wins. s = 1 when splitting is not allowed.
+__device__ int choose_splits_warp(int tiles, int kblocks, int sms, bool allow, int lane) {
+  const int smax = min(allow ? kMaxSplits : 1, kblocks);
+  unsigned cost = 0xFFFFFFFFu;
+  const int s = lane + 1;
+  if (tiles > 0 && s <= smax) {
+    const unsigned units = static_cast<unsigned>(tiles) * static_cast<unsigned>(s);
+    const unsigned waves = (units + sms - 1) / static_cast<unsigned>(sms);
+    cost = waves * static_cast<unsigned>((kblocks + s - 1) / s + kSplitOverhead);
   }
-  return best;
+  const unsigned best = __reduce_min_sync(0xFFFFFFFFu, cost);
+  const unsigned pick = __reduce_min_sync(0xFFFFFFFFu, cost == best ? static_cast<unsigned>(s) : 0xFFFFFFFFu);
+  return (tiles > 0 && best != 0xFFFFFFFFu) ? static_cast<int>(pick) : 1;
 }
 
 // Exclusive scan of v[0..n) (n <= 32*chunk) by one warp; total written to v_out[n].
@@ -156,26 +155,32 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     }
   }
 
-  // widest token tile: the GEMMs size their stage ring from it
+  // widest token tile (the GEMMs size their stage ring from it) and the split-K
+  // factors: warps 0 and 1 of the block
   __syncthreads();
   if (warp == 0) {
     int m = 0;
     for (int e = lane; e < E; e += 32) m = max(m, min(a.BN, s_count[e]));
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (lane == 0) a.header[kHdrMaxRows] = (m + kPadRows - 1) / kPadRows * kPadRows;
-  }
-  if (tid == 0) {
     const int nblocks = s_nboff[E];
     const int rows_used = s_poff[E];
     const int t1 = nblocks * a.fblocks1;
-    const int t2 = nblocks * a.fblocks2;
-    a.header[kHdrRowsUsed] = rows_used;
-    a.header[kHdrTiles1] = t1;
-    a.header[kHdrSplits1] = choose_splits(t1, a.kblocks1, a.num_sms, rows_used <= a.ws1_rows_cap);
-    a.header[kHdrTiles2] = t2;
-    a.header[kHdrSplits2] = choose_splits(t2, a.kblocks2, a.num_sms, true);
-    a.header[kHdrTokenBlocks] = nblocks;
+    const int s1 = choose_splits_warp(t1, a.kblocks1, a.num_sms, rows_used <= a.ws1_rows_cap, lane);
+    if (lane == 0) {
+      a.header[kHdrMaxRows] = (m + kPadRows - 1) / kPadRows * kPadRows;
+      a.header[kHdrRowsUsed] = rows_used;
+      a.header[kHdrTiles1] = t1;
+      a.header[kHdrSplits1] = s1;
+      a.header[kHdrTokenBlocks] = nblocks;
+    }
+  } else if (warp == 1) {
+    const int t2 = s_nboff[E] * a.fblocks2;
+    const int s2 = choose_splits_warp(t2, a.kblocks2, a.num_sms, true, lane);
+    if (lane == 0) {
+      a.header[kHdrTiles2] = t2;
+      a.header[kHdrSplits2] = s2;
+    }
   }
 }
 

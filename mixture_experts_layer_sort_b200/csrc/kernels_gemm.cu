@@ -116,16 +116,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  int n_cap, stage_bytes, STAGES;
-  ring_geometry<C>(a.header[kHdrMaxRows], BN, a.max_stages, n_cap, stage_bytes, STAGES);
   // TMEM accumulators: buffer b starts at column 256*b. Two buffers let the MMA of
   // the next unit run while the epilogue drains this one; gate_up needs two
   // accumulators (gate, up) per buffer, so it double-buffers only up to 128 tokens.
-  const int nbuf = kGateUp ? (n_cap <= 128 ? 2 : 1) : 2;
-  const uint32_t up_col = kGateUp ? (nbuf == 2 ? 128u : 256u) : 0u;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::kMaxStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -147,96 +143,130 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // When the previous kernel wrote the tile list, nobody reads it before waiting.
+  if (a.wait_first) {
+    pdl_wait();
+    pdl_trigger();
+  }
+  int n_cap, stage_bytes, STAGES;
+  ring_geometry<C>(a.header[kHdrMaxRows], BN, a.max_stages, n_cap, stage_bytes, STAGES);
+  const int nbuf = kGateUp ? (n_cap <= 128 ? 2 : 1) : 2;
+  const uint32_t up_col = kGateUp ? (nbuf == 2 ? 128u : 256u) : 0u;
+
   const int T = a.header[a.hdr_tiles];
   const int S = a.header[a.hdr_splits];
   const int units = T * S;
 
-  // Everyone but the producer waits for the previous kernel here. The tile list and
-  // header come from the align kernel, at least two launches back, so they are
+  // Everyone but the producer warp waits for the previous kernel here. The tile list
+  // and header come from the align kernel, at least two launches back, so they are
   // complete already (see pdl_wait in sm100.cuh).
-  if (threadIdx.x != 0) {
+  if (warp != 0 && !a.wait_first) {
     pdl_wait();
     pdl_trigger();
   }
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();   // weights stream through once
-      const uint64_t pol_b = l2_policy_evict_last();    // activations are re-read per tile
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool failed = false;
-      // Weights never depend on the previous kernel, activations do: the first
-      // STAGES weight loads go out before waiting for it, their activation loads after.
-      bool waited = false;
-      int npend = 0;
-      int pend_stage[C::kMaxStages], pend_kc[C::kMaxStages], pend_row[C::kMaxStages], pend_nb[C::kMaxStages];
-      auto release_pending = [&]() {
-        pdl_wait();
-        pdl_trigger();
-        waited = true;
-        for (int i = 0; i < npend; ++i) {
-          uint8_t* bdst = smem + pend_stage[i] * stage_bytes + C::kATiles * C::kABytes;
-          for (int j = 0; j < pend_nb[i]; ++j)
-            tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[pend_stage[i]], pend_kc[i], pend_row[i] + 16 * j,
-                        pol_b);
-        }
-        npend = 0;
-      };
-      for (int u = blockIdx.x; u < units && !failed; u += gridDim.x) {
-        const Unit un = load_unit(a, u, S, n_cap);
-        if (!un.ok) continue;
-        const int nb16 = (un.t.n_valid + 15) >> 4;
-        // first tiled-weight block of this unit's row block (W_gate / W_down) and of W_up
-        const int wtile = (un.t.expert * a.w_rblocks + un.t.fblock) * a.kblocks;
-        const int wtile_up = (un.t.expert * a.w_rblocks + a.up_rblock + un.t.fblock) * a.kblocks;
-        const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
-        for (int kb = un.kb0; kb < un.kb1; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
-            report_error(a.err, kErrWaitEmpty);
-            *abort_flag = 1;
-            failed = true;
-            break;
-          }
-          uint8_t* st = smem + stage * stage_bytes;
-          mbar_arrive_expect_tx(&full[stage], tx);
-          const int kc = kb * C::kKPerBlock;
-          tma_load_2d(st, &tm_w, &full[stage], 0, (wtile + kb) * kTileRows, pol_w);
-          if constexpr (kGateUp)
-            tma_load_2d(st + C::kABytes, &tm_w, &full[stage], 0, (wtile_up + kb) * kTileRows, pol_w);
-          if (waited) {
-            uint8_t* bdst = st + C::kATiles * C::kABytes;
-            for (int j = 0; j < nb16; ++j)
-              tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[stage], kc, un.t.row_start + 16 * j, pol_b);
-          } else {
-            pend_stage[npend] = stage;
-            pend_kc[npend] = kc;
-            pend_row[npend] = un.t.row_start;
-            pend_nb[npend] = nb16;
-            if (++npend == STAGES) release_pending();
-          }
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+    // ------------------------------------------------------------ TMA producer (one warp)
+    // Lane 0 owns the stage barriers and issues the weight loads; the activation rows
+    // of a stage are spread over the 32 lanes.
+    const uint64_t pol_w = l2_policy_evict_first();   // weights stream through once
+    const uint64_t pol_b = l2_policy_evict_last();    // activations are re-read per tile
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool failed = false;
+    // Weights never depend on the previous kernel, activations do: the first
+    // STAGES weight loads go out before waiting for it, their activation loads after.
+    bool waited = a.wait_first != 0;
+    int npend = 0;
+    int pend_stage[C::kMaxStages], pend_kc[C::kMaxStages], pend_row[C::kMaxStages], pend_nb[C::kMaxStages];
+    // direct mode: x row (token) of activation rows lane, lane+32, lane+64, lane+96 of
+    // the current unit; pad rows re-read row 0 (their columns are never stored)
+    int tok[4] = {0, 0, 0, 0};
+    auto load_b = [&](int stg, int kc, int row_start, int nb) {
+      uint8_t* bdst = smem + stg * stage_bytes + C::kATiles * C::kABytes;
+      if (a.direct_pairs == nullptr) {
+        for (int j = lane; j < nb; j += 32)
+          tma_load_2d(bdst + j * 16 * kRowBytes, &tm_b, &full[stg], kc, row_start + 16 * j, pol_b);
+      } else {
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = lane + 32 * i;
+          if (j < nb * 16) tma_load_2d(bdst + j * kRowBytes, &tm_b, &full[stg], kc, tok[i], pol_b);
         }
       }
-      if (!waited) release_pending();
-      if (failed) {
-        // let the copies already in flight land before the CTA's shared memory goes away
-        int zero = 0;
-        int st = stage, ph = static_cast<int>(phase);
-        const int pending = issued < STAGES ? issued : STAGES;
-        for (int i = 0; i < pending; ++i) {
-          if (--st < 0) {
-            st = STAGES - 1;
-            ph ^= 1;
-          }
-          mbar_wait_bounded(&full[st], static_cast<uint32_t>(ph), &zero, 1ll << 26);
+    };
+    auto release_pending = [&]() {
+      pdl_wait();
+      pdl_trigger();
+      waited = true;
+      for (int i = 0; i < npend; ++i) load_b(pend_stage[i], pend_kc[i], pend_row[i], pend_nb[i]);
+      npend = 0;
+    };
+    for (int u = blockIdx.x; u < units && !failed; u += gridDim.x) {
+      const Unit un = load_unit(a, u, S, n_cap);
+      if (!un.ok) continue;
+      const int nb16 = (un.t.n_valid + 15) >> 4;
+      // first tiled-weight block of this unit's row block (W_gate / W_down) and of W_up
+      const int wtile = (un.t.expert * a.w_rblocks + un.t.fblock) * a.kblocks;
+      const int wtile_up = (un.t.expert * a.w_rblocks + a.up_rblock + un.t.fblock) * a.kblocks;
+      const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
+      if (a.direct_pairs != nullptr) {
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = lane + 32 * i;
+          tok[i] = j < un.t.n_valid ? __ldcg(a.direct_pairs + un.t.row_start + j) / a.k : 0;
         }
+      }
+      for (int kb = un.kb0; kb < un.kb1; ++kb) {
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag) ? 1 : 0;
+          if (!ok) {
+            report_error(a.err, kErrWaitEmpty);
+            *abort_flag = 1;
+          } else {
+            uint8_t* st = smem + stage * stage_bytes;
+            mbar_arrive_expect_tx(&full[stage], tx);
+            tma_load_2d(st, &tm_w, &full[stage], 0, (wtile + kb) * kTileRows, pol_w);
+            if constexpr (kGateUp)
+              tma_load_2d(st + C::kABytes, &tm_w, &full[stage], 0, (wtile_up + kb) * kTileRows, pol_w);
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) {
+          failed = true;
+          break;
+        }
+        const int kc = kb * C::kKPerBlock;
+        if (waited) {
+          load_b(stage, kc, un.t.row_start, nb16);
+        } else {
+          pend_stage[npend] = stage;
+          pend_kc[npend] = kc;
+          pend_row[npend] = un.t.row_start;
+          pend_nb[npend] = nb16;
+          if (++npend == STAGES) release_pending();
+        }
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!waited) release_pending();
+    if (failed && lane == 0) {
+      // let the copies already in flight land before the CTA's shared memory goes away
+      int zero = 0;
+      int st = stage, ph = static_cast<int>(phase);
+      const int pending = issued < STAGES ? issued : STAGES;
+      for (int i = 0; i < pending; ++i) {
+        if (--st < 0) {
+          st = STAGES - 1;
+          ph ^= 1;
+        }
+        mbar_wait_bounded(&full[st], static_cast<uint32_t>(ph), &zero, 1ll << 26);
       }
     }
   } else if (warp == 1) {

@@ -20,35 +20,25 @@ namespace moe {
 namespace {
 
 constexpr int kRouteWarps = 8;
-constexpr int kRouteMaxPerLane = 16;   // E <= 512 logits = 16 per lane
 
-// Orderable key of (logit, expert id): larger key = better. Higher logits first,
-// equal logits by ascending id, -0.0 equal to +0.0, NaN below -inf. Key 0 means
-// "no candidate".
-__device__ __forceinline__ unsigned long long route_key(float v, int e) {
+// Orderable 32-bit key of a logit: larger key = larger logit, -0.0 equal to +0.0,
+// NaN (key 1) below -inf (key 0x007FFFFF); key 0 means "no candidate".
+__device__ __forceinline__ unsigned route_key(float v) {
+  if (v != v) return 1u;
   unsigned b = __float_as_uint(v);
   if (v == 0.0f) b = 0u;
-  unsigned ord;
-  if (v != v) ord = 0u;
-  else ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return (static_cast<unsigned long long>(ord) << 32) | (0xFFFFFFFFu - static_cast<unsigned>(e));
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ float key_logit(unsigned long long key) {
-  const unsigned ord = static_cast<unsigned>(key >> 32);
-  const unsigned b = (ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord;
-  return __uint_as_float(b);
+__device__ __forceinline__ float key_logit(unsigned key) {
+  if (key == 1u) return __uint_as_float(0x7FC00000u);
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    v = other > v ? other : v;
-  }
-  return v;
-}
-
+// One warp per token; lane l holds logits l, l+32, ... (NPL of them). Each of the k
+// picks takes the largest key over the warp (redux max), then the lowest expert id
+// holding that key (redux min); the owning lane then rescans its own few logits.
+template <int NPL>
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -57,27 +47,43 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   if (t >= a.M) return;
 
   const float* row = a.logits + static_cast<size_t>(t) * a.E;
-  unsigned long long key[kRouteMaxPerLane];
+  unsigned key[NPL];
   #pragma unroll
-  for (int i = 0; i < kRouteMaxPerLane; ++i) {
+  for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
-    key[i] = (e < a.E) ? route_key(__ldg(row + e), e) : 0ull;
+    key[i] = (e < a.E) ? route_key(row[e]) : 0u;
   }
+  unsigned best = 0u;
+  int best_i = 0;
+  #pragma unroll
+  for (int i = 0; i < NPL; ++i)
+    if (key[i] > best) {
+      best = key[i];
+      best_i = i;
+    }
 
   int my_id = 0;
   float my_logit = 0.f;
   for (int j = 0; j < a.k; ++j) {
-    unsigned long long best = 0ull;
-    #pragma unroll
-    for (int i = 0; i < kRouteMaxPerLane; ++i) best = key[i] > best ? key[i] : best;
-    best = warp_max_u64(best);
-    const int id = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFu));
-    #pragma unroll
-    for (int i = 0; i < kRouteMaxPerLane; ++i)
-      if (lane + 32 * i == id) key[i] = 0ull;
+    const unsigned vmax = __reduce_max_sync(0xFFFFFFFFu, best);
+    const unsigned cand = (best == vmax) ? static_cast<unsigned>(lane + 32 * best_i) : 0xFFFFFFFFu;
+    const int id = static_cast<int>(__reduce_min_sync(0xFFFFFFFFu, cand));
     if (lane == j) {
       my_id = id;
-      my_logit = key_logit(best);
+      my_logit = key_logit(vmax);
+    }
+    if ((id & 31) == lane) {        // this lane's best was taken: rescan its logits
+      #pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (i == best_i) key[i] = 0u;
+      best = 0u;
+      best_i = 0;
+      #pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (key[i] > best) {
+          best = key[i];
+          best_i = i;
+        }
     }
   }
   // slot 0 holds the largest selected logit
@@ -96,7 +102,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     const uint4* xr = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
     float m = 0.f;
     for (int i = lane; i < a.H / 8; i += 32) {
-      const uint4 v = __ldg(xr + i);
+      const uint4 v = xr[i];
       const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
       #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -217,7 +223,12 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   const int grid = (a.M + kRouteWarps - 1) / kRouteWarps;
-  return launch_kernel(route_kernel, dim3(grid), dim3(kRouteWarps * 32), 0, s, a);
+  const dim3 g(grid), b(kRouteWarps * 32);
+  if (a.E <= 32) return launch_kernel(route_kernel<1>, g, b, 0, s, a);
+  if (a.E <= 64) return launch_kernel(route_kernel<2>, g, b, 0, s, a);
+  if (a.E <= 128) return launch_kernel(route_kernel<4>, g, b, 0, s, a);
+  if (a.E <= 256) return launch_kernel(route_kernel<8>, g, b, 0, s, a);
+  return launch_kernel(route_kernel<16>, g, b, 0, s, a);
 }
 
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s) {

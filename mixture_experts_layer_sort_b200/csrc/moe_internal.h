@@ -92,6 +92,8 @@ struct GemmArgs {
   const float* topk_w;
   int k, P;
   int max_stages;          // upper bound of the stage ring depth (<= the kernel's own maximum)
+  int wait_first;          // 1: the previous kernel wrote the tile list (wait before reading it)
+  const int* direct_pairs; // gate_up only: B rows are x rows of token pairs[row]/k (x map box = 1 row)
   int* err;
 };
 
