@@ -50,7 +50,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default="decode",
-                    choices=["tiny", "decode", "decode_fp8", "large_decode", "prefill", "prefill_fp8"])
+                    choices=["tiny", "decode", "decode_fp8", "large_decode", "prefill", "prefill_fp8",
+                             "prefill_e48", "prefill_e48_fp8"])
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -61,11 +62,12 @@ def parse_args():
 
 def workload_spec(name):
     from mixture_experts_layer_sort_b200 import synth
-    if name == "prefill_fp8":
-        wl = synth.WORKLOADS["prefill"]
-        return wl, "fp8"
-    wl = synth.WORKLOADS[name]
-    return wl, wl.dtypes[0]
+    if name in synth.WORKLOADS:
+        wl = synth.WORKLOADS[name]
+        return wl, wl.dtypes[0]
+    if name.endswith("_fp8") and name[:-4] in synth.WORKLOADS:
+        return synth.WORKLOADS[name[:-4]], "fp8"
+    raise KeyError(name)
 
 
 def read_peaks():
@@ -308,6 +310,10 @@ def main():
     layer = MoELayer(wl.E, wl.k, wl.H, wl.I, dtype)
     layer.load_weights(wg, wu, wd)
     layer.reserve(max(Ms))
+    if args.no_cpu_baseline or rank != 0 or ws != 1:
+        del wg, wu, wd                       # the layer holds its own copy
+        wg = wu = wd = None
+        torch.cuda.empty_cache()
     toks = {M: synth.make_tokens(wl.E, wl.H, M, seed=seed, device=dev, zipf_s=wl.zipf_s) for M in Ms}
     outs = {M: torch.empty((M, wl.H), dtype=torch.bfloat16, device=dev) for M in Ms}
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)

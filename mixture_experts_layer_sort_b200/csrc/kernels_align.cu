@@ -22,21 +22,32 @@ constexpr int kAlignThreads = 1024;
 constexpr int kAlignWarps = kAlignThreads / 32;
 constexpr int kSplitOverhead = 2;   // per-unit fixed cost, in K-block equivalents
 
-// Split-K factor of one GEMM, chosen by a whole warp: lane l prices s = l + 1 as
-// waves(tiles * s over the SMs) * (K blocks per split + fixed per-unit cost), and
-// the cheapest (smallest s on ties) wins. s = 1 when splitting is not allowed.
-__device__ int choose_splits_warp(int tiles, int kblocks, int sms, bool allow, int lane) {
+// Split-K factor of one GEMM, chosen by a whole warp: lane l prices s = l + 1 in
+// bytes moved per SM: waves(tiles * s over the SMs) * (K blocks per split + 2) *
+// bytes of a K block, plus, for a split, the partial sums it adds to and (gate_up)
+// reads back from memory. The cheapest (smallest s on ties) wins; s = 1 when
+// splitting is not allowed.
+__device__ int choose_splits_warp(int tiles, int kblocks, int sms, bool allow, int kblock_bytes,
+                                  int split_bytes, int lane) {
   const int smax = min(allow ? kMaxSplits : 1, kblocks);
-  unsigned cost = 0xFFFFFFFFu;
+  unsigned long long cost = ~0ull;
   const int s = lane + 1;
   if (tiles > 0 && s <= smax) {
     const unsigned units = static_cast<unsigned>(tiles) * static_cast<unsigned>(s);
     const unsigned waves = (units + sms - 1) / static_cast<unsigned>(sms);
-    cost = waves * static_cast<unsigned>((kblocks + s - 1) / s + kSplitOverhead);
+    const unsigned long long per_unit =
+        static_cast<unsigned long long>((kblocks + s - 1) / s + kSplitOverhead) * kblock_bytes +
+        (s > 1 ? static_cast<unsigned long long>(split_bytes) : 0ull);
+    cost = waves * per_unit;
   }
-  const unsigned best = __reduce_min_sync(0xFFFFFFFFu, cost);
+  unsigned long long best = cost;
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+    best = other < best ? other : best;
+  }
   const unsigned pick = __reduce_min_sync(0xFFFFFFFFu, cost == best ? static_cast<unsigned>(s) : 0xFFFFFFFFu);
-  return (tiles > 0 && best != 0xFFFFFFFFu) ? static_cast<int>(pick) : 1;
+  return (tiles > 0 && best != ~0ull) ? static_cast<int>(pick) : 1;
 }
 
 // Exclusive scan of v[0..n) (n <= 32*chunk) by one warp; total written to v_out[n].
@@ -166,7 +177,11 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     const int nblocks = s_nboff[E];
     const int rows_used = s_poff[E];
     const int t1 = nblocks * a.fblocks1;
-    const int s1 = choose_splits_warp(t1, a.kblocks1, a.num_sms, rows_used <= a.ws1_rows_cap, lane);
+    // mean token rows per tile; gate_up K block = two 16 KB weight tiles + n rows of x;
+    // a split gate_up tile adds and reads back n x 256 fp32 partial sums
+    const int n_mean = nblocks > 0 ? (a.P + nblocks - 1) / nblocks : 0;
+    const int s1 = choose_splits_warp(t1, a.kblocks1, a.num_sms, rows_used <= a.ws1_rows_cap,
+                                      2 * 16384 + n_mean * 128, n_mean * 256 * 4 * 2, lane);
     if (lane == 0) {
       a.header[kHdrMaxRows] = (m + kPadRows - 1) / kPadRows * kPadRows;
       a.header[kHdrRowsUsed] = rows_used;
@@ -175,8 +190,12 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
       a.header[kHdrTokenBlocks] = nblocks;
     }
   } else if (warp == 1) {
-    const int t2 = s_nboff[E] * a.fblocks2;
-    const int s2 = choose_splits_warp(t2, a.kblocks2, a.num_sms, true, lane);
+    const int nblocks = s_nboff[E];
+    const int t2 = nblocks * a.fblocks2;
+    const int n_mean = nblocks > 0 ? (a.P + nblocks - 1) / nblocks : 0;
+    // down: a split only adds more fp32 partial sums to the accumulator
+    const int s2 = choose_splits_warp(t2, a.kblocks2, a.num_sms, true, 16384 + n_mean * 128, n_mean * 128 * 4,
+                                      lane);
     if (lane == 0) {
       a.header[kHdrTiles2] = t2;
       a.header[kHdrSplits2] = s2;

@@ -40,13 +40,21 @@ constexpr int kEpiThreads = 128;
 
 template <bool kGateUp, bool kFP8, int BN>
 struct Cfg {
-  static constexpr int kATiles = kGateUp ? 2 : 1;
+  // two 128-row weight tiles per stage share one activation tile: W_gate and W_up
+  // rows of the same features (gate_up), or two consecutive 128-row blocks of
+  // W_down (down), so each activation byte brought in feeds 256 weight rows
+  static constexpr int kATiles = 2;
   static constexpr int kABytes = kTileRows * kRowBytes;            // 16 KB per weight tile
-  static constexpr int kAccCols = kGateUp ? 2 * BN : BN;
+  static constexpr int kAccCols = 2 * BN;
   static constexpr int kTmemCols = 512;   // two accumulator buffers of up to 256 columns
   // shared memory: [alignment slack][1 KB barriers and flags][stage ring]
   static constexpr int kSmemBytes = 232448;                         // the sm_100 opt-in maximum
-  static constexpr int kBarrierBytes = 1024;
+  // [0, 1 KB): barriers and flags; [1 KB, 3 KB): two slots of the down epilogue's
+  // per-column token row (int, 256 columns each); [3 KB, 5 KB): two slots of its
+  // scaled routing weights (float); the stage ring starts at 6 KB (1024-aligned)
+  static constexpr int kColTableOffset = 1024;
+  static constexpr int kColTableBytes = 2 * 2 * 256 * 4;
+  static constexpr int kBarrierBytes = 6144;
   static constexpr int kRingBytes = kSmemBytes - 1024 - kBarrierBytes;
   static constexpr int kMaxStages = 16;
   static constexpr int kKPerBlock = kFP8 ? 128 : 64;                // elements in one 128-byte row
@@ -54,7 +62,9 @@ struct Cfg {
   static constexpr int kMmasPerBlock = kRowBytes / kMmaKBytes;
   static_assert(kAccCols <= 512, "TMEM holds 512 columns");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N of an M=128 MMA");
-  static_assert(2 * kMaxStages * 8 + 32 + 4 + 16 <= kBarrierBytes, "barrier area");
+  static_assert(2 * kMaxStages * 8 + 32 + 4 + 16 <= kColTableOffset, "barrier area");
+  static_assert(kColTableOffset + kColTableBytes <= kBarrierBytes && kBarrierBytes % 1024 == 0,
+                "column tables must end before the 1024-aligned stage ring");
   static_assert(kATiles * kABytes + BN * kRowBytes <= kRingBytes / 2, "at least two stages");
 };
 
@@ -112,6 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   int* flags = reinterpret_cast<int*>(tmem_slot + 1);   // [0] abort, [1] last arriver, [2..3] wait outcome
   volatile int* abort_flag = flags;
+  int* col_tok = reinterpret_cast<int*>(base + C::kColTableOffset);           // [2][256]
+  float* col_w = reinterpret_cast<float*>(base + C::kColTableOffset + 2048);  // [2][256]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -150,8 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   int n_cap, stage_bytes, STAGES;
   ring_geometry<C>(a.header[kHdrMaxRows], BN, a.max_stages, n_cap, stage_bytes, STAGES);
-  const int nbuf = kGateUp ? (n_cap <= 128 ? 2 : 1) : 2;
-  const uint32_t up_col = kGateUp ? (nbuf == 2 ? 128u : 256u) : 0u;
+  // two accumulators per buffer (one per weight tile), double-buffered up to 128 tokens
+  const int nbuf = n_cap <= 128 ? 2 : 1;
+  const uint32_t up_col = nbuf == 2 ? 128u : 256u;
 
   const int T = a.header[a.hdr_tiles];
   const int S = a.header[a.hdr_splits];
@@ -207,9 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit un = load_unit(a, u, S, n_cap);
       if (!un.ok) continue;
       const int nb16 = (un.t.n_valid + 15) >> 4;
-      // first tiled-weight block of this unit's row block (W_gate / W_down) and of W_up
-      const int wtile = (un.t.expert * a.w_rblocks + un.t.fblock) * a.kblocks;
-      const int wtile_up = (un.t.expert * a.w_rblocks + a.up_rblock + un.t.fblock) * a.kblocks;
+      // first tiled-weight block of the unit's two weight row blocks; a second block
+      // past the end of the tensor reads zeros and is not stored by the epilogue
+      const int rb0 = un.t.fblock * a.rb_step;
+      const int wtile = (un.t.expert * a.w_rblocks + rb0) * a.kblocks;
+      const int wtile_up = (un.t.expert * a.w_rblocks + rb0 + a.second_rb) * a.kblocks;
       const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
       if (a.direct_pairs != nullptr) {
         #pragma unroll
@@ -229,8 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* st = smem + stage * stage_bytes;
             mbar_arrive_expect_tx(&full[stage], tx);
             tma_load_2d(st, &tm_w, &full[stage], 0, (wtile + kb) * kTileRows, pol_w);
-            if constexpr (kGateUp)
-              tma_load_2d(st + C::kABytes, &tm_w, &full[stage], 0, (wtile_up + kb) * kTileRows, pol_w);
+            tma_load_2d(st + C::kABytes, &tm_w, &full[stage], 0, (wtile_up + kb) * kTileRows, pol_w);
           }
         }
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -308,11 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = sdesc_k_sw128(b0 + koff);
             if constexpr (kFP8) mma_e4m3(d_tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
             else mma_bf16(d_tmem, sdesc_k_sw128(a0 + koff), bd, idesc, accum);
-            if constexpr (kGateUp) {
-              const uint64_t ad1 = sdesc_k_sw128(a0 + C::kABytes + koff);
-              if constexpr (kFP8) mma_e4m3(d_tmem + up_col, ad1, bd, idesc, accum);
-              else mma_bf16(d_tmem + up_col, ad1, bd, idesc, accum);
-            }
+            const uint64_t ad1 = sdesc_k_sw128(a0 + C::kABytes + koff);
+            if constexpr (kFP8) mma_e4m3(d_tmem + up_col, ad1, bd, idesc, accum);
+            else mma_bf16(d_tmem + up_col, ad1, bd, idesc, accum);
           }
           mma_commit(&empty[stage]);   // frees the stage once these MMAs have read it
           if (++stage == STAGES) {
@@ -347,6 +359,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // so that all of them leave together if the wait gives up. The flag slot
       // alternates per unit: no thread can be two units ahead of another.
       volatile int* okf = flags + 2 + (iter & 1);
+      int* s_tok = col_tok + 256 * (iter & 1);
+      float* s_w = col_w + 256 * (iter & 1);
+      if constexpr (!kGateUp) {
+        // token row and scaled routing weight of every column, loaded once per unit
+        // while the MMAs still run (slot alternates per unit, like okf)
+        float scale = 1.f;
+        if constexpr (kFP8) scale = __ldg(a.w_scales + un.t.expert * 3 + 2) * sh;
+        for (int j = epi_tid; j < un.t.n_valid; j += kEpiThreads) {
+          const int p = __ldg(a.padded_pairs + un.t.row_start + j);
+          s_tok[j] = p / a.k;
+          s_w[j] = __ldg(a.topk_w + p) * scale;
+        }
+      }
       const int buf = nbuf == 2 ? (iter & 1) : 0;
       const uint32_t acc_phase = nbuf == 2 ? ((iter >> 1) & 1) : (iter & 1);
       const uint32_t t_lane = t_lane0 + 256u * buf;
@@ -415,46 +440,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           named_bar_sync(1, kEpiThreads);
           if (flags[1]) {
             __threadfence();
-            for (int n = 0; n < n_valid; ++n) {
-              const size_t r = static_cast<size_t>(un.t.row_start + n);
-              float* pg = a.ws1 + r * ld_ws + col;
-              float* pu = pg + a.I;
-              const float gs = ld_cg_f32(pg), us = ld_cg_f32(pu);
-              *pg = 0.f;
-              *pu = 0.f;
-              const float hv = silu(gs * sg) * (us * su);
-              const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
-              a.h[r * a.I + col] = hb;
-              if constexpr (kFP8) lmax = fmaxf(lmax, fabsf(__bfloat162float(hb)));
+            // 8 columns per batch: all 16 loads (L2, bypassing L1) are in flight together
+            for (int n0 = 0; n0 < n_valid; n0 += 8) {
+              float gs[8], us[8];
+              #pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                gs[j] = 0.f;
+                us[j] = 0.f;
+                if (n0 + j < n_valid) {
+                  const float* pg = a.ws1 + static_cast<size_t>(un.t.row_start + n0 + j) * ld_ws + col;
+                  gs[j] = __ldcg(pg);
+                  us[j] = __ldcg(pg + a.I);
+                }
+              }
+              #pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (n0 + j < n_valid) {
+                  const size_t r = static_cast<size_t>(un.t.row_start + n0 + j);
+                  float* pg = a.ws1 + r * ld_ws + col;
+                  __stcg(pg, 0.f);
+                  __stcg(pg + a.I, 0.f);
+                  const float hv = silu(gs[j] * sg) * (us[j] * su);
+                  const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+                  a.h[r * a.I + col] = hb;
+                  if constexpr (kFP8) lmax = fmaxf(lmax, fabsf(__bfloat162float(hb)));
+                }
+              }
             }
           }
         }
       } else {
-        float scale = 1.f;
-        if constexpr (kFP8) scale = __ldg(a.w_scales + e * 3 + 2) * sh;
+        // rows of the first weight block go to features f*256 + row, the second block's
+        // to f*256 + 128 + row, when that block exists (H/128 odd: the last tile has one)
+        const int col0 = un.t.fblock * 2 * kTileRows + row;
+        const bool has2 = (un.t.fblock * 2 + 1) * kTileRows < a.H;
         for (int c0 = 0; c0 < n_valid; c0 += 16) {
-          float y[16];
+          float y[16], y2[16];
           __syncwarp();
           tmem_ld16(t_lane + c0, y);
+          tmem_ld16(t_lane + up_col + c0, y2);
           tmem_ld_wait();
           if (c0 + 16 >= n_valid) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
           }
-          int tok = 0;
-          float wt = 0.f;
-          if (lane < 16 && c0 + lane < n_valid) {
-            const int p = __ldg(a.padded_pairs + un.t.row_start + c0 + lane);
-            tok = p / a.k;
-            wt = __ldg(a.topk_w + p) * scale;
-          }
           #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int tj = __shfl_sync(0xFFFFFFFFu, tok, j);
-            const float wj = __shfl_sync(0xFFFFFFFFu, wt, j);
-            if (c0 + j < n_valid) red_add_f32(a.acc + static_cast<size_t>(tj) * a.H + col, y[j] * wj);
-          }
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < n_valid) {
+              float* dst = a.acc + static_cast<size_t>(s_tok[c0 + j]) * a.H + col0;
+              red_add_f32(dst, y[j] * s_w[c0 + j]);
+              if (has2) red_add_f32(dst + kTileRows, y2[j] * s_w[c0 + j]);
+            }
         }
       }
     }
@@ -474,9 +511,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Variant table: the widest token tile BN (TMEM columns, epilogue range). The stage
-// ring depth follows the actual widest tile at run time (ring_geometry).
-constexpr int kBnSmall = 32, kBnMedium = 128, kBnLarge = 256;
+// One tile variant: up to 256 token rows per tile (the largest N of an M=128 MMA).
+// Thin batches are not penalised: the stage ring and the TMEM buffering follow the
+// widest token tile of the forward at run time (ring_geometry).
+constexpr int kTokenTile = 256;
 
 template <bool kGateUp, bool kFP8, int BN>
 cudaError_t launch_one(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int grid, cudaStream_t s) {
@@ -495,22 +533,21 @@ cudaError_t configure_one() {
 template <bool kGateUp, bool kFP8>
 cudaError_t launch_variant(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int variant, int grid,
                            cudaStream_t s) {
-  if (variant == kVariantSmall) return launch_one<kGateUp, kFP8, kBnSmall>(a, w, b, grid, s);
-  if (variant == kVariantMedium) return launch_one<kGateUp, kFP8, kBnMedium>(a, w, b, grid, s);
-  return launch_one<kGateUp, kFP8, kBnLarge>(a, w, b, grid, s);
+  (void)variant;
+  return launch_one<kGateUp, kFP8, kTokenTile>(a, w, b, grid, s);
 }
 
 template <bool kGateUp, bool kFP8>
 cudaError_t configure_all() {
-  cudaError_t e;
-  if ((e = configure_one<kGateUp, kFP8, kBnSmall>()) != cudaSuccess) return e;
-  if ((e = configure_one<kGateUp, kFP8, kBnMedium>()) != cudaSuccess) return e;
-  return configure_one<kGateUp, kFP8, kBnLarge>();
+  return configure_one<kGateUp, kFP8, kTokenTile>();
 }
 
 }  // namespace
 
-int variant_bn(int v) { return v == kVariantSmall ? kBnSmall : v == kVariantMedium ? kBnMedium : kBnLarge; }
+int variant_bn(int v) {
+  (void)v;
+  return kTokenTile;
+}
 
 cudaError_t gemm_configure() {
   cudaError_t e;

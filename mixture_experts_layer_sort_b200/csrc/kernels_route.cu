@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
 }
 
 // out = bf16(acc); acc = 0 for the next forward; reset the FP8 amax words.
+// Four float4 of acc per thread per step, all loaded before any is stored.
 __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -207,15 +208,26 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
   const long long n4 = a.n / 4;
   float4* acc4 = reinterpret_cast<float4*>(a.acc);
   uint2* out4 = reinterpret_cast<uint2*>(a.out);
-  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += static_cast<long long>(gridDim.x) * 256) {
-    const float4 v = acc4[i];
-    acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
-    uint2 o;
-    o.x = *reinterpret_cast<const unsigned*>(&lo);
-    o.y = *reinterpret_cast<const unsigned*>(&hi);
-    out4[i] = o;
+  const long long T = static_cast<long long>(gridDim.x) * 256;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += 4 * T) {
+    float4 v[4];
+    #pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (i + j * T < n4) v[j] = __ldcg(acc4 + i + j * T);
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long q = i + j * T;
+      if (q < n4) {
+        __stcg(acc4 + q, zero);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(v[j].x, v[j].y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(v[j].z, v[j].w);
+        uint2 o;
+        o.x = *reinterpret_cast<const unsigned*>(&lo);
+        o.y = *reinterpret_cast<const unsigned*>(&hi);
+        out4[q] = o;
+      }
+    }
   }
 }
 

@@ -334,7 +334,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   aa.k = L->k;
   aa.BN = BN;
   aa.fblocks1 = L->I / moe::kTileRows;
-  aa.fblocks2 = L->H / moe::kTileRows;
+  aa.fblocks2 = (L->H / moe::kTileRows + 1) / 2;
   const int kper = fp8 ? 128 : 64;
   aa.kblocks1 = L->H / kper;
   aa.kblocks2 = L->I / kper;
@@ -398,7 +398,8 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g1.hdr_splits = moe::kHdrSplits1;
   g1.kblocks = aa.kblocks1;
   g1.w_rblocks = 2 * L->I / moe::kTileRows;
-  g1.up_rblock = L->I / moe::kTileRows;
+  g1.rb_step = 1;
+  g1.second_rb = L->I / moe::kTileRows;
   g1.max_stages = moe::gemm_max_stages(true);
   g1.wait_first = direct ? 1 : 0;
   g1.direct_pairs = direct ? L->pairs : nullptr;
@@ -431,7 +432,8 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g2.hdr_splits = moe::kHdrSplits2;
   g2.kblocks = aa.kblocks2;
   g2.w_rblocks = L->H / moe::kTileRows;
-  g2.up_rblock = 0;
+  g2.rb_step = 2;
+  g2.second_rb = 1;
   g2.max_stages = moe::gemm_max_stages(false);
   {
     KernelTimer kt(L, 5, st);

@@ -48,7 +48,7 @@ struct AlignArgs {
   const int* topk_ids;     // [P]
   int P, E, k;
   int BN;                  // token rows per tile (the variant's N)
-  int fblocks1, fblocks2;  // I/128 and H/128
+  int fblocks1, fblocks2;  // tiles across the output features: I/128 (gate_up), ceil(H/256) (down)
   int kblocks1, kblocks2;  // K blocks of gate_up (H) and down (I)
   int num_sms;
   int ws1_rows_cap;        // split-K of gate_up needs rows_used <= this
@@ -76,7 +76,8 @@ struct GemmArgs {
   int hdr_tiles, hdr_splits;
   int kblocks;             // K blocks over the whole reduction
   int w_rblocks;           // 128-row blocks of one expert's weights (2I/128 or H/128)
-  int up_rblock;           // gate_up: first row block of W_up inside an expert (I/128); else 0
+  int rb_step;             // tile row block f covers weight row blocks f*rb_step and
+  int second_rb;           //   f*rb_step + second_rb (gate_up: 1 and I/128; down: 2 and 1)
   // gate_up epilogue
   __nv_bfloat16* h;        // [rows_cap, I]
   int I;

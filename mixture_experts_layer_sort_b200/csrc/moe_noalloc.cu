@@ -93,7 +93,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   const long long rows_cap = P + Emin * (moe::kPadRows - 1);
   const long long nblocks = (P + BN - 1) / BN + Emin;
   const long long t1 = nblocks * (v.I / moe::kTileRows);
-  const long long t2 = nblocks * (v.H / moe::kTileRows);
+  const long long t2 = nblocks * ((v.H / moe::kTileRows + 1) / 2);
   const long long ws1_rows = std::min(rows_cap, kSplitRowsMax);
   const size_t el = v.fp8 ? 1 : 2;
 
@@ -152,7 +152,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   aa.k = v.k;
   aa.BN = BN;
   aa.fblocks1 = v.I / moe::kTileRows;
-  aa.fblocks2 = v.H / moe::kTileRows;
+  aa.fblocks2 = (v.H / moe::kTileRows + 1) / 2;
   aa.kblocks1 = v.H / kper;
   aa.kblocks2 = v.I / kper;
   aa.num_sms = v.num_sms;
@@ -200,7 +200,8 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g1.hdr_splits = moe::kHdrSplits1;
   g1.kblocks = aa.kblocks1;
   g1.w_rblocks = 2 * v.I / moe::kTileRows;
-  g1.up_rblock = v.I / moe::kTileRows;
+  g1.rb_step = 1;
+  g1.second_rb = v.I / moe::kTileRows;
   g1.max_stages = moe::gemm_max_stages(true);
   NA_CUDA(moe::launch_gemm1(g1, v.tm_w13, tm_x, v.fp8, variant, v.num_sms, st));
 
@@ -223,7 +224,8 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g2.hdr_splits = moe::kHdrSplits2;
   g2.kblocks = aa.kblocks2;
   g2.w_rblocks = v.H / moe::kTileRows;
-  g2.up_rblock = 0;
+  g2.rb_step = 2;
+  g2.second_rb = 1;
   g2.max_stages = moe::gemm_max_stages(false);
   NA_CUDA(moe::launch_gemm2(g2, v.tm_wd, tm_h, v.fp8, variant, v.num_sms, st));
 

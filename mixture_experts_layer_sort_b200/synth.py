@@ -52,6 +52,12 @@ WORKLOADS = {
     "prefill": Workload("prefill", E=256, k=8, H=7168, I=2048, Ms=(4096,), w_std=0.01,
                         dtypes=("bf16", "fp8"),
                         description="prefill, E=256 top-8, H=7168, I=2048, M=4096, bf16 and e4m3"),
+    # profiling stand-in for prefill: same H, I and tokens per expert (~128) and the same
+    # schedule (no split-K), 3/16 of the experts, so a multi-pass profiler capture holds
+    # ~4 GB instead of 23 GB
+    "prefill_e48": Workload("prefill_e48", E=48, k=8, H=7168, I=2048, Ms=(768,), w_std=0.01,
+                            dtypes=("bf16", "fp8"),
+                            description="prefill-shaped profiling case, E=48 top-8, H=7168, I=2048, M=768"),
 }
 
 
