@@ -57,6 +57,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--only-M", type=int, default=None, help="run a single batch size of the workload")
+    ap.add_argument("--fused-decode", action="store_true", help="single-launch decode path (bf16, M <= 64)")
     return ap.parse_args()
 
 
@@ -281,7 +282,7 @@ def traffic_from_profile(kernel_src_hash):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for name in ("kernels_gemm.cu", "sm100.cuh", "moe_internal.h"):
+    for name in ("kernels_gemm.cu", "gemm_pipeline.cuh", "sm100.cuh", "moe_internal.h"):
         with open(os.path.join(ROOT, "mixture_experts_layer_sort_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -310,6 +311,8 @@ def main():
     layer = MoELayer(wl.E, wl.k, wl.H, wl.I, dtype)
     layer.load_weights(wg, wu, wd)
     layer.reserve(max(Ms))
+    if args.fused_decode:
+        layer.set_fused_decode(True)
     if args.no_cpu_baseline or rank != 0 or ws != 1:
         del wg, wu, wd                       # the layer holds its own copy
         wg = wu = wd = None

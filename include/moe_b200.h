@@ -141,6 +141,16 @@ MOE_API int moe_forward_host(moe_layer* layer, const void* x_host, const float* 
 MOE_API int moe_forward_noalloc(moe_layer* layer, const void* x, const float* router_logits, int M,
                                 void* out, void* stream);
 
+/* Select the single-launch decode path for this handle (enable = 1) or the default
+ * kernel chain (enable = 0). The single-launch path runs a whole bf16 forward of up
+ * to 64 tokens (M*topk <= 512, E <= 512) in one cooperative persistent kernel that
+ * routes, groups, gathers and runs both grouped GEMMs with device-side dependency
+ * counters ("fused MoE kernels combine routing, data movement and expert
+ * calculations into fewer GPU operations": toolboxkart.tech, "AWS SageMaker MoE
+ * kernel optimizations H200", section "Why MoE inference needs specialized
+ * kernels"). Other batches and FP8 layers keep the chain. Same results either way. */
+MOE_API int moe_set_fused_decode(moe_layer* layer, int enable);
+
 /* Text of a status code (static storage). */
 MOE_API const char* moe_status_string(int status);
 

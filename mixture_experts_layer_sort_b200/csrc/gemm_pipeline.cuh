@@ -1,0 +1,588 @@
+// gemm_pipeline.cuh - the warp-specialised tcgen05 pipeline behind both grouped GEMMs
+// of the MoE layer, written once and used by the stand-alone grouped kernel
+// (kernels_gemm.cu) and by the single-launch decode kernel (kernels_decode.cu).
+//
+// Orientation: every tile is "swap-AB". The expert's weight rows fill the MMA's
+// M = 128 slot and the expert's few tokens are the N dimension (16..256), i.e. the
+// kernel computes D^T = W * X^T instead of X * W^T. (A B)^T = B^T A^T changes no
+// arithmetic (kongchang.com, "MoE Kernel Engineering Optimization Practices on
+// Amazon SageMaker AI", section "Swap-AB: Making WGMMA Run at Full Utilization");
+// it keeps the tensor-core rows busy when decode gives an expert a handful of
+// tokens (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section
+// "1. Swap-AB makes better use of the WGMMA tile"; aib.vote, "AWS SageMaker MoE
+// kernel optimizations", second paragraph). On sm_100 N reaches 256, so the same
+// orientation also covers prefill (~128-256 tokens per expert).
+//
+// A stage holds two 128-row weight tiles that share one activation tile: the W_gate
+// and W_up rows of the same 128 features (gate_up), or two consecutive 128-row
+// blocks of W_down (down). Two TMEM accumulators take the two products. The gate_up
+// epilogue forms h = silu(g) * u ("fuses scaling, matrix multiplication ... into one
+// GPU pass", aib.vote page, third paragraph); the down epilogue scales by the
+// routing weight and scatter-adds into the fp32 token accumulator ("expert
+// aggregation").
+//
+// Roles: warp 0 = TMA producer (lane 0 owns the stage barriers and the weight loads,
+// the activation rows of a stage are spread over the lanes), warp 1 = TMEM owner and
+// MMA issuer, warps 2-5 = epilogue (TMEM lane quadrant = warp % 4). Units (a tile,
+// or one K range of a split tile) come from a unit source; dependencies of the
+// activation operand and completion signals come from hooks, so that one kernel can
+// run both GEMMs back to back.
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace pipe {
+
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kTokenTile = 256;   // widest token tile: the largest N of an M=128 MMA
+
+template <bool kFP8>
+struct Cfg {
+  static constexpr int kATiles = 2;
+  static constexpr int kABytes = kTileRows * kRowBytes;             // 16 KB per weight tile
+  static constexpr int kTmemCols = 512;                              // two buffers x two accumulators
+  static constexpr int kSmemBytes = 232448;                          // the sm_100 opt-in maximum
+  // [0, 1 KB): barriers and flags; [1 KB, 3 KB): two slots of the down epilogue's
+  // per-column token row (int, 256 columns each); [3 KB, 5 KB): two slots of its
+  // scaled routing weights (float); then the caller's extra bytes, then the ring
+  static constexpr int kColTableOffset = 1024;
+  static constexpr int kFixedBytes = 6144;
+  static constexpr int kMaxStages = 16;
+  static constexpr int kKPerBlock = kFP8 ? 128 : 64;                 // elements in one 128-byte row
+  static constexpr int kMmaKBytes = 32;                              // K of one MMA = 32 bytes
+  static constexpr int kMmasPerBlock = kRowBytes / kMmaKBytes;
+  static_assert(2 * kMaxStages * 8 + 32 + 4 + 16 <= kColTableOffset, "barrier area");
+  static_assert(kColTableOffset + 2 * 2 * 256 * 4 <= kFixedBytes, "column tables");
+};
+
+struct Shared {
+  uint8_t* ring;          // stage ring, 1024-aligned
+  uint64_t* full;         // [kMaxStages]
+  uint64_t* empty;        // [kMaxStages]
+  uint64_t* acc_full;     // [2]
+  uint64_t* acc_empty;    // [2]
+  uint32_t* tmem_slot;
+  int* flags;             // [0] abort, [1] last arriver, [2..3] epilogue wait outcome
+  int* col_tok;           // [2][256]
+  float* col_w;           // [2][256]
+  uint8_t* extra;         // caller's region (1024-aligned), or the ring when none
+  int ring_bytes;
+};
+
+template <class C>
+__device__ __forceinline__ Shared carve(uint8_t* raw, int extra_bytes) {
+  Shared s;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.full = reinterpret_cast<uint64_t*>(base);
+  s.empty = s.full + C::kMaxStages;
+  s.acc_full = s.empty + C::kMaxStages;
+  s.acc_empty = s.acc_full + 2;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.acc_empty + 2);
+  s.flags = reinterpret_cast<int*>(s.tmem_slot + 1);
+  s.col_tok = reinterpret_cast<int*>(base + C::kColTableOffset);
+  s.col_w = reinterpret_cast<float*>(base + C::kColTableOffset + 2048);
+  const int extra = (extra_bytes + 1023) & ~1023;
+  s.extra = base + C::kFixedBytes;
+  s.ring = base + C::kFixedBytes + extra;
+  s.ring_bytes = C::kSmemBytes - 1024 - C::kFixedBytes - extra;
+  return s;
+}
+
+// Barrier init (one thread) and TMEM allocation (warp 1), then a CTA-wide sync.
+template <class C>
+__device__ __forceinline__ uint32_t prologue(const Shared& s, int warp) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kMaxStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s.acc_full[b], 1);
+      mbar_init(&s.acc_empty[b], kEpiThreads / 32);
+    }
+    for (int i = 0; i < 4; ++i) s.flags[i] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s.tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *s.tmem_slot;
+}
+
+template <class C>
+__device__ __forceinline__ void teardown(uint32_t tmem, int warp) {
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Stage ring: a stage holds the two weight tiles plus n_max rows of activations
+// (n_max = widest token tile of the forward), so thin decode batches get a deeper
+// ring than prefill. Two TMEM buffers (columns 0 and 256) when a buffer's two
+// accumulators fit 256 columns, i.e. up to 128 tokens.
+struct Ring {
+  int n_cap, stage_bytes, stages, nbuf;
+  uint32_t up_col;
+};
+
+template <class C>
+__device__ __forceinline__ Ring make_ring(int n_max, int max_stages, int ring_bytes) {
+  Ring r;
+  r.n_cap = n_max < 16 ? 16 : (n_max > kTokenTile ? kTokenTile : ((n_max + 15) & ~15));
+  r.stage_bytes = (C::kATiles * C::kABytes + r.n_cap * kRowBytes + 1023) & ~1023;
+  r.stages = ring_bytes / r.stage_bytes;
+  if (r.stages > C::kMaxStages) r.stages = C::kMaxStages;
+  if (max_stages >= 2 && r.stages > max_stages) r.stages = max_stages;
+  r.nbuf = r.n_cap <= 128 ? 2 : 1;
+  r.up_col = r.nbuf == 2 ? 128u : 256u;
+  return r;
+}
+
+struct Unit {
+  Tile t;
+  int tile;      // index of the tile (split-K counter)
+  int S;         // splits of the tile
+  int kb0, kb1;  // K blocks of this unit
+  bool ok;       // tile passed its bounds check (every role skips a bad unit alike)
+};
+
+__device__ __forceinline__ Unit make_unit(const Tile& t, int tile, int s, int S, int kblocks, int n_cap) {
+  Unit x;
+  x.t = t;
+  x.tile = tile;
+  x.S = S;
+  x.kb0 = s * kblocks / S;
+  x.kb1 = (s + 1) * kblocks / S;
+  x.ok = t.n_valid >= 1 && t.n_valid <= n_cap && x.kb1 > x.kb0;
+  return x;
+}
+
+// Units of a tile list in global memory (written by the align kernel).
+struct GlobalTiles {
+  const Tile* tiles;
+  int T, S, kblocks;
+  __device__ __forceinline__ int units() const { return T * S; }
+  __device__ __forceinline__ Unit unit(int u, int n_cap) const {
+    const int t = u / S;
+    return make_unit(tiles[t], t, u - t * S, S, kblocks, n_cap);
+  }
+};
+
+__device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
+
+__device__ __forceinline__ float scale_from_amax(unsigned bits) {
+  const float amax = __uint_as_float(bits);
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+}
+
+// ------------------------------------------------------------------------ producer
+struct ProducerState {
+  int stage = 0;
+  uint32_t phase = 0;
+  int issued = 0;
+  bool failed = false;
+};
+
+// Hooks (all lanes call them uniformly):
+//   int dep(const Unit&)  - key of the activation operand's dependency
+//   bool ready(int dep)   - non-blocking check
+//   bool wait(int dep)    - blocking (bounded) wait; false when it gave up
+template <class C, class Src, class Hooks>
+__device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const CUtensorMap* tm_b, const Shared& sh,
+                             const Ring& rg, const Src& src, Hooks& hk, ProducerState& ps, volatile int* abort_flag,
+                             int lane) {
+  const uint64_t pol_w = l2_policy_evict_first();   // weights stream through once
+  const uint64_t pol_b = l2_policy_evict_last();    // activations are re-read per tile
+  // Activation loads whose dependency is not met yet wait in a queue (their weight
+  // loads are already out); the queue is released in order once it fills the ring.
+  int npend = 0;
+  int pend_stage[C::kMaxStages], pend_kc[C::kMaxStages], pend_row[C::kMaxStages], pend_nb[C::kMaxStages],
+      pend_dep[C::kMaxStages];
+  // direct mode: x row (token) of activation rows lane, lane+32, lane+64, lane+96 of
+  // the current unit; pad rows re-read row 0 (their columns are never stored)
+  int tok[4] = {0, 0, 0, 0};
+  auto load_b = [&](int stg, int kc, int row_start, int nb) {
+    uint8_t* bdst = sh.ring + stg * rg.stage_bytes + C::kATiles * C::kABytes;
+    if (a.direct_pairs == nullptr) {
+      for (int j = lane; j < nb; j += 32)
+        tma_load_2d(bdst + j * 16 * kRowBytes, tm_b, &sh.full[stg], kc, row_start + 16 * j, pol_b);
+    } else {
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = lane + 32 * i;
+        if (j < nb * 16) tma_load_2d(bdst + j * kRowBytes, tm_b, &sh.full[stg], kc, tok[i], pol_b);
+      }
+    }
+  };
+  // issue queued activation loads in order while their dependencies are met
+  auto drain = [&](bool block) -> bool {
+    int i = 0;
+    for (; i < npend; ++i) {
+      if (!hk.ready(pend_dep[i])) {
+        if (!block) break;
+        if (!hk.wait(pend_dep[i])) return false;
+      }
+      load_b(pend_stage[i], pend_kc[i], pend_row[i], pend_nb[i]);
+    }
+    for (int j = i; j < npend; ++j) {
+      pend_stage[j - i] = pend_stage[j];
+      pend_kc[j - i] = pend_kc[j];
+      pend_row[j - i] = pend_row[j];
+      pend_nb[j - i] = pend_nb[j];
+      pend_dep[j - i] = pend_dep[j];
+    }
+    npend -= i;
+    return true;
+  };
+  const int units = src.units();
+  for (int u = blockIdx.x; u < units && !ps.failed; u += gridDim.x) {
+    const Unit un = src.unit(u, rg.n_cap);
+    if (!un.ok) continue;
+    const int nb16 = (un.t.n_valid + 15) >> 4;
+    // first tiled-weight block of the unit's two weight row blocks; a second block
+    // past the end of the tensor reads zeros and is not stored by the epilogue
+    const int rb0 = un.t.fblock * a.rb_step;
+    const int wtile = (un.t.expert * a.w_rblocks + rb0) * a.kblocks;
+    const int wtile2 = (un.t.expert * a.w_rblocks + rb0 + a.second_rb) * a.kblocks;
+    const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
+    const int dep = hk.dep(un);
+    if (a.direct_pairs != nullptr) {
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = lane + 32 * i;
+        tok[i] = j < un.t.n_valid ? __ldcg(a.direct_pairs + un.t.row_start + j) / a.k : 0;
+      }
+    }
+    for (int kb = un.kb0; kb < un.kb1; ++kb) {
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait_bounded(&sh.empty[ps.stage], ps.phase ^ 1u, abort_flag) ? 1 : 0;
+        if (!ok) {
+          report_error(a.err, kErrWaitEmpty);
+          *abort_flag = 1;
+        } else {
+          uint8_t* st = sh.ring + ps.stage * rg.stage_bytes;
+          mbar_arrive_expect_tx(&sh.full[ps.stage], tx);
+          tma_load_2d(st, tm_w, &sh.full[ps.stage], 0, (wtile + kb) * kTileRows, pol_w);
+          tma_load_2d(st + C::kABytes, tm_w, &sh.full[ps.stage], 0, (wtile2 + kb) * kTileRows, pol_w);
+        }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) {
+        ps.failed = true;
+        break;
+      }
+      const int kc = kb * C::kKPerBlock;
+      if (npend > 0 && !drain(false)) ps.failed = true;
+      if (!ps.failed && npend == 0 && hk.ready(dep)) {
+        load_b(ps.stage, kc, un.t.row_start, nb16);
+      } else if (!ps.failed) {
+        pend_stage[npend] = ps.stage;
+        pend_kc[npend] = kc;
+        pend_row[npend] = un.t.row_start;
+        pend_nb[npend] = nb16;
+        pend_dep[npend] = dep;
+        if (++npend == rg.stages && !drain(true)) ps.failed = true;
+      }
+      if (ps.failed) {
+        if (lane == 0) {
+          report_error(a.err, kErrWaitDep);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      ++ps.issued;
+      if (++ps.stage == rg.stages) {
+        ps.stage = 0;
+        ps.phase ^= 1u;
+      }
+    }
+  }
+  if (!ps.failed && npend > 0 && !drain(true)) {
+    ps.failed = true;
+    if (lane == 0) {
+      report_error(a.err, kErrWaitDep);
+      *abort_flag = 1;
+    }
+  }
+}
+
+// After a failure: let the copies already in flight land before shared memory goes away.
+template <class C>
+__device__ void producer_quiesce(const Shared& sh, const Ring& rg, const ProducerState& ps, int lane) {
+  if (!ps.failed || lane != 0) return;
+  int zero = 0;
+  int st = ps.stage, ph = static_cast<int>(ps.phase);
+  const int pending = ps.issued < rg.stages ? ps.issued : rg.stages;
+  for (int i = 0; i < pending; ++i) {
+    if (--st < 0) {
+      st = rg.stages - 1;
+      ph ^= 1;
+    }
+    mbar_wait_bounded(&sh.full[st], static_cast<uint32_t>(ph), &zero, 1ll << 26);
+  }
+}
+
+// ------------------------------------------------------------------------ MMA issuer
+struct MmaState {
+  int stage = 0;
+  uint32_t phase = 0;
+  int it = 0;
+  bool failed = false;
+};
+
+template <class C, bool kFP8, class Src>
+__device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, const Src& src, MmaState& ms,
+                        uint32_t tmem, volatile int* abort_flag) {
+  const int units = src.units();
+  for (int u = blockIdx.x; u < units && !ms.failed; u += gridDim.x) {
+    const Unit un = src.unit(u, rg.n_cap);
+    if (!un.ok) continue;
+    const uint32_t n_pad = static_cast<uint32_t>((un.t.n_valid + 15) & ~15);
+    const uint32_t idesc = idesc_make(kFP8 ? 0u : 1u, 128u, n_pad);
+    const int buf = rg.nbuf == 2 ? (ms.it & 1) : 0;
+    const uint32_t acc_phase = rg.nbuf == 2 ? ((ms.it >> 1) & 1) : (ms.it & 1);
+    const uint32_t d_tmem = tmem + 256u * buf;
+    ++ms.it;
+    if (!mbar_wait_bounded(&sh.acc_empty[buf], acc_phase ^ 1u, abort_flag)) {
+      report_error(a.err, kErrWaitAccEmpty);
+      *abort_flag = 1;
+      ms.failed = true;
+      break;
+    }
+    tc_fence_after();
+    for (int kb = un.kb0; kb < un.kb1; ++kb) {
+      if (!mbar_wait_bounded(&sh.full[ms.stage], ms.phase, abort_flag)) {
+        report_error(a.err, kErrWaitFull);
+        *abort_flag = 1;
+        ms.failed = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sh.ring + ms.stage * rg.stage_bytes);
+      const uint32_t b0 = a0 + C::kATiles * C::kABytes;
+      #pragma unroll
+      for (int kk = 0; kk < C::kMmasPerBlock; ++kk) {
+        const uint32_t koff = kk * C::kMmaKBytes;
+        const uint32_t accum = (kb > un.kb0 || kk > 0) ? 1u : 0u;
+        const uint64_t bd = sdesc_k_sw128(b0 + koff);
+        const uint64_t ad0 = sdesc_k_sw128(a0 + koff);
+        const uint64_t ad1 = sdesc_k_sw128(a0 + C::kABytes + koff);
+        if constexpr (kFP8) {
+          mma_e4m3(d_tmem, ad0, bd, idesc, accum);
+          mma_e4m3(d_tmem + rg.up_col, ad1, bd, idesc, accum);
+        } else {
+          mma_bf16(d_tmem, ad0, bd, idesc, accum);
+          mma_bf16(d_tmem + rg.up_col, ad1, bd, idesc, accum);
+        }
+      }
+      mma_commit(&sh.empty[ms.stage]);   // frees the stage once these MMAs have read it
+      if (++ms.stage == rg.stages) {
+        ms.stage = 0;
+        ms.phase ^= 1u;
+      }
+    }
+    if (ms.failed) break;
+    mma_commit(&sh.acc_full[buf]);       // accumulator complete
+  }
+}
+
+// ------------------------------------------------------------------------ epilogue
+struct EpiState {
+  int iter = 0;
+  float lmax = 0.f;     // FP8 gate_up: max |h| written by this thread
+  bool failed = false;
+};
+
+// Hooks:
+//   column(const Unit&, int j, float scale, int& tok, float& w) - down: token row and
+//        scaled routing weight of column j
+//   static constexpr bool kSignalTiles; tile_done(const Unit&, int epi_tid) - gate_up:
+//        called by every epilogue thread once the tile's h rows are written and fenced
+//   static constexpr bool kTokenCompletion; down_done(const Unit&, const int* s_tok,
+//        int epi_tid) - down: called by every epilogue thread after the unit's adds
+template <class C, bool kGateUp, bool kFP8, class Src, class Hooks>
+__device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg, const Src& src, Hooks& hk,
+                             EpiState& es, uint32_t tmem, volatile int* abort_flag, int warp, int lane) {
+  const int q = warp & 3;                       // TMEM lane quadrant of this warp
+  const int row = q * 32 + lane;                // weight row inside the tile
+  const uint32_t t_lane0 = tmem + (static_cast<uint32_t>(q * 32) << 16);
+  const int epi_tid = threadIdx.x - 64;
+  float sx = 1.f, sh_scale = 1.f;
+  if constexpr (kFP8) {
+    sx = scale_from_amax(*a.amax_x);
+    if constexpr (!kGateUp) sh_scale = scale_from_amax(*a.amax_h);
+  }
+  const int units = src.units();
+  for (int u = blockIdx.x; u < units && !es.failed; u += gridDim.x) {
+    const Unit un = src.unit(u, rg.n_cap);
+    if (!un.ok) {
+      if (epi_tid == 0) report_error(a.err, kErrBadTile);
+      continue;
+    }
+    // One thread waits; the named barrier hands the outcome to the other 127, so
+    // that all of them leave together if the wait gives up. Flag and column-table
+    // slots alternate per unit: no thread can be two units ahead of another.
+    volatile int* okf = sh.flags + 2 + (es.iter & 1);
+    int* s_tok = sh.col_tok + 256 * (es.iter & 1);
+    float* s_w = sh.col_w + 256 * (es.iter & 1);
+    if constexpr (!kGateUp) {
+      // token row and scaled routing weight of every column, once per unit, while
+      // the MMAs still run
+      float scale = 1.f;
+      if constexpr (kFP8) scale = __ldg(a.w_scales + un.t.expert * 3 + 2) * sh_scale;
+      for (int j = epi_tid; j < un.t.n_valid; j += kEpiThreads) hk.column(un, j, scale, s_tok[j], s_w[j]);
+    }
+    const int buf = rg.nbuf == 2 ? (es.iter & 1) : 0;
+    const uint32_t acc_phase = rg.nbuf == 2 ? ((es.iter >> 1) & 1) : (es.iter & 1);
+    const uint32_t t_lane = t_lane0 + 256u * buf;
+    ++es.iter;
+    if (epi_tid == 0) *okf = mbar_wait_bounded(&sh.acc_full[buf], acc_phase, abort_flag) ? 1 : 0;
+    named_bar_sync(1, kEpiThreads);
+    if (*okf == 0) {
+      if (epi_tid == 0) {
+        report_error(a.err, kErrWaitAccFull);
+        *abort_flag = 1;
+      }
+      es.failed = true;
+      break;
+    }
+    tc_fence_after();
+    const int n_valid = un.t.n_valid;
+    const int e = un.t.expert;
+
+    if constexpr (kGateUp) {
+      const int col = un.t.fblock * kTileRows + row;
+      float sg = 1.f, su = 1.f;
+      if constexpr (kFP8) {
+        sg = __ldg(a.w_scales + e * 3 + 0) * sx;
+        su = __ldg(a.w_scales + e * 3 + 1) * sx;
+      }
+      const bool split = un.S > 1;
+      const size_t ld_ws = static_cast<size_t>(2) * a.I;
+      for (int c0 = 0; c0 < n_valid; c0 += 16) {
+        float g[16], v[16];
+        __syncwarp();
+        tmem_ld16(t_lane + c0, g);
+        tmem_ld16(t_lane + rg.up_col + c0, v);
+        tmem_ld_wait();
+        if (c0 + 16 >= n_valid) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+        }
+        #pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c0 + j;
+          if (n < n_valid) {
+            const size_t r = static_cast<size_t>(un.t.row_start + n);
+            if (split) {
+              red_add_f32(a.ws1 + r * ld_ws + col, g[j]);
+              red_add_f32(a.ws1 + r * ld_ws + a.I + col, v[j]);
+            } else {
+              const float hv = silu(g[j] * sg) * (v[j] * su);
+              const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+              a.h[r * a.I + col] = hb;
+              if constexpr (kFP8) es.lmax = fmaxf(es.lmax, fabsf(__bfloat162float(hb)));
+            }
+          }
+        }
+      }
+      bool wrote = !split;
+      if (split) {
+        // the last of the splits of this tile finishes it from the partial sums
+        __threadfence();
+        named_bar_sync(1, kEpiThreads);
+        if (epi_tid == 0) {
+          const int old = atomicAdd(a.tile_counters + un.tile, 1);
+          const int last = (old == un.S - 1) ? 1 : 0;
+          if (last) a.tile_counters[un.tile] = 0;
+          sh.flags[1] = last;
+        }
+        named_bar_sync(1, kEpiThreads);
+        if (sh.flags[1]) {
+          wrote = true;
+          __threadfence();
+          // 8 columns per batch: all 16 loads (L2, bypassing L1) are in flight together
+          for (int n0 = 0; n0 < n_valid; n0 += 8) {
+            float gs[8], us[8];
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              gs[j] = 0.f;
+              us[j] = 0.f;
+              if (n0 + j < n_valid) {
+                const float* pg = a.ws1 + static_cast<size_t>(un.t.row_start + n0 + j) * ld_ws + col;
+                gs[j] = __ldcg(pg);
+                us[j] = __ldcg(pg + a.I);
+              }
+            }
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (n0 + j < n_valid) {
+                const size_t r = static_cast<size_t>(un.t.row_start + n0 + j);
+                float* pg = a.ws1 + r * ld_ws + col;
+                __stcg(pg, 0.f);
+                __stcg(pg + a.I, 0.f);
+                const float hv = silu(gs[j] * sg) * (us[j] * su);
+                const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+                a.h[r * a.I + col] = hb;
+                if constexpr (kFP8) es.lmax = fmaxf(es.lmax, fabsf(__bfloat162float(hb)));
+              }
+            }
+          }
+        }
+      }
+      if constexpr (Hooks::kSignalTiles) {
+        if (wrote) hk.tile_done(un, epi_tid);
+      }
+    } else {
+      // rows of the first weight block go to features f*256 + row, the second block's
+      // to f*256 + 128 + row, when that block exists (H/128 odd: the last tile has one)
+      const int col0 = un.t.fblock * 2 * kTileRows + row;
+      const bool has2 = (un.t.fblock * 2 + 1) * kTileRows < a.H;
+      for (int c0 = 0; c0 < n_valid; c0 += 16) {
+        float y[16], y2[16];
+        __syncwarp();
+        tmem_ld16(t_lane + c0, y);
+        tmem_ld16(t_lane + rg.up_col + c0, y2);
+        tmem_ld_wait();
+        if (c0 + 16 >= n_valid) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+        }
+        #pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c0 + j < n_valid) {
+            float* dst = a.acc + static_cast<size_t>(s_tok[c0 + j]) * a.H + col0;
+            red_add_f32(dst, y[j] * s_w[c0 + j]);
+            if (has2) red_add_f32(dst + kTileRows, y2[j] * s_w[c0 + j]);
+          }
+      }
+      if constexpr (Hooks::kTokenCompletion) hk.down_done(un, s_tok, epi_tid);
+    }
+  }
+}
+
+// FP8 gate_up: fold this thread's max |h| into the global amax word.
+__device__ __forceinline__ void publish_amax(unsigned* amax, float lmax, int lane) {
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
+  if (lane == 0 && lmax > 0.f) atomicMax(amax, __float_as_uint(lmax));
+}
+
+}  // namespace pipe
+}  // namespace moe

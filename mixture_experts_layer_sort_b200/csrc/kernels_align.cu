@@ -12,6 +12,7 @@
 // paragraph): it is built on the device from the counts, so the host never
 // learns the routing and no kernel depends on the token count at compile time.
 #include "moe_internal.h"
+#include "route_common.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -20,57 +21,6 @@ namespace {
 
 constexpr int kAlignThreads = 1024;
 constexpr int kAlignWarps = kAlignThreads / 32;
-constexpr int kSplitOverhead = 2;   // per-unit fixed cost, in K-block equivalents
-
-// Split-K factor of one GEMM, chosen by a whole warp: lane l prices s = l + 1 in
-// bytes moved per SM: waves(tiles * s over the SMs) * (K blocks per split + 2) *
-// bytes of a K block, plus, for a split, the partial sums it adds to and (gate_up)
-// reads back from memory. The cheapest (smallest s on ties) wins; s = 1 when
-// splitting is not allowed.
-__device__ int choose_splits_warp(int tiles, int kblocks, int sms, bool allow, int kblock_bytes,
-                                  int split_bytes, int lane) {
-  const int smax = min(allow ? kMaxSplits : 1, kblocks);
-  unsigned long long cost = ~0ull;
-  const int s = lane + 1;
-  if (tiles > 0 && s <= smax) {
-    const unsigned units = static_cast<unsigned>(tiles) * static_cast<unsigned>(s);
-    const unsigned waves = (units + sms - 1) / static_cast<unsigned>(sms);
-    const unsigned long long per_unit =
-        static_cast<unsigned long long>((kblocks + s - 1) / s + kSplitOverhead) * kblock_bytes +
-        (s > 1 ? static_cast<unsigned long long>(split_bytes) : 0ull);
-    cost = waves * per_unit;
-  }
-  unsigned long long best = cost;
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-    best = other < best ? other : best;
-  }
-  const unsigned pick = __reduce_min_sync(0xFFFFFFFFu, cost == best ? static_cast<unsigned>(s) : 0xFFFFFFFFu);
-  return (tiles > 0 && best != ~0ull) ? static_cast<int>(pick) : 1;
-}
-
-// Exclusive scan of v[0..n) (n <= 32*chunk) by one warp; total written to v_out[n].
-__device__ void warp_exclusive_scan(const int* in, int* out, int n, int lane) {
-  const int chunk = (n + 31) / 32;
-  const int lo = lane * chunk;
-  const int hi = min(n, lo + chunk);
-  int local = 0;
-  for (int i = lo; i < hi; ++i) local += in[i];
-  int incl = local;
-  #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  int run = incl - local;
-  for (int i = lo; i < hi; ++i) {
-    out[i] = run;
-    run += in[i];
-  }
-  if (lane == 31) out[n] = incl;
-}
-
 __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   extern __shared__ int sm[];
   const int E = a.E;

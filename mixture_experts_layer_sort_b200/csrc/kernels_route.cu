@@ -13,6 +13,7 @@
 #include <cuda_fp8.h>
 
 #include "moe_internal.h"
+#include "route_common.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -21,23 +22,8 @@ namespace {
 
 constexpr int kRouteWarps = 8;
 
-// Orderable 32-bit key of a logit: larger key = larger logit, -0.0 equal to +0.0,
-// NaN (key 1) below -inf (key 0x007FFFFF); key 0 means "no candidate".
-__device__ __forceinline__ unsigned route_key(float v) {
-  if (v != v) return 1u;
-  unsigned b = __float_as_uint(v);
-  if (v == 0.0f) b = 0u;
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-__device__ __forceinline__ float key_logit(unsigned key) {
-  if (key == 1u) return __uint_as_float(0x7FC00000u);
-  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
-}
-
-// One warp per token; lane l holds logits l, l+32, ... (NPL of them). Each of the k
-// picks takes the largest key over the warp (redux max), then the lowest expert id
-// holding that key (redux min); the owning lane then rescans its own few logits.
+// One warp per token (route_token); FP8 layers also fold the token's max |x| into
+// the per-tensor amax word.
 template <int NPL>
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
@@ -45,57 +31,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   pdl_wait();
   pdl_trigger();
   if (t >= a.M) return;
-
-  const float* row = a.logits + static_cast<size_t>(t) * a.E;
-  unsigned key[NPL];
-  #pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = (e < a.E) ? route_key(row[e]) : 0u;
-  }
-  unsigned best = 0u;
-  int best_i = 0;
-  #pragma unroll
-  for (int i = 0; i < NPL; ++i)
-    if (key[i] > best) {
-      best = key[i];
-      best_i = i;
-    }
-
-  int my_id = 0;
-  float my_logit = 0.f;
-  for (int j = 0; j < a.k; ++j) {
-    const unsigned vmax = __reduce_max_sync(0xFFFFFFFFu, best);
-    const unsigned cand = (best == vmax) ? static_cast<unsigned>(lane + 32 * best_i) : 0xFFFFFFFFu;
-    const int id = static_cast<int>(__reduce_min_sync(0xFFFFFFFFu, cand));
-    if (lane == j) {
-      my_id = id;
-      my_logit = key_logit(vmax);
-    }
-    if ((id & 31) == lane) {        // this lane's best was taken: rescan its logits
-      #pragma unroll
-      for (int i = 0; i < NPL; ++i)
-        if (i == best_i) key[i] = 0u;
-      best = 0u;
-      best_i = 0;
-      #pragma unroll
-      for (int i = 0; i < NPL; ++i)
-        if (key[i] > best) {
-          best = key[i];
-          best_i = i;
-        }
-    }
-  }
-  // slot 0 holds the largest selected logit
-  const float lmax = __shfl_sync(0xFFFFFFFFu, my_logit, 0);
-  float ex = (lane < a.k) ? expf(my_logit - lmax) : 0.f;
-  float sum = ex;
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-  if (lane < a.k) {
-    a.topk_ids[static_cast<size_t>(t) * a.k + lane] = my_id;
-    a.topk_w[static_cast<size_t>(t) * a.k + lane] = ex / sum;
-  }
+  route_token<NPL>(a.logits + static_cast<size_t>(t) * a.E, a.E, a.k, lane, a.topk_ids + static_cast<size_t>(t) * a.k,
+                   a.topk_w + static_cast<size_t>(t) * a.k);
 
   if (a.amax_x != nullptr) {
     // FP8: this token's contribution to max |x|

@@ -55,6 +55,7 @@ struct moe_layer {
   unsigned* amax = nullptr;     // [2] max|x|, max|h| (float bits)
   float* last_scales = nullptr; // [2]
   int* err = nullptr;
+  int* sync = nullptr;          // single-launch decode: counters between its CTAs
   CUtensorMap tm_x{}, tm_h{};
   // staging for moe_forward_host
   void* hx = nullptr;
@@ -63,6 +64,7 @@ struct moe_layer {
   int host_cap = 0;
   // bookkeeping
   int last_M = 0, last_launches = 0, last_variant = 0;
+  bool fused_decode = false;    // single-launch decode path for small bf16 batches
   // per-kernel event timing
   bool profiling = false;
   struct Timed {
@@ -136,6 +138,7 @@ int configure_device(int dev) {
   if (dev < 64 && (g_configured >> dev) & 1ull) return MOE_OK;
   MOE_CUDA(moe::gemm_configure());
   MOE_CUDA(moe::align_configure());
+  MOE_CUDA(moe::decode_configure());
   if (dev < 64) g_configured |= 1ull << dev;
   return MOE_OK;
 }
@@ -210,6 +213,7 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(ws_alloc(L, &L->amax, 2 * 4, true));
   MOE_TRY(ws_alloc(L, &L->last_scales, 2 * 4, false));
   MOE_TRY(ws_alloc(L, &L->err, 4, true));
+  MOE_TRY(ws_alloc(L, &L->sync, moe::decode_sync_words(L->E, cap) * 4, true));
   const float ones[2] = {1.f, 1.f};
   MOE_CUDA(cudaMemcpy(L->last_scales, ones, sizeof(ones), cudaMemcpyHostToDevice));
   MOE_TRY(encode_map(&L->tm_x, L->x_perm, is_fp8(L), L->H, L->rows_cap, 16));
@@ -302,8 +306,74 @@ bool direct_x_disabled() {
   return off;
 }
 
+int decode_stage_cap() {
+  static const int cap = [] {
+    const char* e = std::getenv("MOE_MAX_STAGES_DECODE");
+    return e ? std::atoi(e) : 5;
+  }();
+  return cap;
+}
+
+// The whole layer of a small bf16 batch in one cooperative launch.
+int forward_fused_decode(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
+  moe::DecodeLaunch d{};
+  d.logits = logits;
+  d.x = static_cast<const __nv_bfloat16*>(x);
+  d.out = static_cast<__nv_bfloat16*>(out);
+  d.M = M;
+  d.E = L->E;
+  d.k = L->k;
+  d.H = L->H;
+  d.I = L->I;
+  d.grid = L->num_sms;
+  d.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
+  d.max_stages = decode_stage_cap();
+  d.sync = L->sync;
+  d.x_perm = static_cast<__nv_bfloat16*>(L->x_perm);
+  d.topk_ids = L->topk_ids;
+  d.topk_w = L->topk_w;
+  d.counts = L->counts;
+  d.padded_offsets = L->poff;
+  d.padded_pairs = L->pairs;
+  d.header = L->header;
+  moe::GemmArgs g{};
+  g.h = L->h;
+  g.I = L->I;
+  g.ws1 = L->ws1;
+  g.tile_counters = L->counters;
+  g.acc = L->acc;
+  g.H = L->H;
+  g.k = L->k;
+  g.P = M * L->k;
+  g.err = L->err;
+  d.g1 = g;
+  d.g1.kblocks = L->H / 64;
+  d.g1.w_rblocks = 2 * L->I / moe::kTileRows;
+  d.g1.rb_step = 1;
+  d.g1.second_rb = L->I / moe::kTileRows;
+  d.g2 = g;
+  d.g2.kblocks = L->I / 64;
+  d.g2.w_rblocks = L->H / moe::kTileRows;
+  d.g2.rb_step = 2;
+  d.g2.second_rb = 1;
+  d.tm_w13 = &L->tm_w13;
+  d.tm_wd = &L->tm_wd;
+  d.tm_x = &L->tm_x;
+  d.tm_h = &L->tm_h;
+  {
+    KernelTimer kt(L, 3, st);
+    MOE_CUDA(moe::launch_decode(d, st));
+  }
+  L->last_M = M;
+  L->last_launches = 1;
+  L->last_variant = -1;
+  return MOE_OK;
+}
+
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
+  if (L->fused_decode && !is_fp8(L) && moe::decode_supported(M, L->E, L->k))
+    return forward_fused_decode(L, x, logits, M, out, st);
   const bool fp8 = is_fp8(L);
   const long long P = static_cast<long long>(M) * L->k;
   const int variant = choose_variant(P);
@@ -686,6 +756,12 @@ int moe_get_device_error(moe_layer* L, int* code) {
 }
 
 int moe_last_launch_count(moe_layer* L) { return L ? L->last_launches : 0; }
+
+int moe_set_fused_decode(moe_layer* L, int enable) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  L->fused_decode = enable != 0;
+  return MOE_OK;
+}
 
 int moe_profile_enable(moe_layer* L, int enable) {
   if (!L) return MOE_ERR_INVALID_ARG;

@@ -153,6 +153,32 @@ cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
 cudaError_t gemm_configure();    // opt-in dynamic shared memory sizes (current device)
 cudaError_t align_configure();
 
+// Single-launch decode path (kernels_decode.cu): the whole layer for M <= 64 bf16
+// tokens in one cooperative persistent kernel.
+struct DecodeLaunch {
+  const float* logits;
+  const __nv_bfloat16* x;
+  __nv_bfloat16* out;
+  int M, E, k, H, I, grid, ws1_rows_cap, max_stages;
+  int* sync;               // decode_sync_words(E, M_cap) ints, zero between launches
+  __nv_bfloat16* x_perm;
+  int* topk_ids;           // routing copies for inspection
+  float* topk_w;
+  int* counts;
+  int* padded_offsets;
+  int* padded_pairs;
+  int* header;
+  GemmArgs g1, g2;
+  const CUtensorMap* tm_w13;
+  const CUtensorMap* tm_wd;
+  const CUtensorMap* tm_x;
+  const CUtensorMap* tm_h;
+};
+bool decode_supported(int M, int E, int k);
+size_t decode_sync_words(int E, int M_cap);
+cudaError_t decode_configure();
+cudaError_t launch_decode(const DecodeLaunch& l, cudaStream_t st);
+
 // Weight preparation (load time, not on the forward path). Stored weights are
 // tiled: tile (e, rb, kb) = rows [rb*128, +128) x bytes [kb*128, +128) of expert e,
 // 16 KB contiguous (rows in order), tiles ordered e, then rb, then kb. This is the

@@ -18,6 +18,8 @@ enum DeviceError : int {
   kErrWaitAccFull = 0x103,    // epilogue gave up waiting for the accumulator
   kErrWaitAccEmpty = 0x104,   // MMA warp gave up waiting for the epilogue
   kErrBadTile = 0x105,        // a tile descriptor failed its bounds check
+  kErrWaitDep = 0x106,        // producer gave up waiting for an activation dependency
+  kErrWaitGrid = 0x107,       // a CTA gave up waiting for the other CTAs of its grid
 };
 
 __device__ __forceinline__ void report_error(int* err, int code) {

@@ -113,6 +113,10 @@ class MoELayer:
             self.handle, _ptr(x_cpu), _ptr(logits_cpu), M, _ptr(out_cpu), _stream(stream)))
         return out_cpu
 
+    def set_fused_decode(self, enable: bool = True):
+        """Single-launch decode path (bf16, M <= 64) instead of the kernel chain."""
+        self._check("moe_set_fused_decode", self.lib.moe_set_fused_decode(self.handle, 1 if enable else 0))
+
     @property
     def last_launch_count(self) -> int:
         return self.lib.moe_last_launch_count(self.handle)

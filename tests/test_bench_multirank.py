@@ -1,0 +1,69 @@
+"""The N > 1 path of bench.py on the CPU: two gloo ranks exercise the barrier and the
+max-over-ranks timing reduction (the layer itself needs no collective: each rank is
+an independent replica), and the reference arm exits on non-zero ranks."""
+
+import os
+import socket
+import sys
+import types
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, results):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        mx = bench.max_over_ranks(1.5 + rank, world)   # rank r reports 1.5 + r
+        results[rank] = mx
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    mgr = mp.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    mp.spawn(_rank_main, args=(2, port, results), nprocs=2, join=True)
+    assert dict(results) == {0: 2.5, 1: 2.5}
+
+
+def test_single_rank_helpers_are_no_ops():
+    sys.path.insert(0, ROOT)
+    import bench
+    bench.barrier(1)
+    assert bench.max_over_ranks(3.25, 1) == 3.25
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    sys.path.insert(0, ROOT)
+    import bench
+    args = types.SimpleNamespace(workload="tiny", steps=1, warmup=0, seed=0, gpus=2)
+    assert bench.reference_arm(args, ws=2, rank=1) == 0     # no work, no output
+
+
+def test_reference_arm_prints_one_line(capsys):
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    args = types.SimpleNamespace(workload="tiny", steps=1, warmup=0, seed=0, gpus=1)
+    assert bench.reference_arm(args, ws=1, rank=0) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
