@@ -36,14 +36,31 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
+  // small batches (M <= 64): stable ranks from per-expert token masks (the k experts
+  // of a token are distinct, so the rank of pair (t, j) inside its expert is the
+  // number of earlier tokens routed there); the per-warp table is reused for them
+  const int M = a.P / a.k;
+  const bool small = M <= 64;
+  unsigned* s_mask = reinterpret_cast<unsigned*>(s_wc);   // [E][2] when small
   for (int e = tid; e < E; e += kAlignThreads) {
     s_count[e] = 0;
     s_base[e] = 0;
+    if (small) {
+      s_mask[2 * e] = 0u;
+      s_mask[2 * e + 1] = 0u;
+    }
   }
   pdl_wait();
   pdl_trigger();
   __syncthreads();
-  for (int p = tid; p < a.P; p += kAlignThreads) atomicAdd(&s_count[a.topk_ids[p]], 1);
+  for (int p = tid; p < a.P; p += kAlignThreads) {
+    const int e = a.topk_ids[p];
+    atomicAdd(&s_count[e], 1);
+    if (small) {
+      const int t = p / a.k;
+      atomicOr(&s_mask[2 * e + (t >> 5)], 1u << (t & 31));
+    }
+  }
   __syncthreads();
   for (int e = tid; e < E; e += kAlignThreads) {
     const int n = s_count[e];
@@ -55,10 +72,19 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   if (warp == 1) warp_exclusive_scan(s_nb, s_nboff, E, lane);
   __syncthreads();
 
-  // Stable scatter, 1024 pairs per chunk: rank inside the warp from the match
-  // mask, plus the counts of earlier warps in this chunk, plus earlier chunks.
+  if (small) {
+    for (int p = tid; p < a.P; p += kAlignThreads) {
+      const int e = a.topk_ids[p];
+      const int t = p / a.k;
+      const unsigned lo = t < 32 ? (s_mask[2 * e] & ((1u << t) - 1u)) : s_mask[2 * e];
+      const unsigned hi = t < 32 ? 0u : (s_mask[2 * e + 1] & ((1u << (t - 32)) - 1u));
+      a.padded_pairs[s_poff[e] + __popc(lo) + __popc(hi)] = p;
+    }
+  }
+  // Otherwise a stable scatter, 1024 pairs per chunk: rank inside the warp from the
+  // match mask, plus the counts of earlier warps in this chunk, plus earlier chunks.
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int c0 = 0; c0 < a.P; c0 += kAlignThreads) {
+  for (int c0 = 0; !small && c0 < a.P; c0 += kAlignThreads) {
     for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) s_wc[i] = 0;
     __syncthreads();
     const int p = c0 + tid;
