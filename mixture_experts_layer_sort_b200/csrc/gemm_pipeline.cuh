@@ -159,25 +159,85 @@ struct Unit {
   bool ok;       // tile passed its bounds check (every role skips a bad unit alike)
 };
 
-__device__ __forceinline__ Unit make_unit(const Tile& t, int tile, int s, int S, int kblocks, int n_cap) {
+__device__ __forceinline__ Unit make_unit_range(const Tile& t, int tile, int kb0, int kb1, int S, int n_cap) {
   Unit x;
   x.t = t;
   x.tile = tile;
   x.S = S;
-  x.kb0 = s * kblocks / S;
-  x.kb1 = (s + 1) * kblocks / S;
-  x.ok = t.n_valid >= 1 && t.n_valid <= n_cap && x.kb1 > x.kb0;
+  x.kb0 = kb0;
+  x.kb1 = kb1;
+  x.ok = t.n_valid >= 1 && t.n_valid <= n_cap && kb1 > kb0;
   return x;
 }
 
-// Units of a tile list in global memory (written by the align kernel).
+// Split s of S equal K ranges of a tile.
+__device__ __forceinline__ Unit make_unit(const Tile& t, int tile, int s, int S, int kblocks, int n_cap) {
+  return make_unit_range(t, tile, s * kblocks / S, (s + 1) * kblocks / S, S, n_cap);
+}
+
+// The units of CTA blockIdx.x (of gridDim.x) over a tile list in global memory
+// written by the align kernel; count() of them, unit(i) in the order every role of
+// the CTA walks them. Two ways of dealing them out, chosen by S:
+//  - S >= 1: each tile is cut into S equal K ranges and the T*S units go round-robin.
+//  - S == 0, balanced: the T tiles minus the last one to two waves go round-robin as
+//    whole tiles. The K blocks of the remaining tiles are cut into one contiguous
+//    range per CTA of equal length (to one K block), so that every CTA streams the
+//    same weight bytes whatever T is. A tile whose K blocks fall into the ranges of
+//    several CTAs is a split tile with S = that number of CTAs. A CTA takes its range
+//    first, so that the split tiles' partial-sum fix-ups overlap the whole tiles.
 struct GlobalTiles {
   const Tile* tiles;
-  int T, S, kblocks;
-  __device__ __forceinline__ int units() const { return T * S; }
-  __device__ __forceinline__ Unit unit(int u, int n_cap) const {
-    const int t = u / S;
-    return make_unit(tiles[t], t, u - t * S, S, kblocks, n_cap);
+  int T, S, K;
+  int bal_tiles;           // tiles [0, bal_tiles) form the balanced region
+  int g_bal;               // CTAs that share it (each with a non-empty range)
+  int bal_total;           // its K blocks
+  int x0, x1;              // this CTA's K-block range in it
+  int n_bal, n_whole;      // this CTA's units: pieces of the range, then whole tiles
+
+  // The balanced region holds fewer than two waves of tiles of at most 256 K blocks,
+  // so c * bal_total stays far below 2^31 for any grid of up to a few hundred CTAs.
+  __device__ __forceinline__ GlobalTiles(const Tile* tiles_, int T_, int S_, int K_)
+      : tiles(tiles_), T(T_), S(S_), K(K_), bal_tiles(0), g_bal(0), bal_total(0), x0(0), x1(0), n_bal(0),
+        n_whole(0) {
+    if (S != 0 || T <= 0 || K <= 0) return;
+    const int G = static_cast<int>(gridDim.x);
+    const int c = static_cast<int>(blockIdx.x);
+    const int waves = T / G, rem = T - waves * G;
+    bal_tiles = rem == 0 ? 0 : (waves == 0 ? T : rem + G);
+    bal_total = bal_tiles * K;
+    g_bal = bal_total < G ? bal_total : G;
+    if (c < g_bal) {
+      x0 = c * bal_total / g_bal;
+      x1 = (c + 1) * bal_total / g_bal;
+      n_bal = (x1 - 1) / K - x0 / K + 1;
+    }
+    const int whole = T - bal_tiles;
+    n_whole = c < whole ? (whole - 1 - c) / G + 1 : 0;
+  }
+  // the CTA whose range holds K block x of the balanced region
+  __device__ __forceinline__ int owner(int x) const { return ((x + 1) * g_bal - 1) / bal_total; }
+  __device__ __forceinline__ int count() const {
+    if (S == 0) return n_bal + n_whole;
+    const int n = T * S, c = static_cast<int>(blockIdx.x);
+    return c < n ? (n - 1 - c) / static_cast<int>(gridDim.x) + 1 : 0;
+  }
+  __device__ __forceinline__ Unit unit(int i, int n_cap) const {
+    if (S != 0) {
+      const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+      const int t = u / S;
+      return make_unit(tiles[t], t, u - t * S, S, K, n_cap);
+    }
+    if (i < n_bal) {
+      const int t = x0 / K + i;
+      const int kb0 = i == 0 ? x0 - t * K : 0;
+      const int last = x1 - 1;
+      const int kb1 = t == last / K ? last - t * K + 1 : K;
+      const int first = t * K;
+      const int sharers = owner(first + K - 1) - owner(first) + 1;
+      return make_unit_range(tiles[t], t, kb0, kb1, sharers, n_cap);
+    }
+    const int t = bal_tiles + static_cast<int>(blockIdx.x) + (i - n_bal) * static_cast<int>(gridDim.x);
+    return make_unit_range(tiles[t], t, 0, K, 1, n_cap);
   }
 };
 
@@ -247,9 +307,9 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
     npend -= i;
     return true;
   };
-  const int units = src.units();
-  for (int u = blockIdx.x; u < units && !ps.failed; u += gridDim.x) {
-    const Unit un = src.unit(u, rg.n_cap);
+  const int n_units = src.count();
+  for (int i = 0; i < n_units && !ps.failed; ++i) {
+    const Unit un = src.unit(i, rg.n_cap);
     if (!un.ok) continue;
     const int nb16 = (un.t.n_valid + 15) >> 4;
     // first tiled-weight block of the unit's two weight row blocks; a second block
@@ -347,9 +407,9 @@ struct MmaState {
 template <class C, bool kFP8, class Src>
 __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, const Src& src, MmaState& ms,
                         uint32_t tmem, volatile int* abort_flag) {
-  const int units = src.units();
-  for (int u = blockIdx.x; u < units && !ms.failed; u += gridDim.x) {
-    const Unit un = src.unit(u, rg.n_cap);
+  const int n_units = src.count();
+  for (int i = 0; i < n_units && !ms.failed; ++i) {
+    const Unit un = src.unit(i, rg.n_cap);
     if (!un.ok) continue;
     const uint32_t n_pad = static_cast<uint32_t>((un.t.n_valid + 15) & ~15);
     const uint32_t idesc = idesc_make(kFP8 ? 0u : 1u, 128u, n_pad);
@@ -426,9 +486,9 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
     sx = scale_from_amax(*a.amax_x);
     if constexpr (!kGateUp) sh_scale = scale_from_amax(*a.amax_h);
   }
-  const int units = src.units();
-  for (int u = blockIdx.x; u < units && !es.failed; u += gridDim.x) {
-    const Unit un = src.unit(u, rg.n_cap);
+  const int n_units = src.count();
+  for (int i = 0; i < n_units && !es.failed; ++i) {
+    const Unit un = src.unit(i, rg.n_cap);
     if (!un.ok) {
       if (epi_tid == 0) report_error(a.err, kErrBadTile);
       continue;

@@ -20,6 +20,12 @@ namespace moe {
 namespace {
 
 constexpr int kAlignThreads = 1024;
+// The balanced schedule (split factor 0) serves from one to kBalancedWaves waves of
+// tiles. With more, round-robin leaves every CTA within one tile of the mean (< 1/8
+// of its work) and the cut tiles would cost more than they save; with less than one
+// wave, an equal split of every tile (the cost model's factor) needs fewer partial
+// sums for the same balance.
+constexpr int kBalancedWaves = 8;
 constexpr int kAlignWarps = kAlignThreads / 32;
 __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   extern __shared__ int sm[];
@@ -156,8 +162,13 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     // mean token rows per tile; gate_up K block = two 16 KB weight tiles + n rows of x;
     // a split gate_up tile adds and reads back n x 256 fp32 partial sums
     const int n_mean = nblocks > 0 ? (a.P + nblocks - 1) / nblocks : 0;
-    const int s1 = choose_splits_warp(t1, a.kblocks1, a.num_sms, rows_used <= a.ws1_rows_cap,
-                                      2 * 16384 + n_mean * 128, n_mean * 256 * 4 * 2, lane);
+    // balanced schedule (split factor 0) for one to kBalancedWaves waves of tiles when
+    // the partial sums fit the workspace; otherwise the cost model's split factor
+    const bool allow = rows_used <= a.ws1_rows_cap;
+    const bool bal1 = allow && t1 >= a.num_sms && t1 < kBalancedWaves * a.num_sms;
+    const int s1 = (!a.uniform_splits && bal1) ? 0
+                                     : choose_splits_warp(t1, a.kblocks1, a.num_sms, allow,
+                                                          2 * 16384 + n_mean * 128, n_mean * 256 * 4 * 2, lane);
     if (lane == 0) {
       a.header[kHdrMaxRows] = (m + kPadRows - 1) / kPadRows * kPadRows;
       a.header[kHdrRowsUsed] = rows_used;
@@ -170,8 +181,10 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     const int t2 = nblocks * a.fblocks2;
     const int n_mean = nblocks > 0 ? (a.P + nblocks - 1) / nblocks : 0;
     // down: a split only adds more fp32 partial sums to the accumulator
-    const int s2 = choose_splits_warp(t2, a.kblocks2, a.num_sms, true, 16384 + n_mean * 128, n_mean * 128 * 4,
-                                      lane);
+    const bool bal2 = t2 >= a.num_sms && t2 < kBalancedWaves * a.num_sms;
+    const int s2 = (!a.uniform_splits && bal2) ? 0
+                                     : choose_splits_warp(t2, a.kblocks2, a.num_sms, true, 16384 + n_mean * 128,
+                                                          n_mean * 128 * 4, lane);
     if (lane == 0) {
       a.header[kHdrTiles2] = t2;
       a.header[kHdrSplits2] = s2;

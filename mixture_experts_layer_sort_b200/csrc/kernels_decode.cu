@@ -96,8 +96,13 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 struct SmemTiles {
   const Sched* s;
   int fb, T, S, kblocks;
-  __device__ __forceinline__ int units() const { return T * S; }
-  __device__ __forceinline__ Unit unit(int u, int n_cap) const {
+  // units u = blockIdx.x + i * gridDim.x of the T*S, round-robin
+  __device__ __forceinline__ int count() const {
+    const int n = T * S, c = static_cast<int>(blockIdx.x);
+    return c < n ? (n - 1 - c) / static_cast<int>(gridDim.x) + 1 : 0;
+  }
+  __device__ __forceinline__ Unit unit(int i, int n_cap) const {
+    const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
     const int t = u / S;
     const int ai = t / fb;
     Tile tile;

@@ -2,11 +2,13 @@
 // SwiGLU epilogue, down with the routing-weight scatter-add epilogue), one launch
 // each, on the tcgen05 pipeline of gemm_pipeline.cuh.
 //
-// Work units are the align kernel's tiles, each optionally split along K (split-K)
-// so that small batches still stream weights through every SM. A persistent grid of
-// one CTA per SM walks units blockIdx.x, +gridDim.x, ... With programmatic dependent
-// launch, the weight loads of the first stages go out before the kernel waits for
-// its predecessor; only the activation loads wait.
+// Work units are the align kernel's tiles or K ranges of them (split-K), so that
+// small batches still stream weights through every SM. A persistent grid of one CTA
+// per SM takes its units from the balanced schedule of GlobalTiles: whole tiles
+// round-robin, and the last one to two waves cut into equal K-block ranges, so that
+// every CTA streams the same weight bytes. With programmatic dependent launch, the
+// weight loads of the first stages go out before the kernel waits for its
+// predecessor; only the activation loads wait.
 #include "gemm_pipeline.cuh"
 
 namespace moe {
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_trigger();
   }
   const Ring rg = make_ring<C>(a.header[kHdrMaxRows], a.max_stages, sh.ring_bytes);
-  const GlobalTiles src{a.tiles, a.header[a.hdr_tiles], a.header[a.hdr_splits], a.kblocks};
+  const GlobalTiles src(a.tiles, a.header[a.hdr_tiles], a.header[a.hdr_splits], a.kblocks);
   // Everyone but the producer warp waits for the previous kernel here. Otherwise the
   // tile list comes from the align kernel, at least two launches back, and is
   // complete already (see pdl_wait in sm100.cuh).

@@ -82,51 +82,73 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&v)[8]) {
   }
 }
 
-// One warp per padded row: copy (or quantise) the token's x row into x_perm.
+// Row copies (gather, h quantise): 128 threads per row, two rows per 256-thread block.
+// A thread loads up to 8 of the row's 16-byte vectors (8 bf16 each) before it stores
+// any, so a row costs one memory round trip per 8 x 128 vectors, and the per-element
+// work (the FP8 division) is spread over 128 threads instead of one warp.
+constexpr int kRowThreads = 128;
+constexpr int kRowsPerBlock = 256 / kRowThreads;
+
+template <bool kFP8, bool kCoherent>
+__device__ __forceinline__ void copy_row(const uint4* __restrict__ src, void* __restrict__ dst, int n8, float s,
+                                         int t) {
+  for (int base = t; base < n8; base += kRowThreads * 8) {
+    uint4 v[8];
+    #pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (base + kRowThreads * j < n8) v[j] = kCoherent ? __ldcg(src + base + kRowThreads * j) : __ldg(src + base + kRowThreads * j);
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = base + kRowThreads * j;
+      if (i < n8) {
+        if constexpr (!kFP8) {
+          reinterpret_cast<uint4*>(dst)[i] = v[j];
+        } else {
+          float f[8];
+          bf16x8_to_f32(v[j], f);
+          reinterpret_cast<uint2*>(dst)[i] = quant8(f, s);
+        }
+      }
+    }
+  }
+}
+
+// x_perm row r = the x row of the token of padded pair r (or its e4m3 codes).
 template <bool kFP8>
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kRowsPerBlock + threadIdx.x / kRowThreads;
+  const int t = threadIdx.x % kRowThreads;
   pdl_wait();
   pdl_trigger();
-  if (r >= a.rows_bound || r >= a.header[kHdrRowsUsed]) return;
+  if (r >= a.rows_bound) return;
+  // independent loads issued together (rows past rows_used hold stale but in-bounds pairs)
+  const int used = a.header[kHdrRowsUsed];
   const int p = a.padded_pairs[r];
-  if (p >= a.P) return;   // pad row: never read by an output column
-  const int t = p / a.k;
-  const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
-  const int nvec = a.H / 8;
+  const unsigned amax = kFP8 ? *a.amax_x : 0u;
+  if (r >= used || p >= a.P) return;   // unused row, or a pad row: never read by an output column
+  const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(p / a.k) * a.H);
   if constexpr (!kFP8) {
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.x_perm) +
-                                          static_cast<size_t>(r) * a.H);
-    for (int i = lane; i < nvec; i += 32) dst[i] = __ldg(src + i);
+    copy_row<false, false>(src, static_cast<__nv_bfloat16*>(a.x_perm) + static_cast<size_t>(r) * a.H, a.H / 8, 1.f, t);
   } else {
-    const float s = scale_from_amax(*a.amax_x);
-    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.x_perm) +
-                                          static_cast<size_t>(r) * a.H);
-    for (int i = lane; i < nvec; i += 32) {
-      float v[8];
-      bf16x8_to_f32(__ldg(src + i), v);
-      dst[i] = quant8(v, s);
-    }
+    copy_row<true, false>(src, static_cast<uint8_t*>(a.x_perm) + static_cast<size_t>(r) * a.H, a.H / 8,
+                          scale_from_amax(amax), t);
   }
 }
 
 // FP8: h (bf16) -> e4m3 codes with s_h = amax(h)/448 over the valid rows.
 __global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kRowsPerBlock + threadIdx.x / kRowThreads;
+  const int t = threadIdx.x % kRowThreads;
   pdl_wait();
   pdl_trigger();
-  if (r >= a.rows_bound || r >= a.header[kHdrRowsUsed]) return;
-  if (a.padded_pairs[r] >= a.P) return;
-  const float s = scale_from_amax(*a.amax_h);
-  const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(r) * a.I);
-  uint2* dst = reinterpret_cast<uint2*>(a.h_q + static_cast<size_t>(r) * a.I);
-  for (int i = lane; i < a.I / 8; i += 32) {
-    float v[8];
-    bf16x8_to_f32(src[i], v);
-    dst[i] = quant8(v, s);
-  }
+  if (r >= a.rows_bound) return;
+  const int used = a.header[kHdrRowsUsed];
+  const int p = a.padded_pairs[r];
+  const unsigned amax = *a.amax_h;
+  if (r >= used || p >= a.P) return;
+  // h was written by the previous kernel: coherent loads, not the read-only path
+  copy_row<true, true>(reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(r) * a.I),
+                       a.h_q + static_cast<size_t>(r) * a.I, a.I / 8, scale_from_amax(amax), t);
 }
 
 // out = bf16(acc); acc = 0 for the next forward; reset the FP8 amax words.
@@ -181,13 +203,13 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s) {
-  const int grid = (a.rows_bound + 7) / 8;
+  const int grid = (a.rows_bound + kRowsPerBlock - 1) / kRowsPerBlock;
   if (fp8) return launch_kernel(gather_kernel<true>, dim3(grid), dim3(256), 0, s, a);
   return launch_kernel(gather_kernel<false>, dim3(grid), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s) {
-  const int grid = (a.rows_bound + 7) / 8;
+  const int grid = (a.rows_bound + kRowsPerBlock - 1) / kRowsPerBlock;
   return launch_kernel(quant_h_kernel, dim3(grid), dim3(256), 0, s, a);
 }
 

@@ -410,6 +410,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   aa.kblocks2 = L->I / kper;
   aa.num_sms = L->num_sms;
   aa.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
+  aa.uniform_splits = moe::uniform_splits() ? 1 : 0;
   aa.counts = L->counts;
   aa.padded_offsets = L->poff;
   aa.padded_pairs = L->pairs;
@@ -535,6 +536,14 @@ bool moe::pdl_enabled() {
   static const bool on = [] {
     const char* e = std::getenv("MOE_DISABLE_PDL");
     return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+bool moe::uniform_splits() {
+  static const bool on = [] {
+    const char* e = std::getenv("MOE_UNIFORM_SPLITS");
+    return e && e[0] == '1';
   }();
   return on;
 }

@@ -52,6 +52,7 @@ struct AlignArgs {
   int kblocks1, kblocks2;  // K blocks of gate_up (H) and down (I)
   int num_sms;
   int ws1_rows_cap;        // split-K of gate_up needs rows_used <= this
+  int uniform_splits;      // 1: one split-K factor per GEMM from a cost model; 0: balanced
   int* counts;             // [E]
   int* padded_offsets;     // [E+1]
   int* padded_pairs;       // [rows_cap]
@@ -119,6 +120,8 @@ struct FinalizeArgs {
 // in the environment: the kernel may be scheduled before its predecessor in the stream
 // finishes, and orders itself with griddepcontrol (see sm100.cuh).
 bool pdl_enabled();
+// MOE_UNIFORM_SPLITS=1 replaces the balanced unit schedule by one split factor per GEMM
+bool uniform_splits();
 int gemm_max_stages(bool gate_up);   // ring depth cap (MOE_MAX_STAGES1/2 override, for tuning)
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,

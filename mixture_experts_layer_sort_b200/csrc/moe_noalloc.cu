@@ -157,6 +157,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   aa.kblocks2 = v.I / kper;
   aa.num_sms = v.num_sms;
   aa.ws1_rows_cap = static_cast<int>(ws1_rows);
+  aa.uniform_splits = moe::uniform_splits() ? 1 : 0;
   aa.counts = counts;
   aa.padded_offsets = poff;
   aa.padded_pairs = pairs;
