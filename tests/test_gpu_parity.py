@@ -129,3 +129,39 @@ def test_tiny_large_variant(tiny):
     check_routing(tiny, logits, M)
     ref, _ = oracle_full(tiny, x, logits, fp8=False)
     check_output(out, ref, "bf16")
+
+
+def test_topk_equals_E():
+    # every token routed to every expert: P = M*E pairs, each expert sees all tokens
+    c = Case(8, 8, 256, 512, "bf16", w_std=0.02)
+    try:
+        for M in (1, 33):
+            x, logits = tokens(c.E, c.H, M, seed=40 + M)
+            out = c.run(x, logits)
+            dbg, _ = check_routing(c, logits, M)
+            assert np.all(dbg["counts"].cpu().numpy() == M)
+            ref, _ = oracle_full(c, x, logits, fp8=False)
+            check_output(out, ref, "bf16")
+    finally:
+        c.close()
+
+
+@pytest.mark.parametrize("E,k,H,I,dtype,Ms", [
+    (512, 16, 128, 128, "bf16", (1, 37, 130)),    # the largest E and topk, the smallest H and I
+    (512, 16, 128, 128, "fp8", (37,)),
+    (4, 2, 16384, 128, "bf16", (5,)),             # the largest H (256 K blocks of gate_up)
+    (2, 1, 128, 16384, "bf16", (3, 20)),          # the largest I (128 gate_up row blocks, 256 K blocks of down)
+    (2, 1, 128, 16384, "fp8", (20,)),
+])
+def test_size_limits(E, k, H, I, dtype, Ms):
+    c = Case(E, k, H, I, dtype, w_std=0.02)
+    try:
+        for M in Ms:
+            x, logits = tokens(c.E, c.H, M, seed=M + E)
+            out = c.run(x, logits)
+            check_routing(c, logits, M)
+            ref, _ = oracle_full(c, x, logits, fp8=(dtype == "fp8"))
+            check_output(out, ref, dtype)
+        assert c.layer.device_error() == 0
+    finally:
+        c.close()

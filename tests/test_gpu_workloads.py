@@ -84,3 +84,26 @@ def test_prefill_bf16_sampled(large):
     ref = O.moe_forward(x.float().cpu().numpy(), logits.cpu().numpy(), large.k, provider=large.provider,
                         tokens=rows)
     check_output(out, ref, "bf16", rows=rows)
+
+
+@pytest.mark.slow
+def test_prefill_fp8_sampled(large):
+    # the prefill layer quantised to e4m3 from the same bf16 weights; s_x and s_h are
+    # per-tensor over the whole batch, so the oracle still evaluates every pair's h
+    from mixture_experts_layer_sort_b200 import MoELayer
+    M = 4096
+    layer = MoELayer(large.E, large.k, large.H, large.I, "fp8")
+    try:
+        layer.load_weights(large.wg, large.wu, large.wd)
+        x, logits = tokens(large.E, large.H, M, seed=1)
+        out = layer.forward(x, logits)
+        torch.cuda.synchronize()
+        dbg = layer.debug_routing(M)
+        rows = sorted(np.random.default_rng(1).choice(M, size=32, replace=False).tolist())
+        ref, inter = O.moe_forward(x.float().cpu().numpy(), logits.cpu().numpy(), large.k,
+                                   provider=large.provider, fp8=True, tokens=rows, return_intermediates=True)
+        assert np.array_equal(dbg["ids"].cpu().numpy(), inter["ids"]), "expert ids differ"
+        assert np.float32(dbg["s_x"]) == inter["s_x"], "s_x differs"
+        check_output(out, ref, "fp8", rows=rows)
+    finally:
+        layer.close()
