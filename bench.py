@@ -384,6 +384,20 @@ def main():
     step_ms = [sum(per_M_ms[M][s] for M in Ms) for s in range(args.steps)]
     ms_per_step = max_over_ranks(statistics.mean(step_ms), ws)
 
+    # ---------------------------------------------------------------- eager launches (no graph), same workload
+    eager_ms = {M: [] for M in Ms}
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            for M in Ms:
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                layer.forward(*toks[M], out=outs[M])
+                e1.record(stream)
+                eager_ms[M].append((e0, e1))
+    torch.cuda.synchronize()
+    eager_ms = {M: statistics.median(a.elapsed_time(b) for a, b in v) for M, v in eager_ms.items()}
+
     # ---------------------------------------------------------------- per-kernel events (same workload, eager)
     layer.profile_enable(True)
     prof_steps = max(3, min(args.steps, 20))
@@ -444,7 +458,10 @@ def main():
     for M in Ms:
         t = statistics.mean(per_M_ms[M])
         b = alg_bytes_layer(wl, dtype, M, A[M])
-        per_M[str(M)] = {"ms": t, "tokens_per_s": M / (t / 1e3), "active_experts": A[M],
+        srt = sorted(per_M_ms[M])
+        per_M[str(M)] = {"ms": t, "ms_p50": statistics.median(srt),
+                         "ms_p95": srt[min(len(srt) - 1, int(round(0.95 * (len(srt) - 1))))],
+                         "ms_eager": eager_ms[M], "tokens_per_s": M / (t / 1e3), "active_experts": A[M],
                          "alg_GB": b / 1e9, "alg_GBps": b / (t / 1e3) / 1e9,
                          "roofline_frac": (b / (hbm_gbs * 1e9)) / (t / 1e3), "launches": launches_per_M[M]}
 

@@ -122,7 +122,14 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   if (tid == 0) a.padded_offsets[E] = s_poff[E];
 
   // Tiles: for expert e, its token blocks b and weight row blocks f, in the
-  // order (e, f, b) so that tiles sharing a weight tile are neighbours.
+  // order (e, f, b) so that tiles sharing a weight tile are neighbours. The down
+  // tiles go in feature slabs: (slab, e, f, b), slab s covering row blocks
+  // [s*F/S, (s+1)*F/S). Every tile of a slab adds into the same columns of the fp32
+  // accumulator, so with S slabs only 1/S of the accumulator is live in L2 at a time
+  // (a large batch's accumulator would otherwise not stay in L2 between the k
+  // contributions to each token); the price is reading each expert's h once per slab.
+  const int nblocks_all = s_nboff[E];
+  const int S2 = a.acc_slabs < 1 ? 1 : a.acc_slabs;
   for (int e = warp; e < E; e += kAlignWarps) {
     const int n = s_count[e];
     const int nb = s_nb[e];
@@ -144,7 +151,9 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
       t.fblock = f;
       t.row_start = s_poff[e] + b * a.BN;
       t.n_valid = min(a.BN, n - b * a.BN);
-      a.tiles2[static_cast<size_t>(base) * a.fblocks2 + idx] = t;
+      const int sl = ((f + 1) * S2 - 1) / a.fblocks2;      // the slab holding row block f
+      const int f0 = sl * a.fblocks2 / S2, f1 = (sl + 1) * a.fblocks2 / S2;
+      a.tiles2[static_cast<size_t>(nblocks_all) * f0 + static_cast<size_t>(base) * (f1 - f0) + (f - f0) * nb + b] = t;
     }
   }
 

@@ -370,6 +370,21 @@ int forward_fused_decode(moe_layer* L, const void* x, const float* logits, int M
   return MOE_OK;
 }
 
+// Feature slabs of the down tile order: enough that one slab of the fp32 accumulator
+// (M x H x 4 bytes / slabs) stays well inside the 126 MB L2 next to the streamed
+// weights and the live activations.
+constexpr long long kAccSlabBytes = 64ll << 20;
+
+int acc_slabs(int M, int H, int fblocks2) {
+  static const int forced = [] {
+    const char* e = std::getenv("MOE_ACC_SLABS");   // fixed slab count (1 = expert-major order)
+    return e ? std::atoi(e) : 0;
+  }();
+  const long long bytes = static_cast<long long>(M) * H * 4;
+  const long long s = forced > 0 ? forced : (bytes + kAccSlabBytes - 1) / kAccSlabBytes;
+  return static_cast<int>(std::max(1ll, std::min<long long>(s, fblocks2)));
+}
+
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
   if (L->fused_decode && !is_fp8(L) && moe::decode_supported(M, L->E, L->k))
@@ -410,6 +425,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   aa.kblocks2 = L->I / kper;
   aa.num_sms = L->num_sms;
   aa.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
+  aa.acc_slabs = acc_slabs(M, L->H, aa.fblocks2);
   aa.uniform_splits = moe::uniform_splits() ? 1 : 0;
   aa.counts = L->counts;
   aa.padded_offsets = L->poff;

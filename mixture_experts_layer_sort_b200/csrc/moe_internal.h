@@ -52,6 +52,7 @@ struct AlignArgs {
   int kblocks1, kblocks2;  // K blocks of gate_up (H) and down (I)
   int num_sms;
   int ws1_rows_cap;        // split-K of gate_up needs rows_used <= this
+  int acc_slabs;           // down tiles ordered in this many feature slabs (<= fblocks2; 0 or 1: none)
   int uniform_splits;      // 1: one split-K factor per GEMM from a cost model; 0: balanced
   int* counts;             // [E]
   int* padded_offsets;     // [E+1]
