@@ -19,12 +19,13 @@ of a top-k softmax MoE layer with SwiGLU experts:
              weights = full softmax restricted to those k and renormalised;
 2. permute - pair ids p = t*k + j grouped by expert, ascending p inside each
              expert, optionally padded to a tile of BT rows;
-3. FP8     - per-tensor e4m3 quantisation of weights (one scale per expert and
-             tensor), of x and of the intermediate h ("FP8 tensor-quantized
-             fused MoE", same page, section "2. FP8 backend routing changes
-             which kernel path runs"; E4M3 = 4 exponent and 3 mantissa bits,
-             kongchang.com, "MoE Kernel Engineering Optimization Practices on
-             Amazon SageMaker AI", section "Triton Backend Routing");
+3. FP8     - per-tensor e4m3 (or e5m2) quantisation of weights (one scale per
+             expert and tensor), of x and of the intermediate h ("FP8
+             tensor-quantized fused MoE", same page, section "2. FP8 backend
+             routing changes which kernel path runs"; E4M3 = 4 exponent and 3
+             mantissa bits, E5M2 = 5 and 2, kongchang.com, "MoE Kernel
+             Engineering Optimization Practices on Amazon SageMaker AI", section
+             "Triton Backend Routing");
 4. experts - h = silu(W_gate x) * (W_up x), y = W_down h;
 5. combine - out_t = sum_j w_tj * y_(t,j), the routing-weight scale applied
              after the down projection ("fuses scaling, matrix multiplication,
@@ -36,7 +37,7 @@ Making WGMMA Run at Full Utilization") changes no arithmetic, so the oracle has
 a single GEMM orientation.
 
 Precision: fp64 throughout, except that every step that turns a float into an
-integer code (the e4m3 quantisation of weights, x and h) is taken in IEEE fp32,
+integer code (the FP8 quantisation of weights, x and h) is taken in IEEE fp32,
 the precision in which the kernels take it.
 
 Every function here is pinned by the CPU tests in ``tests/test_oracle_*.py``
@@ -51,6 +52,10 @@ import numpy as np
 E4M3_MAX = 448.0          # largest finite e4m3 magnitude (exponent 1111, mantissa 110)
 E4M3_MIN_NORMAL_EXP = -6  # 2^-6 is the smallest normal e4m3 magnitude
 E4M3_SUBNORMAL_STEP = 2.0 ** -9
+
+E5M2_MAX = 57344.0        # largest finite e5m2 magnitude (exponent 11110, mantissa 11)
+E5M2_MIN_NORMAL_EXP = -14
+E5M2_SUBNORMAL_STEP = 2.0 ** -16
 
 
 # --------------------------------------------------------------------------- routing
@@ -170,33 +175,88 @@ def e4m3_encode(v: np.ndarray) -> np.ndarray:
     return code.astype(np.uint8)
 
 
-def per_tensor_scale(t: np.ndarray) -> np.float32:
-    """s = amax(|t|) / 448 in fp32; an all-zero tensor takes s = 1."""
+# --------------------------------------------------------------------------- e5m2 codec
+# The second FP8 variant the kongchang.com page names ("MoE Kernel Engineering
+# Optimization Practices on Amazon SageMaker AI", section "Triton Backend Routing: A
+# Practical Path to FP8 Quantization"): 5 exponent bits and 2 mantissa bits, a wider
+# range than E4M3 at lower precision. Bias 15 (the IEEE-style layout of the OCP 8-bit
+# floating-point definition): exponent field 0 is subnormal (m * 2^-16), field 31 is
+# infinity (m = 0) or NaN; the largest finite magnitude is 1.75 * 2^15 = 57344.
+def e5m2_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each e5m2 code: 1 sign, 5 exponent (bias 15), 2 mantissa bits. Returns float64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    ex = (c >> 2) & 0x1F
+    man = c & 0x3
+    normal = (1.0 + man / 4.0) * np.exp2(ex - 15.0)
+    sub = man * E5M2_SUBNORMAL_STEP
+    mag = np.where(ex == 0, sub, normal)
+    mag = np.where(ex == 31, np.where(man == 0, np.inf, np.nan), mag)
+    return sign * mag
+
+
+def e5m2_encode(v: np.ndarray) -> np.ndarray:
+    """Round fp32 values to e5m2: round to nearest, ties to even, saturating.
+
+    Magnitudes above 57344 (infinity included) become 57344 (code 0x7B); NaN
+    becomes the NaN code 0x7F with the input's sign bit. Works on the exact value
+    of each fp32 input (held in fp64).
+    """
+    f = np.asarray(v, dtype=np.float32)
+    neg = np.signbit(f)
+    nan = np.isnan(f)
+    a = np.abs(f.astype(np.float64))
+    a = np.where(nan, 0.0, np.minimum(a, E5M2_MAX))
+    _, ex = np.frexp(a)
+    e = ex.astype(np.int64) - 1                      # a in [2^e, 2^(e+1))
+    subnormal = a < 2.0 ** E5M2_MIN_NORMAL_EXP
+    # quantum of the grid at a: 2^-16 below the normal range, 2^(e-2) above
+    step = np.where(subnormal, E5M2_SUBNORMAL_STEP, np.exp2((e - 2).astype(np.float64)))
+    q = np.rint(a / step).astype(np.int64)           # ties to even
+    code_sub = q                                     # q == 4 lands on 2^-14, code 0x04
+    carry = q == 8                                   # normal q in [4, 8]; 8 is the next binade
+    e_n = np.where(carry, e + 1, e)
+    q_n = np.where(carry, 4, q)
+    code_norm = ((e_n + 15) << 2) | (q_n - 4)
+    code = np.where(subnormal, code_sub, code_norm)
+    code = np.where(a == 0.0, 0, code)
+    code = np.where(nan, 0x7F, code)
+    code = code | np.where(neg, 0x80, 0)
+    return code.astype(np.uint8)
+
+
+# name -> (encode, decode, largest finite magnitude)
+FP8_FORMATS = {"e4m3": (e4m3_encode, e4m3_decode, E4M3_MAX), "e5m2": (e5m2_encode, e5m2_decode, E5M2_MAX)}
+
+
+def per_tensor_scale(t: np.ndarray, fmt: str = "e4m3") -> np.float32:
+    """s = amax(|t|) / (largest finite value of the format) in fp32; an all-zero
+    tensor takes s = 1."""
+    fmax = FP8_FORMATS[fmt][2]
     a = np.float32(np.max(np.abs(np.asarray(t, dtype=np.float32)))) if np.size(t) else np.float32(0)
     if a == 0:
         return np.float32(1.0)
-    return np.float32(a) / np.float32(E4M3_MAX)
+    return np.float32(a) / np.float32(fmax)
 
 
-def quantize(t: np.ndarray, s: np.float32) -> np.ndarray:
-    """e4m3 codes of t / s, the division in IEEE fp32."""
+def quantize(t: np.ndarray, s: np.float32, fmt: str = "e4m3") -> np.ndarray:
+    """FP8 codes of t / s, the division in IEEE fp32."""
     q = np.asarray(t, dtype=np.float32) / np.float32(s)
-    return e4m3_encode(q.astype(np.float32))
+    return FP8_FORMATS[fmt][0](q.astype(np.float32))
 
 
-_E4M3_TABLE = None
+_DECODE_TABLES = {}
 
 
-def dequantize(codes: np.ndarray, s) -> np.ndarray:
-    """decode(code) * s in fp64; the decode goes through a 256-entry table of
-    e4m3_decode, which is the same function evaluated once per code."""
-    global _E4M3_TABLE
-    if _E4M3_TABLE is None:
-        _E4M3_TABLE = e4m3_decode(np.arange(256, dtype=np.uint8))
-    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)] * float(s)
+def dequantize(codes: np.ndarray, s, fmt: str = "e4m3") -> np.ndarray:
+    """decode(code) * s in fp64; the decode goes through a 256-entry table of the
+    format's decode function, which is the same function evaluated once per code."""
+    if fmt not in _DECODE_TABLES:
+        _DECODE_TABLES[fmt] = FP8_FORMATS[fmt][1](np.arange(256, dtype=np.uint8))
+    return _DECODE_TABLES[fmt][np.asarray(codes, dtype=np.uint8)] * float(s)
 
 
-def quantize_expert_weights(W: np.ndarray):
+def quantize_expert_weights(W: np.ndarray, fmt: str = "e4m3"):
     """One scale per expert for a stacked weight tensor W [E, rows, cols].
 
     Returns (scales [E] float32, codes [E, rows, cols] uint8).
@@ -206,9 +266,9 @@ def quantize_expert_weights(W: np.ndarray):
     scales = np.zeros(E, dtype=np.float32)
     codes = np.zeros(W.shape, dtype=np.uint8)
     for e in range(E):
-        s = per_tensor_scale(W[e])
+        s = per_tensor_scale(W[e], fmt)
         scales[e] = s
-        codes[e] = quantize(W[e], s)
+        codes[e] = quantize(W[e], s, fmt)
     return scales, codes
 
 
@@ -246,7 +306,7 @@ def _map_experts(fn, experts, threads):
 
 def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
                 provider=None, tokens=None, return_intermediates=False, threads=None,
-                weight_cache=None):
+                weight_cache=None, fp8_format="e4m3"):
     """The layer's output in fp64.
 
     x       [M, H]  bf16 values (any float array holding them)
@@ -254,7 +314,7 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
     w_gate  [E, I, H], w_up [E, I, H], w_down [E, H, I] (bf16 values), or
     provider(e) -> (w_gate[e], w_up[e], w_down[e]) for weights too large to
             hold on the host at once.
-    fp8     emulate the per-tensor e4m3 path: each weight tensor of each
+    fp8     emulate the per-tensor FP8 path: each weight tensor of each
             expert quantised with its own scale, x quantised with one scale
             over all M*H elements, h quantised with one scale over all valid
             (token, slot) rows; dequantised values feed the fp64 arithmetic.
@@ -263,6 +323,7 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
             (FP8) s_h are still computed over the whole batch, as defined.
     threads experts are independent, so they may be evaluated on several
             threads (default: the CPU count); no result depends on it.
+    fp8_format  "e4m3" (default) or "e5m2": the code format of every FP8 tensor.
     weight_cache  optional dict reused across calls with the same weights: it
             keeps each expert's FP8 scales and codes so that they are not
             recomputed (the values are identical either way).
@@ -281,10 +342,11 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
     inter = {"ids": ids, "w": w, "counts": counts, "offsets": offsets,
              "sorted_pairs": sorted_pairs}
 
+    fmt = fp8_format
     if fp8:
-        s_x = per_tensor_scale(x)
-        x_codes = quantize(x, s_x)
-        xin = dequantize(x_codes, s_x)
+        s_x = per_tensor_scale(x, fmt)
+        x_codes = quantize(x, s_x, fmt)
+        xin = dequantize(x_codes, s_x, fmt)
         inter["s_x"] = s_x
         inter["x_codes"] = x_codes
         inter["w_scales"] = np.zeros((E, 3), dtype=np.float32)
@@ -307,11 +369,11 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
         if q is None:
             q = []
             for t in W.get(e):
-                st = per_tensor_scale(t)
-                q.append((st, quantize(t, st)))
+                st = per_tensor_scale(t, fmt)
+                q.append((st, quantize(t, st, fmt)))
             if weight_cache is not None:
                 weight_cache[e] = q
-        return tuple(dequantize(c, st) for st, c in q), tuple(st for st, _ in q)
+        return tuple(dequantize(c, st, fmt) for st, c in q), tuple(st for st, _ in q)
 
     active = [e for e in range(E) if counts[e] > 0]
 
@@ -350,7 +412,7 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
                 Y[int(p)] = Ym[i]
 
     if fp8:
-        s_h = np.float32(1.0) if h_amax == 0 else np.float32(h_amax) / np.float32(E4M3_MAX)
+        s_h = np.float32(1.0) if h_amax == 0 else np.float32(h_amax) / np.float32(FP8_FORMATS[fmt][2])
         inter["s_h"] = s_h
 
         # pass 2: quantised h through the dequantised down projection
@@ -361,7 +423,7 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
                 return []
             d_w = expert_weights(e)[0][2]
             Hm = np.stack([h_rows[p] for p in pairs])
-            Hm = dequantize(quantize(Hm.astype(np.float32), s_h), s_h)
+            Hm = dequantize(quantize(Hm.astype(np.float32), s_h, fmt), s_h, fmt)
             Ym = Hm @ d_w.T
             return [(p, Ym[i]) for i, p in enumerate(pairs)]
 

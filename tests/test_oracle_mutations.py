@@ -64,3 +64,20 @@ def test_rounding_half_away_from_zero_is_caught(monkeypatch):
     v = bits.view(np.float32)
     v = v[np.isfinite(v)]
     assert not np.array_equal(O.e4m3_encode(v), torch_codes(v))
+
+
+def test_e5m2_wrong_bias_is_caught(monkeypatch):
+    # an e5m2 decode with exponent bias 16 instead of 15 disagrees with torch's decode
+    real = O.e5m2_decode
+    monkeypatch.setattr(O, "e5m2_decode", lambda c: real(c) * 0.5)
+    from tests.test_oracle_e5m2 import test_decode_every_code_matches_torch
+    with pytest.raises(AssertionError):
+        test_decode_every_code_matches_torch()
+
+
+def test_e5m2_scale_with_the_e4m3_maximum_is_caught(monkeypatch):
+    # a quantiser that divides amax by 448 for e5m2 too fails the torch-based weight pin
+    monkeypatch.setitem(O.FP8_FORMATS, "e5m2", (O.e5m2_encode, O.e5m2_decode, O.E4M3_MAX))
+    from tests.test_oracle_e5m2 import test_expert_weight_quantiser_matches_torch
+    with pytest.raises(AssertionError):
+        test_expert_weight_quantiser_matches_torch((3, 64, 32))
