@@ -50,8 +50,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default="decode",
-                    choices=["tiny", "decode", "decode_fp8", "large_decode", "prefill", "prefill_fp8",
-                             "prefill_e48", "prefill_e48_fp8"])
+                    choices=["tiny", "decode", "decode_fp8", "decode_e5m2", "large_decode", "prefill",
+                             "prefill_fp8", "prefill_e48", "prefill_e48_fp8"])
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -81,15 +81,23 @@ def read_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def is_fp8(dtype):
+    return dtype in ("fp8", "fp8_e5m2")
+
+
+def fp8_format(dtype):
+    return "e5m2" if dtype == "fp8_e5m2" else "e4m3"
+
+
 def weight_bytes(wl, dtype):
-    return 1 if dtype == "fp8" else 2
+    return 1 if is_fp8(dtype) else 2
 
 
 def alg_bytes_layer(wl, dtype, M, A):
     """Algorithmic bytes of one forward: active-expert weights, FP8 scales, x, out, logits."""
     bw = weight_bytes(wl, dtype)
     b = A * 3 * wl.H * wl.I * bw + M * wl.H * 2 * 2 + M * wl.E * 4
-    if dtype == "fp8":
+    if is_fp8(dtype):
         b += 3 * wl.E * 4
     return b
 
@@ -208,7 +216,8 @@ def time_oracle_sweep(wl, dtype, host_weights, tokens_per_M, budget_s=30.0, max_
     for _ in range(max_reps):
         t0 = time.time()
         for M, (x, l) in tokens_per_M.items():
-            O.moe_forward(x, l, wl.k, *host_weights, fp8=(dtype == "fp8"), weight_cache=cache)
+            O.moe_forward(x, l, wl.k, *host_weights, fp8=is_fp8(dtype), fp8_format=fp8_format(dtype),
+                          weight_cache=cache)
         times.append(time.time() - t0)
         if time.time() - t_start > budget_s:
             break
@@ -238,13 +247,13 @@ def reference_arm(args, ws, rank):
     cache = {}
     for _ in range(max(args.warmup, 0)):
         for M, (x, l) in toks.items():
-            O.moe_forward(x, l, wl.k, *host, fp8=(dtype == "fp8"), weight_cache=cache)
+            O.moe_forward(x, l, wl.k, *host, fp8=is_fp8(dtype), fp8_format=fp8_format(dtype), weight_cache=cache)
         break   # one warm-up sweep is enough for the CPU path (fills the FP8 weight cache)
     times = []
     for _ in range(args.steps):
         t0 = time.time()
         for M, (x, l) in toks.items():
-            O.moe_forward(x, l, wl.k, *host, fp8=(dtype == "fp8"), weight_cache=cache)
+            O.moe_forward(x, l, wl.k, *host, fp8=is_fp8(dtype), fp8_format=fp8_format(dtype), weight_cache=cache)
         times.append(time.time() - t0)
     sec = statistics.mean(times)
     value = tokens / sec
@@ -447,7 +456,8 @@ def main():
 
     # ---------------------------------------------------------------- CPU oracle on the same sweep
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline and args.workload in ("tiny", "decode", "decode_fp8"):
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and args.workload in ("tiny", "decode", "decode_fp8",
+                                                                               "decode_e5m2"):
         host_w = [synth.bf16_to_f32_numpy(w) for w in (wg, wu, wd)]
         tpm = {M: (toks[M][0].float().cpu().numpy(), toks[M][1].cpu().numpy()) for M in Ms}
         sec, reps = time_oracle_sweep(wl, dtype, host_w, tpm)
@@ -476,7 +486,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if dtype == "bf16" else "e4m3",
+        "dtype": "bf16" if dtype == "bf16" else fp8_format(dtype),
         "data": "synthetic",
         "config": {"workload": wl.description + f", one step = one forward at each M in {Ms}",
                    "E": wl.E, "topk": wl.k, "H": wl.H, "I": wl.I, "Ms": Ms, "global_batch": tokens_per_step * ws,

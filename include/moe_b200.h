@@ -16,11 +16,13 @@
  *               order ("fuses scaling, matrix multiplication, and expert aggregation
  *               into one GPU pass", aib.vote, "AWS SageMaker MoE kernel
  *               optimizations", third paragraph).
- * The FP8 variant stores weights as e4m3 with one fp32 scale per expert tensor and
- * quantises x and h per tensor on the fly ("FP8 tensor-quantized fused MoE",
- * toolboxkart.tech page, section "2. FP8 backend routing changes which kernel path
- * runs"; E4M3 format: kongchang.com, "MoE Kernel Engineering Optimization Practices
- * on Amazon SageMaker AI", section "Triton Backend Routing").
+ * The FP8 variants store weights as 8-bit floats with one fp32 scale per expert
+ * tensor and quantise x and h per tensor on the fly ("FP8 tensor-quantized fused
+ * MoE", toolboxkart.tech page, section "2. FP8 backend routing changes which kernel
+ * path runs"), in one of the two formats the kongchang.com page names ("MoE Kernel
+ * Engineering Optimization Practices on Amazon SageMaker AI", section "Triton
+ * Backend Routing: A Practical Path to FP8 Quantization"): E4M3 (4 exponent and 3
+ * mantissa bits, largest finite 448) or E5M2 (5 and 2, largest finite 57344).
  *
  * The token count M is a runtime argument of every call: no kernel is compiled,
  * specialised or re-encoded per M ("Removing repeat compilation can reduce
@@ -54,8 +56,9 @@ typedef struct moe_layer moe_layer;   /* opaque handle */
 
 typedef enum {
   MOE_DTYPE_BF16 = 0,       /* bf16 weights and activations, fp32 accumulation        */
-  MOE_DTYPE_FP8_E4M3 = 1    /* e4m3 weights (per expert-tensor scale), e4m3 activations
+  MOE_DTYPE_FP8_E4M3 = 1,   /* e4m3 weights (per expert-tensor scale), e4m3 activations
                                (per-tensor dynamic scale), fp32 accumulation           */
+  MOE_DTYPE_FP8_E5M2 = 2    /* the same with e5m2 codes for weights and activations    */
 } moe_dtype;
 
 typedef enum {
@@ -80,15 +83,17 @@ MOE_API int moe_destroy(moe_layer* layer);
 /* Copy bf16 expert weights into library-owned memory (device pointers):
  *   w_gate [E, I, H], w_up [E, I, H], w_down [E, H, I], each row-major bf16.
  * For an FP8 layer the library quantises them: one fp32 scale per (expert, tensor)
- * s = amax|W| / 448 (s = 1 for an all-zero tensor), codes = e4m3(W / s) with an IEEE
- * fp32 division, round-to-nearest-even, saturating to +-448.
+ * s = amax|W| / F (F = 448 for e4m3, 57344 for e5m2; s = 1 for an all-zero tensor),
+ * codes = fp8(W / s) with an IEEE fp32 division, round-to-nearest-even, saturating
+ * to +-F.
  * Runs on `stream` and synchronises it before returning; the caller may free the
  * sources afterwards. Calling it again replaces the weights. */
 MOE_API int moe_load_weights(moe_layer* layer, const void* w_gate, const void* w_up,
                      const void* w_down, void* stream);
 
-/* Load already-quantised e4m3 weights into an FP8 layer (device pointers):
- *   q_gate [E, I, H], q_up [E, I, H], q_down [E, H, I] (uint8 e4m3 codes) and
+/* Load already-quantised weights into an FP8 layer (device pointers):
+ *   q_gate [E, I, H], q_up [E, I, H], q_down [E, H, I] (uint8 codes in the layer's
+ *   format, e4m3 or e5m2) and
  *   scales [E, 3] fp32 (gate, up, down scale of each expert; host pointer).
  * Weight value = decode(code) * scale. Synchronises `stream`. */
 MOE_API int moe_load_weights_fp8(moe_layer* layer, const void* q_gate, const void* q_up,
@@ -186,11 +191,11 @@ MOE_API int moe_debug_routing(moe_layer* layer, int* topk_ids, float* topk_w, in
                       int* tile_rows);
 
 /* Test access: copy the permuted activations of the last forward (device buffer of
- * padded_offsets[E] rows of H elements: bf16, or e4m3 codes for FP8 layers), and
+ * padded_offsets[E] rows of H elements: bf16, or FP8 codes for FP8 layers), and
  * the intermediate h (rows of I bf16 values) when h_out is not NULL. */
 MOE_API int moe_debug_activations(moe_layer* layer, void* x_perm_out, void* h_out);
 
-/* Test access: copy the stored weights (device buffers): FP8 layers give e4m3 codes
+/* Test access: copy the stored weights (device buffers): FP8 layers give their codes
  * q_gate/q_up [E,I,H], q_down [E,H,I] and scales_host [E,3]; bf16 layers give the
  * bf16 copies and leave scales_host untouched. Any pointer may be NULL. */
 MOE_API int moe_debug_weights(moe_layer* layer, void* gate_out, void* up_out, void* down_out,

@@ -29,8 +29,7 @@
 // run both GEMMs back to back.
 #pragma once
 
-#include <cuda_fp8.h>
-
+#include "fp8_format.cuh"
 #include "moe_internal.h"
 #include "sm100.cuh"
 
@@ -243,11 +242,6 @@ struct GlobalTiles {
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
 
-__device__ __forceinline__ float scale_from_amax(unsigned bits) {
-  const float amax = __uint_as_float(bits);
-  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-}
-
 // ------------------------------------------------------------------------ producer
 struct ProducerState {
   int stage = 0;
@@ -412,7 +406,8 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
     const Unit un = src.unit(i, rg.n_cap);
     if (!un.ok) continue;
     const uint32_t n_pad = static_cast<uint32_t>((un.t.n_valid + 15) & ~15);
-    const uint32_t idesc = idesc_make(kFP8 ? 0u : 1u, 128u, n_pad);
+    // operand format: bf16 = 1 under kind::f16; the FP8 format code under kind::f8f6f4
+    const uint32_t idesc = idesc_make(kFP8 ? static_cast<uint32_t>(a.f8) : 1u, 128u, n_pad);
     const int buf = rg.nbuf == 2 ? (ms.it & 1) : 0;
     const uint32_t acc_phase = rg.nbuf == 2 ? ((ms.it >> 1) & 1) : (ms.it & 1);
     const uint32_t d_tmem = tmem + 256u * buf;
@@ -442,8 +437,8 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
         const uint64_t ad0 = sdesc_k_sw128(a0 + koff);
         const uint64_t ad1 = sdesc_k_sw128(a0 + C::kABytes + koff);
         if constexpr (kFP8) {
-          mma_e4m3(d_tmem, ad0, bd, idesc, accum);
-          mma_e4m3(d_tmem + rg.up_col, ad1, bd, idesc, accum);
+          mma_f8(d_tmem, ad0, bd, idesc, accum);
+          mma_f8(d_tmem + rg.up_col, ad1, bd, idesc, accum);
         } else {
           mma_bf16(d_tmem, ad0, bd, idesc, accum);
           mma_bf16(d_tmem + rg.up_col, ad1, bd, idesc, accum);
@@ -483,8 +478,8 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
   const int epi_tid = threadIdx.x - 64;
   float sx = 1.f, sh_scale = 1.f;
   if constexpr (kFP8) {
-    sx = scale_from_amax(*a.amax_x);
-    if constexpr (!kGateUp) sh_scale = scale_from_amax(*a.amax_h);
+    sx = fp8_scale_from_amax(*a.amax_x, a.f8);
+    if constexpr (!kGateUp) sh_scale = fp8_scale_from_amax(*a.amax_h, a.f8);
   }
   const int n_units = src.count();
   for (int i = 0; i < n_units && !es.failed; ++i) {

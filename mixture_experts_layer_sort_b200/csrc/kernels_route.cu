@@ -8,9 +8,10 @@
 // experts by their softmax renormalised over the selection.
 //
 // FP8: per-tensor ("tensor-quantized", same page, section "2. FP8 backend routing
-// changes which kernel path runs") e4m3 codes, s = amax/448, codes = RNE(v / s)
-// saturated to +-448, the division in IEEE fp32.
-#include <cuda_fp8.h>
+// changes which kernel path runs") E4M3 or E5M2 codes, s = amax / (the format's
+// largest finite value), codes = RNE(v / s) saturated, the division in IEEE fp32
+// (fp8_format.cuh).
+#include "fp8_format.cuh"
 
 #include "moe_internal.h"
 #include "route_common.cuh"
@@ -53,19 +54,14 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   }
 }
 
-__device__ __forceinline__ float scale_from_amax(unsigned amax_bits) {
-  const float amax = __uint_as_float(amax_bits);
-  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-}
-
-// 8 fp32 values -> 8 e4m3 codes (RNE, saturating), v[i] / s with IEEE division.
-__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
+// 8 fp32 values -> 8 FP8 codes (RNE, saturating), v[i] / s with IEEE division.
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, int f8) {
   uint2 r;
   unsigned short c[4];
   #pragma unroll
   for (int q = 0; q < 4; ++q) {
     float2 f = make_float2(__fdiv_rn(v[2 * q], s), __fdiv_rn(v[2 * q + 1], s));
-    c[q] = static_cast<unsigned short>(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3));
+    c[q] = fp8x2(f, f8);
   }
   r.x = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
   r.y = static_cast<unsigned>(c[2]) | (static_cast<unsigned>(c[3]) << 16);
@@ -91,7 +87,7 @@ constexpr int kRowsPerBlock = 256 / kRowThreads;
 
 template <bool kFP8, bool kCoherent>
 __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, void* __restrict__ dst, int n8, float s,
-                                         int t) {
+                                         int f8, int t) {
   for (int base = t; base < n8; base += kRowThreads * 8) {
     uint4 v[8];
     #pragma unroll
@@ -106,7 +102,7 @@ __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, void* __
         } else {
           float f[8];
           bf16x8_to_f32(v[j], f);
-          reinterpret_cast<uint2*>(dst)[i] = quant8(f, s);
+          reinterpret_cast<uint2*>(dst)[i] = quant8(f, s, f8);
         }
       }
     }
@@ -128,10 +124,11 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
   if (r >= used || p >= a.P) return;   // unused row, or a pad row: never read by an output column
   const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(p / a.k) * a.H);
   if constexpr (!kFP8) {
-    copy_row<false, false>(src, static_cast<__nv_bfloat16*>(a.x_perm) + static_cast<size_t>(r) * a.H, a.H / 8, 1.f, t);
+    copy_row<false, false>(src, static_cast<__nv_bfloat16*>(a.x_perm) + static_cast<size_t>(r) * a.H, a.H / 8, 1.f, 0,
+                           t);
   } else {
     copy_row<true, false>(src, static_cast<uint8_t*>(a.x_perm) + static_cast<size_t>(r) * a.H, a.H / 8,
-                          scale_from_amax(amax), t);
+                          fp8_scale_from_amax(amax, a.f8), a.f8, t);
   }
 }
 
@@ -148,7 +145,7 @@ __global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
   if (r >= used || p >= a.P) return;
   // h was written by the previous kernel: coherent loads, not the read-only path
   copy_row<true, true>(reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(r) * a.I),
-                       a.h_q + static_cast<size_t>(r) * a.I, a.I / 8, scale_from_amax(amax), t);
+                       a.h_q + static_cast<size_t>(r) * a.I, a.I / 8, fp8_scale_from_amax(amax, a.f8), a.f8, t);
 }
 
 // out = bf16(acc); acc = 0 for the next forward; reset the FP8 amax words.
@@ -158,8 +155,8 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
   pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.amax != nullptr) {
     if (a.last_scales != nullptr) {
-      a.last_scales[0] = scale_from_amax(a.amax[0]);
-      a.last_scales[1] = scale_from_amax(a.amax[1]);
+      a.last_scales[0] = fp8_scale_from_amax(a.amax[0], a.f8);
+      a.last_scales[1] = fp8_scale_from_amax(a.amax[1], a.f8);
     }
     a.amax[0] = 0u;
     a.amax[1] = 0u;

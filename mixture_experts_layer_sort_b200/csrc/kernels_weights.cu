@@ -9,10 +9,10 @@
 //
 // FP8 ("tensor-quantized", toolboxkart.tech, "AWS SageMaker MoE kernel
 // optimizations H200", section "2. FP8 backend routing changes which kernel path
-// runs"): one scale per expert tensor s = amax/448 (1 for an all-zero tensor),
-// codes = RNE(w / s) saturated to +-448, the division in IEEE fp32.
-#include <cuda_fp8.h>
-
+// runs"): one scale per expert tensor s = amax / (the format's largest finite value,
+// 448 for E4M3, 57344 for E5M2; 1 for an all-zero tensor), codes = RNE(w / s)
+// saturated, the division in IEEE fp32 (fp8_format.cuh).
+#include "fp8_format.cuh"
 #include "moe_internal.h"
 
 namespace moe {
@@ -25,7 +25,7 @@ __device__ __forceinline__ long long tiled_offset(const TileGeom& g, long long e
   return (tile * 128 + (r & 127)) * 128 + (byte & 127);
 }
 
-__global__ void __launch_bounds__(1024) weight_amax_kernel(const __nv_bfloat16* w, long long per_expert,
+__global__ void __launch_bounds__(1024) weight_amax_kernel(int f8, const __nv_bfloat16* w, long long per_expert,
                                                            float* scales, int stride) {
   const int e = blockIdx.x;
   const uint4* src = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * per_expert);
@@ -48,14 +48,14 @@ __global__ void __launch_bounds__(1024) weight_amax_kernel(const __nv_bfloat16* 
     m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (threadIdx.x == 0) scales[static_cast<size_t>(e) * stride] = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
+    if (threadIdx.x == 0) scales[static_cast<size_t>(e) * stride] = fp8_scale_from_amax(__float_as_uint(m), f8);
   }
 }
 
-// 8 bf16 -> 8 e4m3 codes (8 bytes) per thread, written at their tiled position.
-__global__ void __launch_bounds__(256) weight_quant_tiled_kernel(const __nv_bfloat16* w, TileGeom g,
+// 8 bf16 -> 8 FP8 codes (8 bytes) per thread, written at their tiled position.
+__global__ void __launch_bounds__(256) weight_quant_tiled_kernel(int f8, const __nv_bfloat16* w, TileGeom g,
                                                                  const float* scales, int stride, uint8_t* dst) {
-  const long long K = g.row_bytes;                 // e4m3: one byte per element
+  const long long K = g.row_bytes;                 // FP8: one byte per element
   const long long per_row = K / 8;
   const long long total = static_cast<long long>(g.E) * g.rows * per_row;
   for (long long i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256) weight_quant_tiled_kernel(const __nv_bflo
     for (int q = 0; q < 4; ++q) {
       const float2 f = __bfloat1622float2(p[q]);
       const float2 d = make_float2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s));
-      c2[q] = static_cast<unsigned short>(__nv_cvt_float2_to_fp8x2(d, __NV_SATFINITE, __NV_E4M3));
+      c2[q] = fp8x2(d, f8);
     }
     uint2 o;
     o.x = static_cast<unsigned>(c2[0]) | (static_cast<unsigned>(c2[1]) << 16);
@@ -104,15 +104,15 @@ int grid_for(long long work) {
 
 }  // namespace
 
-cudaError_t launch_weight_amax(const __nv_bfloat16* w, long long per_expert, int E, float* scales,
+cudaError_t launch_weight_amax(int f8, const __nv_bfloat16* w, long long per_expert, int E, float* scales,
                                int stride, cudaStream_t s) {
-  weight_amax_kernel<<<E, 1024, 0, s>>>(w, per_expert, scales, stride);
+  weight_amax_kernel<<<E, 1024, 0, s>>>(f8, w, per_expert, scales, stride);
   return cudaGetLastError();
 }
 
-cudaError_t launch_weight_quant_tiled(const __nv_bfloat16* w, const TileGeom& g, const float* scales, int stride,
-                                      uint8_t* dst, cudaStream_t s) {
-  weight_quant_tiled_kernel<<<grid_for(g.E * g.rows * (g.row_bytes / 8)), 256, 0, s>>>(w, g, scales, stride, dst);
+cudaError_t launch_weight_quant_tiled(int f8, const __nv_bfloat16* w, const TileGeom& g, const float* scales,
+                                      int stride, uint8_t* dst, cudaStream_t s) {
+  weight_quant_tiled_kernel<<<grid_for(g.E * g.rows * (g.row_bytes / 8)), 256, 0, s>>>(f8, w, g, scales, stride, dst);
   return cudaGetLastError();
 }
 

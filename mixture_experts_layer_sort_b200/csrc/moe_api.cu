@@ -172,7 +172,9 @@ int ws_alloc(moe_layer* L, T** p, size_t bytes, bool zero) {
   return MOE_OK;
 }
 
-bool is_fp8(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E4M3; }
+bool is_fp8(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E4M3 || L->dtype == MOE_DTYPE_FP8_E5M2; }
+// FP8 code format of an FP8 layer (moe::Fp8Format values)
+int fp8_format(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E5M2 ? 1 : 0; }
 
 int choose_variant(long long P) {
   if (P <= 128) return moe::kVariantSmall;
@@ -456,6 +458,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   ga.H = L->H;
   ga.x_perm = L->x_perm;
   ga.amax_x = L->amax;
+  ga.f8 = fp8_format(L);
   if (!direct) {
     KernelTimer kt(L, 2, st);
     MOE_CUDA(moe::launch_gather(ga, fp8, st));
@@ -477,6 +480,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g.topk_w = L->topk_w;
   g.k = L->k;
   g.P = static_cast<int>(P);
+  g.f8 = fp8_format(L);
   g.err = L->err;
 
   moe::GemmArgs g1 = g;
@@ -506,6 +510,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
     qa.P = static_cast<int>(P);
     qa.I = L->I;
     qa.amax_h = L->amax + 1;
+    qa.f8 = fp8_format(L);
     {
       KernelTimer kt(L, 4, st);
       MOE_CUDA(moe::launch_quant_h(qa, st));
@@ -534,6 +539,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   fa.n = static_cast<long long>(M) * L->H;
   fa.amax = fp8 ? L->amax : nullptr;
   fa.last_scales = fp8 ? L->last_scales : nullptr;
+  fa.f8 = fp8_format(L);
   {
     KernelTimer kt(L, 6, st);
     MOE_CUDA(moe::launch_finalize(fa, st));
@@ -585,6 +591,7 @@ int moe_layer_view(const moe_layer* L, moe::LayerView* v) {
   v->device = L->device;
   v->num_sms = L->num_sms;
   v->fp8 = is_fp8(L);
+  v->f8 = fp8_format(L);
   v->loaded = L->loaded;
   v->wscales = L->wscales;
   v->tm_w13 = L->tm_w13;
@@ -617,7 +624,8 @@ int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
   *out = nullptr;
   if (E < 1 || E > 512 || topk < 1 || topk > 16 || topk > E) return MOE_ERR_INVALID_ARG;
   if (H < 128 || I < 128 || H > 16384 || I > 16384 || H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
-  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_FP8_E4M3 && dtype != MOE_DTYPE_FP8_E5M2)
+    return MOE_ERR_INVALID_ARG;
   int dev = 0;
   MOE_CUDA(cudaGetDevice(&dev));
   cudaDeviceProp prop;
@@ -634,7 +642,7 @@ int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
   L->dtype = dtype;
   L->device = dev;
   L->num_sms = prop.multiProcessorCount;
-  const size_t el = dtype == MOE_DTYPE_FP8_E4M3 ? 1 : 2;
+  const size_t el = dtype == MOE_DTYPE_BF16 ? 2 : 1;
   if (cudaMalloc(&L->w13, static_cast<size_t>(E) * 2 * I * H * el) != cudaSuccess ||
       cudaMalloc(&L->wd, static_cast<size_t>(E) * H * I * el) != cudaSuccess ||
       cudaMalloc(&L->wscales, static_cast<size_t>(E) * 3 * sizeof(float)) != cudaSuccess) {
@@ -684,8 +692,8 @@ int moe_load_weights(moe_layer* L, const void* w_gate, const void* w_up, const v
   } else {
     for (int j = 0; j < 3; ++j) {
       const auto* w = static_cast<const __nv_bfloat16*>(src[j]);
-      MOE_CUDA(moe::launch_weight_amax(w, static_cast<long long>(IH), L->E, L->wscales + j, 3, st));
-      MOE_CUDA(moe::launch_weight_quant_tiled(w, geom(L, j), L->wscales + j, 3, static_cast<uint8_t*>(dst[j]), st));
+      MOE_CUDA(moe::launch_weight_amax(fp8_format(L), w, static_cast<long long>(IH), L->E, L->wscales + j, 3, st));
+      MOE_CUDA(moe::launch_weight_quant_tiled(fp8_format(L), w, geom(L, j), L->wscales + j, 3, static_cast<uint8_t*>(dst[j]), st));
     }
   }
   MOE_CUDA(cudaStreamSynchronize(st));

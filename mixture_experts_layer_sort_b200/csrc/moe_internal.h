@@ -68,8 +68,9 @@ struct GatherArgs {
   const int* header;
   int rows_bound;          // grid covers this many rows; rows >= rows_used exit
   int P, k, H;
-  void* x_perm;            // [rows_cap, H] bf16 or e4m3
+  void* x_perm;            // [rows_cap, H] bf16 or FP8 codes
   const unsigned* amax_x;  // FP8 only
+  int f8;                  // FP8 code format (Fp8Format)
 };
 
 struct GemmArgs {
@@ -97,6 +98,7 @@ struct GemmArgs {
   int max_stages;          // upper bound of the stage ring depth (<= the kernel's own maximum)
   int wait_first;          // 1: the previous kernel wrote the tile list (wait before reading it)
   const int* direct_pairs; // gate_up only: B rows are x rows of token pairs[row]/k (x map box = 1 row)
+  int f8;                  // FP8 layers: code format of weights and activations (Fp8Format)
   int* err;
 };
 
@@ -107,6 +109,7 @@ struct QuantHArgs {
   const int* header;
   int rows_bound, P, I;
   const unsigned* amax_h;
+  int f8;                  // FP8 code format (Fp8Format)
 };
 
 struct FinalizeArgs {
@@ -115,6 +118,7 @@ struct FinalizeArgs {
   long long n;             // M*H
   unsigned* amax;          // [2] reset to 0 (may be nullptr)
   float* last_scales;      // [2] s_x, s_h of this forward (may be nullptr)
+  int f8;                  // FP8 code format (Fp8Format)
 };
 
 // Launch with programmatic stream serialisation (PDL) unless MOE_DISABLE_PDL=1 is set
@@ -194,10 +198,10 @@ struct TileGeom {
   int rb_total;         // row blocks per expert in the destination (2I/128 or H/128)
   int rb_offset;        // first destination row block of this source (I/128 for up)
 };
-cudaError_t launch_weight_amax(const __nv_bfloat16* w, long long per_expert, int E,
+cudaError_t launch_weight_amax(int f8, const __nv_bfloat16* w, long long per_expert, int E,
                                float* scales, int stride, cudaStream_t s);
 // bf16 source [E, rows, K] -> e4m3 codes in the tiled layout, per-expert scale scales[e*stride].
-cudaError_t launch_weight_quant_tiled(const __nv_bfloat16* w, const TileGeom& g, const float* scales,
+cudaError_t launch_weight_quant_tiled(int f8, const __nv_bfloat16* w, const TileGeom& g, const float* scales,
                                       int stride, uint8_t* dst, cudaStream_t s);
 // row-major [E, rows, row_bytes] bytes -> tiled layout, and back.
 cudaError_t launch_tile_weights(const void* src, const TileGeom& g, void* dst, cudaStream_t s);
@@ -208,6 +212,7 @@ cudaError_t launch_untile_weights(const void* src, const TileGeom& g, void* dst,
 struct LayerView {
   int E, k, H, I, device, num_sms;
   bool fp8, loaded;
+  int f8;                  // FP8 code format (Fp8Format) when fp8
   const float* wscales;
   CUtensorMap tm_w13, tm_wd;
 };

@@ -176,6 +176,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   ga.H = v.H;
   ga.x_perm = x_perm;
   ga.amax_x = amax;
+  ga.f8 = v.f8;
   NA_CUDA(moe::launch_gather(ga, v.fp8, st));
 
   moe::GemmArgs g{};
@@ -193,6 +194,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g.topk_w = topk_w;
   g.k = v.k;
   g.P = static_cast<int>(P);
+  g.f8 = v.f8;
   g.err = nullptr;
 
   moe::GemmArgs g1 = g;
@@ -216,6 +218,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
     qa.P = static_cast<int>(P);
     qa.I = v.I;
     qa.amax_h = amax + 1;
+    qa.f8 = v.f8;
     NA_CUDA(moe::launch_quant_h(qa, st));
   }
 
@@ -236,6 +239,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   fa.n = static_cast<long long>(M) * v.H;
   fa.amax = nullptr;
   fa.last_scales = nullptr;
+  fa.f8 = v.f8;
   NA_CUDA(moe::launch_finalize(fa, st));
   return MOE_OK;
 }

@@ -149,7 +149,8 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
 }
 
 // Instruction descriptor: fp32 accumulator, A/B format codes (bf16 = 1 under
-// kind::f16; e4m3 = 0 under kind::f8f6f4), both operands K-major, shape M x N.
+// kind::f16; e4m3 = 0, e5m2 = 1 under kind::f8f6f4; A and B always take the same
+// format here), both operands K-major, shape M x N.
 __device__ __forceinline__ uint32_t idesc_make(uint32_t ab_format, uint32_t M, uint32_t N) {
   return (1u << 4) | (ab_format << 7) | (ab_format << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
@@ -164,7 +165,7 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
-__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"

@@ -12,8 +12,9 @@ import torch
 
 from ._lib import load_library, status_string
 
-BF16, FP8 = 0, 1
-_DTYPES = {"bf16": BF16, "fp8": FP8, "e4m3": FP8, BF16: BF16, FP8: FP8}
+BF16, FP8, FP8_E5M2 = 0, 1, 2
+_DTYPES = {"bf16": BF16, "fp8": FP8, "e4m3": FP8, "fp8_e5m2": FP8_E5M2, "e5m2": FP8_E5M2,
+           BF16: BF16, FP8: FP8, FP8_E5M2: FP8_E5M2}
 
 
 class MoEError(RuntimeError):
@@ -55,7 +56,7 @@ class MoELayer:
 
     @property
     def is_fp8(self) -> bool:
-        return self.dtype == FP8
+        return self.dtype in (FP8, FP8_E5M2)
 
     def close(self):
         if getattr(self, "handle", None):

@@ -45,6 +45,9 @@ WORKLOADS = {
     "decode_fp8": Workload("decode_fp8", E=128, k=8, H=2048, I=768, Ms=(1, 8, 32, 64), w_std=0.02,
                            dtypes=("fp8",),
                            description="decode e4m3, E=128 top-8, H=2048, I=768, per-tensor scales"),
+    "decode_e5m2": Workload("decode_e5m2", E=128, k=8, H=2048, I=768, Ms=(1, 8, 32, 64), w_std=0.02,
+                            dtypes=("fp8_e5m2",),
+                            description="decode e5m2, E=128 top-8, H=2048, I=768, per-tensor scales"),
     "large_decode": Workload("large_decode", E=256, k=8, H=7168, I=2048, Ms=(1, 32, 64, 128),
                              w_std=0.01, zipf_s=1.1,
                              description="large decode bf16, E=256 top-8, H=7168, I=2048, "
