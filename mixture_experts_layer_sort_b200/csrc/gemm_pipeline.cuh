@@ -313,13 +313,6 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
     const int wtile2 = (un.t.expert * a.w_rblocks + rb0 + a.second_rb) * a.kblocks;
     const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
     const int dep = hk.dep(un);
-    if (a.direct_pairs != nullptr) {
-      #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int j = lane + 32 * i;
-        tok[i] = j < un.t.n_valid ? __ldcg(a.direct_pairs + un.t.row_start + j) / a.k : 0;
-      }
-    }
     for (int kb = un.kb0; kb < un.kb1; ++kb) {
       int ok = 1;
       if (lane == 0) {
@@ -338,6 +331,14 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
       if (!ok) {
         ps.failed = true;
         break;
+      }
+      if (a.direct_pairs != nullptr && kb == un.kb0) {
+        // the unit's token rows, read while its first weight tiles are in flight
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = lane + 32 * i;
+          tok[i] = j < un.t.n_valid ? __ldcg(a.direct_pairs + un.t.row_start + j) / a.k : 0;
+        }
       }
       const int kc = kb * C::kKPerBlock;
       if (npend > 0 && !drain(false)) ps.failed = true;

@@ -59,12 +59,22 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   pdl_wait();
   pdl_trigger();
   __syncthreads();
-  for (int p = tid; p < a.P; p += kAlignThreads) {
-    const int e = a.topk_ids[p];
-    atomicAdd(&s_count[e], 1);
-    if (small) {
-      const int t = p / a.k;
-      atomicOr(&s_mask[2 * e + (t >> 5)], 1u << (t & 31));
+  const bool chunked = a.chunk_counts != nullptr;
+  if (chunked) {
+    // counts are the sums of the chunks' counts (written by align_count_kernel)
+    for (int e = tid; e < E; e += kAlignThreads) {
+      int n = 0;
+      for (int c = 0; c < a.chunks; ++c) n += a.chunk_counts[static_cast<size_t>(c) * E + e];
+      s_count[e] = n;
+    }
+  } else {
+    for (int p = tid; p < a.P; p += kAlignThreads) {
+      const int e = a.topk_ids[p];
+      atomicAdd(&s_count[e], 1);
+      if (small) {
+        const int t = p / a.k;
+        atomicOr(&s_mask[2 * e + (t >> 5)], 1u << (t & 31));
+      }
     }
   }
   __syncthreads();
@@ -87,10 +97,21 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
       a.padded_pairs[s_poff[e] + __popc(lo) + __popc(hi)] = p;
     }
   }
+  if (chunked) {
+    // the first padded row of every (chunk, expert) group, for align_scatter_kernel
+    for (int e = tid; e < E; e += kAlignThreads) {
+      int run = s_poff[e];
+      for (int c = 0; c < a.chunks; ++c) {
+        const size_t i = static_cast<size_t>(c) * E + e;
+        a.chunk_base[i] = run;
+        run += a.chunk_counts[i];
+      }
+    }
+  }
   // Otherwise a stable scatter, 1024 pairs per chunk: rank inside the warp from the
   // match mask, plus the counts of earlier warps in this chunk, plus earlier chunks.
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int c0 = 0; !small && c0 < a.P; c0 += kAlignThreads) {
+  for (int c0 = 0; !small && !chunked && c0 < a.P; c0 += kAlignThreads) {
     for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) s_wc[i] = 0;
     __syncthreads();
     const int p = c0 + tid;
@@ -201,13 +222,63 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   }
 }
 
+// Multi-block path, step 1: per-expert pair counts of chunk blockIdx.x.
+__global__ void __launch_bounds__(kAlignChunk) align_count_kernel(AlignArgs a) {
+  extern __shared__ int hist[];   // [E]
+  for (int e = threadIdx.x; e < a.E; e += kAlignChunk) hist[e] = 0;
+  pdl_wait();
+  pdl_trigger();
+  __syncthreads();
+  const int p = blockIdx.x * kAlignChunk + threadIdx.x;
+  if (p < a.P) atomicAdd(&hist[a.topk_ids[p]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += kAlignChunk)
+    a.chunk_counts[static_cast<size_t>(blockIdx.x) * a.E + e] = hist[e];
+}
+
+// Multi-block path, step 3: place the pairs of chunk blockIdx.x. Row of pair p =
+// chunk_base[chunk][e] + (pairs of e earlier in the chunk): earlier warps' counts
+// plus the rank inside the warp from the match mask, so the order inside an expert
+// stays ascending in p.
+__global__ void __launch_bounds__(kAlignChunk) align_scatter_kernel(AlignArgs a) {
+  extern __shared__ int wc[];     // [32][E] pairs of e in each warp of the chunk
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 32 * a.E; i += kAlignChunk) wc[i] = 0;
+  pdl_wait();
+  pdl_trigger();
+  __syncthreads();
+  const int p = blockIdx.x * kAlignChunk + threadIdx.x;
+  const bool valid = p < a.P;
+  const int e = valid ? a.topk_ids[p] : 0x7FFFFFFF;
+  const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank == 0) wc[warp * a.E + e] = __popc(peers);
+  __syncthreads();
+  if (valid) {
+    int pos = a.chunk_base[static_cast<size_t>(blockIdx.x) * a.E + e] + rank;
+    for (int w = 0; w < warp; ++w) pos += wc[w * a.E + e];
+    a.padded_pairs[pos] = p;
+  }
+}
+
 }  // namespace
 
 size_t align_smem_bytes(int E) { return static_cast<size_t>(6 * E + 2 + kAlignWarps * E) * sizeof(int); }
 
 cudaError_t align_configure() {
-  return cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(align_smem_bytes(512)));
+  cudaError_t e = cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(align_smem_bytes(512)));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(align_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
+}
+
+cudaError_t launch_align_count(const AlignArgs& a, cudaStream_t s) {
+  return launch_kernel(align_count_kernel, dim3(a.chunks), dim3(kAlignChunk), static_cast<size_t>(a.E) * 4, s, a);
+}
+
+cudaError_t launch_align_scatter(const AlignArgs& a, cudaStream_t s) {
+  return launch_kernel(align_scatter_kernel, dim3(a.chunks), dim3(kAlignChunk), static_cast<size_t>(32) * a.E * 4,
+                       s, a);
 }
 
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t s) {

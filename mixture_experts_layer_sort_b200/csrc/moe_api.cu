@@ -56,6 +56,8 @@ struct moe_layer {
   float* last_scales = nullptr; // [2]
   int* err = nullptr;
   int* sync = nullptr;          // single-launch decode: counters between its CTAs
+  int* chunk_buf = nullptr;     // multi-block align: [2][chunks_cap][E] chunk counts and bases
+  long long chunks_cap = 0;
   CUtensorMap tm_x{}, tm_h{};
   // staging for moe_forward_host
   void* hx = nullptr;
@@ -216,6 +218,8 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(ws_alloc(L, &L->last_scales, 2 * 4, false));
   MOE_TRY(ws_alloc(L, &L->err, 4, true));
   MOE_TRY(ws_alloc(L, &L->sync, moe::decode_sync_words(L->E, cap) * 4, true));
+  L->chunks_cap = (P + moe::kAlignChunk - 1) / moe::kAlignChunk;
+  MOE_TRY(ws_alloc(L, &L->chunk_buf, 2 * L->chunks_cap * L->E * 4, false));
   const float ones[2] = {1.f, 1.f};
   MOE_CUDA(cudaMemcpy(L->last_scales, ones, sizeof(ones), cudaMemcpyHostToDevice));
   MOE_TRY(encode_map(&L->tm_x, L->x_perm, is_fp8(L), L->H, L->rows_cap, 16));
@@ -387,6 +391,10 @@ int acc_slabs(int M, int H, int fblocks2) {
   return static_cast<int>(std::max(1ll, std::min<long long>(s, fblocks2)));
 }
 
+// Up to this many (token, slot) pairs one align block places the pairs itself (one
+// chunk of 1024 pairs after another); beyond, chunks go to blocks of their own.
+constexpr long long kAlignSingleBlockMaxPairs = 8192;
+
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
   if (L->fused_decode && !is_fp8(L) && moe::decode_supported(M, L->E, L->k))
@@ -435,11 +443,27 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   aa.tiles1 = L->tiles1;
   aa.tiles2 = L->tiles2;
   aa.header = L->header;
+  // Large batches take the multi-block path: per-chunk counts, the plan (the align
+  // block itself), then the placement of each chunk's pairs by its own block.
+  const bool chunked = P > kAlignSingleBlockMaxPairs;
+  if (chunked) {
+    aa.chunks = static_cast<int>((P + moe::kAlignChunk - 1) / moe::kAlignChunk);
+    aa.chunk_counts = L->chunk_buf;
+    aa.chunk_base = L->chunk_buf + L->chunks_cap * L->E;
+    KernelTimer kt(L, 1, st);
+    MOE_CUDA(moe::launch_align_count(aa, st));
+    ++launches;
+  }
   {
     KernelTimer kt(L, 1, st);
     MOE_CUDA(moe::launch_align(aa, st));
   }
   ++launches;
+  if (chunked) {
+    KernelTimer kt(L, 1, st);
+    MOE_CUDA(moe::launch_align_scatter(aa, st));
+    ++launches;
+  }
 
   // The smallest bf16 batches (P <= 16) skip the gather: gate_up reads each token's x row
   // itself with 1-row TMA boxes. Measured: faster at M=1, slower from M=4 on (16-row

@@ -60,6 +60,14 @@ struct AlignArgs {
   Tile* tiles1;
   Tile* tiles2;
   int* header;             // [kHdrSlots]
+  // Multi-block path (large batches), when chunk_counts is set: pairs are taken in
+  // chunks of kAlignChunk; align_count_kernel writes each chunk's per-expert counts,
+  // align_kernel then sums them and writes chunk_base (the first padded row of each
+  // (chunk, expert) group) instead of placing the pairs itself, and
+  // align_scatter_kernel places them.
+  int* chunk_counts;       // [chunks, E]
+  int* chunk_base;         // [chunks, E]
+  int chunks;
 };
 
 struct GatherArgs {
@@ -151,6 +159,9 @@ int variant_bn(int v);
 // Kernel launchers (each returns the cudaError_t of its launch).
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t s);
+constexpr int kAlignChunk = 1024;   // pairs per block of the multi-block align path
+cudaError_t launch_align_count(const AlignArgs& a, cudaStream_t s);
+cudaError_t launch_align_scatter(const AlignArgs& a, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s);
 cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8,
                          int variant, int grid, cudaStream_t s);

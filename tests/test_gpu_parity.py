@@ -165,3 +165,18 @@ def test_size_limits(E, k, H, I, dtype, Ms):
         assert c.layer.device_error() == 0
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("E,k,M", [(8, 2, 5000), (64, 8, 1100), (200, 6, 2000)])
+def test_multi_block_align(E, k, M):
+    # more than 8192 pairs: per-chunk counts, the plan block and the per-chunk
+    # placement; the padded permutation must still be the stable one, bit for bit
+    c = Case(E, k, 256, 256, "bf16", w_std=0.02)
+    try:
+        x, logits = tokens(c.E, c.H, M, seed=E + M)
+        out = c.run(x, logits)
+        check_routing(c, logits, M)
+        ref, _ = oracle_full(c, x, logits, fp8=False)
+        check_output(out, ref, "bf16")
+    finally:
+        c.close()
