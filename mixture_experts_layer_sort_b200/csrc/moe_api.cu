@@ -57,6 +57,7 @@ struct moe_layer {
   int* err = nullptr;
   int* sync = nullptr;          // single-launch decode: counters between its CTAs
   int* chunk_buf = nullptr;     // multi-block align: [2][chunks_cap][E] chunk counts and bases
+  uint8_t* xq = nullptr;        // FP8 large batches: x quantised per token [M_cap, H]
   long long chunks_cap = 0;
   CUtensorMap tm_x{}, tm_h{};
   // staging for moe_forward_host
@@ -218,6 +219,7 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(ws_alloc(L, &L->last_scales, 2 * 4, false));
   MOE_TRY(ws_alloc(L, &L->err, 4, true));
   MOE_TRY(ws_alloc(L, &L->sync, moe::decode_sync_words(L->E, cap) * 4, true));
+  if (is_fp8(L)) MOE_TRY(ws_alloc(L, &L->xq, static_cast<size_t>(cap) * L->H, false));
   L->chunks_cap = (P + moe::kAlignChunk - 1) / moe::kAlignChunk;
   MOE_TRY(ws_alloc(L, &L->chunk_buf, 2 * L->chunks_cap * L->E * 4, false));
   const float ones[2] = {1.f, 1.f};
@@ -444,8 +446,21 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   aa.tiles2 = L->tiles2;
   aa.header = L->header;
   // Large batches take the multi-block path: per-chunk counts, the plan (the align
-  // block itself), then the placement of each chunk's pairs by its own block.
+  // block itself), then the placement of each chunk's pairs by its own block. FP8
+  // large batches also quantise x once per token here, so that the gather copies bytes.
   const bool chunked = P > kAlignSingleBlockMaxPairs;
+  if (chunked && fp8) {
+    moe::QuantXArgs qx{};
+    qx.x = static_cast<const __nv_bfloat16*>(x);
+    qx.xq = L->xq;
+    qx.M = M;
+    qx.H = L->H;
+    qx.amax_x = L->amax;
+    qx.f8 = fp8_format(L);
+    KernelTimer kt(L, 2, st);
+    MOE_CUDA(moe::launch_quant_x(qx, st));
+    ++launches;
+  }
   if (chunked) {
     aa.chunks = static_cast<int>((P + moe::kAlignChunk - 1) / moe::kAlignChunk);
     aa.chunk_counts = L->chunk_buf;
@@ -483,6 +498,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   ga.x_perm = L->x_perm;
   ga.amax_x = L->amax;
   ga.f8 = fp8_format(L);
+  ga.xq = (chunked && fp8) ? L->xq : nullptr;
   if (!direct) {
     KernelTimer kt(L, 2, st);
     MOE_CUDA(moe::launch_gather(ga, fp8, st));

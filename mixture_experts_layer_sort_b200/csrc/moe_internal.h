@@ -79,6 +79,15 @@ struct GatherArgs {
   void* x_perm;            // [rows_cap, H] bf16 or FP8 codes
   const unsigned* amax_x;  // FP8 only
   int f8;                  // FP8 code format (Fp8Format)
+  const uint8_t* xq;       // FP8: token rows already quantised [M, H] (copy bytes), or nullptr
+};
+
+struct QuantXArgs {
+  const __nv_bfloat16* x;  // [M, H]
+  uint8_t* xq;             // [M, H] FP8 codes
+  int M, H;
+  const unsigned* amax_x;
+  int f8;
 };
 
 struct GemmArgs {
@@ -168,6 +177,7 @@ cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensor
 cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8,
                          int variant, int grid, cudaStream_t s);
 cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s);
+cudaError_t launch_quant_x(const QuantXArgs& a, cudaStream_t s);
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
 cudaError_t gemm_configure();    // opt-in dynamic shared memory sizes (current device)
 cudaError_t align_configure();

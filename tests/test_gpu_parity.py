@@ -180,3 +180,25 @@ def test_multi_block_align(E, k, M):
         check_output(out, ref, "bf16")
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "fp8_e5m2"])
+def test_fp8_multi_block_x_codes(dtype):
+    # more than 8192 pairs: x is quantised once per token and the gather copies the
+    # codes; every valid row of x_perm must still hold the oracle's codes bit for bit
+    fmt = "e5m2" if dtype == "fp8_e5m2" else "e4m3"
+    c = Case(8, 2, 256, 512, dtype, w_std=0.02)
+    try:
+        M = 5000
+        x, logits = tokens(c.E, c.H, M, seed=77)
+        out = c.run(x, logits)
+        dbg, padded = check_routing(c, logits, M)
+        ref, inter = O.moe_forward(x.float().cpu().numpy(), logits.cpu().numpy(), c.k, provider=c.provider,
+                                   fp8=True, fp8_format=fmt, return_intermediates=True)
+        assert np.float32(dbg["s_x"]) == inter["s_x"], "s_x differs"
+        xp, _ = c.layer.debug_activations(len(padded))
+        valid = padded < M * c.k
+        assert np.array_equal(xp.cpu().numpy()[valid], inter["x_codes"][padded[valid] // c.k]), "x codes differ"
+        check_output(out, ref, "fp8")
+    finally:
+        c.close()
