@@ -39,6 +39,7 @@ namespace pipe {
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kTokenTile = 256;   // widest token tile: the largest N of an M=128 MMA
+static_assert(kTokenTile == kTokenBlock, "the align kernel's token blocks are the GEMM token tiles");
 
 template <bool kFP8>
 struct Cfg {

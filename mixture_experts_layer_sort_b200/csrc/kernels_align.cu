@@ -1,6 +1,8 @@
 // kernels_align.cu - moe_align: group the (token, slot) pairs by expert, pad each
-// group to 16 rows, and build the tile lists and split-K factors of both grouped
-// GEMMs, all in one thread block.
+// group to 16 rows, and build the tile lists and split factors of both grouped
+// GEMMs. Up to 8192 pairs one thread block does everything; larger batches count
+// per chunk of 1024 pairs in blocks of their own, plan in the one block, and place
+// each chunk's pairs in its own block again.
 //
 // "Routing tokens to experts, moving data and combining expert outputs can add
 // work around the matrix multiplications" (toolboxkart.tech, "AWS SageMaker MoE

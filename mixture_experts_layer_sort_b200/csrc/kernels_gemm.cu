@@ -105,11 +105,6 @@ cudaError_t configure_one() {
 
 }  // namespace
 
-int variant_bn(int v) {
-  (void)v;
-  return kTokenTile;
-}
-
 cudaError_t gemm_configure() {
   cudaError_t e;
   if ((e = configure_one<true, false>()) != cudaSuccess) return e;
@@ -118,15 +113,13 @@ cudaError_t gemm_configure() {
   return configure_one<false, true>();
 }
 
-cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8, int variant,
-                         int grid, cudaStream_t s) {
-  (void)variant;
+cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8, int grid,
+                         cudaStream_t s) {
   return fp8 ? launch_one<true, true>(a, w, x, grid, s) : launch_one<true, false>(a, w, x, grid, s);
 }
 
-cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int variant,
-                         int grid, cudaStream_t s) {
-  (void)variant;
+cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int grid,
+                         cudaStream_t s) {
   return fp8 ? launch_one<false, true>(a, w, h, grid, s) : launch_one<false, false>(a, w, h, grid, s);
 }
 

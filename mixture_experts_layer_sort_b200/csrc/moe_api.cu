@@ -1,10 +1,11 @@
 // moe_api.cu - the C ABI (include/moe_b200.h) and the host dispatcher: argument
-// checks, weight storage, workspace sizing, TMA descriptor encoding, the variant
-// table and the launch chain of one forward pass.
+// checks, weight storage, workspace sizing, TMA descriptor encoding and the launch
+// chain of one forward pass.
 //
 // The forward pass is a fixed chain of precompiled kernels; the token count M is
-// a runtime argument of each, and the variant (tile width BN) comes from a fixed
-// table keyed by M*k. Nothing is compiled, specialised or re-encoded per M (the
+// a runtime argument of each, and the tile list, split factors and stage-ring depth
+// are computed on the device from the routing. Nothing is compiled, specialised or
+// re-encoded per M (the
 // pages' third change removes exactly such per-token-count recompiles:
 // toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "3.
 // Removing repeat compilation can reduce first-token delay"). Tensor maps are
@@ -66,7 +67,7 @@ struct moe_layer {
   void* hout = nullptr;
   int host_cap = 0;
   // bookkeeping
-  int last_M = 0, last_launches = 0, last_variant = 0;
+  int last_M = 0, last_launches = 0;
   bool fused_decode = false;    // single-launch decode path for small bf16 batches
   // per-kernel event timing
   bool profiling = false;
@@ -179,12 +180,6 @@ bool is_fp8(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E4M3 || L->dt
 // FP8 code format of an FP8 layer (moe::Fp8Format values)
 int fp8_format(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E5M2 ? 1 : 0; }
 
-int choose_variant(long long P) {
-  if (P <= 128) return moe::kVariantSmall;
-  if (P <= 4096) return moe::kVariantMedium;
-  return moe::kVariantLarge;
-}
-
 int ensure_workspace(moe_layer* L, int M) {
   if (M <= L->M_cap) return MOE_OK;
   int cap = 64;
@@ -195,7 +190,7 @@ int ensure_workspace(moe_layer* L, int M) {
   const long long Emin = std::min<long long>(L->E, P);
   L->P_cap = P;
   L->rows_cap = P + Emin * (moe::kPadRows - 1);
-  L->nblocks_cap = (P + moe::variant_bn(moe::kVariantSmall) - 1) / moe::variant_bn(moe::kVariantSmall) + Emin;
+  L->nblocks_cap = (P + moe::kTokenBlock - 1) / moe::kTokenBlock + Emin;
   L->t1_cap = L->nblocks_cap * (L->I / moe::kTileRows);
   L->t2_cap = L->nblocks_cap * (L->H / moe::kTileRows);
   const long long ws1_limit = (128ll << 20) / (8ll * L->I);
@@ -374,7 +369,6 @@ int forward_fused_decode(moe_layer* L, const void* x, const float* logits, int M
   }
   L->last_M = M;
   L->last_launches = 1;
-  L->last_variant = -1;
   return MOE_OK;
 }
 
@@ -403,8 +397,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
     return forward_fused_decode(L, x, logits, M, out, st);
   const bool fp8 = is_fp8(L);
   const long long P = static_cast<long long>(M) * L->k;
-  const int variant = choose_variant(P);
-  const int BN = moe::variant_bn(variant);
+  const int BN = moe::kTokenBlock;
   const int rows_bound = static_cast<int>(P + std::min<long long>(L->E, P) * (moe::kPadRows - 1));
   int launches = 0;
 
@@ -536,7 +529,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g1.direct_pairs = direct ? L->pairs : nullptr;
   {
     KernelTimer kt(L, 3, st);
-    MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, direct ? tm_xd : L->tm_x, fp8, variant, L->num_sms, st));
+    MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, direct ? tm_xd : L->tm_x, fp8, L->num_sms, st));
   }
   ++launches;
 
@@ -569,7 +562,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g2.max_stages = moe::gemm_max_stages(false);
   {
     KernelTimer kt(L, 5, st);
-    MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, variant, L->num_sms, st));
+    MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, L->num_sms, st));
   }
   ++launches;
 
@@ -588,7 +581,6 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
 
   L->last_M = M;
   L->last_launches = launches;
-  L->last_variant = variant;
   return MOE_OK;
 }
 

@@ -17,9 +17,9 @@ constexpr int kMaxSplits = 16;      // largest split-K factor the scheduler pick
 enum HeaderSlot : int {
   kHdrRowsUsed = 0,     // padded rows in use (= padded_offsets[E])
   kHdrTiles1 = 1,       // gate_up tiles
-  kHdrSplits1 = 2,      // gate_up split-K factor
+  kHdrSplits1 = 2,      // gate_up split-K factor (0 = the balanced schedule)
   kHdrTiles2 = 3,       // down tiles
-  kHdrSplits2 = 4,      // down split-K factor
+  kHdrSplits2 = 4,      // down split-K factor (0 = the balanced schedule)
   kHdrTokenBlocks = 5,  // (expert, token block) pairs
   kHdrMaxRows = 6,      // widest token tile (rows of activations a stage must hold), <= BN
   kHdrSlots = 8
@@ -47,7 +47,7 @@ struct RouteArgs {
 struct AlignArgs {
   const int* topk_ids;     // [P]
   int P, E, k;
-  int BN;                  // token rows per tile (the variant's N)
+  int BN;                  // token rows per tile (kTokenBlock)
   int fblocks1, fblocks2;  // tiles across the output features: I/128 (gate_up), ceil(H/256) (down)
   int kblocks1, kblocks2;  // K blocks of gate_up (H) and down (I)
   int num_sms;
@@ -161,9 +161,9 @@ inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// Variant table: precompiled (BN, stages) choices; picked on the host by M*k.
-enum Variant : int { kVariantSmall = 0, kVariantMedium = 1, kVariantLarge = 2, kNumVariants = 3 };
-int variant_bn(int v);
+// Token rows per GEMM tile: the widest N of an M = 128 MMA. An expert with more
+// tokens gets several token blocks.
+constexpr int kTokenBlock = 256;
 
 // Kernel launchers (each returns the cudaError_t of its launch).
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
@@ -172,10 +172,10 @@ constexpr int kAlignChunk = 1024;   // pairs per block of the multi-block align 
 cudaError_t launch_align_count(const AlignArgs& a, cudaStream_t s);
 cudaError_t launch_align_scatter(const AlignArgs& a, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s);
-cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8,
-                         int variant, int grid, cudaStream_t s);
-cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8,
-                         int variant, int grid, cudaStream_t s);
+cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8, int grid,
+                         cudaStream_t s);
+cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int grid,
+                         cudaStream_t s);
 cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s);
 cudaError_t launch_quant_x(const QuantXArgs& a, cudaStream_t s);
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);

@@ -87,8 +87,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   NA_TRY(scratch_address(v.device, &base));
 
   const long long P = static_cast<long long>(M) * v.k;
-  const int variant = P <= 128 ? moe::kVariantSmall : P <= 4096 ? moe::kVariantMedium : moe::kVariantLarge;
-  const int BN = moe::variant_bn(variant);
+  const int BN = moe::kTokenBlock;
   const long long Emin = std::min<long long>(v.E, P);
   const long long rows_cap = P + Emin * (moe::kPadRows - 1);
   const long long nblocks = (P + BN - 1) / BN + Emin;
@@ -206,7 +205,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g1.rb_step = 1;
   g1.second_rb = v.I / moe::kTileRows;
   g1.max_stages = moe::gemm_max_stages(true);
-  NA_CUDA(moe::launch_gemm1(g1, v.tm_w13, tm_x, v.fp8, variant, v.num_sms, st));
+  NA_CUDA(moe::launch_gemm1(g1, v.tm_w13, tm_x, v.fp8, v.num_sms, st));
 
   if (v.fp8) {
     moe::QuantHArgs qa{};
@@ -231,7 +230,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g2.rb_step = 2;
   g2.second_rb = 1;
   g2.max_stages = moe::gemm_max_stages(false);
-  NA_CUDA(moe::launch_gemm2(g2, v.tm_wd, tm_h, v.fp8, variant, v.num_sms, st));
+  NA_CUDA(moe::launch_gemm2(g2, v.tm_wd, tm_h, v.fp8, v.num_sms, st));
 
   moe::FinalizeArgs fa{};
   fa.acc = acc;

@@ -1,7 +1,8 @@
 """GPU parity of the fused MoE layer against the CPU oracle, through the C ABI.
 
-Sizes span several tiles, ragged tails, split-K and every precompiled variant
-(small / medium / large tile width), in bf16 and FP8.
+Sizes span several tiles, ragged tails, split tiles, one and several 256-row token
+blocks per expert, the single-block and multi-block align paths, in bf16 and FP8,
+plus edge cases and the size limits.
 """
 
 import numpy as np
@@ -35,8 +36,8 @@ def oracle_full(case, x, logits, fp8):
 
 @pytest.mark.parametrize("M", [16, 1, 3, 37, 100, 300, 700])
 def test_tiny_bf16(tiny, M):
-    # M=16: the tiny workload; the others cross the small/medium/large variants,
-    # one and several token blocks per expert, split-K and ragged tails
+    # M=16: the tiny workload; the others cross one and several token blocks per
+    # expert, split tiles and ragged tails
     x, logits = tokens(tiny.E, tiny.H, M, seed=M)
     out = tiny.run(x, logits)
     check_routing(tiny, logits, M)
@@ -121,8 +122,8 @@ def test_repeated_calls_are_stable(tiny):
     assert tiny.layer.device_error() == 0
 
 
-def test_tiny_large_variant(tiny):
-    # M*k > 4096 selects the widest tile variant (256 token rows per tile)
+def test_tiny_many_token_blocks(tiny):
+    # ~625 tokens per expert: three 256-row token blocks per expert, one TMEM buffer
     M = 2500
     x, logits = tokens(tiny.E, tiny.H, M, seed=2500)
     out = tiny.run(x, logits)
