@@ -116,7 +116,10 @@ MOE_API int moe_forward(moe_layer* layer, const void* x, const float* router_log
 
 /* Host-buffer convenience: copies x_host [M,H] bf16 and logits_host [M,E] fp32 to
  * the device, runs moe_forward and copies out [M,H] bf16 back to out_host, all on
- * `stream`, and synchronises it. Pinned host memory gives asynchronous copies. */
+ * `stream`, and synchronises it. With pinned host buffers the copies and the
+ * forward are captured once per (M, buffer addresses) into a CUDA graph that later
+ * calls replay (captured again after new weights, a larger workspace or a switch of
+ * the decode path); pageable buffers are copied eagerly. */
 MOE_API int moe_forward_host(moe_layer* layer, const void* x_host, const float* logits_host,
                      int M, void* out_host, void* stream);
 

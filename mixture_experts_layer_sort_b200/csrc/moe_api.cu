@@ -66,6 +66,19 @@ struct moe_layer {
   float* hl = nullptr;
   void* hout = nullptr;
   int host_cap = 0;
+  // moe_forward_host replays a captured graph of copies + forward for pinned host
+  // buffers, one per (M, host pointers); `graph_gen` counts the changes (weights,
+  // workspace, staging, path switches) that make a captured graph stale
+  struct HostGraph {
+    int M;
+    const void *x, *l;
+    void* out;
+    unsigned gen;
+    cudaGraphExec_t exec;
+  };
+  std::vector<HostGraph> host_graphs;
+  unsigned graph_gen = 0;
+  cudaStream_t capture_stream = nullptr;
   // bookkeeping
   int last_M = 0, last_launches = 0;
   bool fused_decode = false;    // single-launch decode path for small bf16 batches
@@ -186,6 +199,7 @@ int ensure_workspace(moe_layer* L, int M) {
   while (cap < M) cap *= 2;
   MOE_CUDA(cudaDeviceSynchronize());   // the old workspace may still be in use
   free_workspace(L);
+  ++L->graph_gen;
   const long long P = static_cast<long long>(cap) * L->k;
   const long long Emin = std::min<long long>(L->E, P);
   L->P_cap = P;
@@ -227,6 +241,7 @@ int ensure_workspace(moe_layer* L, int M) {
 }
 
 int encode_weight_maps(moe_layer* L) {
+  ++L->graph_gen;
   // tiled storage: rows of 128 bytes, one 128-row box = one contiguous 16 KB tile
   const long long el = is_fp8(L) ? 1 : 2;
   const long long inner = 128 / el;
@@ -701,6 +716,8 @@ int moe_destroy(moe_layer* L) {
   cudaFree(L->hx);
   cudaFree(L->hl);
   cudaFree(L->hout);
+  for (auto& hg : L->host_graphs) cudaGraphExecDestroy(hg.exec);
+  if (L->capture_stream) cudaStreamDestroy(L->capture_stream);
   for (auto& t : L->pending) {
     cudaEventDestroy(t.a);
     cudaEventDestroy(t.b);
@@ -777,6 +794,73 @@ int moe_forward(moe_layer* L, const void* x, const float* logits, int M, void* o
   return forward_impl(L, x, logits, M, out, static_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+bool is_pinned(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+// copies in, forward, copy out: enqueued on `st` (eagerly, or while capturing)
+int host_chain(moe_layer* L, const void* x_host, const float* logits_host, int M, void* out_host, cudaStream_t st) {
+  MOE_CUDA(cudaMemcpyAsync(L->hx, x_host, static_cast<size_t>(M) * L->H * 2, cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaMemcpyAsync(L->hl, logits_host, static_cast<size_t>(M) * L->E * 4, cudaMemcpyHostToDevice, st));
+  MOE_TRY(forward_impl(L, L->hx, L->hl, M, L->hout, st));
+  MOE_CUDA(cudaMemcpyAsync(out_host, L->hout, static_cast<size_t>(M) * L->H * 2, cudaMemcpyDeviceToHost, st));
+  return MOE_OK;
+}
+
+// Graph of host_chain for these buffers (captured on the handle's own stream), or
+// nullptr when it cannot be captured (the call then runs eagerly).
+cudaGraphExec_t host_graph(moe_layer* L, const void* x_host, const float* logits_host, int M, void* out_host) {
+  for (auto& hg : L->host_graphs)
+    if (hg.M == M && hg.x == x_host && hg.l == logits_host && hg.out == out_host && hg.gen == L->graph_gen)
+      return hg.exec;
+  if (!L->capture_stream && cudaStreamCreateWithFlags(&L->capture_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    L->capture_stream = nullptr;
+    return nullptr;
+  }
+  cudaStream_t cs = L->capture_stream;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  const int rc = host_chain(L, x_host, logits_host, M, out_host, cs);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(cs, &graph);
+  cudaGraphExec_t exec = nullptr;
+  if (rc != MOE_OK || e != cudaSuccess || graph == nullptr ||
+      cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+    cudaGetLastError();
+    if (graph) cudaGraphDestroy(graph);
+    return nullptr;
+  }
+  cudaGraphDestroy(graph);
+  // keep at most kHostGraphs; stale generations go first, then the oldest
+  constexpr size_t kHostGraphs = 16;
+  for (size_t i = 0; i < L->host_graphs.size();) {
+    if (L->host_graphs[i].gen != L->graph_gen) {
+      cudaGraphExecDestroy(L->host_graphs[i].exec);
+      L->host_graphs.erase(L->host_graphs.begin() + static_cast<long>(i));
+    } else {
+      ++i;
+    }
+  }
+  if (L->host_graphs.size() >= kHostGraphs) {
+    cudaGraphExecDestroy(L->host_graphs.front().exec);
+    L->host_graphs.erase(L->host_graphs.begin());
+  }
+  L->host_graphs.push_back({M, x_host, logits_host, out_host, L->graph_gen, exec});
+  return exec;
+}
+
+}  // namespace
+
 int moe_forward_host(moe_layer* L, const void* x_host, const float* logits_host, int M, void* out_host,
                      void* stream) {
   if (!L || M < 0) return MOE_ERR_INVALID_ARG;
@@ -796,15 +880,24 @@ int moe_forward_host(moe_layer* L, const void* x_host, const float* logits_host,
     L->hx = L->hout = nullptr;
     L->hl = nullptr;
     L->host_cap = 0;
+    ++L->graph_gen;
     MOE_CUDA(cudaMalloc(&L->hx, static_cast<size_t>(M) * L->H * 2));
     MOE_CUDA(cudaMalloc(&L->hl, static_cast<size_t>(M) * L->E * 4));
     MOE_CUDA(cudaMalloc(&L->hout, static_cast<size_t>(M) * L->H * 2));
     L->host_cap = M;
   }
-  MOE_CUDA(cudaMemcpyAsync(L->hx, x_host, static_cast<size_t>(M) * L->H * 2, cudaMemcpyHostToDevice, st));
-  MOE_CUDA(cudaMemcpyAsync(L->hl, logits_host, static_cast<size_t>(M) * L->E * 4, cudaMemcpyHostToDevice, st));
-  MOE_TRY(forward_impl(L, L->hx, L->hl, M, L->hout, st));
-  MOE_CUDA(cudaMemcpyAsync(out_host, L->hout, static_cast<size_t>(M) * L->H * 2, cudaMemcpyDeviceToHost, st));
+  MOE_TRY(ensure_workspace(L, M));   // (re)allocation happens here, never inside a capture
+  // Pinned buffers: one graph launch instead of three copies and five to ten kernel
+  // launches from the host. Pageable buffers, profiling and the single-launch decode
+  // kernel take the eager path.
+  cudaGraphExec_t exec = nullptr;
+  if (!L->profiling && !L->fused_decode && is_pinned(x_host) && is_pinned(logits_host) && is_pinned(out_host))
+    exec = host_graph(L, x_host, logits_host, M, out_host);
+  if (exec) {
+    MOE_CUDA(cudaGraphLaunch(exec, st));
+  } else {
+    MOE_TRY(host_chain(L, x_host, logits_host, M, out_host, st));
+  }
   MOE_CUDA(cudaStreamSynchronize(st));
   return MOE_OK;
 }
@@ -825,6 +918,7 @@ int moe_last_launch_count(moe_layer* L) { return L ? L->last_launches : 0; }
 int moe_set_fused_decode(moe_layer* L, int enable) {
   if (!L) return MOE_ERR_INVALID_ARG;
   L->fused_decode = enable != 0;
+  ++L->graph_gen;
   return MOE_OK;
 }
 
@@ -837,6 +931,7 @@ int moe_profile_enable(moe_layer* L, int enable) {
     L->prof_n[i] = 0;
   }
   L->profiling = enable != 0;
+  ++L->graph_gen;
   return MOE_OK;
 }
 
