@@ -73,3 +73,16 @@ def test_null_handles_are_rejected(lib):
     assert lib.moe_reserve(None, 4, None) == -1
     assert lib.moe_get_device_error(None, None) == -1
     assert lib.moe_last_launch_count(None) == 0
+
+
+def test_every_entry_point_rejects_a_null_handle(lib):
+    # each returns MOE_ERR_INVALID_ARG before any CUDA call
+    assert lib.moe_forward_host(None, None, None, 4, None, None) == -1
+    assert lib.moe_forward_noalloc(None, None, None, 4, None, None) == -1
+    assert lib.moe_load_weights_fp8(None, None, None, None, None, None) == -1
+    assert lib.moe_set_fused_decode(None, 1) == -1
+    assert lib.moe_profile_enable(None, 1) == -1
+    assert lib.moe_profile_read(None, None, None) == -1
+    assert lib.moe_debug_routing(None, None, None, None, None, None, None, None) == -1
+    assert lib.moe_debug_activations(None, None, None) == -1
+    assert lib.moe_debug_weights(None, None, None, None, None) == -1
