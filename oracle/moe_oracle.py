@@ -1,7 +1,7 @@
 """CPU oracle for the fused Mixture-of-Experts layer.
 
 TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or
-execute this module: only the tests, the smoke check of the graft entry point
+execute this module: only the tests, `__graft_entry__.smoke()`
 and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.
 It shares no code, table or helper with the CUDA library and imports nothing
 from it.
