@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--only-M", type=int, default=None, help="run a single batch size of the workload")
     ap.add_argument("--fused-decode", action="store_true", help="single-launch decode path (bf16, M <= 64)")
+    ap.add_argument("--warm-l2", action="store_true",
+                    help="do not flush L2 between forwards (a labelled warm-cache figure, not the headline)")
     return ap.parse_args()
 
 
@@ -328,7 +330,7 @@ def main():
         torch.cuda.empty_cache()
     toks = {M: synth.make_tokens(wl.E, wl.H, M, seed=seed, device=dev, zipf_s=wl.zipf_s) for M in Ms}
     outs = {M: torch.empty((M, wl.H), dtype=torch.bfloat16, device=dev) for M in Ms}
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES if not args.warm_l2 else 0, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
     tokens_per_step = sum(Ms)
 
@@ -491,7 +493,8 @@ def main():
         "config": {"workload": wl.description + f", one step = one forward at each M in {Ms}",
                    "E": wl.E, "topk": wl.k, "H": wl.H, "I": wl.I, "Ms": Ms, "global_batch": tokens_per_step * ws,
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                   "l2": "flushed (252 MB write) before every forward, outside the timed events",
+                   "l2": ("warm: not flushed between forwards" if args.warm_l2 else
+                          "flushed (252 MB write) before every forward, outside the timed events"),
                    "launch": "CUDA graph replay per M" if graphs else "eager"},
         "roofline": {"bound": "hbm", "kernel": "gate_up grouped GEMM", "achieved": achieved, "peak": hbm_gbs,
                      "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None, "traffic": traffic,
