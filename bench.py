@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default="decode",
                     choices=["tiny", "decode", "decode_fp8", "decode_e5m2", "large_decode", "prefill",
-                             "prefill_fp8", "prefill_e48", "prefill_e48_fp8"])
+                             "prefill_fp8", "prefill_m16384", "prefill_e48", "prefill_e48_fp8"])
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -234,7 +234,7 @@ def reference_arm(args, ws, rank):
     from mixture_experts_layer_sort_b200 import synth
     wl, dtype = workload_spec(args.workload)
     Ms = list(wl.Ms)
-    if args.workload in ("prefill", "prefill_fp8", "large_decode"):
+    if args.workload in ("prefill", "prefill_fp8", "prefill_m16384", "large_decode"):
         print(json.dumps({"impl": "reference", "unavailable": "the CPU oracle needs the 22.5 GB weight set "
                           "on the host; the reference arm runs on the decode workloads"}))
         return 0
@@ -466,16 +466,23 @@ def main():
         cpu = {"value": tokens_per_step / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{reps} full decode sweep(s) M={Ms} ({tokens_per_step} tokens), median"}
 
+    # the layer's roofline: the slower of its algorithmic bytes at the measured copy
+    # bandwidth and its FLOPs at the measured dense peak of its dtype (FP8: twice bf16)
+    tensor_tf = bf16_tf * (2.0 if is_fp8(dtype) else 1.0)
     per_M = {}
     for M in Ms:
         t = statistics.mean(per_M_ms[M])
         b = alg_bytes_layer(wl, dtype, M, A[M])
+        f = alg_flops_layer(wl, M)
+        t_roof = max(b / (hbm_gbs * 1e9), f / (tensor_tf * 1e12))
         srt = sorted(per_M_ms[M])
         per_M[str(M)] = {"ms": t, "ms_p50": statistics.median(srt),
                          "ms_p95": srt[min(len(srt) - 1, int(round(0.95 * (len(srt) - 1))))],
                          "ms_eager": eager_ms[M], "tokens_per_s": M / (t / 1e3), "active_experts": A[M],
                          "alg_GB": b / 1e9, "alg_GBps": b / (t / 1e3) / 1e9,
-                         "roofline_frac": (b / (hbm_gbs * 1e9)) / (t / 1e3), "launches": launches_per_M[M]}
+                         "tflops": f / (t / 1e3) / 1e12, "tensor_frac": f / (t / 1e3) / (tensor_tf * 1e12),
+                         "roofline_bound": "hbm" if b / (hbm_gbs * 1e9) >= f / (tensor_tf * 1e12) else "tensor",
+                         "roofline_frac": t_roof / (t / 1e3), "launches": launches_per_M[M]}
 
     line = {
         "metric": METRIC,

@@ -55,6 +55,11 @@ WORKLOADS = {
     "prefill": Workload("prefill", E=256, k=8, H=7168, I=2048, Ms=(4096,), w_std=0.01,
                         dtypes=("bf16", "fp8"),
                         description="prefill, E=256 top-8, H=7168, I=2048, M=4096, bf16 and e4m3"),
+    # a supplementary compute-heavier point: the prefill layer at 4x the tokens (~512 per
+    # expert, two 256-row token blocks each), where the FLOPs (11.5 TFLOP) outweigh the
+    # weight bytes at the measured peaks
+    "prefill_m16384": Workload("prefill_m16384", E=256, k=8, H=7168, I=2048, Ms=(16384,), w_std=0.01,
+                               description="prefill at M=16384 (compute-bound point), E=256 top-8, H=7168, I=2048"),
     # profiling stand-in for prefill: same H, I and tokens per expert (~128) and the same
     # schedule (no split-K), 3/16 of the experts, so a multi-pass profiler capture holds
     # ~4 GB instead of 23 GB
