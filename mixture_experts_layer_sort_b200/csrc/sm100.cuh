@@ -1,6 +1,7 @@
 // sm100.cuh - thin inline-PTX wrappers for the Blackwell (sm_100a) features the
 // grouped GEMMs use: mbarriers with bounded waits, TMA tile loads, tcgen05 MMA
-// with TMEM accumulators, and TMEM loads. No cluster multicast anywhere.
+// with TMEM accumulators, and TMEM loads. Every TMA load fills only the issuing
+// CTA's own shared memory.
 #pragma once
 
 #include <cuda.h>
