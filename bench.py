@@ -1,18 +1,27 @@
 #!/usr/bin/env python
 """Benchmark of the B200 fused MoE layer.
 
-Default workload (N=1): the decode layer E=128 experts, top-8, H=2048, I=768,
+Headline workload (N=1): the decode layer E=128 experts, top-8, H=2048, I=768,
 bf16 weights (1.2 GB), at the four decode batch sizes M = 1, 4, 16, 64. One
 step = one forward at each of the four M (85 tokens); the L2 cache (126 MB) is
 flushed before every forward by writing a 252 MB buffer, outside the timed
 events. Each forward is replayed from a CUDA graph captured once per M (the
 forward is a fixed launch chain with no host synchronisation).
 
+The same line carries, under "workloads", the other shapes the metric names,
+each measured the same way: decode FP8 e4m3 (M = 1, 8, 32, 64, from the same
+decode weights), the Zipf-skewed large decode layer (E=256, H=7168, I=2048,
+bf16, M = 1, 32, 64, 128) and prefill (the same layer, M = 4096, bf16 and e4m3
+from one bf16 weight set).
+
 Reported (one JSON line, rank 0):
   value      tokens/s over all ranks = N * 85 / (device time of one step)
   roofline   gate_up GEMM (the kernel with the largest share): active-expert
              W_gate+W_up bytes per launch / its CUDA-event duration, against
              the measured HBM copy bandwidth
+  per_M      per batch size: device time (mean, p50, p95), tokens/s and the
+             layer's roofline fraction, against the measured peaks and against
+             the nominal 8 TB/s HBM / datasheet tensor peaks
   e2e        the same metric through moe_forward_host: host->device copies of
              x and logits and the device->host copy of out inside the timing
   cpu_baseline  the CPU oracle timed on the same decode sweep on the host cores
@@ -40,6 +49,9 @@ sys.path.insert(0, ROOT)
 METRIC = "fused-MoE tokens/s and HBM GB/s vs roofline (decode M=1-64, prefill), 1 B200"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_HBM_GBS = 8000.0          # the "~8 TB/s" the layer's target is stated against
+NOMINAL_BF16_TFLOPS = 2250.0      # B200 datasheet dense bf16 (FP8: twice)
+DECODE_TARGET = 0.70              # decode shapes: fraction of the HBM roofline
 L2_FLUSH_BYTES = 252 << 20
 
 
@@ -55,6 +67,8 @@ def parse_args():
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="measure the headline workload only (skip decode FP8, large decode and prefill)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--only-M", type=int, default=None, help="run a single batch size of the workload")
     ap.add_argument("--fused-decode", action="store_true", help="single-launch decode path (bf16, M <= 64)")
@@ -91,14 +105,17 @@ def fp8_format(dtype):
     return "e5m2" if dtype == "fp8_e5m2" else "e4m3"
 
 
-def weight_bytes(wl, dtype):
+def dtype_name(dtype):
+    return "bf16" if dtype == "bf16" else fp8_format(dtype)
+
+
+def weight_bytes(dtype):
     return 1 if is_fp8(dtype) else 2
 
 
 def alg_bytes_layer(wl, dtype, M, A):
     """Algorithmic bytes of one forward: active-expert weights, FP8 scales, x, out, logits."""
-    bw = weight_bytes(wl, dtype)
-    b = A * 3 * wl.H * wl.I * bw + M * wl.H * 2 * 2 + M * wl.E * 4
+    b = A * 3 * wl.H * wl.I * weight_bytes(dtype) + M * wl.H * 2 * 2 + M * wl.E * 4
     if is_fp8(dtype):
         b += 3 * wl.E * 4
     return b
@@ -108,9 +125,29 @@ def alg_flops_layer(wl, M):
     return 6 * M * wl.k * wl.H * wl.I
 
 
+def bench_config(wl, Ms, ws, warm_l2):
+    """The workload description both arms print (the reference arm prints the same dict)."""
+    return {"workload": wl.description + f", one step = one forward at each M in {list(Ms)}",
+            "E": wl.E, "topk": wl.k, "H": wl.H, "I": wl.I, "Ms": list(Ms), "global_batch": sum(Ms) * ws,
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "l2": ("warm: not flushed between forwards" if warm_l2 else
+                   "flushed (252 MB write) before every forward, outside the timed events")}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return None
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed regions run."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -209,31 +246,56 @@ def blas_threads():
 
 
 # ----------------------------------------------------------------------------- oracle timing
-def time_oracle_sweep(wl, dtype, host_weights, tokens_per_M, budget_s=30.0, max_reps=50):
-    """Seconds per decode sweep of the CPU oracle (bounded: at least one sweep)."""
+def time_oracle_sweep(wl, dtype, host_weights, tokens_per_M, budget_s=30.0, max_reps=50, one_thread=False):
+    """Seconds per sweep of the CPU oracle over tokens_per_M (bounded: at least one sweep)."""
+    import contextlib
     from oracle import moe_oracle as O
+    ctx = contextlib.nullcontext()
+    if one_thread:
+        import threadpoolctl
+        ctx = threadpoolctl.threadpool_limits(limits=1)
     cache = {}
     times = []
-    t_start = time.time()
-    for _ in range(max_reps):
-        t0 = time.time()
-        for M, (x, l) in tokens_per_M.items():
-            O.moe_forward(x, l, wl.k, *host_weights, fp8=is_fp8(dtype), fp8_format=fp8_format(dtype),
-                          weight_cache=cache)
-        times.append(time.time() - t0)
-        if time.time() - t_start > budget_s:
-            break
+    with ctx:
+        if is_fp8(dtype):   # fill the FP8 weight cache outside the timing, as the GPU loads once
+            for M, (x, l) in tokens_per_M.items():
+                O.moe_forward(x, l, wl.k, *host_weights, fp8=True, fp8_format=fp8_format(dtype),
+                              weight_cache=cache, threads=1 if one_thread else None)
+        t_start = time.time()
+        for _ in range(max_reps):
+            t0 = time.time()
+            for M, (x, l) in tokens_per_M.items():
+                O.moe_forward(x, l, wl.k, *host_weights, fp8=is_fp8(dtype), fp8_format=fp8_format(dtype),
+                              weight_cache=cache, threads=1 if one_thread else None)
+            times.append(time.time() - t0)
+            if time.time() - t_start > budget_s:
+                break
     return statistics.median(times), len(times)
+
+
+def cpu_baseline_entry(wl, dtype, host_w, toks_np, budget_s, one_thread_Ms=(1, 4)):
+    """The oracle on the host cores: the full sweep on all threads, and a smaller
+    sample on one thread (both bounded), as tokens/s."""
+    Ms = list(toks_np)
+    tokens = sum(Ms)
+    sec, reps = time_oracle_sweep(wl, dtype, host_w, toks_np, budget_s=budget_s)
+    sub = {M: toks_np[M] for M in one_thread_Ms if M in toks_np}
+    sec1, reps1 = time_oracle_sweep(wl, dtype, host_w, sub, budget_s=budget_s / 3, max_reps=5, one_thread=True)
+    return {"value": tokens / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+            "sample": f"{reps} full sweep(s) M={Ms} ({tokens} tokens) on all host threads, median",
+            "one_thread": {"value": sum(sub) / sec1, "unit": "tokens/s", "cores": 1,
+                           "sample": f"{reps1} sweep(s) M={list(sub)} ({sum(sub)} tokens), median"}}
 
 
 def reference_arm(args, ws, rank):
     """The CPU oracle as the reference arm: rank 0 times it, the others exit."""
     if rank != 0:
         return 0
-    import torch
     from mixture_experts_layer_sort_b200 import synth
     wl, dtype = workload_spec(args.workload)
-    Ms = list(wl.Ms)
+    only_M = getattr(args, "only_M", None)
+    Ms = [only_M] if only_M else list(wl.Ms)
     if args.workload in ("prefill", "prefill_fp8", "prefill_m16384", "large_decode"):
         print(json.dumps({"impl": "reference", "unavailable": "the CPU oracle needs the 22.5 GB weight set "
                           "on the host; the reference arm runs on the decode workloads"}))
@@ -247,10 +309,8 @@ def reference_arm(args, ws, rank):
     tokens = sum(Ms)
     from oracle import moe_oracle as O
     cache = {}
-    for _ in range(max(args.warmup, 0)):
-        for M, (x, l) in toks.items():
-            O.moe_forward(x, l, wl.k, *host, fp8=is_fp8(dtype), fp8_format=fp8_format(dtype), weight_cache=cache)
-        break   # one warm-up sweep is enough for the CPU path (fills the FP8 weight cache)
+    for M, (x, l) in toks.items():   # one warm-up sweep (fills the FP8 weight cache)
+        O.moe_forward(x, l, wl.k, *host, fp8=is_fp8(dtype), fp8_format=fp8_format(dtype), weight_cache=cache)
     times = []
     for _ in range(args.steps):
         t0 = time.time()
@@ -263,9 +323,10 @@ def reference_arm(args, ws, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.description + f", M in {Ms} per step", "Ms": Ms, "global_batch": tokens},
+        "config": bench_config(wl, Ms, args.gpus, getattr(args, "warm_l2", False)),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": f"full decode sweep M={Ms} ({tokens} tokens) per step"},
+                         "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+                         "sample": f"full sweep M={Ms} ({tokens} tokens) per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -299,6 +360,205 @@ def kernel_source_hash():
     return h.hexdigest()
 
 
+class Runner:
+    """Times one layer on one workload: graph replay per M with an L2 flush before every
+    forward (outside the events), then an eager pass, then a pass with the library's
+    per-kernel CUDA events (on the forward's stream)."""
+
+    def __init__(self, layer, wl, dtype, Ms, toks, stream, flush, use_graph):
+        import torch
+        self.torch = torch
+        self.layer, self.wl, self.dtype, self.Ms, self.toks = layer, wl, dtype, list(Ms), toks
+        self.stream, self.flush = stream, flush
+        dev = toks[self.Ms[0]][0].device
+        self.outs = {M: torch.empty((M, wl.H), dtype=torch.bfloat16, device=dev) for M in self.Ms}
+        layer.reserve(max(self.Ms))
+        self.A, self.launches = {}, {}
+        with torch.cuda.stream(stream):
+            for M in self.Ms:
+                layer.forward(*toks[M], out=self.outs[M])
+                self.A[M] = int(torch.count_nonzero(layer.debug_routing(M)["counts"]).item())
+                layer.forward(*toks[M], out=self.outs[M])
+                self.launches[M] = layer.last_launch_count
+        torch.cuda.synchronize()
+        self.graphs = {}
+        if use_graph:
+            for M in self.Ms:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    layer.forward(*toks[M], out=self.outs[M])
+                self.graphs[M] = g
+            torch.cuda.synchronize()
+
+    def forward(self, M):
+        if self.graphs:
+            self.graphs[M].replay()
+        else:
+            self.layer.forward(*self.toks[M], out=self.outs[M])
+
+    def step(self, events=None):
+        for i, M in enumerate(self.Ms):
+            self.flush.zero_()
+            if events is not None:
+                events[i][0].record(self.stream)
+            self.forward(M)
+            if events is not None:
+                events[i][1].record(self.stream)
+
+    def warm(self, n):
+        with self.torch.cuda.stream(self.stream):
+            for _ in range(n):
+                self.step()
+        self.torch.cuda.synchronize()
+
+    def timed(self, steps):
+        """Per-M lists of CUDA-event ms over `steps` steps, and the wall time."""
+        torch = self.torch
+        ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in self.Ms]
+              for _ in range(steps)]
+        torch.cuda.synchronize()
+        t0 = time.time()
+        with torch.cuda.stream(self.stream):
+            for s in range(steps):
+                self.step(ev[s])
+        torch.cuda.synchronize()
+        wall = time.time() - t0
+        per_M = {M: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)] for i, M in enumerate(self.Ms)}
+        return per_M, wall
+
+    def eager_ms(self, reps=3):
+        torch = self.torch
+        got = {M: [] for M in self.Ms}
+        with torch.cuda.stream(self.stream):
+            for _ in range(reps):
+                for M in self.Ms:
+                    self.flush.zero_()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(self.stream)
+                    self.layer.forward(*self.toks[M], out=self.outs[M])
+                    e1.record(self.stream)
+                    got[M].append((e0, e1))
+        torch.cuda.synchronize()
+        return {M: statistics.median(a.elapsed_time(b) for a, b in v) for M, v in got.items()}
+
+    def kernel_profile(self, reps):
+        """{kernel: (ms, launches)} over `reps` eager steps, and the gate_up / down
+        algorithmic weight bytes those launches moved."""
+        wl, bw = self.wl, weight_bytes(self.dtype)
+        self.layer.profile_enable(True)
+        gate_bytes = down_bytes = 0.0
+        with self.torch.cuda.stream(self.stream):
+            for _ in range(reps):
+                for M in self.Ms:
+                    self.flush.zero_()
+                    self.layer.forward(*self.toks[M], out=self.outs[M])
+                    gate_bytes += self.A[M] * 2 * wl.H * wl.I * bw
+                    down_bytes += self.A[M] * wl.H * wl.I * bw
+        prof = self.layer.profile_read()
+        self.layer.profile_enable(False)
+        return prof, gate_bytes, down_bytes
+
+    def close(self):
+        self.graphs.clear()
+
+
+def per_M_summary(wl, dtype, Ms, per_M_ms, eager, A, launches, hbm_gbs, bf16_tf):
+    tensor_tf = bf16_tf * (2.0 if is_fp8(dtype) else 1.0)
+    tensor_nom = NOMINAL_BF16_TFLOPS * (2.0 if is_fp8(dtype) else 1.0)
+    out = {}
+    for M in Ms:
+        v = per_M_ms[M]
+        t = statistics.mean(v)
+        srt = sorted(v)
+        b = alg_bytes_layer(wl, dtype, M, A[M])
+        f = alg_flops_layer(wl, M)
+        t_roof = max(b / (hbm_gbs * 1e9), f / (tensor_tf * 1e12))
+        t_nom = max(b / (NOMINAL_HBM_GBS * 1e9), f / (tensor_nom * 1e12))
+        out[str(M)] = {"ms": t, "ms_p50": statistics.median(srt),
+                       "ms_p95": srt[min(len(srt) - 1, int(round(0.95 * (len(srt) - 1))))],
+                       "ms_eager": eager.get(M), "tokens_per_s": M / (t / 1e3), "active_experts": A[M],
+                       "alg_GB": b / 1e9, "alg_GBps": b / (t / 1e3) / 1e9,
+                       "tflops": f / (t / 1e3) / 1e12, "tensor_frac": f / (t / 1e3) / (tensor_tf * 1e12),
+                       "roofline_bound": "hbm" if b / (hbm_gbs * 1e9) >= f / (tensor_tf * 1e12) else "tensor",
+                       "roofline_frac": t_roof / (t / 1e3), "roofline_frac_nominal": t_nom / (t / 1e3),
+                       "launches": launches[M]}
+    return out
+
+
+def measure_workload(name, layer, wl, dtype, Ms, toks, stream, flush, args, hbm_gbs, bf16_tf):
+    """One workload entry of the bench line (an extra workload next to the headline)."""
+    r = Runner(layer, wl, dtype, Ms, toks, stream, flush, use_graph=not args.no_graph)
+    r.warm(max(3, args.warmup))
+    steps = max(5, min(args.steps, 20))
+    per_M_ms, _ = r.timed(steps)
+    eager = r.eager_ms()
+    prof, gate_bytes, down_bytes = r.kernel_profile(max(3, min(steps, 10)))
+    r.close()
+    step_ms = [sum(per_M_ms[M][s] for M in Ms) for s in range(steps)]
+    ms = statistics.mean(step_ms)
+    g_ms, _ = prof["gate_up"]
+    d_ms, _ = prof["down"]
+    tot = sum(v[0] for v in prof.values())
+    gemm = {"gate_up": {"GBps": gate_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else None},
+            "down": {"GBps": down_bytes / (d_ms / 1e3) / 1e9 if d_ms > 0 else None}}
+    for v in gemm.values():
+        v["frac"] = v["GBps"] / hbm_gbs if v["GBps"] else None
+    dom = max(("gate_up", "down"), key=lambda k: prof[k][0])
+    summary = per_M_summary(wl, dtype, Ms, per_M_ms, eager, r.A, r.launches, hbm_gbs, bf16_tf)
+    entry = {"workload": wl.description + f", one step = one forward at each M in {list(Ms)}",
+             "dtype": dtype_name(dtype), "Ms": list(Ms), "steps": steps, "ms_per_step": ms,
+             "tokens_per_s": sum(Ms) / (ms / 1e3), "per_M": summary,
+             "dominant_gemm": dict(kernel=dom, **gemm[dom]), "gemm_event_GBps": gemm,
+             "kernel_share": {k: round(v[0] / tot, 4) for k, v in prof.items() if v[1] > 0} if tot else {},
+             "launches_per_step": sum(r.launches[M] for M in Ms)}
+    if name.startswith("decode"):
+        entry["meets_decode_target"] = {M: summary[str(M)]["roofline_frac"] >= DECODE_TARGET for M in summary}
+    return entry
+
+
+def extra_workloads(args, dev, stream, flush, dec_weights, seed, hbm_gbs, bf16_tf, cpu_on):
+    """Decode FP8 (from the decode weights), large decode and prefill bf16 + FP8 (from one
+    E=256 bf16 weight set), each measured like the headline."""
+    import torch
+    from mixture_experts_layer_sort_b200 import MoELayer, synth
+    res = {}
+    wl = synth.WORKLOADS["decode_fp8"]
+    lay = MoELayer(wl.E, wl.k, wl.H, wl.I, "fp8")
+    lay.load_weights(*dec_weights)
+    toks = {M: synth.make_tokens(wl.E, wl.H, M, seed=seed, device=dev) for M in wl.Ms}
+    res["decode_fp8"] = measure_workload("decode_fp8", lay, wl, "fp8", wl.Ms, toks, stream, flush, args,
+                                         hbm_gbs, bf16_tf)
+    lay.close()
+    if cpu_on:
+        host_w = [synth.bf16_to_f32_numpy(w) for w in dec_weights]
+        tnp = {M: (toks[M][0].float().cpu().numpy(), toks[M][1].cpu().numpy()) for M in wl.Ms}
+        res["decode_fp8"]["cpu_baseline"] = cpu_baseline_entry(wl, "fp8", host_w, tnp, budget_s=10.0,
+                                                               one_thread_Ms=(1, 8))
+    del toks
+
+    wl4, wl5 = synth.WORKLOADS["large_decode"], synth.WORKLOADS["prefill"]
+    wg, wu, wd = synth.make_weights(wl4.E, wl4.H, wl4.I, wl4.w_std, seed=args.seed, device=dev)
+    big = MoELayer(wl4.E, wl4.k, wl4.H, wl4.I, "bf16")
+    big.load_weights(wg, wu, wd)
+    big8 = MoELayer(wl5.E, wl5.k, wl5.H, wl5.I, "fp8")
+    big8.load_weights(wg, wu, wd)
+    del wg, wu, wd
+    torch.cuda.empty_cache()
+    toks = {M: synth.make_tokens(wl4.E, wl4.H, M, seed=seed, device=dev, zipf_s=wl4.zipf_s) for M in wl4.Ms}
+    res["large_decode"] = measure_workload("large_decode", big, wl4, "bf16", wl4.Ms, toks, stream, flush, args,
+                                           hbm_gbs, bf16_tf)
+    del toks
+    toks = {M: synth.make_tokens(wl5.E, wl5.H, M, seed=seed, device=dev) for M in wl5.Ms}
+    res["prefill"] = measure_workload("prefill", big, wl5, "bf16", wl5.Ms, toks, stream, flush, args,
+                                      hbm_gbs, bf16_tf)
+    big.close()
+    res["prefill_fp8"] = measure_workload("prefill_fp8", big8, wl5, "fp8", wl5.Ms, toks, stream, flush, args,
+                                          hbm_gbs, bf16_tf)
+    big8.close()
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     args = parse_args()
     ws, rank, local = dist_setup(args)
@@ -309,7 +569,6 @@ def main():
             dist.destroy_process_group()
         return rc
 
-    import numpy as np
     import torch
 
     from mixture_experts_layer_sort_b200 import MoELayer, synth
@@ -321,109 +580,30 @@ def main():
     wg, wu, wd = synth.make_weights(wl.E, wl.H, wl.I, wl.w_std, seed=args.seed, device=dev)
     layer = MoELayer(wl.E, wl.k, wl.H, wl.I, dtype)
     layer.load_weights(wg, wu, wd)
-    layer.reserve(max(Ms))
     if args.fused_decode:
         layer.set_fused_decode(True)
-    if args.no_cpu_baseline or rank != 0 or ws != 1:
-        del wg, wu, wd                       # the layer holds its own copy
-        wg = wu = wd = None
-        torch.cuda.empty_cache()
     toks = {M: synth.make_tokens(wl.E, wl.H, M, seed=seed, device=dev, zipf_s=wl.zipf_s) for M in Ms}
-    outs = {M: torch.empty((M, wl.H), dtype=torch.bfloat16, device=dev) for M in Ms}
     flush = torch.empty(L2_FLUSH_BYTES if not args.warm_l2 else 0, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
     tokens_per_step = sum(Ms)
+    hbm_gbs, bf16_tf, peak_src = read_peaks()
 
-    # active experts per M (from this forward's own routing counts)
-    A = {}
-    with torch.cuda.stream(stream):
-        for M in Ms:
-            layer.forward(*toks[M], out=outs[M])
-            A[M] = int(torch.count_nonzero(layer.debug_routing(M)["counts"]).item())
-    launches_per_M = {}
-    for M in Ms:
-        with torch.cuda.stream(stream):
-            layer.forward(*toks[M], out=outs[M])
-        launches_per_M[M] = layer.last_launch_count
-    torch.cuda.synchronize()
-
-    graphs = {}
-    if not args.no_graph:
-        for M in Ms:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                layer.forward(*toks[M], out=outs[M])
-            graphs[M] = g
-        torch.cuda.synchronize()
-
-    def run_forward(M):
-        if graphs:
-            graphs[M].replay()
-        else:
-            layer.forward(*toks[M], out=outs[M])
-
-    def step(events=None):
-        for i, M in enumerate(Ms):
-            flush.zero_()
-            if events is not None:
-                events[i][0].record(stream)
-            run_forward(M)
-            if events is not None:
-                events[i][1].record(stream)
-
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
-    torch.cuda.synchronize()
+    run = Runner(layer, wl, dtype, Ms, toks, stream, flush, use_graph=not args.no_graph)
+    run.warm(args.warmup)
 
     # ---------------------------------------------------------------- timed region
-    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in Ms]
-          for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     time.sleep(0.3)
     barrier(ws)
-    torch.cuda.synchronize()
-    t0 = time.time()
-    with torch.cuda.stream(stream):
-        for s in range(args.steps):
-            step(ev[s])
-    torch.cuda.synchronize()
-    wall = time.time() - t0
+    per_M_ms, wall = run.timed(args.steps)
     barrier(ws)
-    per_M_ms = {M: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i, M in enumerate(Ms)}
     step_ms = [sum(per_M_ms[M][s] for M in Ms) for s in range(args.steps)]
     ms_per_step = max_over_ranks(statistics.mean(step_ms), ws)
 
-    # ---------------------------------------------------------------- eager launches (no graph), same workload
-    eager_ms = {M: [] for M in Ms}
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            for M in Ms:
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                layer.forward(*toks[M], out=outs[M])
-                e1.record(stream)
-                eager_ms[M].append((e0, e1))
-    torch.cuda.synchronize()
-    eager_ms = {M: statistics.median(a.elapsed_time(b) for a, b in v) for M, v in eager_ms.items()}
-
-    # ---------------------------------------------------------------- per-kernel events (same workload, eager)
-    layer.profile_enable(True)
+    eager_ms = run.eager_ms()
     prof_steps = max(3, min(args.steps, 20))
-    gate_bytes = 0.0
-    with torch.cuda.stream(stream):
-        for s in range(prof_steps):
-            for M in Ms:
-                flush.zero_()
-                layer.forward(*toks[M], out=outs[M])
-                gate_bytes += A[M] * 2 * wl.H * wl.I * weight_bytes(wl, dtype)
-    prof = layer.profile_read()
-    layer.profile_enable(False)
-    clk = clocks.stop()
-
-    hbm_gbs, bf16_tf, peak_src = read_peaks()
+    prof, gate_bytes, _ = run.kernel_profile(prof_steps)
     g_ms, g_n = prof["gate_up"]
     achieved = gate_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else None
     traffic_tbl = traffic_from_profile(kernel_source_hash())
@@ -431,6 +611,13 @@ def main():
     if traffic_tbl and all(M in traffic_tbl for M in Ms):
         traffic = statistics.mean(traffic_tbl[M] for M in Ms)
     total_prof = sum(v[0] for v in prof.values())
+
+    # ---------------------------------------------------------------- other workloads of the metric
+    workloads = None
+    cpu_on = rank == 0 and ws == 1 and not args.no_cpu_baseline
+    if ws == 1 and not args.no_workloads and args.workload == "decode" and not args.only_M:
+        workloads = extra_workloads(args, dev, stream, flush, (wg, wu, wd), seed, hbm_gbs, bf16_tf, cpu_on)
+    clk = clocks.stop()
 
     # ---------------------------------------------------------------- e2e through host buffers
     e2e = None
@@ -458,32 +645,12 @@ def main():
 
     # ---------------------------------------------------------------- CPU oracle on the same sweep
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline and args.workload in ("tiny", "decode", "decode_fp8",
-                                                                               "decode_e5m2"):
+    if cpu_on and args.workload in ("tiny", "decode", "decode_fp8", "decode_e5m2"):
         host_w = [synth.bf16_to_f32_numpy(w) for w in (wg, wu, wd)]
         tpm = {M: (toks[M][0].float().cpu().numpy(), toks[M][1].cpu().numpy()) for M in Ms}
-        sec, reps = time_oracle_sweep(wl, dtype, host_w, tpm)
-        cpu = {"value": tokens_per_step / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{reps} full decode sweep(s) M={Ms} ({tokens_per_step} tokens), median"}
+        cpu = cpu_baseline_entry(wl, dtype, host_w, tpm, budget_s=30.0)
 
-    # the layer's roofline: the slower of its algorithmic bytes at the measured copy
-    # bandwidth and its FLOPs at the measured dense peak of its dtype (FP8: twice bf16)
-    tensor_tf = bf16_tf * (2.0 if is_fp8(dtype) else 1.0)
-    per_M = {}
-    for M in Ms:
-        t = statistics.mean(per_M_ms[M])
-        b = alg_bytes_layer(wl, dtype, M, A[M])
-        f = alg_flops_layer(wl, M)
-        t_roof = max(b / (hbm_gbs * 1e9), f / (tensor_tf * 1e12))
-        srt = sorted(per_M_ms[M])
-        per_M[str(M)] = {"ms": t, "ms_p50": statistics.median(srt),
-                         "ms_p95": srt[min(len(srt) - 1, int(round(0.95 * (len(srt) - 1))))],
-                         "ms_eager": eager_ms[M], "tokens_per_s": M / (t / 1e3), "active_experts": A[M],
-                         "alg_GB": b / 1e9, "alg_GBps": b / (t / 1e3) / 1e9,
-                         "tflops": f / (t / 1e3) / 1e12, "tensor_frac": f / (t / 1e3) / (tensor_tf * 1e12),
-                         "roofline_bound": "hbm" if b / (hbm_gbs * 1e9) >= f / (tensor_tf * 1e12) else "tensor",
-                         "roofline_frac": t_roof / (t / 1e3), "launches": launches_per_M[M]}
-
+    per_M = per_M_summary(wl, dtype, Ms, per_M_ms, eager_ms, run.A, run.launches, hbm_gbs, bf16_tf)
     line = {
         "metric": METRIC,
         "value": ws * tokens_per_step / (ms_per_step / 1e3),
@@ -495,32 +662,35 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if dtype == "bf16" else fp8_format(dtype),
+        "dtype": dtype_name(dtype),
         "data": "synthetic",
-        "config": {"workload": wl.description + f", one step = one forward at each M in {Ms}",
-                   "E": wl.E, "topk": wl.k, "H": wl.H, "I": wl.I, "Ms": Ms, "global_batch": tokens_per_step * ws,
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                   "l2": ("warm: not flushed between forwards" if args.warm_l2 else
-                          "flushed (252 MB write) before every forward, outside the timed events"),
-                   "launch": "CUDA graph replay per M" if graphs else "eager"},
+        "config": bench_config(wl, Ms, ws, args.warm_l2),
+        "launch": "CUDA graph replay per M" if run.graphs else "eager",
         "roofline": {"bound": "hbm", "kernel": "gate_up grouped GEMM", "achieved": achieved, "peak": hbm_gbs,
                      "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None, "traffic": traffic,
                      "peak_source": f"{peak_src} HBM copy bandwidth",
                      "alg_bytes_per_launch": gate_bytes / max(g_n, 1),
                      "avg_launch_ms": g_ms / max(g_n, 1)},
+        "layer_roofline": {
+            "note": "whole-forward fractions per M (slower of algorithmic bytes at HBM bandwidth and FLOPs at "
+                    "tensor peak); the decode target is >= 0.70 of the HBM roofline",
+            "frac_measured_peaks": {M: round(per_M[M]["roofline_frac"], 4) for M in per_M},
+            "frac_nominal_8TBps": {M: round(per_M[M]["roofline_frac_nominal"], 4) for M in per_M},
+            "worst_frac_measured": min(per_M[M]["roofline_frac"] for M in per_M),
+            "meets_decode_target": {M: per_M[M]["roofline_frac"] >= DECODE_TARGET for M in per_M}},
         "kernel_share": {k: round(v[0] / total_prof, 4) for k, v in prof.items() if v[1] > 0} if total_prof else {},
         "kernel_us_per_step": {k: round(v[0] * 1e3 / prof_steps, 2) for k, v in prof.items() if v[1] > 0},
         "per_M": per_M,
+        "workloads": workloads,
         "e2e": e2e,
-        "gpu_launches": sum(launches_per_M[M] for M in Ms) * args.steps,
+        "gpu_launches": sum(run.launches[M] for M in Ms) * args.steps,
         "cpu_baseline": cpu,
         "clocks": clk,
         "wall_s_timed": wall,
     }
     if rank == 0:
         print(json.dumps(line))
-    for g in graphs.values():
-        del g
+    run.close()
     layer.close()
     if ws > 1:
         import torch.distributed as dist

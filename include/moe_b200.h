@@ -127,9 +127,8 @@ MOE_API int moe_forward_host(moe_layer* layer, const void* x_host, const float* 
  * counterpart to this entry point; it exists for how the library is deployed.)
  * moe_forward allocates its per-call scratch on first use and grows it with cudaMalloc
  * when a larger batch arrives. A caller whose runtime owns all of HBM and forbids later
- * allocations, a caller that is capturing a stream into a CUDA graph, or a caller that
- * cannot afford the device-wide synchronisation of cudaMalloc/cudaFree, uses this entry
- * point instead: same arguments and same result as moe_forward, but every byte of
+ * allocations, or a caller that cannot afford the device-wide synchronisation of
+ * cudaMalloc/cudaFree inside its serving loop, uses this entry point instead: same arguments and same result as moe_forward, but every byte of
  * per-call scratch comes from one fixed 32 MiB array in device memory that the library
  * defines statically. Nothing is allocated or freed by the call.
  *   - Limit: a batch whose scratch exceeds 32 MiB is rejected with MOE_ERR_INVALID_ARG and a
@@ -144,8 +143,12 @@ MOE_API int moe_forward_host(moe_layer* layer, const void* x_host, const float* 
  *     their data in it; each call clears the parts that must start at zero. Two calls
  *     whose work overlaps on the GPU (different streams, or different host threads) race
  *     on the array: keep them stream-ordered.
- *   - Kernel waits are bounded as in moe_forward, but this path does not write the
- *     handle's device error word. */
+ *   - Kernel waits are bounded as in moe_forward. A wait that gives up records its code
+ *     in an error word kept at the start of the array (per device, not per handle);
+ *     moe_get_device_error on any handle of that device reads and clears it.
+ *   - moe_debug_routing and moe_debug_activations describe the last moe_forward call
+ *     only: this path leaves the handle's workspace (and its FP8 s_x / s_h record)
+ *     untouched. */
 MOE_API int moe_forward_noalloc(moe_layer* layer, const void* x, const float* router_logits, int M,
                                 void* out, void* stream);
 
@@ -162,9 +165,14 @@ MOE_API int moe_set_fused_decode(moe_layer* layer, int enable);
 /* Text of a status code (static storage). */
 MOE_API const char* moe_status_string(int status);
 
-/* Synchronise the device and read (then clear) the handle's device error word:
- * 0 when no kernel reported an error; otherwise a code whose low byte names the
- * kernel and wait that gave up (bounded waits never spin forever). */
+/* Synchronise the device and read (then clear) the handle's device error word, or,
+ * when that is clear, the error word of moe_forward_noalloc on the handle's device:
+ * *code = 0 when no kernel reported an error; otherwise a code whose low byte names
+ * the wait that gave up (0x01 stage full, 0x02 stage empty, 0x03 accumulator full,
+ * 0x04 accumulator empty, 0x06 activation dependency, 0x07 grid) or 0x05 (a tile
+ * descriptor failed its bounds check). Bounded waits never spin forever.
+ * Returns MOE_OK when *code is 0, MOE_ERR_DEVICE_TIMEOUT when a wait gave up,
+ * MOE_ERR_CUDA for a failed bounds check or a failed CUDA call. */
 MOE_API int moe_get_device_error(moe_layer* layer, int* code);
 
 /* Number of kernels the last moe_forward launched (0 for M = 0). */

@@ -221,13 +221,14 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   return launch_kernel(route_kernel<16>, g, b, 0, s, a);
 }
 
-// Row kernels: one block per two rows, or (capped) at most 8 blocks per SM of a B200
-// striding over the rows. Measured at prefill size on one box: the bf16 gather (14 KB
+// Row kernels: one block per two rows, or (capped) at most 8 blocks per SM striding
+// over the rows. Measured at prefill size on one box: the bf16 gather (14 KB
 // row copies) is faster uncapped (127 vs 141 us), the FP8 row kernels (quantising,
 // or copying 1-byte rows) capped (x: 116 vs 150 us, h: 68 vs 81 us).
 int row_grid(int rows, bool capped) {
   const int g = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
-  return g < 1 ? 1 : ((capped && g > 148 * 8) ? 148 * 8 : g);
+  const int cap = 8 * sm_count();
+  return g < 1 ? 1 : ((capped && g > cap) ? cap : g);
 }
 
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s) {
@@ -249,7 +250,7 @@ cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s) {
   long long n4 = a.n / 4;
   long long blocks = (n4 + 255) / 256;
   if (blocks < 1) blocks = 1;
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks > 8ll * sm_count()) blocks = 8ll * sm_count();
   return launch_kernel(finalize_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, s, a);
 }
 

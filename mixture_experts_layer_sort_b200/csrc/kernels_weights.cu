@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(256) retile_kernel(const uint8_t* src, TileGeo
 
 int grid_for(long long work) {
   long long b = (work + 255) / 256;
-  if (b > 148 * 32) b = 148 * 32;
+  if (b > 32ll * sm_count()) b = 32ll * sm_count();
   return static_cast<int>(b < 1 ? 1 : b);
 }
 

@@ -8,8 +8,11 @@
 // re-encoded per M (the
 // pages' third change removes exactly such per-token-count recompiles:
 // toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "3.
-// Removing repeat compilation can reduce first-token delay"). Tensor maps are
-// encoded once per weight load and once per workspace allocation.
+// Removing repeat compilation can reduce first-token delay"). Tensor maps of the
+// weights and of the workspace are encoded once per weight load and once per
+// workspace allocation; the one exception is the map over the caller's x that the
+// direct-x path of the smallest bf16 batches encodes on the host per call (a host
+// computation of 128 bytes, no compilation and no device work).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -24,6 +27,7 @@
 
 #include "../../include/moe_b200.h"
 #include "moe_internal.h"
+#include "sm100.cuh"
 
 using moe::Tile;
 
@@ -609,6 +613,17 @@ bool moe::pdl_enabled() {
   return on;
 }
 
+int moe::sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
 bool moe::uniform_splits() {
   static const bool on = [] {
     const char* e = std::getenv("MOE_UNIFORM_SPLITS");
@@ -907,10 +922,16 @@ int moe_get_device_error(moe_layer* L, int* code) {
   *code = 0;
   DeviceGuard g(L->device);
   MOE_CUDA(cudaDeviceSynchronize());
-  if (!L->err) return MOE_OK;
-  MOE_CUDA(cudaMemcpy(code, L->err, 4, cudaMemcpyDeviceToHost));
-  MOE_CUDA(cudaMemset(L->err, 0, 4));
-  return MOE_OK;
+  if (L->err) {
+    MOE_CUDA(cudaMemcpy(code, L->err, 4, cudaMemcpyDeviceToHost));
+    if (*code != 0) MOE_CUDA(cudaMemset(L->err, 0, 4));
+  }
+  int na = 0;
+  MOE_TRY(moe_noalloc_take_error(L->device, &na));
+  if (*code == 0) *code = na;
+  if (*code == 0) return MOE_OK;
+  // a bounded wait that gave up, or (kErrBadTile) a tile that failed its bounds check
+  return *code == moe::kErrBadTile ? MOE_ERR_CUDA : MOE_ERR_DEVICE_TIMEOUT;
 }
 
 int moe_last_launch_count(moe_layer* L) { return L ? L->last_launches : 0; }

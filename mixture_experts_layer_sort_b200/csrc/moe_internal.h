@@ -142,6 +142,8 @@ struct FinalizeArgs {
 // in the environment: the kernel may be scheduled before its predecessor in the stream
 // finishes, and orders itself with griddepcontrol (see sm100.cuh).
 bool pdl_enabled();
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count();
 // MOE_UNIFORM_SPLITS=1 replaces the balanced unit schedule by one split factor per GEMM
 bool uniform_splits();
 int gemm_max_stages(bool gate_up);   // ring depth cap (MOE_MAX_STAGES1/2 override, for tuning)
@@ -242,5 +244,8 @@ struct LayerView {
 
 struct moe_layer;
 int moe_layer_view(const moe_layer* L, moe::LayerView* v);
+// Read and clear the device error word of moe_forward_noalloc on device `dev` (the
+// current device); *code = 0 when that path never ran there.
+int moe_noalloc_take_error(int dev, int* code);
 // 2-D tensor map [rows, inner] of bf16 (or e4m3 when fp8), 128-byte rows per box, box_rows rows.
 int moe_encode_tile_map(CUtensorMap* m, const void* base, bool fp8, long long inner, long long rows, int box_rows);

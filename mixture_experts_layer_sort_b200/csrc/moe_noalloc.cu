@@ -5,10 +5,8 @@
 // split-K partial sums, the fp32 combine accumulator, tile lists) on first use and
 // grows it with cudaMalloc when a larger batch arrives. Some callers cannot let a
 // library do that: a serving runtime that hands out all of HBM to its own pool at
-// start-up and forbids later allocations, code that runs while a stream is being
-// captured into a CUDA graph (where a cudaMalloc is illegal or breaks the capture),
-// and latency-critical loops that cannot afford the device-wide synchronisation a
-// cudaMalloc/cudaFree may bring. For them this entry point takes all per-call
+// start-up and forbids later allocations, and latency-critical loops that cannot
+// afford the device-wide synchronisation a cudaMalloc/cudaFree may bring. For them this entry point takes all per-call
 // scratch from one fixed array in device memory, kScratchBytes large, defined at file
 // scope below. Every GPU that loads the library holds that array until the process
 // exits. The layer's weights are still the ones moe_load_weights stored in the
@@ -53,10 +51,16 @@ int scratch_address(int dev, void** out) {
   return MOE_OK;
 }
 
+// The first 256 bytes of the array hold the device error word of this path (kernels
+// whose bounded waits give up record a code there, first error wins). Calls never
+// clear it: moe_get_device_error reads and clears it (static device memory starts
+// at zero). The per-call scratch is carved from the rest.
+constexpr size_t kErrWordBytes = 256;
+
 // Bump allocator over the scratch array: 256-byte aligned pieces, no device calls.
 struct Carve {
   unsigned char* base;
-  size_t off = 0;
+  size_t off = kErrWordBytes;
   template <class T>
   T* take(size_t bytes) {
     off = (off + 255) & ~size_t(255);
@@ -194,7 +198,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g.k = v.k;
   g.P = static_cast<int>(P);
   g.f8 = v.f8;
-  g.err = nullptr;
+  g.err = static_cast<int*>(base);
 
   moe::GemmArgs g1 = g;
   g1.tiles = tiles1;
@@ -244,6 +248,20 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
 }
 
 }  // namespace
+
+int moe_noalloc_take_error(int dev, int* code) {
+  *code = 0;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_OK;
+  void* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    p = g_scratch_addr[dev];
+  }
+  if (p == nullptr) return MOE_OK;   // the path never ran on this device
+  NA_CUDA(cudaMemcpy(code, p, sizeof(int), cudaMemcpyDeviceToHost));
+  if (*code != 0) NA_CUDA(cudaMemset(p, 0, sizeof(int)));
+  return MOE_OK;
+}
 
 extern "C" int moe_forward_noalloc(moe_layer* layer, const void* x, const float* router_logits, int M,
                                    void* out, void* stream) {

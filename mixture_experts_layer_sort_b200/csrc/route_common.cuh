@@ -71,9 +71,11 @@ __device__ __forceinline__ void route_token(const float* row, int E, int k, int 
         }
     }
   }
-  // slot 0 holds the largest selected logit
+  // slot 0 holds the largest selected logit. When it is -inf, every logit of the
+  // row is -inf (or NaN): the row takes the limit of k equal logits, weight 1/k each.
   const float lmax = __shfl_sync(0xFFFFFFFFu, my_logit, 0);
-  const float ex = (lane < k) ? expf(my_logit - lmax) : 0.f;
+  const bool no_finite = lmax == __uint_as_float(0xFF800000u) || lmax != lmax;
+  const float ex = (lane < k) ? (no_finite ? 1.f : expf(my_logit - lmax)) : 0.f;
   float sum = ex;
   #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);

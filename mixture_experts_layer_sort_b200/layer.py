@@ -136,8 +136,11 @@ class MoELayer:
         return {k: (ms[i], n[i]) for i, k in enumerate(self.KERNEL_SLOTS)}
 
     def device_error(self) -> int:
+        """The device error word (0 = no kernel reported an error); reading clears it."""
         c = ctypes.c_int(0)
-        self._check("moe_get_device_error", self.lib.moe_get_device_error(self.handle, ctypes.byref(c)))
+        rc = self.lib.moe_get_device_error(self.handle, ctypes.byref(c))
+        if rc != 0 and c.value == 0:
+            self._check("moe_get_device_error", rc)
         return c.value
 
     # ------------------------------------------------------------------ test access

@@ -69,6 +69,10 @@ def route(logits: np.ndarray, k: int):
     softmax over all E logits in fp64 (max subtracted), restricted to the
     selected experts and divided by their sum.
 
+    A row whose logits are all -inf has no finite softmax; it takes the limit
+    of a row of k equal logits, i.e. weight 1/k for each selected expert (the
+    k lowest ids, by the tie rule).
+
     Returns (ids [M,k] int32, w [M,k] float64).
     """
     logits = np.asarray(logits, dtype=np.float32)
@@ -80,7 +84,9 @@ def route(logits: np.ndarray, k: int):
     ids = order[:, :k].astype(np.int32)
     l64 = logits.astype(np.float64)
     mx = l64.max(axis=1, keepdims=True)
-    p = np.exp(l64 - mx)
+    all_neg_inf = np.isneginf(mx[:, 0])
+    p = np.exp(l64 - np.where(all_neg_inf[:, None], 0.0, mx))
+    p = np.where(all_neg_inf[:, None], 1.0, p)
     p /= p.sum(axis=1, keepdims=True)
     sel = np.take_along_axis(p, ids.astype(np.int64), axis=1)
     w = sel / sel.sum(axis=1, keepdims=True)

@@ -67,3 +67,7 @@ def test_reference_arm_prints_one_line(capsys):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # the same workload description as the main arm, so both lines name one config
+    from mixture_experts_layer_sort_b200 import synth
+    wl = synth.WORKLOADS["tiny"]
+    assert line["config"] == bench.bench_config(wl, list(wl.Ms), 1, False)

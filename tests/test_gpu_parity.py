@@ -98,6 +98,7 @@ def test_tied_and_negative_infinite_logits(tiny):
     logits[1, :] = -float("inf")
     logits[1, 5] = 1.0
     logits[1, 2] = 1.0
+    logits[2, :] = -float("inf")              # no finite logit: weight 1/k each
     out = tiny.run(x, logits)
     check_routing(tiny, logits, M)
     ref, _ = oracle_full(tiny, x, logits, fp8=False)

@@ -85,6 +85,21 @@ def test_route_negative_infinity_logits():
     assert list(ids[1]) == [0, 2, 5]
 
 
+def test_route_row_of_only_negative_infinity_is_the_equal_logit_limit():
+    # no finite softmax exists; the row must equal the limit of a row of equal
+    # finite logits: the k lowest ids, each with weight 1/k
+    logits = np.full((3, 6), -np.inf, dtype=np.float32)
+    logits[1] = np.float32(-3.0e38)
+    logits[2, 4] = 0.0
+    ids, w = O.route(logits, 4)
+    assert list(ids[0]) == [0, 1, 2, 3]
+    np.testing.assert_array_equal(ids[0], ids[1])
+    np.testing.assert_allclose(w[0], np.full(4, 0.25), rtol=0, atol=0)
+    np.testing.assert_allclose(w[0], w[1], rtol=0, atol=1e-15)
+    assert np.all(np.isfinite(w))
+    assert list(ids[2]) == [4, 0, 1, 2] and w[2, 0] == 1.0 and np.all(w[2, 1:] == 0.0)
+
+
 def brute_permute(ids, E):
     flat = ids.ravel().tolist()
     counts, order = [], []
