@@ -516,6 +516,67 @@ def measure_workload(name, layer, wl, dtype, Ms, toks, stream, flush, args, hbm_
     return entry
 
 
+ROPE_SHAPE = {"NH": 16, "D": 128, "max_pos": 32768, "Ts": (1, 64, 4096, 16384)}
+
+
+def measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on):
+    """The inverse-RoPE + per-head FP8 quantisation kernel at several token counts (one
+    kernel for all of them): device time per call with L2 flushed before each, and the
+    achieved HBM bandwidth over its algorithmic bytes (2D bytes in, D codes + a 4-byte
+    scale out per vector, a 4-byte position per token)."""
+    import numpy as np
+    import torch
+    from mixture_experts_layer_sort_b200 import inv_rope_fp8_quant
+    NH, D, max_pos = ROPE_SHAPE["NH"], ROPE_SHAPE["D"], ROPE_SHAPE["max_pos"]
+    i = torch.arange(D // 2, dtype=torch.float64)
+    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * (10000.0 ** (-2.0 * i / D))[None, :]
+    table = torch.cat([torch.cos(ang), torch.sin(ang)], dim=1).float().to(dev)
+    g = torch.Generator(device=dev).manual_seed(seed)
+    steps = max(5, min(args.steps, 20))
+    per_T = {}
+    for T in ROPE_SHAPE["Ts"]:
+        x = torch.randn((T, NH, D), generator=g, device=dev).to(torch.bfloat16)
+        pos = torch.randint(0, max_pos, (T,), generator=g, device=dev, dtype=torch.int32)
+        codes = torch.empty((T, NH, D), dtype=torch.uint8, device=dev)
+        scales = torch.empty((T, NH), dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                inv_rope_fp8_quant(x, pos, table, codes=codes, scales=scales, stream=stream)
+            ev = []
+            for _ in range(steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                inv_rope_fp8_quant(x, pos, table, codes=codes, scales=scales, stream=stream)
+                e1.record(stream)
+                ev.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = sorted(a.elapsed_time(b) for a, b in ev)
+        mean = statistics.mean(ms)
+        alg = T * NH * (2 * D + D + 4) + T * 4
+        per_T[str(T)] = {"us": mean * 1e3, "us_p50": statistics.median(ms) * 1e3, "alg_MB": alg / 1e6,
+                         "GBps": alg / (mean / 1e3) / 1e9, "frac_hbm": alg / (mean / 1e3) / 1e9 / hbm_gbs}
+    entry = {"workload": f"inverse RoPE + per-head e4m3 quantisation, [T, {NH} heads, {D}] bf16, half-split "
+                         f"pairs, one launch per T in {list(ROPE_SHAPE['Ts'])}",
+             "per_T": per_T, "bound": "hbm", "peak_GBps": hbm_gbs}
+    if cpu_on:
+        from oracle import rope_oracle as R
+        T = 4096
+        x = torch.randn((T, NH, D), generator=g, device=dev).to(torch.bfloat16).float().cpu().numpy()
+        pos = torch.randint(0, max_pos, (T,), generator=g, device=dev, dtype=torch.int32).cpu().numpy()
+        tab = table.cpu().numpy()
+        t0 = time.time()
+        reps = 0
+        while reps < 3 or time.time() - t0 < 2.0:
+            R.inv_rope_fp8_quant(x, pos, tab)
+            reps += 1
+            if time.time() - t0 > 10.0:
+                break
+        entry["cpu_baseline"] = {"value": T * reps / (time.time() - t0), "unit": "tokens/s", "kind": "oracle",
+                                 "cores": 1, "sample": f"{reps} calls at T={T}"}
+    return entry
+
+
 def extra_workloads(args, dev, stream, flush, dec_weights, seed, hbm_gbs, bf16_tf, cpu_on):
     """Decode FP8 (from the decode weights), large decode and prefill bf16 + FP8 (from one
     E=256 bf16 weight set), each measured like the headline."""
@@ -556,6 +617,7 @@ def extra_workloads(args, dev, stream, flush, dec_weights, seed, hbm_gbs, bf16_t
                                           hbm_gbs, bf16_tf)
     big8.close()
     torch.cuda.empty_cache()
+    res["inv_rope_fp8"] = measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on)
     return res
 
 

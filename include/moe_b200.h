@@ -91,6 +91,26 @@ MOE_API int moe_destroy(moe_layer* layer);
 MOE_API int moe_load_weights(moe_layer* layer, const void* w_gate, const void* w_up,
                      const void* w_down, void* stream);
 
+/* Tensor parallelism over the expert intermediate dimension: load shard `shard` of
+ * `num_shards` of a layer whose full intermediate size is I_full = I * num_shards (the
+ * handle was created with I = I_full / num_shards). The pages run the layer at
+ * eight-way tensor parallelism (toolboxkart.tech, "AWS SageMaker MoE kernel
+ * optimizations H200", section "3. Removing repeat compilation can reduce first-token
+ * delay"). From the FULL bf16 tensors (device pointers)
+ *   w_gate [E, I_full, H], w_up [E, I_full, H], w_down [E, H, I_full]
+ * the handle keeps rows [shard*I, (shard+1)*I) of every W_gate[e] and W_up[e] and the
+ * matching columns [shard*I, (shard+1)*I) of every W_down[e]. SwiGLU acts on each
+ * intermediate feature alone and the down projection sums over them, so the layer's
+ * output is the SUM of the shards' outputs (combined by an all-reduce across the
+ * ranks that hold them). Routing depends only on the logits and is the same on every
+ * shard. An FP8 handle quantises its own slice: one scale per (expert, tensor) of the
+ * slice, and its own per-tensor scale of h over its slice of h.
+ * Synchronises `stream`. Returns MOE_ERR_INVALID_ARG when I * num_shards != I_full or
+ * the shard index is out of range. */
+MOE_API int moe_load_weights_shard(moe_layer* layer, const void* w_gate, const void* w_up,
+                                   const void* w_down, int I_full, int shard, int num_shards,
+                                   void* stream);
+
 /* Load already-quantised weights into an FP8 layer (device pointers):
  *   q_gate [E, I, H], q_up [E, I, H], q_down [E, H, I] (uint8 codes in the layer's
  *   format, e4m3 or e5m2) and
@@ -151,6 +171,34 @@ MOE_API int moe_forward_host(moe_layer* layer, const void* x_host, const float* 
  *     untouched. */
 MOE_API int moe_forward_noalloc(moe_layer* layer, const void* x, const float* router_logits, int M,
                                 void* out, void* stream);
+
+/* Inverse rotary position embedding fused with per-head FP8 quantisation, for any
+ * number of tokens (a run-time argument: one precompiled kernel per head size, nothing
+ * compiled or specialised per token count). The pages name this kernel,
+ * _fused_inv_rope_fp8_quant_per_head, as the one that was recompiled for every new
+ * token count until that specialisation was removed (toolboxkart.tech, "AWS SageMaker
+ * MoE kernel optimizations H200", section "3. Removing repeat compilation can reduce
+ * first-token delay"; aib.vote, "AWS SageMaker MoE kernel optimizations", fourth
+ * paragraph). No layer handle is needed; it runs on the current device.
+ *   x         [num_tokens, num_heads, head_dim] bf16 (device), rotated by RoPE
+ *   positions [num_tokens] int32 (device): the position of each token
+ *   cos_sin   [max_pos, head_dim] fp32 (device): row p holds cos of the head_dim/2
+ *             angles of position p, then their sin
+ *   codes     [num_tokens, num_heads, head_dim] uint8 (device), written: FP8 codes
+ *   scales    [num_tokens, num_heads] fp32 (device), written: one scale per vector
+ * Per (token, head) vector y = x rotated back: for each pair (a', b') with the
+ * angle's c, s:  a = a'c + b's,  b = b'c - a's (each product, sum and difference
+ * rounded to fp32 in that order); pairs are (i, i + head_dim/2) when interleaved = 0,
+ * (2i, 2i + 1) when interleaved = 1. Then scale = max|y| / F (F = 448 for
+ * fp8_format = MOE_DTYPE_FP8_E4M3, 57344 for MOE_DTYPE_FP8_E5M2; 1 when y is all
+ * zero) and codes = RNE(y / scale) saturated, the division in IEEE fp32.
+ * A position outside [0, max_pos) gives codes 0 and scale NaN for that token (no
+ * out-of-bounds read). head_dim must be 64, 128 or 256; x, cos_sin and codes 16-byte
+ * aligned. num_tokens = 0 is a no-op. Asynchronous on `stream`; the caller owns every
+ * buffer. Returns MOE_ERR_INVALID_ARG for a bad size, format or pointer. */
+MOE_API int moe_inv_rope_fp8_quant(const void* x, const int* positions, const float* cos_sin, int max_pos,
+                                   int num_tokens, int num_heads, int head_dim, int interleaved,
+                                   int fp8_format, void* codes, float* scales, void* stream);
 
 /* Select the single-launch decode path for this handle (enable = 1) or the default
  * kernel chain (enable = 0). The single-launch path runs a whole bf16 forward of up

@@ -6,11 +6,11 @@ binding over it plus seeded input generators. Importing the package does not
 load the library: ``MoELayer`` does, and raises if it is missing.
 """
 
-__all__ = ["MoELayer", "load_library", "MoEError"]
+__all__ = ["MoELayer", "load_library", "MoEError", "inv_rope_fp8_quant"]
 
 
 def __getattr__(name):
-    if name in ("MoELayer", "MoEError"):
+    if name in ("MoELayer", "MoEError", "inv_rope_fp8_quant"):
         from . import layer
         return getattr(layer, name)
     if name == "load_library":

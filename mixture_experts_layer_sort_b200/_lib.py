@@ -19,6 +19,8 @@ SIGNATURES = {
     "moe_destroy": (_c_int, [_c_void_p]),
     "moe_load_weights": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "moe_load_weights_fp8": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "moe_load_weights_shard": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
+                                        _c_void_p]),
     "moe_reserve": (_c_int, [_c_void_p, _c_int, _c_void_p]),
     "moe_forward": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "moe_forward_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p]),
@@ -33,6 +35,8 @@ SIGNATURES = {
                                    _c_void_p, ctypes.POINTER(ctypes.c_int)]),
     "moe_debug_activations": (_c_int, [_c_void_p, _c_void_p, _c_void_p]),
     "moe_debug_weights": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "moe_inv_rope_fp8_quant": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                        _c_int, _c_void_p, _c_void_p, _c_void_p]),
 }
 
 _lib = None

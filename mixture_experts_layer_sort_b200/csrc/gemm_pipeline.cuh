@@ -175,9 +175,16 @@ __device__ __forceinline__ Unit make_unit(const Tile& t, int tile, int s, int S,
   return make_unit_range(t, tile, s * kblocks / S, (s + 1) * kblocks / S, S, n_cap);
 }
 
-// The units of CTA blockIdx.x (of gridDim.x) over a tile list in global memory
-// written by the align kernel; count() of them, unit(i) in the order every role of
-// the CTA walks them. Two ways of dealing them out, chosen by S:
+// Tile t of a tile list in global memory (written by the align kernel).
+struct GlobalTileFn {
+  const Tile* tiles;
+  __device__ __forceinline__ Tile operator()(int t) const { return tiles[t]; }
+};
+
+// The units of CTA blockIdx.x (of gridDim.x) over T tiles given by a tile function
+// (a list in global memory, or a schedule held in shared memory); count() of them,
+// unit(i) in the order every role of the CTA walks them. Two ways of dealing them
+// out, chosen by S:
 //  - S >= 1: each tile is cut into S equal K ranges and the T*S units go round-robin.
 //  - S == 0, balanced: the T tiles minus the last one to two waves go round-robin as
 //    whole tiles. The K blocks of the remaining tiles are cut into one contiguous
@@ -185,8 +192,9 @@ __device__ __forceinline__ Unit make_unit(const Tile& t, int tile, int s, int S,
 //    same weight bytes whatever T is. A tile whose K blocks fall into the ranges of
 //    several CTAs is a split tile with S = that number of CTAs. A CTA takes its range
 //    first, so that the split tiles' partial-sum fix-ups overlap the whole tiles.
-struct GlobalTiles {
-  const Tile* tiles;
+template <class TileFn>
+struct UnitSchedule {
+  TileFn tiles;
   int T, S, K;
   int bal_tiles;           // tiles [0, bal_tiles) form the balanced region
   int g_bal;               // CTAs that share it (each with a non-empty range)
@@ -196,7 +204,7 @@ struct GlobalTiles {
 
   // The balanced region holds fewer than two waves of tiles of at most 256 K blocks,
   // so c * bal_total stays far below 2^31 for any grid of up to a few hundred CTAs.
-  __device__ __forceinline__ GlobalTiles(const Tile* tiles_, int T_, int S_, int K_)
+  __device__ __forceinline__ UnitSchedule(TileFn tiles_, int T_, int S_, int K_)
       : tiles(tiles_), T(T_), S(S_), K(K_), bal_tiles(0), g_bal(0), bal_total(0), x0(0), x1(0), n_bal(0),
         n_whole(0) {
     if (S != 0 || T <= 0 || K <= 0) return;
@@ -225,7 +233,7 @@ struct GlobalTiles {
     if (S != 0) {
       const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
       const int t = u / S;
-      return make_unit(tiles[t], t, u - t * S, S, K, n_cap);
+      return make_unit(tiles(t), t, u - t * S, S, K, n_cap);
     }
     if (i < n_bal) {
       const int t = x0 / K + i;
@@ -234,11 +242,16 @@ struct GlobalTiles {
       const int kb1 = t == last / K ? last - t * K + 1 : K;
       const int first = t * K;
       const int sharers = owner(first + K - 1) - owner(first) + 1;
-      return make_unit_range(tiles[t], t, kb0, kb1, sharers, n_cap);
+      return make_unit_range(tiles(t), t, kb0, kb1, sharers, n_cap);
     }
     const int t = bal_tiles + static_cast<int>(blockIdx.x) + (i - n_bal) * static_cast<int>(gridDim.x);
-    return make_unit_range(tiles[t], t, 0, K, 1, n_cap);
+    return make_unit_range(tiles(t), t, 0, K, 1, n_cap);
   }
+};
+
+struct GlobalTiles : UnitSchedule<GlobalTileFn> {
+  __device__ __forceinline__ GlobalTiles(const Tile* tiles_, int T_, int S_, int K_)
+      : UnitSchedule<GlobalTileFn>(GlobalTileFn{tiles_}, T_, S_, K_) {}
 };
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
@@ -255,6 +268,9 @@ struct ProducerState {
 //   int dep(const Unit&)  - key of the activation operand's dependency
 //   bool ready(int dep)   - non-blocking check
 //   bool wait(int dep)    - blocking (bounded) wait; false when it gave up
+//   bool direct()         - activation rows are single rows of a [tokens, K] tensor
+//                           (one-row TMA boxes) instead of 16-row boxes of a permuted one
+//   int direct_token(const Unit&, int j) - in direct mode, the tensor row of column j
 template <class C, class Src, class Hooks>
 __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const CUtensorMap* tm_b, const Shared& sh,
                              const Ring& rg, const Src& src, Hooks& hk, ProducerState& ps, volatile int* abort_flag,
@@ -269,9 +285,10 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
   // direct mode: x row (token) of activation rows lane, lane+32, lane+64, lane+96 of
   // the current unit; pad rows re-read row 0 (their columns are never stored)
   int tok[4] = {0, 0, 0, 0};
+  const bool direct = hk.direct();
   auto load_b = [&](int stg, int kc, int row_start, int nb) {
     uint8_t* bdst = sh.ring + stg * rg.stage_bytes + C::kATiles * C::kABytes;
-    if (a.direct_pairs == nullptr) {
+    if (!direct) {
       for (int j = lane; j < nb; j += 32)
         tma_load_2d(bdst + j * 16 * kRowBytes, tm_b, &sh.full[stg], kc, row_start + 16 * j, pol_b);
     } else {
@@ -333,12 +350,12 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
         ps.failed = true;
         break;
       }
-      if (a.direct_pairs != nullptr && kb == un.kb0) {
+      if (direct && kb == un.kb0) {
         // the unit's token rows, read while its first weight tiles are in flight
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int j = lane + 32 * i;
-          tok[i] = j < un.t.n_valid ? __ldcg(a.direct_pairs + un.t.row_start + j) / a.k : 0;
+          tok[i] = j < un.t.n_valid ? hk.direct_token(un, j) : 0;
         }
       }
       const int kc = kb * C::kKPerBlock;
@@ -467,8 +484,9 @@ struct EpiState {
 // Hooks:
 //   column(const Unit&, int j, float scale, int& tok, float& w) - down: token row and
 //        scaled routing weight of column j
-//   static constexpr bool kSignalTiles; tile_done(const Unit&, int epi_tid) - gate_up:
-//        called by every epilogue thread once the tile's h rows are written and fenced
+//   static constexpr bool kSignalTiles; tile_done(const Unit&, int epi_tid, float lmax) -
+//        gate_up: called by every epilogue thread once the tile's h rows are written
+//        (lmax: the thread's running max |h|, FP8)
 //   static constexpr bool kTokenCompletion; down_done(const Unit&, const int* s_tok,
 //        int epi_tid) - down: called by every epilogue thread after the unit's adds
 template <class C, bool kGateUp, bool kFP8, class Src, class Hooks>
@@ -480,8 +498,9 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
   const int epi_tid = threadIdx.x - 64;
   float sx = 1.f, sh_scale = 1.f;
   if constexpr (kFP8) {
-    sx = fp8_scale_from_amax(*a.amax_x, a.f8);
-    if constexpr (!kGateUp) sh_scale = fp8_scale_from_amax(*a.amax_h, a.f8);
+    // written by other CTAs (or kernels): read from L2, not a possibly stale L1 line
+    sx = fp8_scale_from_amax(__ldcg(a.amax_x), a.f8);
+    if constexpr (!kGateUp) sh_scale = fp8_scale_from_amax(__ldcg(a.amax_h), a.f8);
   }
   const int n_units = src.count();
   for (int i = 0; i < n_units && !es.failed; ++i) {
@@ -603,7 +622,7 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
         }
       }
       if constexpr (Hooks::kSignalTiles) {
-        if (wrote) hk.tile_done(un, epi_tid);
+        if (wrote) hk.tile_done(un, epi_tid, es.lmax);
       }
     } else {
       // rows of the first weight block go to features f*256 + row, the second block's

@@ -1,33 +1,41 @@
-// kernels_decode.cu - the whole MoE layer for a decode batch (M <= 64 tokens, bf16)
-// in ONE persistent, cooperative launch: routing, the grouping of (token, slot) pairs
-// by expert, the gather of x into expert order, the gate_up GEMM with SwiGLU, the
-// down GEMM with the routing-weight scatter-add, and the conversion of the finished
-// token rows to bf16.
+// kernels_decode.cu - the whole MoE layer for a decode batch (M <= 64 tokens, bf16 or
+// FP8) in ONE persistent, cooperative launch: routing, the grouping of (token, slot)
+// pairs by expert, the gate_up GEMM with SwiGLU, the down GEMM with the routing-weight
+// scatter-add, and the conversion of the finished token rows to bf16.
 //
 // Fused MoE kernels "combine routing, data movement and expert calculations into
 // fewer GPU operations", cutting launch overhead and intermediate traffic
 // (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "Why MoE
-// inference needs specialized kernels"); at decode sizes the separate kernels' own
-// latency, not bandwidth, dominates, and this kernel removes it.
+// inference needs specialized kernels"). At decode sizes the weights of the selected
+// experts are the only large traffic, and what decides the time is how soon after the
+// launch they start streaming and how little waiting is left once they have arrived.
 //
-// How one launch replaces the chain:
-// - CTA t routes token t and publishes its top-k; once all M tokens are published,
-//   every CTA builds the permutation and both tile schedules itself, in shared
-//   memory. The order inside an expert (ascending token, i.e. ascending pair id)
-//   comes from a per-expert 64-bit token mask.
-// - CTA c gathers rows c, c+G, ... of x into expert order, then bumps a counter.
-// - The gate_up units start streaming weights at once; a unit's activation loads
-//   wait (bounded) until all CTAs have gathered. Each finished gate_up tile bumps its
-//   expert's "h ready" counter.
+// How one launch replaces the chain, per CTA (one per SM, all resident):
+// - Every CTA routes all M tokens itself (the logits are staged in shared memory
+//   first, so that the loads overlap) and builds the grouping and both unit schedules
+//   in shared memory: no CTA waits for another to learn the routing. The order inside
+//   an expert (ascending token, i.e. ascending pair id) comes from a per-expert 64-bit
+//   token mask.
+// - gate_up streams weights at once. Its activation operand is read straight from
+//   the token rows with one-row TMA boxes (no gathered copy): bf16 layers read x;
+//   FP8 layers read e4m3/e5m2 codes of x that CTA t writes for token t once every
+//   token's max |x| is in (two grid counters the producer waits on, bounded, while
+//   the first weight tiles are already in flight).
+// - Each finished gate_up tile bumps its expert's "h ready" counter (and, FP8, a
+//   global count of finished tiles after folding its max |h| into the amax word).
 // - A CTA moves on to its down units as soon as it has issued its gate_up work:
-//   W_down streams in while other CTAs finish gate_up; a down unit's activation
-//   loads wait until every gate_up tile of its expert is done.
-// - The down epilogue adds into the fp32 accumulator and counts, per token, the
-//   contributions still missing; the CTA that completes a token converts its row to
-//   bf16 and re-zeroes it. The last CTA to finish resets the counters.
+//   W_down streams in while other CTAs finish gate_up. bf16: a down unit's activation
+//   loads wait until every gate_up tile of its expert is done. FP8: s_h needs every
+//   h row, so once all gate_up tiles are done each CTA converts its share of the h
+//   rows to codes, and the down activation loads wait for all shares (the FP8 h
+//   quantisation of the chain, without its launch or its extra pass over h).
+// - The down epilogue adds into the fp32 accumulator and counts, per token, the K
+//   blocks added so far; the CTA that completes a token converts its row to bf16 and
+//   re-zeroes it. The last CTA to finish resets the counters.
 // All CTAs must be resident at once (they wait on each other): the launch is
 // cooperative, one CTA per SM. Every wait is bounded and reports through the error
 // word when it gives up.
+#include "fp8_format.cuh"
 #include "gemm_pipeline.cuh"
 #include "route_common.cuh"
 
@@ -36,31 +44,41 @@ namespace moe {
 namespace {
 
 using namespace pipe;
-using C = Cfg<false>;
 
 constexpr int kMaxTokens = 64;     // per-expert token masks are 64 bits
 constexpr int kMaxPairs = 512;
 constexpr int kMaxExperts = 512;
+constexpr int kBalancedWaves = 8;  // as in the chain's align kernel
 
-// Global sync words (zero between launches):
-//   [0] CTAs that finished their gather, [1] CTAs that finished everything,
-//   [2] tokens routed, [3, 3+E) gate_up tiles finished per expert,
-//   [3+E, 3+E+M) down contributions per token
+// Global sync words (zero between launches; the last CTA resets them):
+enum SyncSlot : int {
+  kSyncDone = 0,       // CTAs that finished everything
+  kSyncGateDone = 1,   // FP8: gate_up tiles finished (all experts)
+  kSyncXMax = 2,       // FP8: tokens whose max |x| is folded into the amax word
+  kSyncXq = 3,         // FP8: token rows of x quantised
+  kSyncHq = 4,         // FP8: CTAs that converted their share of h
+  kSyncAmaxX = 5,      // FP8: max |x| (float bits)
+  kSyncAmaxH = 6,      // FP8: max |h| (float bits)
+  kSyncFixed = 8       // then expert_ready [E], then token K-block counts [M]
+};
+
 struct DecodeArgs {
   const float* logits;
   const __nv_bfloat16* x;
   __nv_bfloat16* out;
   int M, E, k, H, I, P;
-  int ws1_rows_cap, max_stages;
+  int ws1_rows_cap, max_stages, f8;
   int* sync;
-  __nv_bfloat16* x_perm;
-  // copies of the routing for inspection (written by CTA 0)
+  uint8_t* xq;             // FP8: [M, H] codes of x
+  uint8_t* hq;             // FP8: [rows, I] codes of h (the down GEMM's activation)
+  // copies of the routing for inspection (written by CTA 0 at the end)
   int* topk_ids;
   float* topk_w;
   int* counts;
   int* padded_offsets;
   int* padded_pairs;
   int* header;
+  float* last_scales;      // FP8: s_x, s_h of this forward
   GemmArgs g1, g2;
 };
 
@@ -70,15 +88,16 @@ struct Sched {
   float w[kMaxPairs];
   int count[kMaxExperts];
   int off[kMaxExperts + 1];       // compact offsets of each expert's pairs
-  int poff[kMaxExperts + 1];      // padded offsets (rows of x_perm / h)
+  int poff[kMaxExperts + 1];      // padded offsets (rows of h)
   int tmp[kMaxExperts + 1];
   int act[kMaxExperts];           // active experts, ascending
   int aidx[kMaxExperts + 1];      // index of each expert among the active ones
   unsigned mask[kMaxExperts][2];  // tokens routed to each expert
   int pairs[kMaxPairs];           // pair ids grouped by expert, ascending inside an expert
   int done[256];                  // tokens completed by the current down unit
+  float red[8];                   // block reduction scratch
   int ndone;
-  int nact, T1, S1, T2, S2, n_max, rows_used, last_cta;
+  int nact, T1, S1, T2, S2, n_max, rows_used, flag;
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -91,28 +110,43 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Units of one GEMM computed from the shared schedule: tile t = (active expert t / fb,
-// row block t % fb); every expert has a single token tile (n_e <= M <= 64).
-struct SmemTiles {
+// Tile t of a GEMM from the shared schedule: tile t = (active expert t / fb, row block
+// t % fb); every expert has a single token tile (n_e <= M <= 64).
+struct SmemTileFn {
   const Sched* s;
-  int fb, T, S, kblocks;
-  // units u = blockIdx.x + i * gridDim.x of the T*S, round-robin
-  __device__ __forceinline__ int count() const {
-    const int n = T * S, c = static_cast<int>(blockIdx.x);
-    return c < n ? (n - 1 - c) / static_cast<int>(gridDim.x) + 1 : 0;
-  }
-  __device__ __forceinline__ Unit unit(int i, int n_cap) const {
-    const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
-    const int t = u / S;
+  int fb;
+  __device__ __forceinline__ Tile operator()(int t) const {
     const int ai = t / fb;
     Tile tile;
     tile.expert = s->act[ai];
     tile.fblock = t - ai * fb;
     tile.row_start = s->poff[tile.expert];
     tile.n_valid = s->count[tile.expert];
-    return make_unit(tile, t, u - t * S, S, kblocks, n_cap);
+    return tile;
   }
 };
+
+// Bounded wait of one thread until *p >= target (acquire); false when it gave up.
+__device__ __forceinline__ bool wait_counter(const int* p, int target, volatile int* abort_flag) {
+  if (ld_acquire(p) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire(p) >= target) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > (1ll << 31)) return false;
+  }
+}
+
+// Warp-uniform: lane 0 checks *p >= target (acquire); every lane gets the answer, and
+// on success every lane orders its later TMA reads after the producers' writes.
+__device__ __forceinline__ bool warp_poll(const int* p, int target) {
+  int v = 0;
+  if ((threadIdx.x & 31) == 0) v = ld_acquire(p) >= target ? 1 : 0;
+  v = __shfl_sync(0xFFFFFFFFu, v, 0);
+  if (v) fence_proxy_async_global();
+  return v != 0;
+}
 
 // Bounded spin of the producer warp on a condition read by lane 0.
 template <class F>
@@ -129,76 +163,82 @@ __device__ __forceinline__ bool spin_until(F cond, volatile int* abort_flag) {
   }
 }
 
-// gate_up: activation rows come from x_perm, complete once every CTA gathered.
+// gate_up: activation rows are token rows of x (bf16) or of its codes (FP8; ready
+// once all M rows are written).
+template <bool kFP8>
 struct GateUpHooks {
   const DecodeArgs* d;
-  int grid;
+  const Sched* s;
   int* expert_ready;
   volatile int* abort_flag;
-  bool gathered = false;
+  bool xready = !kFP8;
   static constexpr bool kSignalTiles = true;
   static constexpr bool kTokenCompletion = false;
+  __device__ __forceinline__ bool direct() const { return true; }
+  __device__ __forceinline__ int direct_token(const Unit& un, int j) const {
+    return s->pairs[s->off[un.t.expert] + j] / d->k;
+  }
   __device__ __forceinline__ int dep(const Unit&) const { return 0; }
   __device__ __forceinline__ bool ready(int) {
-    if (gathered) return true;
-    int v = 0;
-    if ((threadIdx.x & 31) == 0) v = ld_acquire(d->sync) >= grid ? 1 : 0;
-    v = __shfl_sync(0xFFFFFFFFu, v, 0);
-    if (v) {
-      (void)ld_acquire(d->sync);     // every lane observes it before its TMA reads
-      fence_proxy_async_global();
-      gathered = true;
-    }
-    return gathered;
+    if (!xready) xready = warp_poll(d->sync + kSyncXq, d->M);
+    return xready;
   }
   __device__ __forceinline__ bool wait(int dd) {
     if (ready(dd)) return true;
-    const int* p = d->sync;
-    const int g = grid;
-    if (!spin_until([p, g]() { return ld_acquire(p) >= g; }, abort_flag)) return false;
+    const int* p = d->sync + kSyncXq;
+    const int m = d->M;
+    if (!spin_until([p, m]() { return ld_acquire(p) >= m; }, abort_flag)) return false;
     return ready(dd);
   }
   __device__ __forceinline__ void column(const Unit&, int, float, int&, float&) const {}
-  // every epilogue thread: its h stores of the tile are visible (also to TMA reads)
-  // before the expert's counter moves
-  __device__ __forceinline__ void tile_done(const Unit& un, int epi_tid) {
+  // every epilogue thread: its h stores of the tile (and, FP8, its max |h| so far) are
+  // visible, also to TMA reads, before the counters move
+  __device__ __forceinline__ void tile_done(const Unit& un, int epi_tid, float lmax) {
+    if constexpr (kFP8) {
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xFFFFFFFFu, lmax, o));
+      if ((threadIdx.x & 31) == 0 && lmax > 0.f)
+        atomicMax(reinterpret_cast<unsigned*>(d->sync + kSyncAmaxH), __float_as_uint(lmax));
+    }
     fence_proxy_async_global();
     __threadfence();
     named_bar_sync(1, kEpiThreads);
-    if (epi_tid == 0) atomicAdd(expert_ready + un.t.expert, 1);
+    if (epi_tid == 0) {
+      __threadfence();
+      atomicAdd(expert_ready + un.t.expert, 1);
+      if constexpr (kFP8) atomicAdd(d->sync + kSyncGateDone, 1);
+    }
   }
   __device__ __forceinline__ void down_done(const Unit&, const int*, int) {}
 };
 
-// down: activation rows of expert e come from h, complete once all its gate_up
-// tiles are done; tokens are converted by whoever adds their last contribution.
+// down: activation rows of expert e come from h (bf16: complete once all its gate_up
+// tiles are done) or from its codes (FP8: complete once every CTA converted its
+// share); tokens are converted by whoever adds their last K block.
+template <bool kFP8>
 struct DownHooks {
   const DecodeArgs* d;
   Sched* s;
   int* expert_ready;
   int* token_cnt;
-  int fb1, need;      // gate_up tiles per expert; down contributions per token
+  int fb1, need, grid;   // gate_up tiles per expert; K blocks added per token; CTAs
   volatile int* abort_flag;
   int last_ready = -1;
   static constexpr bool kSignalTiles = false;
   static constexpr bool kTokenCompletion = true;
-  __device__ __forceinline__ int dep(const Unit& un) const { return un.t.expert; }
+  __device__ __forceinline__ bool direct() const { return false; }
+  __device__ __forceinline__ int direct_token(const Unit&, int) const { return 0; }
+  __device__ __forceinline__ int dep(const Unit& un) const { return kFP8 ? 0 : un.t.expert; }
   __device__ __forceinline__ bool ready(int e) {
     if (e == last_ready) return true;
-    int v = 0;
-    if ((threadIdx.x & 31) == 0) v = ld_acquire(expert_ready + e) >= fb1 ? 1 : 0;
-    v = __shfl_sync(0xFFFFFFFFu, v, 0);
-    if (v) {
-      (void)ld_acquire(expert_ready + e);
-      fence_proxy_async_global();
-      last_ready = e;
-    }
-    return v != 0;
+    const bool v = kFP8 ? warp_poll(d->sync + kSyncHq, grid) : warp_poll(expert_ready + e, fb1);
+    if (v) last_ready = e;
+    return v;
   }
   __device__ __forceinline__ bool wait(int e) {
     if (ready(e)) return true;
-    const int* p = expert_ready + e;
-    const int f = fb1;
+    const int* p = kFP8 ? d->sync + kSyncHq : expert_ready + e;
+    const int f = kFP8 ? grid : fb1;
     if (!spin_until([p, f]() { return ld_acquire(p) >= f; }, abort_flag)) return false;
     return ready(e);
   }
@@ -207,15 +247,16 @@ struct DownHooks {
     tok = p / d->k;
     w = s->w[p] * scale;
   }
-  __device__ __forceinline__ void tile_done(const Unit&, int) {}
+  __device__ __forceinline__ void tile_done(const Unit&, int, float) {}
   __device__ __forceinline__ void down_done(const Unit& un, const int* s_tok, int epi_tid) {
     __threadfence();                        // this unit's adds happen before the counts move
     named_bar_sync(1, kEpiThreads);
     if (epi_tid == 0) s->ndone = 0;
     named_bar_sync(1, kEpiThreads);
+    const int add = un.kb1 - un.kb0;
     for (int j = epi_tid; j < un.t.n_valid; j += kEpiThreads) {
       const int t = s_tok[j];
-      if (atomicAdd(token_cnt + t, 1) == need - 1) s->done[atomicAdd(&s->ndone, 1)] = t;
+      if (atomicAdd(token_cnt + t, add) == need - add) s->done[atomicAdd(&s->ndone, 1)] = t;
     }
     named_bar_sync(1, kEpiThreads);
     const int nd = s->ndone;
@@ -243,10 +284,42 @@ struct DownHooks {
   }
 };
 
+// 8 fp32 values -> 8 FP8 codes (RNE, saturating), v[i] / s with IEEE division.
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, int f8) {
+  unsigned short c[4];
+  #pragma unroll
+  for (int q = 0; q < 4; ++q) c[q] = fp8x2(make_float2(__fdiv_rn(v[2 * q], s), __fdiv_rn(v[2 * q + 1], s)), f8);
+  uint2 r;
+  r.x = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
+  r.y = static_cast<unsigned>(c[2]) | (static_cast<unsigned>(c[3]) << 16);
+  return r;
+}
+
+// One row of n bf16 values -> codes, by the 128 epilogue threads (n % 8 == 0).
+__device__ __forceinline__ void quant_row(const __nv_bfloat16* src, uint8_t* dst, int n, float s, int f8,
+                                          int epi_tid) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint2* d2 = reinterpret_cast<uint2*>(dst);
+  for (int i = epi_tid; i < n / 8; i += kEpiThreads) {
+    const uint4 u = __ldcg(s4 + i);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+    float f[8];
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 v = __bfloat1622float2(p[q]);
+      f[2 * q] = v.x;
+      f[2 * q + 1] = v.y;
+    }
+    d2[i] = quant8(f, s, f8);
+  }
+}
+
+template <bool kFP8>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_decode_kernel(const __grid_constant__ DecodeArgs d, const __grid_constant__ CUtensorMap tm_w13,
                         const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_h) {
+  using C = Cfg<kFP8>;
   extern __shared__ uint8_t smem_raw[];
   const Shared sh = carve<C>(smem_raw, sizeof(Sched));
   Sched* s = reinterpret_cast<Sched*>(sh.extra);
@@ -255,10 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
   const int G = gridDim.x;
+  const int c = blockIdx.x;
   const int E = d.E, M = d.M, k = d.k, P = d.P;
-  int* route_cnt = d.sync + 2;
-  int* expert_ready = d.sync + 3;
-  int* token_cnt = d.sync + 3 + E;
+  int* expert_ready = d.sync + kSyncFixed;
+  int* token_cnt = expert_ready + E;
   if (tid == 0) {
     tma_prefetch_desc(&tm_w13);
     tma_prefetch_desc(&tm_wd);
@@ -267,42 +340,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const uint32_t tmem = prologue<C>(sh, warp);
 
-  // ---------------------------------------------------------------- routing
-  // CTA c routes tokens c, c+G, ... and publishes them; then everyone reads all
-  for (int t = blockIdx.x; t < M; t += G) {
-    if (warp == 0)
-      route_token_any(d.logits + static_cast<size_t>(t) * E, E, k, lane, d.topk_ids + t * k, d.topk_w + t * k);
+  // ---------------------------------------------------------------- routing, in every CTA
+  // the logits go to shared memory first (all loads in flight together), staged in the
+  // stage ring, which is not in use yet (M * E * 4 <= 128 KB < ring bytes)
+  float* s_logits = reinterpret_cast<float*>(sh.ring);
+  const int n_logits = M * E;
+  for (int i0 = tid; i0 < n_logits; i0 += kThreads * 8) {
+    float v[8];
+    #pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (i0 + j * kThreads < n_logits) v[j] = __ldg(d.logits + i0 + j * kThreads);
+    #pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (i0 + j * kThreads < n_logits) s_logits[i0 + j * kThreads] = v[j];
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int mine = blockIdx.x < M ? (M - 1 - static_cast<int>(blockIdx.x)) / G + 1 : 0;
-    if (mine > 0) atomicAdd(route_cnt, mine);
+  if constexpr (kFP8) {
+    // CTA t < M: max |x| of token t into the amax word
+    if (c < M) {
+      const uint4* xr = reinterpret_cast<const uint4*>(d.x + static_cast<size_t>(c) * d.H);
+      float m = 0.f;
+      for (int i = tid; i < d.H / 8; i += kThreads) {
+        const uint4 u = __ldg(xr + i);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+        #pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(p[q]);
+          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+      }
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (lane == 0) s->red[warp] = m;
+    }
   }
   for (int e = tid; e < E; e += kThreads) {
     s->count[e] = 0;
     s->mask[e][0] = 0u;
     s->mask[e][1] = 0u;
   }
-  if (tid == 0) {
-    const long long t0 = clock64();
-    int ok = 1;
-    while (ld_acquire(route_cnt) < M) {
-      if (clock64() - t0 > (1ll << 31)) {
-        ok = 0;
-        break;
-      }
-      __nanosleep(32);
-    }
-    if (!ok) report_error(d.g1.err, kErrWaitGrid);
-    s->last_cta = ok;                       // reused below as "routing complete"
-  }
   __syncthreads();
-  const bool routed = s->last_cta != 0;
-  for (int p = tid; p < P; p += kThreads) {
-    s->ids[p] = routed ? __ldcg(d.topk_ids + p) : 0;
-    s->w[p] = routed ? __ldcg(d.topk_w + p) : 0.f;
+  if constexpr (kFP8) {
+    if (c < M && tid == 0) {
+      float m = 0.f;
+      for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, s->red[w]);
+      if (m > 0.f) atomicMax(reinterpret_cast<unsigned*>(d.sync + kSyncAmaxX), __float_as_uint(m));
+      __threadfence();
+      atomicAdd(d.sync + kSyncXMax, 1);
+    }
   }
+  for (int t = warp; t < M; t += kThreads / 32)
+    route_token_any(s_logits + static_cast<size_t>(t) * E, E, k, lane, s->ids + t * k, s->w + t * k);
   __syncthreads();
   for (int p = tid; p < P; p += kThreads) {
     const int e = s->ids[p];
@@ -341,7 +428,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int fb2 = (d.H / kTileRows + 1) / 2;
   const int kb1 = d.H / C::kKPerBlock;
   const int kb2 = d.I / C::kKPerBlock;
-  __syncthreads();
   if (warp == 0) {
     int m = 0;
     for (int e = lane; e < E; e += 32) m = max(m, s->count[e]);
@@ -351,8 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rows_used = s->poff[E];
     const int n_mean = A > 0 ? (P + A - 1) / A : 0;
     const int t1 = A * fb1;
-    const int s1 = choose_splits_warp(t1, kb1, G, rows_used <= d.ws1_rows_cap, 2 * 16384 + n_mean * 128,
-                                      n_mean * 256 * 4 * 2, lane);
+    // the chain's rule: the balanced schedule (0) for one to kBalancedWaves waves of
+    // tiles when the partial sums fit, else the cost model's split factor
+    const bool allow = rows_used <= d.ws1_rows_cap;
+    const int s1 = (allow && t1 >= G && t1 < kBalancedWaves * G)
+                       ? 0
+                       : choose_splits_warp(t1, kb1, G, allow, 2 * 16384 + n_mean * 128, n_mean * 256 * 4 * 2, lane);
     if (lane == 0) {
       s->n_max = (m + kPadRows - 1) / kPadRows * kPadRows;
       s->rows_used = rows_used;
@@ -363,16 +453,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int A = s->nact;
     const int n_mean = A > 0 ? (P + A - 1) / A : 0;
     const int t2 = A * fb2;
-    const int s2 = choose_splits_warp(t2, kb2, G, true, 2 * 16384 + n_mean * 128, n_mean * 128 * 4, lane);
+    const int s2 = (t2 >= G && t2 < kBalancedWaves * G)
+                       ? 0
+                       : choose_splits_warp(t2, kb2, G, true, 16384 + n_mean * 128, n_mean * 128 * 4, lane);
     if (lane == 0) {
       s->T2 = t2;
       s->S2 = s2;
     }
   }
-  __syncthreads();
+  // the staged logits are dead from here on: order their generic-proxy accesses before
+  // the TMA writes that reuse the ring
+  fence_proxy_async_smem();
+  __syncthreads();   // the schedule is complete
 
-  // copies of the grouping for inspection
-  if (blockIdx.x == 0) {
+  // ---------------------------------------------------------------- both GEMMs
+  const Ring rg = make_ring<C>(s->n_max, d.max_stages, sh.ring_bytes);
+  const UnitSchedule<SmemTileFn> src1(SmemTileFn{s, fb1}, s->T1, s->S1, kb1);
+  const UnitSchedule<SmemTileFn> src2(SmemTileFn{s, fb2}, s->T2, s->S2, kb2);
+  GateUpHooks<kFP8> h1{&d, s, expert_ready, abort_flag};
+  DownHooks<kFP8> h2{&d, s, expert_ready, token_cnt, fb1, k * fb2 * kb2, G, abort_flag};
+
+  if (warp == 0) {
+    ProducerState ps;
+    run_producer<C>(d.g1, &tm_w13, &tm_x, sh, rg, src1, h1, ps, abort_flag, lane);
+    if (!ps.failed) run_producer<C>(d.g2, &tm_wd, &tm_h, sh, rg, src2, h2, ps, abort_flag, lane);
+    producer_quiesce<C>(sh, rg, ps, lane);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      MmaState ms;
+      run_mma<C, kFP8>(d.g1, sh, rg, src1, ms, tmem, abort_flag);
+      if (!ms.failed) run_mma<C, kFP8>(d.g2, sh, rg, src2, ms, tmem, abort_flag);
+    }
+  } else {
+    const int epi_tid = tid - 64;
+    volatile int* okf = sh.flags + 2;
+    bool ok = true;
+    if constexpr (kFP8) {
+      // x codes: once every token's max |x| is in, CTA t < M quantises token row t;
+      // every CTA needs the final amax before its gate_up epilogue scales by s_x
+      if (epi_tid == 0) *okf = wait_counter(d.sync + kSyncXMax, M, abort_flag) ? 1 : 0;
+      named_bar_sync(1, kEpiThreads);
+      ok = *okf != 0;
+      if (ok && c < M) {
+        const float sx = fp8_scale_from_amax(__ldcg(reinterpret_cast<const unsigned*>(d.sync + kSyncAmaxX)), d.f8);
+        quant_row(d.x + static_cast<size_t>(c) * d.H, d.xq + static_cast<size_t>(c) * d.H, d.H, sx, d.f8, epi_tid);
+        fence_proxy_async_global();
+        __threadfence();
+        named_bar_sync(1, kEpiThreads);
+        if (epi_tid == 0) atomicAdd(d.sync + kSyncXq, 1);
+      }
+      if (!ok && epi_tid == 0) {
+        report_error(d.g1.err, kErrWaitGrid);
+        *abort_flag = 1;
+      }
+    }
+    EpiState es;
+    es.failed = !ok;
+    if (ok) run_epilogue<C, true, kFP8>(d.g1, sh, rg, src1, h1, es, tmem, abort_flag, warp, lane);
+    if constexpr (kFP8) {
+      // h codes: s_h is final once every gate_up tile is done; this CTA converts the
+      // valid h rows c, c + G, ...
+      if (!es.failed) {
+        named_bar_sync(1, kEpiThreads);
+        if (epi_tid == 0) *okf = wait_counter(d.sync + kSyncGateDone, s->T1, abort_flag) ? 1 : 0;
+        named_bar_sync(1, kEpiThreads);
+        if (*okf == 0) {
+          if (epi_tid == 0) {
+            report_error(d.g1.err, kErrWaitGrid);
+            *abort_flag = 1;
+          }
+          es.failed = true;
+        }
+      }
+      if (!es.failed) {
+        const float shs = fp8_scale_from_amax(__ldcg(reinterpret_cast<const unsigned*>(d.sync + kSyncAmaxH)), d.f8);
+        for (int r = c; r < s->rows_used; r += G) {
+          int lo = 0, hi = s->nact - 1;                 // active expert whose padded rows hold r
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s->poff[s->act[mid]] <= r) lo = mid;
+            else hi = mid - 1;
+          }
+          const int e = s->act[lo];
+          if (r - s->poff[e] >= s->count[e]) continue;  // a pad row: never read by a stored column
+          quant_row(d.g1.h + static_cast<size_t>(r) * d.I, d.hq + static_cast<size_t>(r) * d.I, d.I, shs, d.f8,
+                    epi_tid);
+        }
+        fence_proxy_async_global();
+        __threadfence();
+        named_bar_sync(1, kEpiThreads);
+        if (epi_tid == 0) atomicAdd(d.sync + kSyncHq, 1);
+      }
+    }
+    if (!es.failed) run_epilogue<C, false, kFP8>(d.g2, sh, rg, src2, h2, es, tmem, abort_flag, warp, lane);
+  }
+  teardown<C>(tmem, warp);
+
+  // ---------------------------------------------------------------- copies for inspection
+  if (c == 0) {
+    for (int p = tid; p < P; p += kThreads) {
+      d.topk_ids[p] = s->ids[p];
+      d.topk_w[p] = s->w[p];
+    }
     for (int e = tid; e < E; e += kThreads) {
       d.counts[e] = s->count[e];
       d.padded_offsets[e] = s->poff[e];
@@ -384,70 +566,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       d.padded_offsets[E] = s->poff[E];
       d.header[kHdrRowsUsed] = s->rows_used;
+      if constexpr (kFP8) {
+        d.last_scales[0] = fp8_scale_from_amax(__ldcg(reinterpret_cast<const unsigned*>(d.sync + kSyncAmaxX)), d.f8);
+        d.last_scales[1] = fp8_scale_from_amax(__ldcg(reinterpret_cast<const unsigned*>(d.sync + kSyncAmaxH)), d.f8);
+      }
     }
   }
-
-  // ---------------------------------------------------------------- gather
-  // this CTA's rows of x in expert order (pad rows are never read by a stored column)
-  for (int r = blockIdx.x + warp * G; r < s->rows_used; r += G * (kThreads / 32)) {
-    int lo = 0, hi = s->nact - 1;                 // active expert whose padded rows hold r
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s->poff[s->act[mid]] <= r) lo = mid;
-      else hi = mid - 1;
-    }
-    const int e = s->act[lo];
-    const int j = r - s->poff[e];
-    if (j >= s->count[e]) continue;
-    const int tok = s->pairs[s->off[e] + j] / k;
-    const uint4* src = reinterpret_cast<const uint4*>(d.x + static_cast<size_t>(tok) * d.H);
-    uint4* dst = reinterpret_cast<uint4*>(d.x_perm + static_cast<size_t>(r) * d.H);
-    for (int i = lane; i < d.H / 8; i += 32) dst[i] = __ldg(src + i);
-  }
-  fence_proxy_async_global();
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) atomicAdd(d.sync, 1);
-
-  // ---------------------------------------------------------------- both GEMMs
-  const Ring rg = make_ring<C>(s->n_max, d.max_stages, sh.ring_bytes);
-  const SmemTiles src1{s, fb1, s->T1, s->S1, kb1};
-  const SmemTiles src2{s, fb2, s->T2, s->S2, kb2};
-  GateUpHooks h1{&d, G, expert_ready, abort_flag};
-  DownHooks h2{&d, s, expert_ready, token_cnt, fb1, k * fb2 * s->S2, abort_flag};
-
-  if (warp == 0) {
-    ProducerState ps;
-    run_producer<C>(d.g1, &tm_w13, &tm_x, sh, rg, src1, h1, ps, abort_flag, lane);
-    if (!ps.failed) run_producer<C>(d.g2, &tm_wd, &tm_h, sh, rg, src2, h2, ps, abort_flag, lane);
-    producer_quiesce<C>(sh, rg, ps, lane);
-  } else if (warp == 1) {
-    if (lane == 0) {
-      MmaState ms;
-      run_mma<C, false>(d.g1, sh, rg, src1, ms, tmem, abort_flag);
-      if (!ms.failed) run_mma<C, false>(d.g2, sh, rg, src2, ms, tmem, abort_flag);
-    }
-  } else {
-    EpiState es;
-    run_epilogue<C, true, false>(d.g1, sh, rg, src1, h1, es, tmem, abort_flag, warp, lane);
-    if (!es.failed) run_epilogue<C, false, false>(d.g2, sh, rg, src2, h2, es, tmem, abort_flag, warp, lane);
-  }
-  teardown<C>(tmem, warp);
 
   // ---------------------------------------------------------------- last CTA resets
+  __syncthreads();
   if (tid == 0) {
     __threadfence();
-    s->last_cta = atomicAdd(d.sync + 1, 1) == G - 1 ? 1 : 0;
+    s->flag = atomicAdd(d.sync + kSyncDone, 1) == G - 1 ? 1 : 0;
   }
   __syncthreads();
-  if (s->last_cta) {
+  if (s->flag) {
     __threadfence();
     for (int e = tid; e < E; e += kThreads) expert_ready[e] = 0;
     for (int t = tid; t < M; t += kThreads) token_cnt[t] = 0;
     if (tid == 0) {
-      d.sync[0] = 0;
-      d.sync[1] = 0;
-      d.sync[2] = 0;
+      for (int i = 1; i < kSyncFixed; ++i) d.sync[i] = 0;
+      __threadfence();
+      d.sync[kSyncDone] = 0;
     }
   }
 }
@@ -456,10 +596,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool decode_supported(int M, int E, int k) { return M >= 1 && M <= kMaxTokens && E <= kMaxExperts && M * k <= kMaxPairs; }
 
-size_t decode_sync_words(int E, int M_cap) { return static_cast<size_t>(3 + E + M_cap); }
+size_t decode_sync_words(int E, int M_cap) { return static_cast<size_t>(kSyncFixed + E + M_cap); }
 
 cudaError_t decode_configure() {
-  return cudaFuncSetAttribute(fused_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<false>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(fused_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<true>::kSmemBytes);
 }
 
 cudaError_t launch_decode(const DecodeLaunch& l, cudaStream_t st) {
@@ -475,27 +619,34 @@ cudaError_t launch_decode(const DecodeLaunch& l, cudaStream_t st) {
   d.P = l.M * l.k;
   d.ws1_rows_cap = l.ws1_rows_cap;
   d.max_stages = l.max_stages;
+  d.f8 = l.f8;
   d.sync = l.sync;
-  d.x_perm = l.x_perm;
+  d.xq = l.xq;
+  d.hq = l.hq;
   d.topk_ids = l.topk_ids;
   d.topk_w = l.topk_w;
   d.counts = l.counts;
   d.padded_offsets = l.padded_offsets;
   d.padded_pairs = l.padded_pairs;
   d.header = l.header;
+  d.last_scales = l.last_scales;
   d.g1 = l.g1;
   d.g2 = l.g2;
+  // the FP8 amax words live in the sync block (reset by the kernel's last CTA)
+  d.g1.amax_x = d.g2.amax_x = reinterpret_cast<unsigned*>(l.sync + kSyncAmaxX);
+  d.g1.amax_h = d.g2.amax_h = reinterpret_cast<unsigned*>(l.sync + kSyncAmaxH);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(l.grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.dynamicSmemBytes = l.fp8 ? Cfg<true>::kSmemBytes : Cfg<false>::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fused_decode_kernel, d, *l.tm_w13, *l.tm_wd, *l.tm_x, *l.tm_h);
+  if (l.fp8) return cudaLaunchKernelEx(&cfg, fused_decode_kernel<true>, d, *l.tm_w13, *l.tm_wd, *l.tm_x, *l.tm_h);
+  return cudaLaunchKernelEx(&cfg, fused_decode_kernel<false>, d, *l.tm_w13, *l.tm_wd, *l.tm_x, *l.tm_h);
 }
 
 }  // namespace moe

@@ -38,7 +38,11 @@ struct PdlHooks {
     tok = p / a->k;
     w = __ldg(a->topk_w + p) * scale;
   }
-  __device__ __forceinline__ void tile_done(const Unit&, int) {}
+  __device__ __forceinline__ bool direct() const { return a->direct_pairs != nullptr; }
+  __device__ __forceinline__ int direct_token(const Unit& un, int j) const {
+    return __ldcg(a->direct_pairs + un.t.row_start + j) / a->k;
+  }
+  __device__ __forceinline__ void tile_done(const Unit&, int, float) {}
   __device__ __forceinline__ void down_done(const Unit&, const int*, int) {}
 };
 

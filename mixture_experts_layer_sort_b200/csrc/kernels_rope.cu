@@ -1,0 +1,234 @@
+// kernels_rope.cu - inverse rotary position embedding fused with per-head FP8
+// quantisation, for any number of tokens (a run-time argument: one precompiled kernel
+// per head size, nothing specialised or rebuilt per token count).
+//
+// The pages name this kernel, `_fused_inv_rope_fp8_quant_per_head`, as the one that
+// used to be recompiled for every new token count, costing time to first token at
+// eight-way tensor parallelism until its variable-length parameters were kept out of
+// the specialisation (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200",
+// section "3. Removing repeat compilation can reduce first-token delay"; aib.vote,
+// "AWS SageMaker MoE kernel optimizations", fourth paragraph). They give only the
+// name; what it computes here, per (token t, head h) vector of D values:
+//   1. undo the rotation by the angles of position p = positions[t]: for each pair
+//      (a', b') and its angle's c = cos, s = sin from the table row p
+//      (cos in columns [0, D/2), sin in [D/2, D)):  a = a'c + b's,  b = b'c - a's,
+//      each product, sum and difference rounded to fp32 in that order;
+//      pairs are (i, i + D/2) (half-split) or (2i, 2i + 1) (interleaved);
+//   2. one FP8 scale per vector: s = max|y| / F (F = 448 e4m3, 57344 e5m2; 1 for an
+//      all-zero vector), codes = RNE(y / s) saturated, the division in IEEE fp32.
+// A position outside [0, max_pos) has no table row: its vector gets codes 0 and a
+// NaN scale (no out-of-bounds read).
+//
+// Layout and roofline: one warp per vector, lane l holding D/32 consecutive values (so
+// a warp's load of a vector is one coalesced 2D-byte access and the half-split
+// partner of lane l is lane l ^ 16); four vectors per warp are in flight at once. The
+// kernel moves 2D bytes in and D + 4 bytes out per vector (the table rows are shared
+// by a token's heads and stay in cache): it is HBM-bound.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <type_traits>
+
+#include "../../include/moe_b200.h"
+#include "fp8_format.cuh"
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRopeThreads = 256;
+constexpr int kRopeUnroll = 4;     // vectors per warp in flight
+
+struct RopeArgs {
+  const __nv_bfloat16* x;   // [T, NH, D]
+  const int* positions;     // [T]
+  const float* cos_sin;     // [max_pos, D]
+  uint8_t* codes;           // [T, NH, D]
+  float* scales;            // [T, NH]
+  long long nvec;           // T * NH
+  int NH, max_pos, f8;
+  int interleaved;
+};
+
+template <int CH>
+struct Vec {
+  float v[CH];
+};
+
+// CH consecutive bf16 values (4, 8 or 16 bytes) -> fp32
+template <int CH>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&v)[CH]) {
+  if constexpr (CH == 2) {
+    const __nv_bfloat162 u = *reinterpret_cast<const __nv_bfloat162*>(p);
+    const float2 f = __bfloat1622float2(u);
+    v[0] = f.x;
+    v[1] = f.y;
+  } else {
+    using U = typename std::conditional<CH == 4, uint2, uint4>::type;
+    const U u = __ldg(reinterpret_cast<const U*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+    #pragma unroll
+    for (int q = 0; q < CH / 2; ++q) {
+      const float2 f = __bfloat1622float2(h[q]);
+      v[2 * q] = f.x;
+      v[2 * q + 1] = f.y;
+    }
+  }
+}
+
+template <int CH>
+__device__ __forceinline__ void load_f32(const float* p, float (&v)[CH]) {
+  #pragma unroll
+  for (int q = 0; q < CH; q += 2) {
+    const float2 f = __ldg(reinterpret_cast<const float2*>(p + q));
+    v[q] = f.x;
+    v[q + 1] = f.y;
+  }
+}
+
+template <int CH>
+__device__ __forceinline__ void store_codes(uint8_t* p, const unsigned short (&c)[CH / 2]) {
+  if constexpr (CH == 2) {
+    *reinterpret_cast<unsigned short*>(p) = c[0];
+  } else if constexpr (CH == 4) {
+    *reinterpret_cast<unsigned*>(p) = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
+  } else {
+    uint2 o;
+    o.x = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
+    o.y = static_cast<unsigned>(c[2]) | (static_cast<unsigned>(c[3]) << 16);
+    *reinterpret_cast<uint2*>(p) = o;
+  }
+}
+
+// D = 32 * CH values per vector.
+template <int CH>
+__global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) {
+  constexpr int D = 32 * CH;
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const long long gwarp = (static_cast<long long>(blockIdx.x) * kRopeThreads + threadIdx.x) >> 5;
+  const long long nwarps = static_cast<long long>(gridDim.x) * (kRopeThreads / 32);
+  const float fmax = fp8_max(a.f8);
+  // angle index of this lane's first value: half-split pairs value i with i + D/2
+  // (angle i mod D/2), interleaved pairs 2i with 2i + 1 (angle i)
+  const int ang0 = a.interleaved ? lane * CH / 2 : (lane & 15) * CH;
+  const bool upper = lane >= 16;   // half-split: this lane holds the b' of its pairs
+  for (long long v0 = gwarp * kRopeUnroll; v0 < a.nvec; v0 += nwarps * kRopeUnroll) {
+    float x[kRopeUnroll][CH];
+    int pos[kRopeUnroll];
+    #pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const long long v = v0 + u;
+      pos[u] = -1;
+      if (v < a.nvec) {
+        load_bf16<CH>(a.x + v * D + lane * CH, x[u]);
+        pos[u] = __ldg(a.positions + v / a.NH);
+      }
+    }
+    #pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const long long v = v0 + u;
+      if (v >= a.nvec) break;   // warp-uniform
+      const bool valid = pos[u] >= 0 && pos[u] < a.max_pos;
+      float y[CH];
+      if (valid) {
+        const float* row = a.cos_sin + static_cast<long long>(pos[u]) * D;
+        if (a.interleaved) {
+          float c[CH / 2], s[CH / 2];
+          #pragma unroll
+          for (int q = 0; q < CH / 2; ++q) {
+            c[q] = __ldg(row + ang0 + q);
+            s[q] = __ldg(row + D / 2 + ang0 + q);
+          }
+          #pragma unroll
+          for (int q = 0; q < CH / 2; ++q) {
+            const float pa = x[u][2 * q], pb = x[u][2 * q + 1];
+            y[2 * q] = __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
+            y[2 * q + 1] = __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]));
+          }
+        } else {
+          float c[CH], s[CH];
+          load_f32<CH>(row + ang0, c);
+          load_f32<CH>(row + D / 2 + ang0, s);
+          #pragma unroll
+          for (int q = 0; q < CH; ++q) {
+            const float other = __shfl_xor_sync(0xFFFFFFFFu, x[u][q], 16);
+            const float pa = upper ? other : x[u][q];
+            const float pb = upper ? x[u][q] : other;
+            y[q] = upper ? __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]))
+                         : __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
+          }
+        }
+      } else {   // (valid is the same for the whole warp: the shuffles above stay uniform)
+        #pragma unroll
+        for (int q = 0; q < CH; ++q) y[q] = 0.f;
+      }
+      float m = 0.f;
+      #pragma unroll
+      for (int q = 0; q < CH; ++q) m = fmaxf(m, fabsf(y[q]));
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      const float sc = m == 0.f ? 1.f : __fdiv_rn(m, fmax);
+      unsigned short cd[CH / 2];
+      #pragma unroll
+      for (int q = 0; q < CH / 2; ++q)
+        cd[q] = valid ? fp8x2(make_float2(__fdiv_rn(y[2 * q], sc), __fdiv_rn(y[2 * q + 1], sc)), a.f8)
+                      : static_cast<unsigned short>(0);
+      store_codes<CH>(a.codes + v * D + lane * CH, cd);
+      if (lane == 0) a.scales[v] = valid ? sc : __int_as_float(0x7FC00000);
+    }
+  }
+}
+
+template <int CH>
+cudaError_t launch_rope(const RopeArgs& a, cudaStream_t s) {
+  const long long per_block = (kRopeThreads / 32) * kRopeUnroll;
+  long long blocks = (a.nvec + per_block - 1) / per_block;
+  const long long cap = 8ll * sm_count();
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_kernel(inv_rope_fp8_kernel<CH>, dim3(static_cast<unsigned>(blocks)), dim3(kRopeThreads), 0, s, a);
+}
+
+bool aligned(const void* p, unsigned bytes) { return (reinterpret_cast<uintptr_t>(p) & (bytes - 1)) == 0; }
+
+}  // namespace
+
+}  // namespace moe
+
+extern "C" int moe_inv_rope_fp8_quant(const void* x, const int* positions, const float* cos_sin, int max_pos,
+                                      int num_tokens, int num_heads, int head_dim, int interleaved, int fp8_format,
+                                      void* codes, float* scales, void* stream) {
+  if (num_tokens < 0 || num_heads < 1 || max_pos < 1 || (interleaved != 0 && interleaved != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return MOE_ERR_INVALID_ARG;
+  if (fp8_format != MOE_DTYPE_FP8_E4M3 && fp8_format != MOE_DTYPE_FP8_E5M2) return MOE_ERR_INVALID_ARG;
+  if (num_tokens == 0) return MOE_OK;
+  if (!x || !positions || !cos_sin || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  if (!moe::aligned(x, 16) || !moe::aligned(cos_sin, 16) || !moe::aligned(codes, 16) || !moe::aligned(positions, 4) ||
+      !moe::aligned(scales, 4))
+    return MOE_ERR_INVALID_ARG;
+  moe::RopeArgs a{};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.positions = positions;
+  a.cos_sin = cos_sin;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = scales;
+  a.nvec = static_cast<long long>(num_tokens) * num_heads;
+  a.NH = num_heads;
+  a.max_pos = max_pos;
+  a.f8 = fp8_format == MOE_DTYPE_FP8_E5M2 ? moe::kFp8E5M2 : moe::kFp8E4M3;
+  a.interleaved = interleaved;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = head_dim == 64 ? moe::launch_rope<2>(a, st)
+                                 : (head_dim == 128 ? moe::launch_rope<4>(a, st) : moe::launch_rope<8>(a, st));
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "moe_inv_rope_fp8_quant: launch failed: %s\n", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}

@@ -25,13 +25,22 @@ __device__ __forceinline__ long long tiled_offset(const TileGeom& g, long long e
   return (tile * 128 + (r & 127)) * 128 + (byte & 127);
 }
 
-__global__ void __launch_bounds__(1024) weight_amax_kernel(int f8, const __nv_bfloat16* w, long long per_expert,
-                                                           float* scales, int stride) {
+// Byte offset, in the row-major side, of byte `b` of row r of expert e.
+__device__ __forceinline__ long long rowmajor_offset(const TileGeom& g, long long e, long long r, long long b) {
+  return e * g.src_expert_stride + r * g.src_row_stride + g.src_offset + b;
+}
+
+// scales[e * stride] = amax of expert e's rows (bf16, row-major side of g; K = row_bytes
+// elements per row, the stored layout being FP8) / the format's largest finite value.
+__global__ void __launch_bounds__(1024) weight_amax_kernel(int f8, const uint8_t* w, TileGeom g, float* scales,
+                                                           int stride) {
   const int e = blockIdx.x;
-  const uint4* src = reinterpret_cast<const uint4*>(w + static_cast<size_t>(e) * per_expert);
+  const long long per_row = g.row_bytes / 8;       // 16-byte vectors of 8 bf16 per row
   float m = 0.f;
-  for (long long i = threadIdx.x; i < per_expert / 8; i += blockDim.x) {
-    const uint4 u = __ldg(src + i);
+  for (long long i = threadIdx.x; i < g.rows * per_row; i += blockDim.x) {
+    const long long r = i / per_row;
+    const long long c = (i - r * per_row) * 16;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(w + rowmajor_offset(g, e, r, c)));
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
     #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -53,7 +62,7 @@ __global__ void __launch_bounds__(1024) weight_amax_kernel(int f8, const __nv_bf
 }
 
 // 8 bf16 -> 8 FP8 codes (8 bytes) per thread, written at their tiled position.
-__global__ void __launch_bounds__(256) weight_quant_tiled_kernel(int f8, const __nv_bfloat16* w, TileGeom g,
+__global__ void __launch_bounds__(256) weight_quant_tiled_kernel(int f8, const uint8_t* w, TileGeom g,
                                                                  const float* scales, int stride, uint8_t* dst) {
   const long long K = g.row_bytes;                 // FP8: one byte per element
   const long long per_row = K / 8;
@@ -64,7 +73,8 @@ __global__ void __launch_bounds__(256) weight_quant_tiled_kernel(int f8, const _
     const long long e = row / g.rows;
     const long long r = row - e * g.rows;
     const float s = __ldg(scales + e * stride);
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(w) + i);
+    // 8 bf16 source values = 16 bytes at column c of the row-major source
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(w + rowmajor_offset(g, e, r, 2 * c)));
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
     unsigned short c2[4];
     #pragma unroll
@@ -91,8 +101,9 @@ __global__ void __launch_bounds__(256) retile_kernel(const uint8_t* src, TileGeo
     const long long e = row / g.rows;
     const long long r = row - e * g.rows;
     const long long t = tiled_offset(g, e, r, b);
-    if constexpr (kToTiled) *reinterpret_cast<uint4*>(dst + t) = __ldg(reinterpret_cast<const uint4*>(src) + i);
-    else reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(src + t);
+    const long long m = rowmajor_offset(g, e, r, b);
+    if constexpr (kToTiled) *reinterpret_cast<uint4*>(dst + t) = __ldg(reinterpret_cast<const uint4*>(src + m));
+    else *reinterpret_cast<uint4*>(dst + m) = *reinterpret_cast<const uint4*>(src + t);
   }
 }
 
@@ -104,15 +115,16 @@ int grid_for(long long work) {
 
 }  // namespace
 
-cudaError_t launch_weight_amax(int f8, const __nv_bfloat16* w, long long per_expert, int E, float* scales,
-                               int stride, cudaStream_t s) {
-  weight_amax_kernel<<<E, 1024, 0, s>>>(f8, w, per_expert, scales, stride);
+cudaError_t launch_weight_amax(int f8, const __nv_bfloat16* w, const TileGeom& g, float* scales, int stride,
+                               cudaStream_t s) {
+  weight_amax_kernel<<<g.E, 1024, 0, s>>>(f8, reinterpret_cast<const uint8_t*>(w), g, scales, stride);
   return cudaGetLastError();
 }
 
 cudaError_t launch_weight_quant_tiled(int f8, const __nv_bfloat16* w, const TileGeom& g, const float* scales,
                                       int stride, uint8_t* dst, cudaStream_t s) {
-  weight_quant_tiled_kernel<<<grid_for(g.E * g.rows * (g.row_bytes / 8)), 256, 0, s>>>(f8, w, g, scales, stride, dst);
+  weight_quant_tiled_kernel<<<grid_for(g.E * g.rows * (g.row_bytes / 8)), 256, 0, s>>>(
+      f8, reinterpret_cast<const uint8_t*>(w), g, scales, stride, dst);
   return cudaGetLastError();
 }
 

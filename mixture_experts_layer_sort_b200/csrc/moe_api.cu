@@ -65,6 +65,7 @@ struct moe_layer {
   uint8_t* xq = nullptr;        // FP8 large batches: x quantised per token [M_cap, H]
   long long chunks_cap = 0;
   CUtensorMap tm_x{}, tm_h{};
+  CUtensorMap tm_xq{};          // FP8 single-launch decode: token rows of xq, one-row boxes
   // staging for moe_forward_host
   void* hx = nullptr;
   float* hl = nullptr;
@@ -240,6 +241,7 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(encode_map(&L->tm_x, L->x_perm, is_fp8(L), L->H, L->rows_cap, 16));
   MOE_TRY(encode_map(&L->tm_h, is_fp8(L) ? static_cast<void*>(L->h_q) : static_cast<void*>(L->h), is_fp8(L),
                      L->I, L->rows_cap, 16));
+  if (is_fp8(L)) MOE_TRY(encode_map(&L->tm_xq, L->xq, true, L->H, cap, 1));
   L->M_cap = cap;
   return MOE_OK;
 }
@@ -254,8 +256,12 @@ int encode_weight_maps(moe_layer* L) {
   return MOE_OK;
 }
 
-// Tile geometry of the three stored tensors: W_gate and W_up share w13 (up rows after gate rows).
-moe::TileGeom geom(const moe_layer* L, int which) {
+// Tile geometry of the three stored tensors: W_gate and W_up share w13 (up rows after
+// gate rows). The row-major side has elements of src_el bytes (2 for a bf16 source, 1
+// for FP8 codes) and is the full tensor of I_full intermediate features, of which the
+// handle holds shard `shard` of I_full / I: rows [shard*I, (shard+1)*I) of W_gate and
+// W_up, columns [shard*I, (shard+1)*I) of W_down. A whole tensor is shard 0 of I.
+moe::TileGeom geom(const moe_layer* L, int which, long long src_el, long long I_full, int shard) {
   const long long el = is_fp8(L) ? 1 : 2;
   moe::TileGeom g{};
   g.E = L->E;
@@ -264,13 +270,41 @@ moe::TileGeom geom(const moe_layer* L, int which) {
     g.row_bytes = L->H * el;
     g.rb_total = 2 * L->I / moe::kTileRows;
     g.rb_offset = which == 0 ? 0 : L->I / moe::kTileRows;
+    g.src_row_stride = L->H * src_el;
+    g.src_expert_stride = I_full * L->H * src_el;
+    g.src_offset = static_cast<long long>(shard) * L->I * L->H * src_el;
   } else {
     g.rows = L->H;
     g.row_bytes = L->I * el;
     g.rb_total = L->H / moe::kTileRows;
     g.rb_offset = 0;
+    g.src_row_stride = I_full * src_el;
+    g.src_expert_stride = L->H * I_full * src_el;
+    g.src_offset = static_cast<long long>(shard) * L->I * src_el;
   }
   return g;
+}
+
+moe::TileGeom geom(const moe_layer* L, int which) {
+  return geom(L, which, is_fp8(L) ? 1 : 2, L->I, 0);
+}
+
+// Weights of shard `shard` (I_full = I * shards) from bf16 sources: tiled copies, or
+// per-(expert, tensor) scales and codes of the shard's own slice (FP8).
+int load_bf16_sources(moe_layer* L, const void* const src[3], long long I_full, int shard, cudaStream_t st) {
+  void* dst[3] = {L->w13, L->w13, L->wd};
+  for (int j = 0; j < 3; ++j) {
+    const moe::TileGeom g = geom(L, j, 2, I_full, shard);
+    if (!is_fp8(L)) {
+      MOE_CUDA(moe::launch_tile_weights(src[j], g, dst[j], st));
+    } else {
+      const auto* w = static_cast<const __nv_bfloat16*>(src[j]);
+      MOE_CUDA(moe::launch_weight_amax(fp8_format(L), w, g, L->wscales + j, 3, st));
+      MOE_CUDA(moe::launch_weight_quant_tiled(fp8_format(L), w, g, L->wscales + j, 3, static_cast<uint8_t*>(dst[j]),
+                                              st));
+    }
+  }
+  return MOE_OK;
 }
 
 cudaEvent_t pool_event(moe_layer* L) {
@@ -328,6 +362,16 @@ bool direct_x_disabled() {
   return off;
 }
 
+// Whether new handles take the single-launch decode path for the batches it supports
+// (MOE_FUSED_DECODE=0 or 1 overrides the default).
+bool fused_decode_default() {
+  static const bool on = [] {
+    const char* e = std::getenv("MOE_FUSED_DECODE");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
+}
+
 int decode_stage_cap() {
   static const int cap = [] {
     const char* e = std::getenv("MOE_MAX_STAGES_DECODE");
@@ -336,8 +380,14 @@ int decode_stage_cap() {
   return cap;
 }
 
-// The whole layer of a small bf16 batch in one cooperative launch.
+// The whole layer of a decode batch in one cooperative launch.
 int forward_fused_decode(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
+  const bool fp8 = is_fp8(L);
+  const int kper = fp8 ? 128 : 64;
+  // gate_up reads token rows with one-row boxes: of the caller's x (bf16), or of the
+  // codes of x the kernel writes into the workspace (FP8; map encoded with it)
+  CUtensorMap tm_xd{};
+  if (!fp8) MOE_TRY(encode_map(&tm_xd, x, false, L->H, M, 1));
   moe::DecodeLaunch d{};
   d.logits = logits;
   d.x = static_cast<const __nv_bfloat16*>(x);
@@ -350,8 +400,12 @@ int forward_fused_decode(moe_layer* L, const void* x, const float* logits, int M
   d.grid = L->num_sms;
   d.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
   d.max_stages = decode_stage_cap();
+  d.fp8 = fp8;
+  d.f8 = fp8_format(L);
   d.sync = L->sync;
-  d.x_perm = static_cast<__nv_bfloat16*>(L->x_perm);
+  d.xq = L->xq;
+  d.hq = L->h_q;
+  d.last_scales = L->last_scales;
   d.topk_ids = L->topk_ids;
   d.topk_w = L->topk_w;
   d.counts = L->counts;
@@ -368,19 +422,21 @@ int forward_fused_decode(moe_layer* L, const void* x, const float* logits, int M
   g.k = L->k;
   g.P = M * L->k;
   g.err = L->err;
+  g.w_scales = L->wscales;
+  g.f8 = fp8_format(L);
   d.g1 = g;
-  d.g1.kblocks = L->H / 64;
+  d.g1.kblocks = L->H / kper;
   d.g1.w_rblocks = 2 * L->I / moe::kTileRows;
   d.g1.rb_step = 1;
   d.g1.second_rb = L->I / moe::kTileRows;
   d.g2 = g;
-  d.g2.kblocks = L->I / 64;
+  d.g2.kblocks = L->I / kper;
   d.g2.w_rblocks = L->H / moe::kTileRows;
   d.g2.rb_step = 2;
   d.g2.second_rb = 1;
   d.tm_w13 = &L->tm_w13;
   d.tm_wd = &L->tm_wd;
-  d.tm_x = &L->tm_x;
+  d.tm_x = fp8 ? &L->tm_xq : &tm_xd;
   d.tm_h = &L->tm_h;
   {
     KernelTimer kt(L, 3, st);
@@ -412,7 +468,7 @@ constexpr long long kAlignSingleBlockMaxPairs = 8192;
 
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
-  if (L->fused_decode && !is_fp8(L) && moe::decode_supported(M, L->E, L->k))
+  if (L->fused_decode && M <= L->num_sms && moe::decode_supported(M, L->E, L->k))
     return forward_fused_decode(L, x, logits, M, out, st);
   const bool fp8 = is_fp8(L);
   const long long P = static_cast<long long>(M) * L->k;
@@ -704,6 +760,7 @@ int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
   L->dtype = dtype;
   L->device = dev;
   L->num_sms = prop.multiProcessorCount;
+  L->fused_decode = fused_decode_default();
   const size_t el = dtype == MOE_DTYPE_BF16 ? 2 : 1;
   if (cudaMalloc(&L->w13, static_cast<size_t>(E) * 2 * I * H * el) != cudaSuccess ||
       cudaMalloc(&L->wd, static_cast<size_t>(E) * H * I * el) != cudaSuccess ||
@@ -747,19 +804,26 @@ int moe_load_weights(moe_layer* L, const void* w_gate, const void* w_up, const v
   if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
   DeviceGuard g(L->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t IH = static_cast<size_t>(L->I) * L->H;
   L->loaded = false;
   const void* src[3] = {w_gate, w_up, w_down};
-  void* dst[3] = {L->w13, L->w13, L->wd};
-  if (!is_fp8(L)) {
-    for (int j = 0; j < 3; ++j) MOE_CUDA(moe::launch_tile_weights(src[j], geom(L, j), dst[j], st));
-  } else {
-    for (int j = 0; j < 3; ++j) {
-      const auto* w = static_cast<const __nv_bfloat16*>(src[j]);
-      MOE_CUDA(moe::launch_weight_amax(fp8_format(L), w, static_cast<long long>(IH), L->E, L->wscales + j, 3, st));
-      MOE_CUDA(moe::launch_weight_quant_tiled(fp8_format(L), w, geom(L, j), L->wscales + j, 3, static_cast<uint8_t*>(dst[j]), st));
-    }
-  }
+  MOE_TRY(load_bf16_sources(L, src, L->I, 0, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  MOE_TRY(encode_weight_maps(L));
+  L->loaded = true;
+  return MOE_OK;
+}
+
+int moe_load_weights_shard(moe_layer* L, const void* w_gate, const void* w_up, const void* w_down, int I_full,
+                           int shard, int num_shards, void* stream) {
+  if (!L || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
+  if (num_shards < 1 || shard < 0 || shard >= num_shards) return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(L->I) * num_shards != I_full) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  L->loaded = false;
+  const void* src[3] = {w_gate, w_up, w_down};
+  MOE_TRY(load_bf16_sources(L, src, I_full, shard, st));
   MOE_CUDA(cudaStreamSynchronize(st));
   MOE_TRY(encode_weight_maps(L));
   L->loaded = true;

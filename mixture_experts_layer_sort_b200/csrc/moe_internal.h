@@ -184,15 +184,19 @@ cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
 cudaError_t gemm_configure();    // opt-in dynamic shared memory sizes (current device)
 cudaError_t align_configure();
 
-// Single-launch decode path (kernels_decode.cu): the whole layer for M <= 64 bf16
-// tokens in one cooperative persistent kernel.
+// Single-launch decode path (kernels_decode.cu): the whole layer for M <= 64 tokens
+// (bf16 or FP8) in one cooperative persistent kernel.
 struct DecodeLaunch {
   const float* logits;
   const __nv_bfloat16* x;
   __nv_bfloat16* out;
   int M, E, k, H, I, grid, ws1_rows_cap, max_stages;
+  bool fp8;
+  int f8;                  // FP8 code format (Fp8Format)
   int* sync;               // decode_sync_words(E, M_cap) ints, zero between launches
-  __nv_bfloat16* x_perm;
+  uint8_t* xq;             // FP8: [M_cap, H] codes of x (tm_x maps it, one-row boxes)
+  uint8_t* hq;             // FP8: [rows_cap, I] codes of h (tm_h maps it)
+  float* last_scales;      // FP8: [2] s_x, s_h of the forward
   int* topk_ids;           // routing copies for inspection
   float* topk_w;
   int* counts;
@@ -202,8 +206,8 @@ struct DecodeLaunch {
   GemmArgs g1, g2;
   const CUtensorMap* tm_w13;
   const CUtensorMap* tm_wd;
-  const CUtensorMap* tm_x;
-  const CUtensorMap* tm_h;
+  const CUtensorMap* tm_x;   // token rows of x (bf16) or of xq (FP8), one-row boxes
+  const CUtensorMap* tm_h;   // h (bf16) or its codes (FP8), 16-row boxes
 };
 bool decode_supported(int M, int E, int k);
 size_t decode_sync_words(int E, int M_cap);
@@ -220,9 +224,14 @@ struct TileGeom {
   long long row_bytes;  // bytes of one stored row (K * element size)
   int rb_total;         // row blocks per expert in the destination (2I/128 or H/128)
   int rb_offset;        // first destination row block of this source (I/128 for up)
+  // Row-major side (the source of a load, the destination of an un-tiling), possibly a
+  // slice of a larger tensor: row r of expert e starts at byte
+  // e * src_expert_stride + r * src_row_stride + src_offset. All three are multiples of 16.
+  long long src_expert_stride, src_row_stride, src_offset;
 };
-cudaError_t launch_weight_amax(int f8, const __nv_bfloat16* w, long long per_expert, int E,
-                               float* scales, int stride, cudaStream_t s);
+// scales[e * stride] from the bf16 rows of g's row-major side (K = g.row_bytes elements).
+cudaError_t launch_weight_amax(int f8, const __nv_bfloat16* w, const TileGeom& g, float* scales, int stride,
+                               cudaStream_t s);
 // bf16 source [E, rows, K] -> e4m3 codes in the tiled layout, per-expert scale scales[e*stride].
 cudaError_t launch_weight_quant_tiled(int f8, const __nv_bfloat16* w, const TileGeom& g, const float* scales,
                                       int stride, uint8_t* dst, cudaStream_t s);

@@ -78,6 +78,18 @@ class MoELayer:
         self._check("moe_load_weights", self.lib.moe_load_weights(
             self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), _stream(stream)))
 
+    def load_weights_shard(self, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, shard: int,
+                           num_shards: int, stream=None):
+        """Shard `shard` of `num_shards` over the intermediate dimension, from the FULL bf16
+        device tensors W_gate [E,I_full,H], W_up [E,I_full,H], W_down [E,H,I_full]
+        (I_full = I * num_shards); the slicing happens in the library's load kernels."""
+        I_full = self.I * num_shards
+        for t, shape in ((w_gate, (self.E, I_full, self.H)), (w_up, (self.E, I_full, self.H)),
+                         (w_down, (self.E, self.H, I_full))):
+            assert t.is_cuda and t.dtype == torch.bfloat16 and tuple(t.shape) == shape and t.is_contiguous()
+        self._check("moe_load_weights_shard", self.lib.moe_load_weights_shard(
+            self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), I_full, shard, num_shards, _stream(stream)))
+
     def load_weights_fp8(self, q_gate, q_up, q_down, scales, stream=None):
         """uint8 e4m3 codes (device) and scales [E,3] fp32 (host)."""
         sc = torch.as_tensor(scales, dtype=torch.float32).contiguous().cpu()
@@ -179,3 +191,22 @@ class MoELayer:
         self._check("moe_debug_weights", self.lib.moe_debug_weights(
             self.handle, _ptr(g), _ptr(u), _ptr(d), sc.data_ptr()))
         return g, u, d, sc
+
+
+def inv_rope_fp8_quant(x: torch.Tensor, positions: torch.Tensor, cos_sin: torch.Tensor, interleaved: bool = False,
+                       fmt: str = "e4m3", codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                       stream=None):
+    """moe_inv_rope_fp8_quant: x [T, NH, D] bf16, positions [T] int32, cos_sin [max_pos, D]
+    fp32 (device) -> (codes [T, NH, D] uint8, scales [T, NH] fp32)."""
+    lib = load_library()
+    T, NH, D = x.shape
+    if codes is None:
+        codes = torch.empty((T, NH, D), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((T, NH), dtype=torch.float32, device=x.device)
+    rc = lib.moe_inv_rope_fp8_quant(_ptr(x), _ptr(positions), _ptr(cos_sin), cos_sin.shape[0], T, NH, D,
+                                    1 if interleaved else 0, _DTYPES[fmt], _ptr(codes), _ptr(scales),
+                                    _stream(stream))
+    if rc != 0:
+        raise MoEError("moe_inv_rope_fp8_quant", rc)
+    return codes, scales

@@ -449,3 +449,41 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
         inter["h_rows"] = h_rows
         return out, inter
     return out
+
+
+# --------------------------------------------------------------------------- tensor parallelism
+def shard_weights(w_gate, w_up, w_down, shard: int, num_shards: int):
+    """Slice `shard` of `num_shards` over the intermediate dimension I: rows
+    [g*I/G, (g+1)*I/G) of every W_gate[e] and W_up[e], the same columns of every
+    W_down[e] (the eight-way tensor parallelism the pages deploy the layer with,
+    toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "3.
+    Removing repeat compilation can reduce first-token delay")."""
+    I = np.asarray(w_gate).shape[1]
+    if I % num_shards:
+        raise ValueError("I must divide into the shards")
+    a, b = shard * I // num_shards, (shard + 1) * I // num_shards
+    return (np.asarray(w_gate)[:, a:b, :], np.asarray(w_up)[:, a:b, :], np.asarray(w_down)[:, :, a:b])
+
+
+def moe_forward_tp(x, logits, k, w_gate=None, w_up=None, w_down=None, *, num_shards: int, provider=None,
+                   fp8=False, fp8_format="e4m3"):
+    """The layer split over `num_shards` ranks by the intermediate dimension: each rank
+    is a layer of its slice (routing is the same everywhere: it reads only the logits),
+    and the combine adds the ranks' outputs. SwiGLU acts per intermediate feature and
+    the down projection sums over features, so in exact arithmetic the bf16 result is
+    the unsharded layer's. FP8 ranks quantise their own slice (weights) and their own
+    h, so the FP8 result is the sum of the ranks' FP8 layers. Weights as stacked
+    arrays, or provider(e) -> (w_gate[e], w_up[e], w_down[e]) of the FULL layer."""
+    out = None
+    for g in range(num_shards):
+        if provider is None:
+            kw = dict(zip(("w_gate", "w_up", "w_down"), shard_weights(w_gate, w_up, w_down, g, num_shards)))
+        else:
+            def sliced(e, g=g):
+                gw, uw, dw = (np.asarray(t) for t in provider(e))
+                sub = shard_weights(gw[None], uw[None], dw[None], g, num_shards)
+                return sub[0][0], sub[1][0], sub[2][0]
+            kw = {"provider": sliced}
+        part = moe_forward(x, logits, k, fp8=fp8, fp8_format=fp8_format, **kw)
+        out = part if out is None else out + part
+    return out

@@ -86,3 +86,17 @@ def test_every_entry_point_rejects_a_null_handle(lib):
     assert lib.moe_debug_routing(None, None, None, None, None, None, None, None) == -1
     assert lib.moe_debug_activations(None, None, None) == -1
     assert lib.moe_debug_weights(None, None, None, None, None) == -1
+
+
+@pytest.mark.parametrize("max_pos,T,NH,D,inter,fmt", [
+    (16, -1, 4, 128, 0, 1), (16, 4, 0, 128, 0, 1), (0, 4, 4, 128, 0, 1), (16, 4, 4, 96, 0, 1),
+    (16, 4, 4, 512, 0, 1), (16, 4, 4, 128, 2, 1), (16, 4, 4, 128, 0, 0), (16, 4, 4, 128, 0, 3)])
+def test_inv_rope_rejects_bad_arguments_without_a_gpu(lib, max_pos, T, NH, D, inter, fmt):
+    # every check happens before any CUDA call
+    assert lib.moe_inv_rope_fp8_quant(16, 16, 16, max_pos, T, NH, D, inter, fmt, 16, 16, None) == -1
+
+
+def test_inv_rope_rejects_null_or_misaligned_pointers(lib):
+    assert lib.moe_inv_rope_fp8_quant(None, 16, 16, 16, 4, 4, 128, 0, 1, 16, 16, None) == -1
+    assert lib.moe_inv_rope_fp8_quant(24, 16, 16, 16, 4, 4, 128, 0, 1, 16, 16, None) == -1   # x not 16-aligned
+    assert lib.moe_inv_rope_fp8_quant(16, 16, 16, 16, 0, 4, 128, 0, 1, None, None, None) == 0   # no tokens: no-op
