@@ -58,7 +58,9 @@ typedef enum {
   MOE_DTYPE_BF16 = 0,       /* bf16 weights and activations, fp32 accumulation        */
   MOE_DTYPE_FP8_E4M3 = 1,   /* e4m3 weights (per expert-tensor scale), e4m3 activations
                                (per-tensor dynamic scale), fp32 accumulation           */
-  MOE_DTYPE_FP8_E5M2 = 2    /* the same with e5m2 codes for weights and activations    */
+  MOE_DTYPE_FP8_E5M2 = 2,   /* the same with e5m2 codes for weights and activations    */
+  MOE_DTYPE_MIXED_E4M3 = 3  /* a precision per expert, bf16 or e4m3: see
+                               moe_load_weights_mixed                                  */
 } moe_dtype;
 
 typedef enum {
@@ -90,6 +92,23 @@ MOE_API int moe_destroy(moe_layer* layer);
  * sources afterwards. Calling it again replaces the weights. */
 MOE_API int moe_load_weights(moe_layer* layer, const void* w_gate, const void* w_up,
                      const void* w_down, void* stream);
+
+/* Load a layer created with MOE_DTYPE_MIXED_E4M3, choosing the precision of each
+ * expert: expert_fp8 [E] (host, one byte per expert) is nonzero for an expert kept as
+ * e4m3 codes, zero for one kept in bf16. Experts differ in their numerical ranges,
+ * and the kongchang.com page describes deciding per expert (or per computation stage)
+ * which ones run in FP8 and which keep a higher precision ("MoE Kernel Engineering
+ * Optimization Practices on Amazon SageMaker AI", section "Triton Backend Routing: A
+ * Practical Path to FP8 Quantization"). Sources are the bf16 tensors of
+ * moe_load_weights (device pointers). An FP8 expert takes the FP8 path of an e4m3
+ * layer: one scale per (expert, tensor), e4m3 codes of x with s_x over all of x, and
+ * of its h rows with s_h = max|h| / 448 over the valid h rows of the FP8 experts only;
+ * a bf16 expert takes the bf16 path. Each grouped GEMM then runs as two launches, one
+ * per precision. Synchronises `stream`. MOE_ERR_INVALID_ARG for another dtype;
+ * moe_load_weights, moe_load_weights_fp8, moe_load_weights_shard reject a mixed layer,
+ * moe_forward_noalloc returns MOE_ERR_UNSUPPORTED for it and moe_debug_weights too. */
+MOE_API int moe_load_weights_mixed(moe_layer* layer, const void* w_gate, const void* w_up,
+                                   const void* w_down, const unsigned char* expert_fp8, void* stream);
 
 /* Tensor parallelism over the expert intermediate dimension: load shard `shard` of
  * `num_shards` of a layer whose full intermediate size is I_full = I * num_shards (the

@@ -19,6 +19,7 @@ SIGNATURES = {
     "moe_destroy": (_c_int, [_c_void_p]),
     "moe_load_weights": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "moe_load_weights_fp8": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "moe_load_weights_mixed": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "moe_load_weights_shard": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
                                         _c_void_p]),
     "moe_reserve": (_c_int, [_c_void_p, _c_int, _c_void_p]),

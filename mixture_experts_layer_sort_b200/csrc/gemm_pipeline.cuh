@@ -327,8 +327,9 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
     // first tiled-weight block of the unit's two weight row blocks; a second block
     // past the end of the tensor reads zeros and is not stored by the epilogue
     const int rb0 = un.t.fblock * a.rb_step;
-    const int wtile = (un.t.expert * a.w_rblocks + rb0) * a.kblocks;
-    const int wtile2 = (un.t.expert * a.w_rblocks + rb0 + a.second_rb) * a.kblocks;
+    const int et = a.w_expert_tiles > 0 ? static_cast<int>(a.w_expert_tiles) : a.w_rblocks * a.kblocks;
+    const int wtile = un.t.expert * et + rb0 * a.kblocks;
+    const int wtile2 = un.t.expert * et + (rb0 + a.second_rb) * a.kblocks;
     const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
     const int dep = hk.dep(un);
     for (int kb = un.kb0; kb < un.kb1; ++kb) {

@@ -39,6 +39,13 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   int* s_nb = s_base + E;               // [E]   token blocks of e
   int* s_nboff = s_nb + E;              // [E+1]
   int* s_wc = s_nboff + E + 1;          // [32][E] per-warp counts of the current chunk
+  // precision per expert: token blocks of the FP8 experts and their offsets, then of the
+  // bf16 experts (the FP8 experts' tiles go first in each tile list)
+  int* s_nb8 = s_wc + kAlignWarps * E;  // [E]
+  int* s_nboff8 = s_nb8 + E;            // [E+1]
+  int* s_nbbf = s_nboff8 + E + 1;       // [E]
+  int* s_nboffbf = s_nbbf + E;          // [E+1]
+  const bool mixed = a.eflags != nullptr;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -84,10 +91,17 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
     const int n = s_count[e];
     s_padded[e] = (n + kPadRows - 1) / kPadRows * kPadRows;
     s_nb[e] = (n + a.BN - 1) / a.BN;
+    if (mixed) {
+      const bool f8 = a.eflags[e] != 0;
+      s_nb8[e] = f8 ? s_nb[e] : 0;
+      s_nbbf[e] = f8 ? 0 : s_nb[e];
+    }
   }
   __syncthreads();
   if (warp == 0) warp_exclusive_scan(s_padded, s_poff, E, lane);
   if (warp == 1) warp_exclusive_scan(s_nb, s_nboff, E, lane);
+  if (mixed && warp == 2) warp_exclusive_scan(s_nb8, s_nboff8, E, lane);
+  if (mixed && warp == 3) warp_exclusive_scan(s_nbbf, s_nboffbf, E, lane);
   __syncthreads();
 
   if (small) {
@@ -152,12 +166,14 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
   // (a large batch's accumulator would otherwise not stay in L2 between the k
   // contributions to each token); the price is reading each expert's h once per slab.
   const int nblocks_all = s_nboff[E];
-  const int S2 = a.acc_slabs < 1 ? 1 : a.acc_slabs;
+  // (a layer with a precision per expert keeps one slab: each of its two parts must
+  // be one contiguous run of tiles)
+  const int S2 = (mixed || a.acc_slabs < 1) ? 1 : a.acc_slabs;
   for (int e = warp; e < E; e += kAlignWarps) {
     const int n = s_count[e];
     const int nb = s_nb[e];
     if (nb == 0) continue;
-    const int base = s_nboff[e];
+    const int base = !mixed ? s_nboff[e] : (a.eflags[e] != 0 ? s_nboff8[e] : s_nboff8[E] + s_nboffbf[e]);
     for (int idx = lane; idx < nb * a.fblocks1; idx += 32) {
       const int f = idx / nb, b = idx - f * nb;
       Tile t;
@@ -207,6 +223,25 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_kernel(AlignArgs a) {
       a.header[kHdrTiles1] = t1;
       a.header[kHdrSplits1] = s1;
       a.header[kHdrTokenBlocks] = nblocks;
+    }
+  } else if (mixed && warp >= 2 && warp < 6) {
+    // the FP8 part and the bf16 part of each list, each with its own split factor
+    // (the rule of warps 0 and 1 below with the part's tiles and K blocks)
+    const bool gate = warp < 4, f8 = (warp & 1) == 0;
+    const int nb_part = f8 ? s_nboff8[E] : s_nboffbf[E];
+    const int nblocks = s_nboff[E];
+    const int n_mean = nblocks > 0 ? (a.P + nblocks - 1) / nblocks : 0;
+    const int t = nb_part * (gate ? a.fblocks1 : a.fblocks2);
+    const int kb = gate ? (f8 ? a.kblocks1_f8 : a.kblocks1) : (f8 ? a.kblocks2_f8 : a.kblocks2);
+    const int kbytes = (gate ? 2 * 16384 : 16384) + n_mean * 128;
+    const int sbytes = gate ? n_mean * 256 * 4 * 2 : n_mean * 128 * 4;
+    const bool allow = !gate || s_poff[E] <= a.ws1_rows_cap;
+    const bool bal = allow && t >= a.num_sms && t < kBalancedWaves * a.num_sms;
+    const int sp = (!a.uniform_splits && bal) ? 0 : choose_splits_warp(t, kb, a.num_sms, allow, kbytes, sbytes, lane);
+    if (lane == 0) {
+      const int slot = gate ? (f8 ? kHdrTiles1F8 : kHdrTiles1BF) : (f8 ? kHdrTiles2F8 : kHdrTiles2BF);
+      a.header[slot] = t;
+      a.header[slot + 1] = sp;
     }
   } else if (warp == 1) {
     const int nblocks = s_nboff[E];
@@ -265,7 +300,7 @@ __global__ void __launch_bounds__(kAlignChunk) align_scatter_kernel(AlignArgs a)
 
 }  // namespace
 
-size_t align_smem_bytes(int E) { return static_cast<size_t>(6 * E + 2 + kAlignWarps * E) * sizeof(int); }
+size_t align_smem_bytes(int E) { return static_cast<size_t>(10 * E + 4 + kAlignWarps * E) * sizeof(int); }
 
 cudaError_t align_configure() {
   cudaError_t e = cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

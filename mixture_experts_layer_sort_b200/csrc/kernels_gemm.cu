@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_trigger();
   }
   const Ring rg = make_ring<C>(a.header[kHdrMaxRows], a.max_stages, sh.ring_bytes);
-  const GlobalTiles src(a.tiles, a.header[a.hdr_tiles], a.header[a.hdr_splits], a.kblocks);
+  const int t_off = a.hdr_tile_offset > 0 ? a.header[a.hdr_tile_offset] : 0;
+  const GlobalTiles src(a.tiles + t_off, a.header[a.hdr_tiles], a.header[a.hdr_splits], a.kblocks);
   // Everyone but the producer warp waits for the previous kernel here. Otherwise the
   // tile list comes from the align kernel, at least two launches back, and is
   // complete already (see pdl_wait in sm100.cuh).

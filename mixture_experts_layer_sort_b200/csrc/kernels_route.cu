@@ -141,6 +141,29 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
   }
 }
 
+// A precision per expert: row r of a pair routed to an FP8 expert gets the codes of
+// its token's x row in x_perm8; a pair of a bf16 expert gets the bf16 row in x_perm.
+__global__ void __launch_bounds__(256) gather_mixed_kernel(GatherArgs a) {
+  const int t = threadIdx.x % kRowThreads;
+  pdl_wait();
+  pdl_trigger();
+  const int used = a.header[kHdrRowsUsed];
+  const float s = fp8_scale_from_amax(*a.amax_x, a.f8);
+  const int bound = used < a.rows_bound ? used : a.rows_bound;
+  for (int r = blockIdx.x * kRowsPerBlock + threadIdx.x / kRowThreads; r < bound;
+       r += gridDim.x * kRowsPerBlock) {
+    const int p = a.padded_pairs[r];
+    if (p >= a.P) continue;   // a pad row: never read by an output column
+    const size_t tok = static_cast<size_t>(p / a.k);
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + tok * a.H);
+    if (a.eflags[a.topk_ids[p]] != 0)
+      copy_row<true, false>(src, a.x_perm8 + static_cast<size_t>(r) * a.H, a.H / 8, s, a.f8, t);
+    else
+      copy_row<false, false>(src, static_cast<__nv_bfloat16*>(a.x_perm) + static_cast<size_t>(r) * a.H, a.H / 8,
+                             1.f, 0, t);
+  }
+}
+
 // FP8, large batches: the M token rows of x -> FP8 codes with s_x = amax(x)/F, once
 // per token instead of once per (token, slot) pair.
 __global__ void __launch_bounds__(256) quant_x_kernel(QuantXArgs a) {
@@ -163,7 +186,9 @@ __global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
   const int bound = used < a.rows_bound ? used : a.rows_bound;
   for (int r = blockIdx.x * kRowsPerBlock + threadIdx.x / kRowThreads; r < bound;
        r += gridDim.x * kRowsPerBlock) {
-    if (a.padded_pairs[r] >= a.P) continue;
+    const int p = a.padded_pairs[r];
+    if (p >= a.P) continue;
+    if (a.eflags != nullptr && a.eflags[a.topk_ids[p]] == 0) continue;   // a bf16 expert's row
     // h was written by the previous kernel: coherent loads, not the read-only path
     copy_row<true, true>(reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(r) * a.I),
                          a.h_q + static_cast<size_t>(r) * a.I, a.I / 8, s, a.f8, t);
@@ -232,6 +257,8 @@ int row_grid(int rows, bool capped) {
 }
 
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s) {
+  if (a.eflags != nullptr)
+    return launch_kernel(gather_mixed_kernel, dim3(row_grid(a.rows_bound, true)), dim3(256), 0, s, a);
   const int grid = row_grid(a.rows_bound, fp8);
   if (fp8) return launch_kernel(gather_kernel<true>, dim3(grid), dim3(256), 0, s, a);
   return launch_kernel(gather_kernel<false>, dim3(grid), dim3(256), 0, s, a);

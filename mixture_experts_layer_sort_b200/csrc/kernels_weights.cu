@@ -21,7 +21,8 @@ namespace {
 
 __device__ __forceinline__ long long tiled_offset(const TileGeom& g, long long e, long long r, long long byte) {
   const long long kbn = g.row_bytes / 128;
-  const long long tile = (e * g.rb_total + g.rb_offset + r / 128) * kbn + byte / 128;
+  const long long slot = g.expert_tiles > 0 ? g.expert_tiles : g.rb_total * kbn;
+  const long long tile = e * slot + (g.rb_offset + r / 128) * kbn + byte / 128;
   return (tile * 128 + (r & 127)) * 128 + (byte & 127);
 }
 
@@ -35,6 +36,7 @@ __device__ __forceinline__ long long rowmajor_offset(const TileGeom& g, long lon
 __global__ void __launch_bounds__(1024) weight_amax_kernel(int f8, const uint8_t* w, TileGeom g, float* scales,
                                                            int stride) {
   const int e = blockIdx.x;
+  if (g.expert_mask != nullptr && g.expert_mask[e] != g.mask_value) return;
   const long long per_row = g.row_bytes / 8;       // 16-byte vectors of 8 bf16 per row
   float m = 0.f;
   for (long long i = threadIdx.x; i < g.rows * per_row; i += blockDim.x) {
@@ -72,6 +74,7 @@ __global__ void __launch_bounds__(256) weight_quant_tiled_kernel(int f8, const u
     const long long c = (i - row * per_row) * 8;
     const long long e = row / g.rows;
     const long long r = row - e * g.rows;
+    if (g.expert_mask != nullptr && g.expert_mask[e] != g.mask_value) continue;
     const float s = __ldg(scales + e * stride);
     // 8 bf16 source values = 16 bytes at column c of the row-major source
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(w + rowmajor_offset(g, e, r, 2 * c)));
@@ -100,6 +103,7 @@ __global__ void __launch_bounds__(256) retile_kernel(const uint8_t* src, TileGeo
     const long long b = (i - row * per_row) * 16;
     const long long e = row / g.rows;
     const long long r = row - e * g.rows;
+    if (g.expert_mask != nullptr && g.expert_mask[e] != g.mask_value) continue;
     const long long t = tiled_offset(g, e, r, b);
     const long long m = rowmajor_offset(g, e, r, b);
     if constexpr (kToTiled) *reinterpret_cast<uint4*>(dst + t) = __ldg(reinterpret_cast<const uint4*>(src + m));

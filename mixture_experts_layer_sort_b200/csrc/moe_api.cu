@@ -26,6 +26,7 @@
 #include <vector>
 
 #include "../../include/moe_b200.h"
+#include "fp8_format.cuh"
 #include "moe_internal.h"
 #include "sm100.cuh"
 
@@ -38,6 +39,7 @@ struct moe_layer {
   void* w13 = nullptr;          // [E, 2I, H] gate rows then up rows of each expert (bf16 or e4m3)
   void* wd = nullptr;           // [E, H, I]
   float* wscales = nullptr;     // [E, 3] FP8 scales (device)
+  int* eflags = nullptr;        // [E] precision per expert (1 = FP8), layers with a precision per expert
   CUtensorMap tm_w13{}, tm_wd{};
   // workspace, sized for M_cap tokens
   int M_cap = 0;
@@ -66,6 +68,8 @@ struct moe_layer {
   long long chunks_cap = 0;
   CUtensorMap tm_x{}, tm_h{};
   CUtensorMap tm_xq{};          // FP8 single-launch decode: token rows of xq, one-row boxes
+  uint8_t* x_perm8 = nullptr;   // precision per expert: FP8 codes of the FP8 experts' rows [rows_cap, H]
+  CUtensorMap tm_x8{}, tm_hq{}; // precision per expert: maps of x_perm8 and of h_q
   // staging for moe_forward_host
   void* hx = nullptr;
   float* hl = nullptr;
@@ -195,6 +199,8 @@ int ws_alloc(moe_layer* L, T** p, size_t bytes, bool zero) {
 }
 
 bool is_fp8(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E4M3 || L->dtype == MOE_DTYPE_FP8_E5M2; }
+// a precision per expert (bf16 or e4m3): weights in bf16-sized slots, both kernel kinds
+bool is_mixed(const moe_layer* L) { return L->dtype == MOE_DTYPE_MIXED_E4M3; }
 // FP8 code format of an FP8 layer (moe::Fp8Format values)
 int fp8_format(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E5M2 ? 1 : 0; }
 
@@ -225,7 +231,8 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(ws_alloc(L, &L->header, moe::kHdrSlots * 4, true));
   MOE_TRY(ws_alloc(L, &L->x_perm, L->rows_cap * L->H * el, true));
   MOE_TRY(ws_alloc(L, &L->h, L->rows_cap * L->I * 2, true));
-  if (is_fp8(L)) MOE_TRY(ws_alloc(L, &L->h_q, L->rows_cap * L->I, true));
+  if (is_fp8(L) || is_mixed(L)) MOE_TRY(ws_alloc(L, &L->h_q, L->rows_cap * L->I, true));
+  if (is_mixed(L)) MOE_TRY(ws_alloc(L, &L->x_perm8, L->rows_cap * L->H, true));
   MOE_TRY(ws_alloc(L, &L->ws1, L->ws1_rows_cap * 2 * L->I * 4, true));
   MOE_TRY(ws_alloc(L, &L->counters, L->t1_cap * 4, true));
   MOE_TRY(ws_alloc(L, &L->acc, static_cast<size_t>(cap) * L->H * 4, true));
@@ -242,6 +249,10 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(encode_map(&L->tm_h, is_fp8(L) ? static_cast<void*>(L->h_q) : static_cast<void*>(L->h), is_fp8(L),
                      L->I, L->rows_cap, 16));
   if (is_fp8(L)) MOE_TRY(encode_map(&L->tm_xq, L->xq, true, L->H, cap, 1));
+  if (is_mixed(L)) {
+    MOE_TRY(encode_map(&L->tm_x8, L->x_perm8, true, L->H, L->rows_cap, 16));
+    MOE_TRY(encode_map(&L->tm_hq, L->h_q, true, L->I, L->rows_cap, 16));
+  }
   L->M_cap = cap;
   return MOE_OK;
 }
@@ -466,8 +477,11 @@ int acc_slabs(int M, int H, int fblocks2) {
 // chunk of 1024 pairs after another); beyond, chunks go to blocks of their own.
 constexpr long long kAlignSingleBlockMaxPairs = 8192;
 
+int forward_mixed(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st);
+
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
+  if (is_mixed(L)) return forward_mixed(L, x, logits, M, out, st);
   if (L->fused_decode && M <= L->num_sms && moe::decode_supported(M, L->E, L->k))
     return forward_fused_decode(L, x, logits, M, out, st);
   const bool fp8 = is_fp8(L);
@@ -659,6 +673,193 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   return MOE_OK;
 }
 
+// A layer with a precision per expert (bf16 or e4m3; the per-expert FP8 choice of the
+// kongchang.com page, "MoE Kernel Engineering Optimization Practices on Amazon
+// SageMaker AI", section "Triton Backend Routing: A Practical Path to FP8
+// Quantization"). Every expert's weights sit in a bf16-sized slot (an FP8 expert's
+// codes in its first half); the align kernel lists the FP8 experts' tiles first, then
+// the bf16 experts', and each GEMM runs as two launches, one per precision, over its
+// own part of the list:
+//   route (+ max|x|) -> align -> gather (bf16 rows or FP8 codes per row) ->
+//   gate_up FP8 -> gate_up bf16 -> quant_h (FP8 experts' rows; s_h over them) ->
+//   down FP8 -> down bf16 -> finalize
+int forward_mixed(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
+  const long long P = static_cast<long long>(M) * L->k;
+  const int rows_bound = static_cast<int>(P + std::min<long long>(L->E, P) * (moe::kPadRows - 1));
+  const int f8 = moe::kFp8E4M3;
+  int launches = 0;
+
+  moe::RouteArgs ra{};
+  ra.logits = logits;
+  ra.x = static_cast<const __nv_bfloat16*>(x);
+  ra.M = M;
+  ra.E = L->E;
+  ra.k = L->k;
+  ra.H = L->H;
+  ra.topk_ids = L->topk_ids;
+  ra.topk_w = L->topk_w;
+  ra.amax_x = L->amax;
+  {
+    KernelTimer kt(L, 0, st);
+    MOE_CUDA(moe::launch_route(ra, st));
+  }
+  ++launches;
+
+  moe::AlignArgs aa{};
+  aa.topk_ids = L->topk_ids;
+  aa.P = static_cast<int>(P);
+  aa.E = L->E;
+  aa.k = L->k;
+  aa.BN = moe::kTokenBlock;
+  aa.fblocks1 = L->I / moe::kTileRows;
+  aa.fblocks2 = (L->H / moe::kTileRows + 1) / 2;
+  aa.kblocks1 = L->H / 64;
+  aa.kblocks2 = L->I / 64;
+  aa.kblocks1_f8 = L->H / 128;
+  aa.kblocks2_f8 = L->I / 128;
+  aa.num_sms = L->num_sms;
+  aa.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
+  aa.acc_slabs = 1;
+  aa.uniform_splits = moe::uniform_splits() ? 1 : 0;
+  aa.counts = L->counts;
+  aa.padded_offsets = L->poff;
+  aa.padded_pairs = L->pairs;
+  aa.tiles1 = L->tiles1;
+  aa.tiles2 = L->tiles2;
+  aa.header = L->header;
+  aa.eflags = L->eflags;
+  {
+    KernelTimer kt(L, 1, st);
+    MOE_CUDA(moe::launch_align(aa, st));
+  }
+  ++launches;
+
+  moe::GatherArgs ga{};
+  ga.x = static_cast<const __nv_bfloat16*>(x);
+  ga.padded_pairs = L->pairs;
+  ga.header = L->header;
+  ga.rows_bound = rows_bound;
+  ga.P = static_cast<int>(P);
+  ga.k = L->k;
+  ga.H = L->H;
+  ga.x_perm = L->x_perm;
+  ga.amax_x = L->amax;
+  ga.f8 = f8;
+  ga.eflags = L->eflags;
+  ga.topk_ids = L->topk_ids;
+  ga.x_perm8 = L->x_perm8;
+  {
+    KernelTimer kt(L, 2, st);
+    MOE_CUDA(moe::launch_gather(ga, false, st));
+  }
+  ++launches;
+
+  moe::GemmArgs g{};
+  g.header = L->header;
+  g.h = L->h;
+  g.I = L->I;
+  g.ws1 = L->ws1;
+  g.tile_counters = L->counters;
+  g.amax_h = L->amax + 1;
+  g.amax_x = L->amax;
+  g.w_scales = L->wscales;
+  g.acc = L->acc;
+  g.H = L->H;
+  g.padded_pairs = L->pairs;
+  g.topk_w = L->topk_w;
+  g.k = L->k;
+  g.P = static_cast<int>(P);
+  g.f8 = f8;
+  g.err = L->err;
+
+  // gate_up: FP8 experts, then bf16 experts (bf16-sized expert slots in both)
+  moe::GemmArgs g1 = g;
+  g1.tiles = L->tiles1;
+  g1.w_rblocks = 2 * L->I / moe::kTileRows;
+  g1.w_expert_tiles = static_cast<long long>(g1.w_rblocks) * (L->H / 64);
+  g1.rb_step = 1;
+  g1.second_rb = L->I / moe::kTileRows;
+  g1.max_stages = moe::gemm_max_stages(true);
+  moe::GemmArgs g1f = g1;
+  g1f.hdr_tiles = moe::kHdrTiles1F8;
+  g1f.hdr_splits = moe::kHdrSplits1F8;
+  g1f.kblocks = L->H / 128;
+  moe::GemmArgs g1b = g1;
+  g1b.hdr_tile_offset = moe::kHdrTiles1F8;
+  g1b.hdr_tiles = moe::kHdrTiles1BF;
+  g1b.hdr_splits = moe::kHdrSplits1BF;
+  g1b.kblocks = L->H / 64;
+  {
+    KernelTimer kt(L, 3, st);
+    MOE_CUDA(moe::launch_gemm1(g1f, L->tm_w13, L->tm_x8, true, L->num_sms, st));
+  }
+  {
+    KernelTimer kt(L, 3, st);
+    MOE_CUDA(moe::launch_gemm1(g1b, L->tm_w13, L->tm_x, false, L->num_sms, st));
+  }
+  launches += 2;
+
+  moe::QuantHArgs qa{};
+  qa.h = L->h;
+  qa.h_q = L->h_q;
+  qa.padded_pairs = L->pairs;
+  qa.header = L->header;
+  qa.rows_bound = rows_bound;
+  qa.P = static_cast<int>(P);
+  qa.I = L->I;
+  qa.amax_h = L->amax + 1;
+  qa.f8 = f8;
+  qa.eflags = L->eflags;
+  qa.topk_ids = L->topk_ids;
+  {
+    KernelTimer kt(L, 4, st);
+    MOE_CUDA(moe::launch_quant_h(qa, st));
+  }
+  ++launches;
+
+  moe::GemmArgs g2 = g;
+  g2.tiles = L->tiles2;
+  g2.w_rblocks = L->H / moe::kTileRows;
+  g2.w_expert_tiles = static_cast<long long>(g2.w_rblocks) * (L->I / 64);
+  g2.rb_step = 2;
+  g2.second_rb = 1;
+  g2.max_stages = moe::gemm_max_stages(false);
+  moe::GemmArgs g2f = g2;
+  g2f.hdr_tiles = moe::kHdrTiles2F8;
+  g2f.hdr_splits = moe::kHdrSplits2F8;
+  g2f.kblocks = L->I / 128;
+  moe::GemmArgs g2b = g2;
+  g2b.hdr_tile_offset = moe::kHdrTiles2F8;
+  g2b.hdr_tiles = moe::kHdrTiles2BF;
+  g2b.hdr_splits = moe::kHdrSplits2BF;
+  g2b.kblocks = L->I / 64;
+  {
+    KernelTimer kt(L, 5, st);
+    MOE_CUDA(moe::launch_gemm2(g2f, L->tm_wd, L->tm_hq, true, L->num_sms, st));
+  }
+  {
+    KernelTimer kt(L, 5, st);
+    MOE_CUDA(moe::launch_gemm2(g2b, L->tm_wd, L->tm_h, false, L->num_sms, st));
+  }
+  launches += 2;
+
+  moe::FinalizeArgs fa{};
+  fa.acc = L->acc;
+  fa.out = static_cast<__nv_bfloat16*>(out);
+  fa.n = static_cast<long long>(M) * L->H;
+  fa.amax = L->amax;
+  fa.last_scales = L->last_scales;
+  fa.f8 = f8;
+  {
+    KernelTimer kt(L, 6, st);
+    MOE_CUDA(moe::launch_finalize(fa, st));
+  }
+  ++launches;
+  L->last_M = M;
+  L->last_launches = launches;
+  return MOE_OK;
+}
+
 }  // namespace
 
 bool moe::pdl_enabled() {
@@ -709,6 +910,7 @@ int moe_layer_view(const moe_layer* L, moe::LayerView* v) {
   v->device = L->device;
   v->num_sms = L->num_sms;
   v->fp8 = is_fp8(L);
+  v->mixed = is_mixed(L);
   v->f8 = fp8_format(L);
   v->loaded = L->loaded;
   v->wscales = L->wscales;
@@ -742,7 +944,8 @@ int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
   *out = nullptr;
   if (E < 1 || E > 512 || topk < 1 || topk > 16 || topk > E) return MOE_ERR_INVALID_ARG;
   if (H < 128 || I < 128 || H > 16384 || I > 16384 || H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
-  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_FP8_E4M3 && dtype != MOE_DTYPE_FP8_E5M2)
+  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_FP8_E4M3 && dtype != MOE_DTYPE_FP8_E5M2 &&
+      dtype != MOE_DTYPE_MIXED_E4M3)
     return MOE_ERR_INVALID_ARG;
   int dev = 0;
   MOE_CUDA(cudaGetDevice(&dev));
@@ -761,13 +964,15 @@ int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
   L->device = dev;
   L->num_sms = prop.multiProcessorCount;
   L->fused_decode = fused_decode_default();
-  const size_t el = dtype == MOE_DTYPE_BF16 ? 2 : 1;
+  const size_t el = (dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_MIXED_E4M3) ? 2 : 1;
   if (cudaMalloc(&L->w13, static_cast<size_t>(E) * 2 * I * H * el) != cudaSuccess ||
       cudaMalloc(&L->wd, static_cast<size_t>(E) * H * I * el) != cudaSuccess ||
-      cudaMalloc(&L->wscales, static_cast<size_t>(E) * 3 * sizeof(float)) != cudaSuccess) {
+      cudaMalloc(&L->wscales, static_cast<size_t>(E) * 3 * sizeof(float)) != cudaSuccess ||
+      (dtype == MOE_DTYPE_MIXED_E4M3 && cudaMalloc(&L->eflags, static_cast<size_t>(E) * sizeof(int)) != cudaSuccess)) {
     cudaFree(L->w13);
     cudaFree(L->wd);
     cudaFree(L->wscales);
+    cudaFree(L->eflags);
     delete L;
     return MOE_ERR_OOM;
   }
@@ -785,6 +990,7 @@ int moe_destroy(moe_layer* L) {
   cudaFree(L->w13);
   cudaFree(L->wd);
   cudaFree(L->wscales);
+  cudaFree(L->eflags);
   cudaFree(L->hx);
   cudaFree(L->hl);
   cudaFree(L->hout);
@@ -801,6 +1007,7 @@ int moe_destroy(moe_layer* L) {
 
 int moe_load_weights(moe_layer* L, const void* w_gate, const void* w_up, const void* w_down, void* stream) {
   if (!L || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
+  if (is_mixed(L)) return MOE_ERR_INVALID_ARG;   // needs the per-expert choice: moe_load_weights_mixed
   if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
   DeviceGuard g(L->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -813,9 +1020,46 @@ int moe_load_weights(moe_layer* L, const void* w_gate, const void* w_up, const v
   return MOE_OK;
 }
 
+int moe_load_weights_mixed(moe_layer* L, const void* w_gate, const void* w_up, const void* w_down,
+                           const unsigned char* expert_fp8, void* stream) {
+  if (!L || !w_gate || !w_up || !w_down || !expert_fp8) return MOE_ERR_INVALID_ARG;
+  if (!is_mixed(L)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(L->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  L->loaded = false;
+  std::vector<int> flags(static_cast<size_t>(L->E));
+  for (int e = 0; e < L->E; ++e) flags[e] = expert_fp8[e] ? 1 : 0;
+  MOE_CUDA(cudaMemcpyAsync(L->eflags, flags.data(), flags.size() * sizeof(int), cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaStreamSynchronize(st));   // `flags` is pageable host memory
+  const void* src[3] = {w_gate, w_up, w_down};
+  void* dst[3] = {L->w13, L->w13, L->wd};
+  for (int j = 0; j < 3; ++j) {
+    // bf16 experts: tiled copies into their slots
+    moe::TileGeom gb = geom(L, j, 2, L->I, 0);
+    gb.expert_mask = L->eflags;
+    gb.mask_value = 0;
+    MOE_CUDA(moe::launch_tile_weights(src[j], gb, dst[j], st));
+    // FP8 experts: scale and e4m3 codes of their tensors, in the first half of a bf16-sized slot
+    moe::TileGeom gf = gb;
+    gf.expert_tiles = gb.rb_total * (gb.row_bytes / 128);
+    gf.row_bytes = gb.row_bytes / 2;
+    gf.mask_value = 1;
+    const auto* w = static_cast<const __nv_bfloat16*>(src[j]);
+    MOE_CUDA(moe::launch_weight_amax(moe::kFp8E4M3, w, gf, L->wscales + j, 3, st));
+    MOE_CUDA(moe::launch_weight_quant_tiled(moe::kFp8E4M3, w, gf, L->wscales + j, 3, static_cast<uint8_t*>(dst[j]),
+                                            st));
+  }
+  MOE_CUDA(cudaStreamSynchronize(st));
+  MOE_TRY(encode_weight_maps(L));
+  L->loaded = true;
+  return MOE_OK;
+}
+
 int moe_load_weights_shard(moe_layer* L, const void* w_gate, const void* w_up, const void* w_down, int I_full,
                            int shard, int num_shards, void* stream) {
   if (!L || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
+  if (is_mixed(L)) return MOE_ERR_INVALID_ARG;
   if (num_shards < 1 || shard < 0 || shard >= num_shards) return MOE_ERR_INVALID_ARG;
   if (static_cast<long long>(L->I) * num_shards != I_full) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
@@ -1069,6 +1313,7 @@ int moe_debug_activations(moe_layer* L, void* x_perm_out, void* h_out) {
 int moe_debug_weights(moe_layer* L, void* gate_out, void* up_out, void* down_out, float* scales_host) {
   if (!L) return MOE_ERR_INVALID_ARG;
   if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  if (is_mixed(L)) return MOE_ERR_UNSUPPORTED;
   DeviceGuard g(L->device);
   MOE_CUDA(cudaDeviceSynchronize());
   void* outs[3] = {gate_out, up_out, down_out};

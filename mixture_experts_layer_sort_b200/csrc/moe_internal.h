@@ -22,7 +22,17 @@ enum HeaderSlot : int {
   kHdrSplits2 = 4,      // down split-K factor (0 = the balanced schedule)
   kHdrTokenBlocks = 5,  // (expert, token block) pairs
   kHdrMaxRows = 6,      // widest token tile (rows of activations a stage must hold), <= BN
-  kHdrSlots = 8
+  // layers with a precision per expert: the tile lists hold the FP8 experts' tiles
+  // first, then the bf16 experts' tiles; count and split factor of each part
+  kHdrTiles1F8 = 8,
+  kHdrSplits1F8 = 9,
+  kHdrTiles1BF = 10,
+  kHdrSplits1BF = 11,
+  kHdrTiles2F8 = 12,
+  kHdrSplits2F8 = 13,
+  kHdrTiles2BF = 14,
+  kHdrSplits2BF = 15,
+  kHdrSlots = 16
 };
 
 // One output tile of a grouped GEMM: weight rows [fblock*128, +128) of expert
@@ -68,6 +78,11 @@ struct AlignArgs {
   int* chunk_counts;       // [chunks, E]
   int* chunk_base;         // [chunks, E]
   int chunks;
+  // Precision per expert (nullptr: one precision for the layer): eflags[e] = 1 for an
+  // FP8 expert. The tile lists then hold the FP8 experts' tiles first; kblocks1/2 are
+  // the bf16 K blocks and kblocks1_f8/2_f8 the FP8 ones (128-byte rows of each).
+  const int* eflags;
+  int kblocks1_f8, kblocks2_f8;
 };
 
 struct GatherArgs {
@@ -80,6 +95,11 @@ struct GatherArgs {
   const unsigned* amax_x;  // FP8 only
   int f8;                  // FP8 code format (Fp8Format)
   const uint8_t* xq;       // FP8: token rows already quantised [M, H] (copy bytes), or nullptr
+  // precision per expert (nullptr: none): rows of FP8 experts get codes in x_perm8,
+  // the others bf16 copies in x_perm
+  const int* eflags;
+  const int* topk_ids;     // [P] expert of each pair (with eflags)
+  uint8_t* x_perm8;        // [rows_cap, H] FP8 codes (with eflags)
 };
 
 struct QuantXArgs {
@@ -96,6 +116,9 @@ struct GemmArgs {
   int hdr_tiles, hdr_splits;
   int kblocks;             // K blocks over the whole reduction
   int w_rblocks;           // 128-row blocks of one expert's weights (2I/128 or H/128)
+  long long w_expert_tiles; // stored tiles per expert slot (0: w_rblocks * kblocks; more
+                            //   when FP8 experts sit in bf16-sized slots)
+  int hdr_tile_offset;     // header slot holding the index of this GEMM's first tile (0: none)
   int rb_step;             // tile row block f covers weight row blocks f*rb_step and
   int second_rb;           //   f*rb_step + second_rb (gate_up: 1 and I/128; down: 2 and 1)
   // gate_up epilogue
@@ -127,6 +150,8 @@ struct QuantHArgs {
   int rows_bound, P, I;
   const unsigned* amax_h;
   int f8;                  // FP8 code format (Fp8Format)
+  const int* eflags;       // precision per expert (nullptr: none): only FP8 experts' rows
+  const int* topk_ids;     // [P] (with eflags)
 };
 
 struct FinalizeArgs {
@@ -224,6 +249,9 @@ struct TileGeom {
   long long row_bytes;  // bytes of one stored row (K * element size)
   int rb_total;         // row blocks per expert in the destination (2I/128 or H/128)
   int rb_offset;        // first destination row block of this source (I/128 for up)
+  long long expert_tiles;  // stored tiles per expert slot (0: rb_total * row_bytes / 128)
+  const int* expert_mask;  // when set, only experts e with expert_mask[e] == mask_value
+  int mask_value;
   // Row-major side (the source of a load, the destination of an un-tiling), possibly a
   // slice of a larger tensor: row r of expert e starts at byte
   // e * src_expert_stride + r * src_row_stride + src_offset. All three are multiples of 16.
@@ -243,7 +271,7 @@ cudaError_t launch_untile_weights(const void* src, const TileGeom& g, void* dst,
 // entry points that live outside moe_api.cu.
 struct LayerView {
   int E, k, H, I, device, num_sms;
-  bool fp8, loaded;
+  bool fp8, mixed, loaded;
   int f8;                  // FP8 code format (Fp8Format) when fp8
   const float* wscales;
   CUtensorMap tm_w13, tm_wd;

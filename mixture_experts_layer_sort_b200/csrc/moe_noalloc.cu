@@ -268,6 +268,7 @@ extern "C" int moe_forward_noalloc(moe_layer* layer, const void* x, const float*
   moe::LayerView v;
   if (!layer || M < 0 || moe_layer_view(layer, &v) != MOE_OK) return MOE_ERR_INVALID_ARG;
   if (!v.loaded) return MOE_ERR_NOT_LOADED;
+  if (v.mixed) return MOE_ERR_UNSUPPORTED;   // a precision per expert runs through moe_forward only
   if (M == 0) return MOE_OK;
   auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
   if (!x || !router_logits || !out || misaligned(x) || misaligned(router_logits) || misaligned(out))

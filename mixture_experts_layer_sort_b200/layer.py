@@ -12,9 +12,9 @@ import torch
 
 from ._lib import load_library, status_string
 
-BF16, FP8, FP8_E5M2 = 0, 1, 2
-_DTYPES = {"bf16": BF16, "fp8": FP8, "e4m3": FP8, "fp8_e5m2": FP8_E5M2, "e5m2": FP8_E5M2,
-           BF16: BF16, FP8: FP8, FP8_E5M2: FP8_E5M2}
+BF16, FP8, FP8_E5M2, MIXED = 0, 1, 2, 3
+_DTYPES = {"bf16": BF16, "fp8": FP8, "e4m3": FP8, "fp8_e5m2": FP8_E5M2, "e5m2": FP8_E5M2, "mixed": MIXED,
+           BF16: BF16, FP8: FP8, FP8_E5M2: FP8_E5M2, MIXED: MIXED}
 
 
 class MoEError(RuntimeError):
@@ -77,6 +77,15 @@ class MoELayer:
             assert t.is_cuda and t.dtype == torch.bfloat16 and tuple(t.shape) == shape and t.is_contiguous()
         self._check("moe_load_weights", self.lib.moe_load_weights(
             self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), _stream(stream)))
+
+    def load_weights_mixed(self, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, expert_fp8,
+                           stream=None):
+        """A "mixed" layer: bf16 device tensors as for load_weights, and expert_fp8 [E]
+        booleans (host) choosing e4m3 (True) or bf16 (False) per expert."""
+        flags = torch.as_tensor([1 if f else 0 for f in expert_fp8], dtype=torch.uint8)
+        assert flags.numel() == self.E
+        self._check("moe_load_weights_mixed", self.lib.moe_load_weights_mixed(
+            self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), flags.data_ptr(), _stream(stream)))
 
     def load_weights_shard(self, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, shard: int,
                            num_shards: int, stream=None):

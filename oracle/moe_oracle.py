@@ -312,7 +312,7 @@ def _map_experts(fn, experts, threads):
 
 def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
                 provider=None, tokens=None, return_intermediates=False, threads=None,
-                weight_cache=None, fp8_format="e4m3"):
+                weight_cache=None, fp8_format="e4m3", expert_fp8=None):
     """The layer's output in fp64.
 
     x       [M, H]  bf16 values (any float array holding them)
@@ -324,6 +324,14 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
             expert quantised with its own scale, x quantised with one scale
             over all M*H elements, h quantised with one scale over all valid
             (token, slot) rows; dequantised values feed the fp64 arithmetic.
+    expert_fp8  optional [E] booleans, a precision per expert instead of one for
+            the layer (the per-expert choice of FP8 or higher precision the
+            kongchang.com page describes, "MoE Kernel Engineering Optimization
+            Practices on Amazon SageMaker AI", section "Triton Backend Routing: A
+            Practical Path to FP8 Quantization"): FP8 experts take the FP8
+            path above, the others the bf16 path. s_x is over all of x; s_h is
+            over the valid h rows of the FP8 experts only (the rows that feed an
+            FP8 down projection). When given, `fp8` is ignored.
     tokens  optional list of token indices whose output rows are wanted; the
             other rows come back as NaN. Routing, the permutation, s_x and
             (FP8) s_h are still computed over the whole batch, as defined.
@@ -348,16 +356,21 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
     inter = {"ids": ids, "w": w, "counts": counts, "offsets": offsets,
              "sorted_pairs": sorted_pairs}
 
+    if expert_fp8 is None:
+        expert_fp8 = np.full(E, bool(fp8))
+    expert_fp8 = np.asarray(expert_fp8, dtype=bool)
+    any_fp8 = bool(expert_fp8.any())
+
     fmt = fp8_format
-    if fp8:
+    x64 = x.astype(np.float64)
+    xq = None
+    if any_fp8:
         s_x = per_tensor_scale(x, fmt)
         x_codes = quantize(x, s_x, fmt)
-        xin = dequantize(x_codes, s_x, fmt)
+        xq = dequantize(x_codes, s_x, fmt)
         inter["s_x"] = s_x
         inter["x_codes"] = x_codes
         inter["w_scales"] = np.zeros((E, 3), dtype=np.float32)
-    else:
-        xin = x.astype(np.float64)
 
     want = np.ones(M, dtype=bool) if tokens is None else np.zeros(M, dtype=bool)
     if tokens is not None:
@@ -368,7 +381,7 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
         threads = os.cpu_count() or 1
 
     def expert_weights(e):
-        if not fp8:
+        if not expert_fp8[e]:
             g_w, u_w, d_w = W.get(e)
             return g_w.astype(np.float64), u_w.astype(np.float64), d_w.astype(np.float64)
         q = weight_cache.get(e) if weight_cache is not None else None
@@ -383,25 +396,26 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
 
     active = [e for e in range(E) if counts[e] > 0]
 
-    # pass 1: gate/up projections and SwiGLU. FP8 needs every valid h row for
-    # the amax behind s_h; the bf16 path only needs the wanted tokens' pairs.
+    # pass 1: gate/up projections and SwiGLU. An FP8 expert needs every valid h row
+    # for the amax behind s_h; a bf16 expert only needs the wanted tokens' pairs.
     def pass1(e):
+        f8 = bool(expert_fp8[e])
         n = int(counts[e])
         pairs = sorted_pairs[offsets[e]:offsets[e] + n]
         sel = want[pairs // k]
-        if not fp8 and not sel.any():
+        if not f8 and not sel.any():
             return e, None
-        if fp8:
+        if f8:
             (g_w, u_w, d_w), sc = expert_weights(e)
             inter["w_scales"][e] = sc
         else:
             g_w, u_w, d_w = expert_weights(e)
-        rows = pairs if fp8 else pairs[sel]
-        X = xin[rows // k]
+        rows = pairs if f8 else pairs[sel]
+        X = (xq if f8 else x64)[rows // k]
         Hh = silu(X @ g_w.T) * (X @ u_w.T)
-        amax = np.float32(np.max(np.abs(Hh.astype(np.float32)))) if fp8 else None
+        amax = np.float32(np.max(np.abs(Hh.astype(np.float32)))) if f8 else None
         keep = {int(p): Hh[i] for i, p in enumerate(rows) if want[p // k]}
-        Ym = None if fp8 else Hh @ d_w.T      # bf16 path: down projection right away
+        Ym = None if f8 else Hh @ d_w.T       # bf16 expert: down projection right away
         return e, (rows, keep, amax, Ym)
 
     h_rows, Y = {}, {}
@@ -411,17 +425,17 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
             continue
         rows, keep, amax, Ym = res
         h_rows.update(keep)
-        if fp8:
+        if expert_fp8[e]:
             h_amax = max(h_amax, amax)
         else:
             for i, p in enumerate(rows):
                 Y[int(p)] = Ym[i]
 
-    if fp8:
+    if any_fp8:
         s_h = np.float32(1.0) if h_amax == 0 else np.float32(h_amax) / np.float32(FP8_FORMATS[fmt][2])
         inter["s_h"] = s_h
 
-        # pass 2: quantised h through the dequantised down projection
+        # pass 2: quantised h of the FP8 experts through their dequantised down projection
         def pass2(e):
             n = int(counts[e])
             pairs = [int(p) for p in sorted_pairs[offsets[e]:offsets[e] + n] if want[int(p) // k]]
@@ -433,7 +447,7 @@ def moe_forward(x, logits, k, w_gate=None, w_up=None, w_down=None, *, fp8=False,
             Ym = Hm @ d_w.T
             return [(p, Ym[i]) for i, p in enumerate(pairs)]
 
-        for res in _map_experts(pass2, active, threads):
+        for res in _map_experts(pass2, [e for e in active if expert_fp8[e]], threads):
             for p, y in res:
                 Y[p] = y
 

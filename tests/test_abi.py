@@ -58,7 +58,7 @@ def test_status_strings(lib):
 @pytest.mark.parametrize("E,k,H,I,dt", [
     (0, 1, 256, 256, 0), (513, 8, 256, 256, 0), (8, 0, 256, 256, 0), (8, 9, 256, 256, 0),
     (8, 17, 256, 256, 0), (32, 17, 256, 256, 0), (8, 2, 200, 256, 0), (8, 2, 256, 100, 0),
-    (8, 2, 0, 256, 0), (8, 2, 256, 256, 3), (8, 2, 32768, 256, 0)])
+    (8, 2, 0, 256, 0), (8, 2, 256, 256, 4), (8, 2, 256, 256, -1), (8, 2, 32768, 256, 0)])
 def test_create_rejects_bad_shapes_without_a_gpu(lib, E, k, H, I, dt):
     h = ctypes.c_void_p()
     assert lib.moe_create(E, k, H, I, dt, ctypes.byref(h)) == -1
