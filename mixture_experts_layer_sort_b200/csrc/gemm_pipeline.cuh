@@ -56,7 +56,7 @@ struct Cfg {
   static constexpr int kKPerBlock = kFP8 ? 128 : 64;                 // elements in one 128-byte row
   static constexpr int kMmaKBytes = 32;                              // K of one MMA = 32 bytes
   static constexpr int kMmasPerBlock = kRowBytes / kMmaKBytes;
-  static_assert(2 * kMaxStages * 8 + 32 + 4 + 16 <= kColTableOffset, "barrier area");
+  static_assert(2 * kMaxStages * 8 + 40 + 4 + 16 <= kColTableOffset, "barrier area");
   static_assert(kColTableOffset + 2 * 2 * 256 * 4 <= kFixedBytes, "column tables");
 };
 
@@ -66,6 +66,7 @@ struct Shared {
   uint64_t* empty;        // [kMaxStages]
   uint64_t* acc_full;     // [2]
   uint64_t* acc_empty;    // [2]
+  uint64_t* drain;        // MMA warp, after a failure: completion of every MMA it issued
   uint32_t* tmem_slot;
   int* flags;             // [0] abort, [1] last arriver, [2..3] epilogue wait outcome
   int* col_tok;           // [2][256]
@@ -82,7 +83,8 @@ __device__ __forceinline__ Shared carve(uint8_t* raw, int extra_bytes) {
   s.empty = s.full + C::kMaxStages;
   s.acc_full = s.empty + C::kMaxStages;
   s.acc_empty = s.acc_full + 2;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.acc_empty + 2);
+  s.drain = s.acc_empty + 2;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
   s.flags = reinterpret_cast<int*>(s.tmem_slot + 1);
   s.col_tok = reinterpret_cast<int*>(base + C::kColTableOffset);
   s.col_w = reinterpret_cast<float*>(base + C::kColTableOffset + 2048);
@@ -105,6 +107,7 @@ __device__ __forceinline__ uint32_t prologue(const Shared& s, int warp) {
       mbar_init(&s.acc_full[b], 1);
       mbar_init(&s.acc_empty[b], kEpiThreads / 32);
     }
+    mbar_init(s.drain, 1);
     for (int i = 0; i < 4; ++i) s.flags[i] = 0;
     fence_barrier_init();
   }
@@ -256,6 +259,12 @@ struct GlobalTiles : UnitSchedule<GlobalTileFn> {
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
 
+// SM cycles a pipeline wait may take before it gives up (GemmArgs::wait_budget, 0 = the
+// default of about a second).
+__device__ __forceinline__ long long wait_budget(const GemmArgs& a) {
+  return a.wait_budget > 0 ? a.wait_budget : (1ll << 31);
+}
+
 // ------------------------------------------------------------------------ producer
 struct ProducerState {
   int stage = 0;
@@ -286,6 +295,9 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
   // the current unit; pad rows re-read row 0 (their columns are never stored)
   int tok[4] = {0, 0, 0, 0};
   const bool direct = hk.direct();
+  // nb: 16-row boxes, or in direct mode the number of valid rows (rows past them are
+  // not loaded: an MMA output column depends on its own activation row only, and the
+  // columns of pad rows are never stored)
   auto load_b = [&](int stg, int kc, int row_start, int nb) {
     uint8_t* bdst = sh.ring + stg * rg.stage_bytes + C::kATiles * C::kABytes;
     if (!direct) {
@@ -295,7 +307,7 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
       #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int j = lane + 32 * i;
-        if (j < nb * 16) tma_load_2d(bdst + j * kRowBytes, tm_b, &sh.full[stg], kc, tok[i], pol_b);
+        if (j < nb) tma_load_2d(bdst + j * kRowBytes, tm_b, &sh.full[stg], kc, tok[i], pol_b);
       }
     }
   };
@@ -330,12 +342,14 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
     const int et = a.w_expert_tiles > 0 ? static_cast<int>(a.w_expert_tiles) : a.w_rblocks * a.kblocks;
     const int wtile = un.t.expert * et + rb0 * a.kblocks;
     const int wtile2 = un.t.expert * et + (rb0 + a.second_rb) * a.kblocks;
-    const uint32_t tx = C::kATiles * C::kABytes + nb16 * 16 * kRowBytes;
+    // activation rows of a stage: 16-row boxes, or (direct mode) the valid rows alone
+    const int nrows = direct ? un.t.n_valid : nb16;
+    const uint32_t tx = C::kATiles * C::kABytes + (direct ? un.t.n_valid : nb16 * 16) * kRowBytes;
     const int dep = hk.dep(un);
     for (int kb = un.kb0; kb < un.kb1; ++kb) {
       int ok = 1;
       if (lane == 0) {
-        ok = mbar_wait_bounded(&sh.empty[ps.stage], ps.phase ^ 1u, abort_flag) ? 1 : 0;
+        ok = mbar_wait_bounded(&sh.empty[ps.stage], ps.phase ^ 1u, abort_flag, wait_budget(a)) ? 1 : 0;
         if (!ok) {
           report_error(a.err, kErrWaitEmpty);
           *abort_flag = 1;
@@ -352,6 +366,9 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
         break;
       }
       if (direct && kb == un.kb0) {
+        // queued activation loads read the previous unit's token rows: issue them
+        // (waiting for their dependency) before the rows change
+        if (npend > 0 && !drain(true)) ps.failed = true;
         // the unit's token rows, read while its first weight tiles are in flight
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -360,14 +377,14 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
         }
       }
       const int kc = kb * C::kKPerBlock;
-      if (npend > 0 && !drain(false)) ps.failed = true;
+      if (!ps.failed && npend > 0 && !drain(false)) ps.failed = true;
       if (!ps.failed && npend == 0 && hk.ready(dep)) {
-        load_b(ps.stage, kc, un.t.row_start, nb16);
+        load_b(ps.stage, kc, un.t.row_start, nrows);
       } else if (!ps.failed) {
         pend_stage[npend] = ps.stage;
         pend_kc[npend] = kc;
         pend_row[npend] = un.t.row_start;
-        pend_nb[npend] = nb16;
+        pend_nb[npend] = nrows;
         pend_dep[npend] = dep;
         if (++npend == rg.stages && !drain(true)) ps.failed = true;
       }
@@ -375,6 +392,13 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
         if (lane == 0) {
           report_error(a.err, kErrWaitDep);
           *abort_flag = 1;
+        }
+        // this stage's weight loads are out: count it, so that producer_quiesce waits
+        // for them before the CTA leaves
+        ++ps.issued;
+        if (++ps.stage == rg.stages) {
+          ps.stage = 0;
+          ps.phase ^= 1u;
         }
         break;
       }
@@ -432,7 +456,7 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
     const uint32_t acc_phase = rg.nbuf == 2 ? ((ms.it >> 1) & 1) : (ms.it & 1);
     const uint32_t d_tmem = tmem + 256u * buf;
     ++ms.it;
-    if (!mbar_wait_bounded(&sh.acc_empty[buf], acc_phase ^ 1u, abort_flag)) {
+    if (!mbar_wait_bounded(&sh.acc_empty[buf], acc_phase ^ 1u, abort_flag, wait_budget(a))) {
       report_error(a.err, kErrWaitAccEmpty);
       *abort_flag = 1;
       ms.failed = true;
@@ -440,7 +464,7 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
     }
     tc_fence_after();
     for (int kb = un.kb0; kb < un.kb1; ++kb) {
-      if (!mbar_wait_bounded(&sh.full[ms.stage], ms.phase, abort_flag)) {
+      if (!mbar_wait_bounded(&sh.full[ms.stage], ms.phase, abort_flag, wait_budget(a))) {
         report_error(a.err, kErrWaitFull);
         *abort_flag = 1;
         ms.failed = true;
@@ -473,6 +497,16 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
     if (ms.failed) break;
     mma_commit(&sh.acc_full[buf]);       // accumulator complete
   }
+}
+
+// After the MMA thread gave up: make every MMA it issued complete (they write TMEM and
+// arrive on stage barriers) before the CTA frees TMEM and leaves. tcgen05.commit
+// tracks all earlier MMAs of the thread; the wait is bounded as well.
+__device__ __forceinline__ void mma_drain(const Shared& sh, const MmaState& ms) {
+  if (!ms.failed) return;
+  int zero = 0;
+  mma_commit(sh.drain);
+  mbar_wait_bounded(sh.drain, 0u, &zero, 1ll << 26);
 }
 
 // ------------------------------------------------------------------------ epilogue
@@ -527,7 +561,7 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
     const uint32_t acc_phase = rg.nbuf == 2 ? ((es.iter >> 1) & 1) : (es.iter & 1);
     const uint32_t t_lane = t_lane0 + 256u * buf;
     ++es.iter;
-    if (epi_tid == 0) *okf = mbar_wait_bounded(&sh.acc_full[buf], acc_phase, abort_flag) ? 1 : 0;
+    if (epi_tid == 0) *okf = mbar_wait_bounded(&sh.acc_full[buf], acc_phase, abort_flag, wait_budget(a)) ? 1 : 0;
     named_bar_sync(1, kEpiThreads);
     if (*okf == 0) {
       if (epi_tid == 0) {

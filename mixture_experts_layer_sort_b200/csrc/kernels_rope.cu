@@ -19,11 +19,12 @@
 // A position outside [0, max_pos) has no table row: its vector gets codes 0 and a
 // NaN scale (no out-of-bounds read).
 //
-// Layout and roofline: one warp per vector, lane l holding D/32 consecutive values (so
-// a warp's load of a vector is one coalesced 2D-byte access and the half-split
-// partner of lane l is lane l ^ 16); four vectors per warp are in flight at once. The
-// kernel moves 2D bytes in and D + 4 bytes out per vector (the table rows are shared
-// by a token's heads and stay in cache): it is HBM-bound.
+// Layout and roofline: one warp per token; lane l holds D/32 consecutive values of a
+// head vector (a warp's load of a vector is one coalesced 2D-byte access and the
+// half-split partner of lane l is lane l ^ 16). The position and the table row are
+// read once per token, and eight head vectors of the token are in flight at once.
+// The kernel moves 2D bytes in and D + 4 bytes out per vector, plus 4 + 4D bytes per
+// token: it is HBM-bound.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -40,7 +41,7 @@ namespace moe {
 namespace {
 
 constexpr int kRopeThreads = 256;
-constexpr int kRopeUnroll = 4;     // vectors per warp in flight
+constexpr int kRopeUnroll = 8;     // heads of a token per warp in flight
 
 struct RopeArgs {
   const __nv_bfloat16* x;   // [T, NH, D]
@@ -103,7 +104,9 @@ __device__ __forceinline__ void store_codes(uint8_t* p, const unsigned short (&c
   }
 }
 
-// D = 32 * CH values per vector.
+// D = 32 * CH values per vector. One warp per token: the position and the token's
+// cos/sin row are loaded once, then the token's heads kRopeUnroll at a time, all
+// their loads issued before any value is used.
 template <int CH>
 __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) {
   constexpr int D = 32 * CH;
@@ -117,77 +120,79 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) 
   // (angle i mod D/2), interleaved pairs 2i with 2i + 1 (angle i)
   const int ang0 = a.interleaved ? lane * CH / 2 : (lane & 15) * CH;
   const bool upper = lane >= 16;   // half-split: this lane holds the b' of its pairs
-  for (long long v0 = gwarp * kRopeUnroll; v0 < a.nvec; v0 += nwarps * kRopeUnroll) {
-    float x[kRopeUnroll][CH];
-    int pos[kRopeUnroll];
-    #pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      const long long v = v0 + u;
-      pos[u] = -1;
-      if (v < a.nvec) {
-        load_bf16<CH>(a.x + v * D + lane * CH, x[u]);
-        pos[u] = __ldg(a.positions + v / a.NH);
+  const long long T = a.nvec / a.NH;
+  for (long long t = gwarp; t < T; t += nwarps) {
+    const int pos = __ldg(a.positions + t);       // the same for the whole warp
+    const bool valid = pos >= 0 && pos < a.max_pos;
+    // this lane's angles: CH of them (half-split) or CH/2 (interleaved)
+    float c[CH], s[CH];
+    if (valid) {
+      const float* row = a.cos_sin + static_cast<long long>(pos) * D;
+      if (a.interleaved) {
+        #pragma unroll
+        for (int q = 0; q < CH / 2; ++q) {
+          c[q] = __ldg(row + ang0 + q);
+          s[q] = __ldg(row + D / 2 + ang0 + q);
+        }
+      } else {
+        load_f32<CH>(row + ang0, c);
+        load_f32<CH>(row + D / 2 + ang0, s);
       }
     }
-    #pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      const long long v = v0 + u;
-      if (v >= a.nvec) break;   // warp-uniform
-      const bool valid = pos[u] >= 0 && pos[u] < a.max_pos;
-      float y[CH];
-      if (valid) {
-        const float* row = a.cos_sin + static_cast<long long>(pos[u]) * D;
-        if (a.interleaved) {
-          float c[CH / 2], s[CH / 2];
-          #pragma unroll
-          for (int q = 0; q < CH / 2; ++q) {
-            c[q] = __ldg(row + ang0 + q);
-            s[q] = __ldg(row + D / 2 + ang0 + q);
+    for (int h0 = 0; h0 < a.NH; h0 += kRopeUnroll) {
+      float x[kRopeUnroll][CH];
+      #pragma unroll
+      for (int u = 0; u < kRopeUnroll; ++u)
+        if (h0 + u < a.NH) load_bf16<CH>(a.x + (t * a.NH + h0 + u) * D + lane * CH, x[u]);
+      #pragma unroll
+      for (int u = 0; u < kRopeUnroll; ++u) {
+        if (h0 + u >= a.NH) break;   // warp-uniform
+        const long long v = t * a.NH + h0 + u;
+        float y[CH];
+        if (valid) {
+          if (a.interleaved) {
+            #pragma unroll
+            for (int q = 0; q < CH / 2; ++q) {
+              const float pa = x[u][2 * q], pb = x[u][2 * q + 1];
+              y[2 * q] = __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
+              y[2 * q + 1] = __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]));
+            }
+          } else {
+            #pragma unroll
+            for (int q = 0; q < CH; ++q) {
+              const float other = __shfl_xor_sync(0xFFFFFFFFu, x[u][q], 16);
+              const float pa = upper ? other : x[u][q];
+              const float pb = upper ? x[u][q] : other;
+              y[q] = upper ? __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]))
+                           : __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
+            }
           }
+        } else {   // (valid is the same for the whole warp: the shuffles above stay uniform)
           #pragma unroll
-          for (int q = 0; q < CH / 2; ++q) {
-            const float pa = x[u][2 * q], pb = x[u][2 * q + 1];
-            y[2 * q] = __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
-            y[2 * q + 1] = __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]));
-          }
-        } else {
-          float c[CH], s[CH];
-          load_f32<CH>(row + ang0, c);
-          load_f32<CH>(row + D / 2 + ang0, s);
-          #pragma unroll
-          for (int q = 0; q < CH; ++q) {
-            const float other = __shfl_xor_sync(0xFFFFFFFFu, x[u][q], 16);
-            const float pa = upper ? other : x[u][q];
-            const float pb = upper ? x[u][q] : other;
-            y[q] = upper ? __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]))
-                         : __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
-          }
+          for (int q = 0; q < CH; ++q) y[q] = 0.f;
         }
-      } else {   // (valid is the same for the whole warp: the shuffles above stay uniform)
+        float m = 0.f;
         #pragma unroll
-        for (int q = 0; q < CH; ++q) y[q] = 0.f;
+        for (int q = 0; q < CH; ++q) m = fmaxf(m, fabsf(y[q]));
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        const float sc = m == 0.f ? 1.f : __fdiv_rn(m, fmax);
+        unsigned short cd[CH / 2];
+        #pragma unroll
+        for (int q = 0; q < CH / 2; ++q)
+          cd[q] = valid ? fp8x2(make_float2(__fdiv_rn(y[2 * q], sc), __fdiv_rn(y[2 * q + 1], sc)), a.f8)
+                        : static_cast<unsigned short>(0);
+        store_codes<CH>(a.codes + v * D + lane * CH, cd);
+        if (lane == 0) a.scales[v] = valid ? sc : __int_as_float(0x7FC00000);
       }
-      float m = 0.f;
-      #pragma unroll
-      for (int q = 0; q < CH; ++q) m = fmaxf(m, fabsf(y[q]));
-      #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-      const float sc = m == 0.f ? 1.f : __fdiv_rn(m, fmax);
-      unsigned short cd[CH / 2];
-      #pragma unroll
-      for (int q = 0; q < CH / 2; ++q)
-        cd[q] = valid ? fp8x2(make_float2(__fdiv_rn(y[2 * q], sc), __fdiv_rn(y[2 * q + 1], sc)), a.f8)
-                      : static_cast<unsigned short>(0);
-      store_codes<CH>(a.codes + v * D + lane * CH, cd);
-      if (lane == 0) a.scales[v] = valid ? sc : __int_as_float(0x7FC00000);
     }
   }
 }
 
 template <int CH>
 cudaError_t launch_rope(const RopeArgs& a, cudaStream_t s) {
-  const long long per_block = (kRopeThreads / 32) * kRopeUnroll;
-  long long blocks = (a.nvec + per_block - 1) / per_block;
+  const long long per_block = kRopeThreads / 32;   // tokens per block and round
+  long long blocks = (a.nvec / a.NH + per_block - 1) / per_block;
   const long long cap = 8ll * sm_count();
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;

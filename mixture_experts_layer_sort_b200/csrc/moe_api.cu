@@ -206,6 +206,7 @@ int fp8_format(const moe_layer* L) { return L->dtype == MOE_DTYPE_FP8_E5M2 ? 1 :
 
 int ensure_workspace(moe_layer* L, int M) {
   if (M <= L->M_cap) return MOE_OK;
+  if (moe::fail_workspace_alloc()) return MOE_ERR_OOM;   // injected failure (tests): nothing allocated
   int cap = 64;
   while (cap < M) cap *= 2;
   MOE_CUDA(cudaDeviceSynchronize());   // the old workspace may still be in use
@@ -433,6 +434,7 @@ int forward_fused_decode(moe_layer* L, const void* x, const float* logits, int M
   g.k = L->k;
   g.P = M * L->k;
   g.err = L->err;
+  g.wait_budget = moe::wait_budget_cycles();
   g.w_scales = L->wscales;
   g.f8 = fp8_format(L);
   d.g1 = g;
@@ -604,6 +606,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g.P = static_cast<int>(P);
   g.f8 = fp8_format(L);
   g.err = L->err;
+  g.wait_budget = moe::wait_budget_cycles();
 
   moe::GemmArgs g1 = g;
   g1.tiles = L->tiles1;
@@ -771,6 +774,7 @@ int forward_mixed(moe_layer* L, const void* x, const float* logits, int M, void*
   g.P = static_cast<int>(P);
   g.f8 = f8;
   g.err = L->err;
+  g.wait_budget = moe::wait_budget_cycles();
 
   // gate_up: FP8 experts, then bf16 experts (bf16-sized expert slots in both)
   moe::GemmArgs g1 = g;
@@ -868,6 +872,16 @@ bool moe::pdl_enabled() {
     return !(e && e[0] == '1');
   }();
   return on;
+}
+
+long long moe::wait_budget_cycles() {
+  const char* e = std::getenv("MOE_WAIT_BUDGET_CYCLES");
+  return e ? std::atoll(e) : 0;
+}
+
+bool moe::fail_workspace_alloc() {
+  const char* e = std::getenv("MOE_TEST_FAIL_WORKSPACE");
+  return e != nullptr && e[0] == '1';
 }
 
 int moe::sm_count() {

@@ -140,6 +140,7 @@ struct GemmArgs {
   const int* direct_pairs; // gate_up only: B rows are x rows of token pairs[row]/k (x map box = 1 row)
   int f8;                  // FP8 layers: code format of weights and activations (Fp8Format)
   int* err;
+  long long wait_budget;   // SM cycles a pipeline wait may take (0: about a second)
 };
 
 struct QuantHArgs {
@@ -172,6 +173,13 @@ int sm_count();
 // MOE_UNIFORM_SPLITS=1 replaces the balanced unit schedule by one split factor per GEMM
 bool uniform_splits();
 int gemm_max_stages(bool gate_up);   // ring depth cap (MOE_MAX_STAGES1/2 override, for tuning)
+// Budget of the GEMMs' pipeline waits in SM cycles: 0 (the default, about a second)
+// unless MOE_WAIT_BUDGET_CYCLES is set; read at every forward, so that a test can make
+// a wait run out on purpose and then restore the default in the same process.
+long long wait_budget_cycles();
+// MOE_TEST_FAIL_WORKSPACE=1 (read at every forward): the workspace allocation reports
+// an out-of-memory failure without allocating (a host-side failure injection for tests).
+bool fail_workspace_alloc();
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                                  Args... args) {

@@ -199,6 +199,7 @@ int forward_noalloc(const moe::LayerView& v, const void* x, const float* logits,
   g.P = static_cast<int>(P);
   g.f8 = v.f8;
   g.err = static_cast<int*>(base);
+  g.wait_budget = moe::wait_budget_cycles();
 
   moe::GemmArgs g1 = g;
   g1.tiles = tiles1;
