@@ -542,15 +542,23 @@ def measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on):
         with torch.cuda.stream(stream):
             for _ in range(3):
                 inv_rope_fp8_quant(x, pos, table, codes=codes, scales=scales, stream=stream)
+        torch.cuda.synchronize()
+        # replayed from a CUDA graph like the layer, so that no host launch gap is timed
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            inv_rope_fp8_quant(x, pos, table, codes=codes, scales=scales, stream=stream)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
             ev = []
             for _ in range(steps):
                 flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                inv_rope_fp8_quant(x, pos, table, codes=codes, scales=scales, stream=stream)
+                graph.replay()
                 e1.record(stream)
                 ev.append((e0, e1))
         torch.cuda.synchronize()
+        del graph
         ms = sorted(a.elapsed_time(b) for a, b in ev)
         mean = statistics.mean(ms)
         alg = T * NH * (2 * D + D + 4) + T * 4

@@ -66,12 +66,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed. Gives up after
 // roughly `budget_cycles` SM clock cycles, or as soon as *abort is set by another
-// role of the CTA; returns false in both cases. Never spins forever.
+// role of the CTA; returns false in both cases. Never spins forever. try_wait may
+// suspend the thread for a while inside the instruction, so a short budget (a test
+// that makes waits run out on purpose) polls with test_wait and reads the clock after
+// every poll instead.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort,
                                                   long long budget_cycles = (1ll << 31)) {
+  if (budget_cycles < (1ll << 20)) {
+    const long long t0 = clock64();
+    while (true) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (*abort) return false;
+      if (clock64() - t0 > budget_cycles) return false;
+    }
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
