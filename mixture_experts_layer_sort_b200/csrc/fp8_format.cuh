@@ -24,6 +24,31 @@ __device__ __forceinline__ float fp8_scale_from_amax(unsigned amax_bits, int fmt
   return amax == 0.f ? 1.f : __fdiv_rn(amax, fp8_max(fmt));
 }
 
+// Division of many values by one scale s, correctly rounded like an IEEE fp32 division
+// but with one reciprocal per scale: Markstein's division (the theorem that, with r the
+// correctly rounded reciprocal of s and q = RN(y * r), the remainder y - q * s is exact
+// in one fused multiply-add and RN(q + rem * r) is the correctly rounded quotient;
+// P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34 (1990); Handbook of Floating-Point Arithmetic,
+// Muller et al., chapter on division). It holds for normal s away from the ends of the
+// range, which `ScaleDiv` checks once, falling back to __fdiv_rn. A zero remainder
+// keeps q itself (and the sign of a zero quotient). The tests compare every code with
+// a plain IEEE division.
+struct ScaleDiv {
+  float s, r;
+  bool fast;
+  __device__ __forceinline__ explicit ScaleDiv(float s_) : s(s_) {
+    fast = s_ >= 0x1p-120f && s_ <= 0x1p120f;
+    r = fast ? __frcp_rn(s_) : 1.f;
+  }
+  __device__ __forceinline__ float operator()(float y) const {
+    if (!fast) return __fdiv_rn(y, s);
+    const float q = __fmul_rn(y, r);
+    const float rem = __fmaf_rn(-q, s, y);
+    return rem == 0.f ? q : __fmaf_rn(rem, r, q);
+  }
+};
+
 // two fp32 values -> two codes (low byte = v.x), round to nearest even, saturating
 __device__ __forceinline__ unsigned short fp8x2(float2 v, int fmt) {
   return static_cast<unsigned short>(

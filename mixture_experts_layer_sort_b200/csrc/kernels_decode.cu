@@ -284,11 +284,11 @@ struct DownHooks {
   }
 };
 
-// 8 fp32 values -> 8 FP8 codes (RNE, saturating), v[i] / s with IEEE division.
-__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, int f8) {
+// 8 fp32 values -> 8 FP8 codes (RNE, saturating), v[i] / s correctly rounded.
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], const ScaleDiv& dv, int f8) {
   unsigned short c[4];
   #pragma unroll
-  for (int q = 0; q < 4; ++q) c[q] = fp8x2(make_float2(__fdiv_rn(v[2 * q], s), __fdiv_rn(v[2 * q + 1], s)), f8);
+  for (int q = 0; q < 4; ++q) c[q] = fp8x2(make_float2(dv(v[2 * q]), dv(v[2 * q + 1])), f8);
   uint2 r;
   r.x = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
   r.y = static_cast<unsigned>(c[2]) | (static_cast<unsigned>(c[3]) << 16);
@@ -300,6 +300,7 @@ __device__ __forceinline__ void quant_row(const __nv_bfloat16* src, uint8_t* dst
                                           int epi_tid) {
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
   uint2* d2 = reinterpret_cast<uint2*>(dst);
+  const ScaleDiv dv(s);
   for (int i = epi_tid; i < n / 8; i += kEpiThreads) {
     const uint4 u = __ldcg(s4 + i);
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -310,7 +311,7 @@ __device__ __forceinline__ void quant_row(const __nv_bfloat16* src, uint8_t* dst
       f[2 * q] = v.x;
       f[2 * q + 1] = v.y;
     }
-    d2[i] = quant8(f, s, f8);
+    d2[i] = quant8(f, dv, f8);
   }
 }
 

@@ -177,11 +177,11 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) 
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
         const float sc = m == 0.f ? 1.f : __fdiv_rn(m, fmax);
+        const ScaleDiv dv(sc);   // y / sc, correctly rounded, one reciprocal per vector
         unsigned short cd[CH / 2];
         #pragma unroll
         for (int q = 0; q < CH / 2; ++q)
-          cd[q] = valid ? fp8x2(make_float2(__fdiv_rn(y[2 * q], sc), __fdiv_rn(y[2 * q + 1], sc)), a.f8)
-                        : static_cast<unsigned short>(0);
+          cd[q] = valid ? fp8x2(make_float2(dv(y[2 * q]), dv(y[2 * q + 1])), a.f8) : static_cast<unsigned short>(0);
         store_codes<CH>(a.codes + v * D + lane * CH, cd);
         if (lane == 0) a.scales[v] = valid ? sc : __int_as_float(0x7FC00000);
       }
@@ -229,6 +229,7 @@ extern "C" int moe_inv_rope_fp8_quant(const void* x, const int* positions, const
   a.f8 = fp8_format == MOE_DTYPE_FP8_E5M2 ? moe::kFp8E5M2 : moe::kFp8E4M3;
   a.interleaved = interleaved;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  moe::NvtxRange range("moe_inv_rope_fp8_quant");
   cudaError_t e = head_dim == 64 ? moe::launch_rope<2>(a, st)
                                  : (head_dim == 128 ? moe::launch_rope<4>(a, st) : moe::launch_rope<8>(a, st));
   if (e != cudaSuccess) {

@@ -54,13 +54,13 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   }
 }
 
-// 8 fp32 values -> 8 FP8 codes (RNE, saturating), v[i] / s with IEEE division.
-__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, int f8) {
+// 8 fp32 values -> 8 FP8 codes (RNE, saturating), v[i] / s correctly rounded.
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], const ScaleDiv& dv, int f8) {
   uint2 r;
   unsigned short c[4];
   #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    float2 f = make_float2(__fdiv_rn(v[2 * q], s), __fdiv_rn(v[2 * q + 1], s));
+    float2 f = make_float2(dv(v[2 * q]), dv(v[2 * q + 1]));
     c[q] = fp8x2(f, f8);
   }
   r.x = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
@@ -88,6 +88,7 @@ constexpr int kRowsPerBlock = 256 / kRowThreads;
 template <bool kFP8, bool kCoherent>
 __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, void* __restrict__ dst, int n8, float s,
                                          int f8, int t) {
+  const ScaleDiv dv(s);
   for (int base = t; base < n8; base += kRowThreads * 8) {
     uint4 v[8];
     #pragma unroll
@@ -102,7 +103,7 @@ __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, void* __
         } else {
           float f[8];
           bf16x8_to_f32(v[j], f);
-          reinterpret_cast<uint2*>(dst)[i] = quant8(f, s, f8);
+          reinterpret_cast<uint2*>(dst)[i] = quant8(f, dv, f8);
         }
       }
     }

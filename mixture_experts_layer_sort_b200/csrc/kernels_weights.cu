@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(256) weight_quant_tiled_kernel(int f8, const u
     const long long e = row / g.rows;
     const long long r = row - e * g.rows;
     if (g.expert_mask != nullptr && g.expert_mask[e] != g.mask_value) continue;
-    const float s = __ldg(scales + e * stride);
+    const ScaleDiv dv(__ldg(scales + e * stride));
     // 8 bf16 source values = 16 bytes at column c of the row-major source
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(w + rowmajor_offset(g, e, r, 2 * c)));
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(256) weight_quant_tiled_kernel(int f8, const u
     #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 f = __bfloat1622float2(p[q]);
-      const float2 d = make_float2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s));
+      const float2 d = make_float2(dv(f.x), dv(f.y));
       c2[q] = fp8x2(d, f8);
     }
     uint2 o;

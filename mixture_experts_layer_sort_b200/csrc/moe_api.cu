@@ -331,12 +331,17 @@ cudaEvent_t pool_event(moe_layer* L) {
 }
 
 // Records an event pair around one kernel launch when profiling is on.
+// NVTX names of the kernel slots (the profiling slots of moe_profile_read)
+const char* const kSlotNames[MOE_PROFILE_SLOTS] = {"moe route", "moe align", "moe gather", "moe gate_up GEMM",
+                                                   "moe quant_h", "moe down GEMM", "moe finalize"};
+
 struct KernelTimer {
   moe_layer* L;
   int slot;
   cudaStream_t st;
   cudaEvent_t a = nullptr;
-  KernelTimer(moe_layer* l, int s, cudaStream_t stream) : L(l), slot(s), st(stream) {
+  moe::NvtxRange range;
+  KernelTimer(moe_layer* l, int s, cudaStream_t stream) : L(l), slot(s), st(stream), range(kSlotNames[s]) {
     if (L->profiling && (a = pool_event(L)) != nullptr) cudaEventRecord(a, st);
   }
   ~KernelTimer() {
@@ -1128,6 +1133,7 @@ int moe_forward(moe_layer* L, const void* x, const float* logits, int M, void* o
   if (M > (1 << 22) / L->k) return MOE_ERR_INVALID_ARG;
   if (!x || !logits || !out || !aligned16(x) || !aligned16(logits) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   DeviceGuard g(L->device);
+  moe::NvtxRange range("moe_forward");
   return forward_impl(L, x, logits, M, out, static_cast<cudaStream_t>(stream));
 }
 
@@ -1224,6 +1230,7 @@ int moe_forward_host(moe_layer* L, const void* x_host, const float* logits_host,
     L->host_cap = M;
   }
   MOE_TRY(ensure_workspace(L, M));   // (re)allocation happens here, never inside a capture
+  moe::NvtxRange range("moe_forward_host");
   // Pinned buffers: one graph launch instead of three copies and five to ten kernel
   // launches from the host. Pageable buffers, profiling and the single-launch decode
   // kernel take the eager path.

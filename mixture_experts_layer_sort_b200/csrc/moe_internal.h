@@ -4,9 +4,20 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace moe {
+
+// An NVTX range around a host-side scope (a forward pass, one kernel launch, a weight
+// load), so that a timeline tool shows the layer's steps by name. Header-only NVTX3:
+// without a tool attached a push/pop costs a pointer test.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kPadRows = 16;        // every expert's group of rows is padded to 16 (B tile granule)
 constexpr int kTileRows = 128;      // weight rows per GEMM tile (the MMA's M slot)

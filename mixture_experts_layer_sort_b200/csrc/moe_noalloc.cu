@@ -278,6 +278,7 @@ extern "C" int moe_forward_noalloc(moe_layer* layer, const void* x, const float*
   int prev = -1;
   NA_CUDA(cudaGetDevice(&prev));
   if (prev != v.device) NA_CUDA(cudaSetDevice(v.device));
+  moe::NvtxRange range("moe_forward_noalloc");
   const int status = forward_noalloc(v, x, router_logits, M, out, static_cast<cudaStream_t>(stream));
   if (prev != v.device) cudaSetDevice(prev);
   return status;
