@@ -35,6 +35,7 @@
 // All CTAs must be resident at once (they wait on each other): the launch is
 // cooperative, one CTA per SM. Every wait is bounded and reports through the error
 // word when it gives up.
+#include "decode_sched.cuh"
 #include "fp8_format.cuh"
 #include "gemm_pipeline.cuh"
 #include "route_common.cuh"
@@ -44,11 +45,6 @@ namespace moe {
 namespace {
 
 using namespace pipe;
-
-constexpr int kMaxTokens = 64;     // per-expert token masks are 64 bits
-constexpr int kMaxPairs = 512;
-constexpr int kMaxExperts = 512;
-constexpr int kBalancedWaves = 8;  // as in the chain's align kernel
 
 // Global sync words (zero between launches; the last CTA resets them):
 enum SyncSlot : int {
@@ -67,7 +63,7 @@ struct DecodeArgs {
   const __nv_bfloat16* x;
   __nv_bfloat16* out;
   int M, E, k, H, I, P;
-  int ws1_rows_cap, max_stages, f8;
+  int ws1_rows_cap, max_stages, f8, uniform;
   int* sync;
   uint8_t* xq;             // FP8: [M, H] codes of x
   uint8_t* hq;             // FP8: [rows, I] codes of h (the down GEMM's activation)
@@ -82,24 +78,6 @@ struct DecodeArgs {
   GemmArgs g1, g2;
 };
 
-// Shared-memory schedule (the pipeline's "extra" region).
-struct Sched {
-  int ids[kMaxPairs];
-  float w[kMaxPairs];
-  int count[kMaxExperts];
-  int off[kMaxExperts + 1];       // compact offsets of each expert's pairs
-  int poff[kMaxExperts + 1];      // padded offsets (rows of h)
-  int tmp[kMaxExperts + 1];
-  int act[kMaxExperts];           // active experts, ascending
-  int aidx[kMaxExperts + 1];      // index of each expert among the active ones
-  unsigned mask[kMaxExperts][2];  // tokens routed to each expert
-  int pairs[kMaxPairs];           // pair ids grouped by expert, ascending inside an expert
-  int done[256];                  // tokens completed by the current down unit
-  float red[8];                   // block reduction scratch
-  int ndone;
-  int nact, T1, S1, T2, S2, n_max, rows_used, flag;
-};
-
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -109,22 +87,6 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
-
-// Tile t of a GEMM from the shared schedule: tile t = (active expert t / fb, row block
-// t % fb); every expert has a single token tile (n_e <= M <= 64).
-struct SmemTileFn {
-  const Sched* s;
-  int fb;
-  __device__ __forceinline__ Tile operator()(int t) const {
-    const int ai = t / fb;
-    Tile tile;
-    tile.expert = s->act[ai];
-    tile.fblock = t - ai * fb;
-    tile.row_start = s->poff[tile.expert];
-    tile.n_valid = s->count[tile.expert];
-    return tile;
-  }
-};
 
 // Bounded wait of one thread until *p >= target (acquire); false when it gave up.
 __device__ __forceinline__ bool wait_counter(const int* p, int target, volatile int* abort_flag) {
@@ -374,11 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) s->red[warp] = m;
     }
   }
-  for (int e = tid; e < E; e += kThreads) {
-    s->count[e] = 0;
-    s->mask[e][0] = 0u;
-    s->mask[e][1] = 0u;
-  }
+  sched_clear(s, E, tid, kThreads);
   __syncthreads();
   if constexpr (kFP8) {
     if (c < M && tid == 0) {
@@ -392,76 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int t = warp; t < M; t += kThreads / 32)
     route_token_any(s_logits + static_cast<size_t>(t) * E, E, k, lane, s->ids + t * k, s->w + t * k);
   __syncthreads();
-  for (int p = tid; p < P; p += kThreads) {
-    const int e = s->ids[p];
-    const int t = p / k;
-    atomicAdd(&s->count[e], 1);
-    atomicOr(&s->mask[e][t >> 5], 1u << (t & 31));
-  }
-  __syncthreads();
-  if (warp == 0) {
-    warp_exclusive_scan(s->count, s->off, E, lane);
-  } else if (warp == 1) {
-    for (int e = lane; e < E; e += 32) s->act[e] = (s->count[e] + kPadRows - 1) / kPadRows * kPadRows;
-    __syncwarp();
-    warp_exclusive_scan(s->act, s->poff, E, lane);
-  }
-  __syncthreads();
-  if (warp == 0) {
-    for (int e = lane; e < E; e += 32) s->tmp[e] = s->count[e] > 0 ? 1 : 0;
-    __syncwarp();
-    warp_exclusive_scan(s->tmp, s->aidx, E, lane);
-    __syncwarp();
-    for (int e = lane; e < E; e += 32)
-      if (s->count[e] > 0) s->act[s->aidx[e]] = e;
-    if (lane == 0) s->nact = s->aidx[E];
-  }
-  __syncthreads();
-  // stable grouping: rank of pair (t, j) inside expert e = tokens t' < t routed to e
-  for (int p = tid; p < P; p += kThreads) {
-    const int e = s->ids[p];
-    const int t = p / k;
-    const unsigned lo = t < 32 ? (s->mask[e][0] & ((1u << t) - 1u)) : s->mask[e][0];
-    const unsigned hi = t < 32 ? 0u : (s->mask[e][1] & ((1u << (t - 32)) - 1u));
-    s->pairs[s->off[e] + __popc(lo) + __popc(hi)] = p;
-  }
   const int fb1 = d.I / kTileRows;
   const int fb2 = (d.H / kTileRows + 1) / 2;
   const int kb1 = d.H / C::kKPerBlock;
   const int kb2 = d.I / C::kKPerBlock;
-  if (warp == 0) {
-    int m = 0;
-    for (int e = lane; e < E; e += 32) m = max(m, s->count[e]);
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    const int A = s->nact;
-    const int rows_used = s->poff[E];
-    const int n_mean = A > 0 ? (P + A - 1) / A : 0;
-    const int t1 = A * fb1;
-    // the chain's rule: the balanced schedule (0) for one to kBalancedWaves waves of
-    // tiles when the partial sums fit, else the cost model's split factor
-    const bool allow = rows_used <= d.ws1_rows_cap;
-    const int s1 = (allow && t1 >= G && t1 < kBalancedWaves * G)
-                       ? 0
-                       : choose_splits_warp(t1, kb1, G, allow, 2 * 16384 + n_mean * 128, n_mean * 256 * 4 * 2, lane);
-    if (lane == 0) {
-      s->n_max = (m + kPadRows - 1) / kPadRows * kPadRows;
-      s->rows_used = rows_used;
-      s->T1 = t1;
-      s->S1 = s1;
-    }
-  } else if (warp == 1) {
-    const int A = s->nact;
-    const int n_mean = A > 0 ? (P + A - 1) / A : 0;
-    const int t2 = A * fb2;
-    const int s2 = (t2 >= G && t2 < kBalancedWaves * G)
-                       ? 0
-                       : choose_splits_warp(t2, kb2, G, true, 16384 + n_mean * 128, n_mean * 128 * 4, lane);
-    if (lane == 0) {
-      s->T2 = t2;
-      s->S2 = s2;
-    }
-  }
+  sched_build(s, P, E, k, fb1, fb2, kb1, kb2, G, d.ws1_rows_cap, d.uniform, tid, kThreads);
   // the staged logits are dead from here on: order their generic-proxy accesses before
   // the TMA writes that reuse the ring
   fence_proxy_async_smem();
@@ -557,17 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       d.topk_ids[p] = s->ids[p];
       d.topk_w[p] = s->w[p];
     }
-    for (int e = tid; e < E; e += kThreads) {
-      d.counts[e] = s->count[e];
-      d.padded_offsets[e] = s->poff[e];
-      for (int r = s->poff[e]; r < s->poff[e + 1]; ++r) {
-        const int j = r - s->poff[e];
-        d.padded_pairs[r] = j < s->count[e] ? s->pairs[s->off[e] + j] : P;
-      }
-    }
+    sched_publish(s, P, E, d.counts, d.padded_offsets, d.padded_pairs, d.header, tid, kThreads);
     if (tid == 0) {
-      d.padded_offsets[E] = s->poff[E];
-      d.header[kHdrRowsUsed] = s->rows_used;
       if constexpr (kFP8) {
         d.last_scales[0] = fp8_scale_from_amax(__ldcg(reinterpret_cast<const unsigned*>(d.sync + kSyncAmaxX)), d.f8);
         d.last_scales[1] = fp8_scale_from_amax(__ldcg(reinterpret_cast<const unsigned*>(d.sync + kSyncAmaxH)), d.f8);
@@ -596,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-bool decode_supported(int M, int E, int k) { return M >= 1 && M <= kMaxTokens && E <= kMaxExperts && M * k <= kMaxPairs; }
+bool decode_supported(int M, int E, int k) { return sched_supported(M, E, k); }
 
 size_t decode_sync_words(int E, int M_cap) { return static_cast<size_t>(kSyncFixed + E + M_cap); }
 
@@ -622,6 +506,7 @@ cudaError_t launch_decode(const DecodeLaunch& l, cudaStream_t st) {
   d.ws1_rows_cap = l.ws1_rows_cap;
   d.max_stages = l.max_stages;
   d.f8 = l.f8;
+  d.uniform = uniform_splits() ? 1 : 0;
   d.sync = l.sync;
   d.xq = l.xq;
   d.hq = l.hq;

@@ -19,12 +19,13 @@
 // A position outside [0, max_pos) has no table row: its vector gets codes 0 and a
 // NaN scale (no out-of-bounds read).
 //
-// Layout and roofline: one warp per token; lane l holds D/32 consecutive values of a
-// head vector (a warp's load of a vector is one coalesced 2D-byte access and the
-// half-split partner of lane l is lane l ^ 16). The position and the table row are
-// read once per token, and eight head vectors of the token are in flight at once.
-// The kernel moves 2D bytes in and D + 4 bytes out per vector, plus 4 + 4D bytes per
-// token: it is HBM-bound.
+// Layout and roofline: one warp per token; a head vector is spread over D/16 lanes,
+// 16 consecutive values (32 bytes in, 16 bytes of codes out) per lane, so that the
+// per-vector work (the max reduction, the scale, its reciprocal) is shared by 16 values
+// and a warp covers 512/D vectors per pass; the half-split partner of a value sits D/32
+// lanes away. The position and the lane's part of the table row are read once per
+// token, and two passes of vectors are in flight at once. The kernel moves 2D bytes in
+// and D + 4 bytes out per vector, plus 4 + 4D bytes per token: it is HBM-bound.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -41,7 +42,6 @@ namespace moe {
 namespace {
 
 constexpr int kRopeThreads = 256;
-constexpr int kRopeUnroll = 8;     // heads of a token per warp in flight
 
 struct RopeArgs {
   const __nv_bfloat16* x;   // [T, NH, D]
@@ -54,113 +54,97 @@ struct RopeArgs {
   int interleaved;
 };
 
-template <int CH>
-struct Vec {
-  float v[CH];
-};
+constexpr int kEPL = 16;   // values of a head vector per lane
 
-// CH consecutive bf16 values (4, 8 or 16 bytes) -> fp32
-template <int CH>
-__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&v)[CH]) {
-  if constexpr (CH == 2) {
-    const __nv_bfloat162 u = *reinterpret_cast<const __nv_bfloat162*>(p);
-    const float2 f = __bfloat1622float2(u);
-    v[0] = f.x;
-    v[1] = f.y;
-  } else {
-    using U = typename std::conditional<CH == 4, uint2, uint4>::type;
-    const U u = __ldg(reinterpret_cast<const U*>(p));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-    #pragma unroll
-    for (int q = 0; q < CH / 2; ++q) {
-      const float2 f = __bfloat1622float2(h[q]);
-      v[2 * q] = f.x;
-      v[2 * q + 1] = f.y;
-    }
+// 16 consecutive bf16 values (32 bytes) -> fp32
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[kEPL]) {
+  const uint4 u[2] = {__ldg(reinterpret_cast<const uint4*>(p)), __ldg(reinterpret_cast<const uint4*>(p) + 1)};
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(u);
+  #pragma unroll
+  for (int q = 0; q < kEPL / 2; ++q) {
+    const float2 f = __bfloat1622float2(h[q]);
+    v[2 * q] = f.x;
+    v[2 * q + 1] = f.y;
   }
 }
 
-template <int CH>
-__device__ __forceinline__ void load_f32(const float* p, float (&v)[CH]) {
+// n consecutive fp32 values (n a multiple of 4, 16-byte aligned)
+template <int n>
+__device__ __forceinline__ void load_f32(const float* p, float* v) {
   #pragma unroll
-  for (int q = 0; q < CH; q += 2) {
-    const float2 f = __ldg(reinterpret_cast<const float2*>(p + q));
+  for (int q = 0; q < n; q += 4) {
+    const float4 f = __ldg(reinterpret_cast<const float4*>(p + q));
     v[q] = f.x;
     v[q + 1] = f.y;
+    v[q + 2] = f.z;
+    v[q + 3] = f.w;
   }
 }
 
-template <int CH>
-__device__ __forceinline__ void store_codes(uint8_t* p, const unsigned short (&c)[CH / 2]) {
-  if constexpr (CH == 2) {
-    *reinterpret_cast<unsigned short*>(p) = c[0];
-  } else if constexpr (CH == 4) {
-    *reinterpret_cast<unsigned*>(p) = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
-  } else {
-    uint2 o;
-    o.x = static_cast<unsigned>(c[0]) | (static_cast<unsigned>(c[1]) << 16);
-    o.y = static_cast<unsigned>(c[2]) | (static_cast<unsigned>(c[3]) << 16);
-    *reinterpret_cast<uint2*>(p) = o;
-  }
-}
-
-// D = 32 * CH values per vector. One warp per token: the position and the token's
-// cos/sin row are loaded once, then the token's heads kRopeUnroll at a time, all
-// their loads issued before any value is used.
-template <int CH>
+// D values per head vector, L = D / 16 lanes per vector (16 values each), 32 / L vectors
+// per pass of a warp; one warp per token: the position and the lane's part of the
+// token's cos/sin row are loaded once, then the token's heads two passes at a time,
+// all their loads issued before any value is used.
+template <int D>
 __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) {
-  constexpr int D = 32 * CH;
+  constexpr int L = D / kEPL;          // lanes per head vector
+  constexpr int HPW = 32 / L;          // head vectors per pass
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
+  const int hl = lane / L;             // this lane's head vector in a pass
+  const int e0 = (lane % L) * kEPL;    // its values [e0, e0 + 16) of the vector
   const long long gwarp = (static_cast<long long>(blockIdx.x) * kRopeThreads + threadIdx.x) >> 5;
   const long long nwarps = static_cast<long long>(gridDim.x) * (kRopeThreads / 32);
   const float fmax = fp8_max(a.f8);
-  // angle index of this lane's first value: half-split pairs value i with i + D/2
-  // (angle i mod D/2), interleaved pairs 2i with 2i + 1 (angle i)
-  const int ang0 = a.interleaved ? lane * CH / 2 : (lane & 15) * CH;
-  const bool upper = lane >= 16;   // half-split: this lane holds the b' of its pairs
+  // half-split: values i < D/2 pair with i + D/2, which sits L/2 lanes further; a lane
+  // of the upper half holds the b' of its pairs. Interleaved: 2i pairs with 2i + 1.
+  const bool upper = e0 >= D / 2;
+  const int ang0 = a.interleaved ? e0 / 2 : (upper ? e0 - D / 2 : e0);
   const long long T = a.nvec / a.NH;
   for (long long t = gwarp; t < T; t += nwarps) {
     const int pos = __ldg(a.positions + t);       // the same for the whole warp
     const bool valid = pos >= 0 && pos < a.max_pos;
-    // this lane's angles: CH of them (half-split) or CH/2 (interleaved)
-    float c[CH], s[CH];
+    float c[kEPL], s[kEPL];                       // interleaved: the first 8 of each
     if (valid) {
       const float* row = a.cos_sin + static_cast<long long>(pos) * D;
       if (a.interleaved) {
-        #pragma unroll
-        for (int q = 0; q < CH / 2; ++q) {
-          c[q] = __ldg(row + ang0 + q);
-          s[q] = __ldg(row + D / 2 + ang0 + q);
-        }
+        load_f32<kEPL / 2>(row + ang0, c);
+        load_f32<kEPL / 2>(row + D / 2 + ang0, s);
       } else {
-        load_f32<CH>(row + ang0, c);
-        load_f32<CH>(row + D / 2 + ang0, s);
+        load_f32<kEPL>(row + ang0, c);
+        load_f32<kEPL>(row + D / 2 + ang0, s);
       }
     }
-    for (int h0 = 0; h0 < a.NH; h0 += kRopeUnroll) {
-      float x[kRopeUnroll][CH];
+    for (int h0 = 0; h0 < a.NH; h0 += 2 * HPW) {
+      float x[2][kEPL];
       #pragma unroll
-      for (int u = 0; u < kRopeUnroll; ++u)
-        if (h0 + u < a.NH) load_bf16<CH>(a.x + (t * a.NH + h0 + u) * D + lane * CH, x[u]);
+      for (int u = 0; u < 2; ++u) {
+        const int h = h0 + u * HPW + hl;
+        if (h < a.NH) {
+          load16(a.x + (t * a.NH + h) * D + e0, x[u]);
+        } else {
+          #pragma unroll
+          for (int q = 0; q < kEPL; ++q) x[u][q] = 0.f;
+        }
+      }
       #pragma unroll
-      for (int u = 0; u < kRopeUnroll; ++u) {
-        if (h0 + u >= a.NH) break;   // warp-uniform
-        const long long v = t * a.NH + h0 + u;
-        float y[CH];
+      for (int u = 0; u < 2; ++u) {
+        if (h0 + u * HPW >= a.NH) break;          // warp-uniform
+        const int h = h0 + u * HPW + hl;          // lanes past the last head compute zeros
+        float y[kEPL];
         if (valid) {
           if (a.interleaved) {
             #pragma unroll
-            for (int q = 0; q < CH / 2; ++q) {
+            for (int q = 0; q < kEPL / 2; ++q) {
               const float pa = x[u][2 * q], pb = x[u][2 * q + 1];
               y[2 * q] = __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
               y[2 * q + 1] = __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]));
             }
           } else {
             #pragma unroll
-            for (int q = 0; q < CH; ++q) {
-              const float other = __shfl_xor_sync(0xFFFFFFFFu, x[u][q], 16);
+            for (int q = 0; q < kEPL; ++q) {
+              const float other = __shfl_xor_sync(0xFFFFFFFFu, x[u][q], L / 2);
               const float pa = upper ? other : x[u][q];
               const float pb = upper ? x[u][q] : other;
               y[q] = upper ? __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]))
@@ -169,34 +153,41 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) 
           }
         } else {   // (valid is the same for the whole warp: the shuffles above stay uniform)
           #pragma unroll
-          for (int q = 0; q < CH; ++q) y[q] = 0.f;
+          for (int q = 0; q < kEPL; ++q) y[q] = 0.f;
         }
         float m = 0.f;
         #pragma unroll
-        for (int q = 0; q < CH; ++q) m = fmaxf(m, fabsf(y[q]));
+        for (int q = 0; q < kEPL; ++q) m = fmaxf(m, fabsf(y[q]));
         #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        for (int o = L / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
         const float sc = m == 0.f ? 1.f : __fdiv_rn(m, fmax);
         const ScaleDiv dv(sc);   // y / sc, correctly rounded, one reciprocal per vector
-        unsigned short cd[CH / 2];
+        uint4 o;
+        unsigned* ow = reinterpret_cast<unsigned*>(&o);
         #pragma unroll
-        for (int q = 0; q < CH / 2; ++q)
-          cd[q] = valid ? fp8x2(make_float2(dv(y[2 * q]), dv(y[2 * q + 1])), a.f8) : static_cast<unsigned short>(0);
-        store_codes<CH>(a.codes + v * D + lane * CH, cd);
-        if (lane == 0) a.scales[v] = valid ? sc : __int_as_float(0x7FC00000);
+        for (int q = 0; q < kEPL / 4; ++q) {
+          const unsigned short lo = fp8x2(make_float2(dv(y[4 * q]), dv(y[4 * q + 1])), a.f8);
+          const unsigned short hi = fp8x2(make_float2(dv(y[4 * q + 2]), dv(y[4 * q + 3])), a.f8);
+          ow[q] = valid ? (static_cast<unsigned>(lo) | (static_cast<unsigned>(hi) << 16)) : 0u;
+        }
+        if (h < a.NH) {
+          const long long v = t * a.NH + h;
+          *reinterpret_cast<uint4*>(a.codes + v * D + e0) = o;
+          if (e0 == 0) a.scales[v] = valid ? sc : __int_as_float(0x7FC00000);
+        }
       }
     }
   }
 }
 
-template <int CH>
+template <int D>
 cudaError_t launch_rope(const RopeArgs& a, cudaStream_t s) {
   const long long per_block = kRopeThreads / 32;   // tokens per block and round
   long long blocks = (a.nvec / a.NH + per_block - 1) / per_block;
   const long long cap = 8ll * sm_count();
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  return launch_kernel(inv_rope_fp8_kernel<CH>, dim3(static_cast<unsigned>(blocks)), dim3(kRopeThreads), 0, s, a);
+  return launch_kernel(inv_rope_fp8_kernel<D>, dim3(static_cast<unsigned>(blocks)), dim3(kRopeThreads), 0, s, a);
 }
 
 bool aligned(const void* p, unsigned bytes) { return (reinterpret_cast<uintptr_t>(p) & (bytes - 1)) == 0; }
@@ -230,8 +221,8 @@ extern "C" int moe_inv_rope_fp8_quant(const void* x, const int* positions, const
   a.interleaved = interleaved;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   moe::NvtxRange range("moe_inv_rope_fp8_quant");
-  cudaError_t e = head_dim == 64 ? moe::launch_rope<2>(a, st)
-                                 : (head_dim == 128 ? moe::launch_rope<4>(a, st) : moe::launch_rope<8>(a, st));
+  cudaError_t e = head_dim == 64 ? moe::launch_rope<64>(a, st)
+                                 : (head_dim == 128 ? moe::launch_rope<128>(a, st) : moe::launch_rope<256>(a, st));
   if (e != cudaSuccess) {
     std::fprintf(stderr, "moe_inv_rope_fp8_quant: launch failed: %s\n", cudaGetErrorString(e));
     return MOE_ERR_CUDA;

@@ -63,6 +63,7 @@ struct moe_layer {
   float* last_scales = nullptr; // [2]
   int* err = nullptr;
   int* sync = nullptr;          // single-launch decode: counters between its CTAs
+  int* small_sync = nullptr;    // small batches: [M_cap] token K-block counts, then a CTA count
   int* chunk_buf = nullptr;     // multi-block align: [2][chunks_cap][E] chunk counts and bases
   uint8_t* xq = nullptr;        // FP8 large batches: x quantised per token [M_cap, H]
   long long chunks_cap = 0;
@@ -90,7 +91,8 @@ struct moe_layer {
   cudaStream_t capture_stream = nullptr;
   // bookkeeping
   int last_M = 0, last_launches = 0;
-  bool fused_decode = false;    // single-launch decode path for small bf16 batches
+  bool fused_decode = false;    // single-launch decode path for small batches
+  bool last_small = false;      // the last forward took the small-batch path (no gathered x)
   // per-kernel event timing
   bool profiling = false;
   struct Timed {
@@ -165,6 +167,7 @@ int configure_device(int dev) {
   MOE_CUDA(moe::gemm_configure());
   MOE_CUDA(moe::align_configure());
   MOE_CUDA(moe::decode_configure());
+  MOE_CUDA(moe::small_configure());
   if (dev < 64) g_configured |= 1ull << dev;
   return MOE_OK;
 }
@@ -241,6 +244,7 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(ws_alloc(L, &L->last_scales, 2 * 4, false));
   MOE_TRY(ws_alloc(L, &L->err, 4, true));
   MOE_TRY(ws_alloc(L, &L->sync, moe::decode_sync_words(L->E, cap) * 4, true));
+  MOE_TRY(ws_alloc(L, &L->small_sync, (static_cast<size_t>(cap) + 8) * 4, true));
   if (is_fp8(L)) MOE_TRY(ws_alloc(L, &L->xq, static_cast<size_t>(cap) * L->H, false));
   L->chunks_cap = (P + moe::kAlignChunk - 1) / moe::kAlignChunk;
   MOE_TRY(ws_alloc(L, &L->chunk_buf, 2 * L->chunks_cap * L->E * 4, false));
@@ -486,11 +490,150 @@ constexpr long long kAlignSingleBlockMaxPairs = 8192;
 
 int forward_mixed(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st);
 
+// Whether batches that fit the small-batch path take it (MOE_SMALL_BATCH=0 keeps the
+// full chain for them).
+bool small_batch_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("MOE_SMALL_BATCH");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+// A batch of up to 64 tokens: route -> gate_up -> down (FP8: route -> quant_x ->
+// gate_up -> quant_h -> down). The GEMMs build the schedule from the routing
+// themselves, gate_up reads token rows directly, down finishes token rows itself.
+int forward_small(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
+  const bool fp8 = is_fp8(L);
+  const long long P = static_cast<long long>(M) * L->k;
+  int launches = 0;
+
+  moe::RouteArgs ra{};
+  ra.logits = logits;
+  ra.x = static_cast<const __nv_bfloat16*>(x);
+  ra.M = M;
+  ra.E = L->E;
+  ra.k = L->k;
+  ra.H = L->H;
+  ra.topk_ids = L->topk_ids;
+  ra.topk_w = L->topk_w;
+  ra.amax_x = fp8 ? L->amax : nullptr;
+  {
+    KernelTimer kt(L, 0, st);
+    MOE_CUDA(moe::launch_route(ra, st));
+  }
+  ++launches;
+
+  // gate_up's activation rows: the caller's x rows (bf16), or their codes (FP8)
+  CUtensorMap tm_xd{};
+  if (fp8) {
+    moe::QuantXArgs qx{};
+    qx.x = static_cast<const __nv_bfloat16*>(x);
+    qx.xq = L->xq;
+    qx.M = M;
+    qx.H = L->H;
+    qx.amax_x = L->amax;
+    qx.f8 = fp8_format(L);
+    KernelTimer kt(L, 2, st);
+    MOE_CUDA(moe::launch_quant_x(qx, st));
+    ++launches;
+  } else {
+    MOE_TRY(encode_map(&tm_xd, x, false, L->H, M, 1));
+  }
+
+  const int kper = fp8 ? 128 : 64;
+  moe::SmallArgs sa{};
+  sa.topk_ids = L->topk_ids;
+  sa.topk_w = L->topk_w;
+  sa.out = static_cast<__nv_bfloat16*>(out);
+  sa.M = M;
+  sa.E = L->E;
+  sa.k = L->k;
+  sa.H = L->H;
+  sa.I = L->I;
+  sa.P = static_cast<int>(P);
+  sa.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
+  sa.uniform = moe::uniform_splits() ? 1 : 0;
+  sa.f8 = fp8_format(L);
+  sa.token_cnt = L->small_sync;
+  sa.done = L->small_sync + L->M_cap;
+  sa.amax = L->amax;
+  sa.last_scales = L->last_scales;
+  sa.counts = L->counts;
+  sa.padded_offsets = L->poff;
+  sa.padded_pairs = L->pairs;
+  sa.header = L->header;
+  moe::GemmArgs g{};
+  g.h = L->h;
+  g.I = L->I;
+  g.ws1 = L->ws1;
+  g.tile_counters = L->counters;
+  g.amax_h = L->amax + 1;
+  g.amax_x = L->amax;
+  g.w_scales = L->wscales;
+  g.acc = L->acc;
+  g.H = L->H;
+  g.k = L->k;
+  g.P = static_cast<int>(P);
+  g.f8 = fp8_format(L);
+  g.err = L->err;
+  g.wait_budget = moe::wait_budget_cycles();
+
+  moe::SmallArgs s1 = sa;
+  s1.g = g;
+  s1.g.kblocks = L->H / kper;
+  s1.g.w_rblocks = 2 * L->I / moe::kTileRows;
+  s1.g.rb_step = 1;
+  s1.g.second_rb = L->I / moe::kTileRows;
+  s1.g.max_stages = moe::gemm_max_stages(true);
+  {
+    KernelTimer kt(L, 3, st);
+    MOE_CUDA(moe::launch_small_gate_up(s1, L->tm_w13, fp8 ? L->tm_xq : tm_xd, fp8, L->num_sms, st));
+  }
+  ++launches;
+
+  if (fp8) {
+    moe::QuantHArgs qa{};
+    qa.h = L->h;
+    qa.h_q = L->h_q;
+    qa.padded_pairs = L->pairs;
+    qa.header = L->header;
+    qa.rows_bound = static_cast<int>(P + std::min<long long>(L->E, P) * (moe::kPadRows - 1));
+    qa.P = static_cast<int>(P);
+    qa.I = L->I;
+    qa.amax_h = L->amax + 1;
+    qa.f8 = fp8_format(L);
+    KernelTimer kt(L, 4, st);
+    MOE_CUDA(moe::launch_quant_h(qa, st));
+    ++launches;
+  }
+
+  moe::SmallArgs s2 = sa;
+  s2.g = g;
+  s2.g.kblocks = L->I / kper;
+  s2.g.w_rblocks = L->H / moe::kTileRows;
+  s2.g.rb_step = 2;
+  s2.g.second_rb = 1;
+  s2.g.max_stages = moe::gemm_max_stages(false);
+  {
+    KernelTimer kt(L, 5, st);
+    MOE_CUDA(moe::launch_small_down(s2, L->tm_wd, L->tm_h, fp8, L->num_sms, st));
+  }
+  ++launches;
+  L->last_M = M;
+  L->last_launches = launches;
+  L->last_small = true;
+  return MOE_OK;
+}
+
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
+  L->last_small = false;
   if (is_mixed(L)) return forward_mixed(L, x, logits, M, out, st);
   if (L->fused_decode && M <= L->num_sms && moe::decode_supported(M, L->E, L->k))
     return forward_fused_decode(L, x, logits, M, out, st);
+  if (small_batch_enabled() && moe::small_supported(M, L->E, L->k))
+    return forward_small(L, x, logits, M, out, st);
   const bool fp8 = is_fp8(L);
   const long long P = static_cast<long long>(M) * L->k;
   const int BN = moe::kTokenBlock;
@@ -1325,8 +1468,25 @@ int moe_debug_activations(moe_layer* L, void* x_perm_out, void* h_out) {
   int rows = 0;
   MOE_CUDA(cudaMemcpy(&rows, L->header + moe::kHdrRowsUsed, 4, cudaMemcpyDeviceToHost));
   const size_t el = is_fp8(L) ? 1 : 2;
-  if (x_perm_out)
+  if (x_perm_out && L->last_small && is_fp8(L)) {
+    // the small-batch path quantised x once per token and read those rows directly:
+    // lay its codes out in expert order here (the gather kernel copying code rows)
+    moe::GatherArgs ga{};
+    ga.padded_pairs = L->pairs;
+    ga.header = L->header;
+    ga.rows_bound = rows;
+    ga.P = L->last_M * L->k;
+    ga.k = L->k;
+    ga.H = L->H;
+    ga.x_perm = x_perm_out;
+    ga.amax_x = L->amax;
+    ga.f8 = fp8_format(L);
+    ga.xq = L->xq;
+    MOE_CUDA(moe::launch_gather(ga, true, nullptr));
+    MOE_CUDA(cudaDeviceSynchronize());
+  } else if (x_perm_out) {
     MOE_CUDA(cudaMemcpy(x_perm_out, L->x_perm, static_cast<size_t>(rows) * L->H * el, cudaMemcpyDeviceToDevice));
+  }
   if (h_out) MOE_CUDA(cudaMemcpy(h_out, L->h, static_cast<size_t>(rows) * L->I * 2, cudaMemcpyDeviceToDevice));
   return MOE_OK;
 }

@@ -258,6 +258,31 @@ size_t decode_sync_words(int E, int M_cap);
 cudaError_t decode_configure();
 cudaError_t launch_decode(const DecodeLaunch& l, cudaStream_t st);
 
+// Small batches (kernels_small.cu): the grouped GEMMs build the batch's schedule
+// themselves from the routing (no align kernel), gate_up reads token rows directly (no
+// gather) and down finishes token rows itself (no finalize).
+struct SmallArgs {
+  const int* topk_ids;     // [P] from the route kernel
+  const float* topk_w;     // [P]
+  __nv_bfloat16* out;      // down: [M, H]
+  int M, E, k, H, I, P, ws1_rows_cap, uniform, f8;
+  int* token_cnt;          // down: [M] K blocks added per token (zero between calls)
+  int* done;               // down: [1] CTAs finished (zero between calls)
+  unsigned* amax;          // FP8: [2] max|x|, max|h| (reset by down's last CTA)
+  float* last_scales;      // FP8: [2] s_x, s_h of the forward
+  int* counts;             // gate_up (CTA 0): copies of the schedule
+  int* padded_offsets;
+  int* padded_pairs;
+  int* header;
+  GemmArgs g;
+};
+bool small_supported(int M, int E, int k);
+cudaError_t small_configure();
+cudaError_t launch_small_gate_up(const SmallArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8, int grid,
+                                 cudaStream_t s);
+cudaError_t launch_small_down(const SmallArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int grid,
+                              cudaStream_t s);
+
 // Weight preparation (load time, not on the forward path). Stored weights are
 // tiled: tile (e, rb, kb) = rows [rb*128, +128) x bytes [kb*128, +128) of expert e,
 // 16 KB contiguous (rows in order), tiles ordered e, then rb, then kb. This is the
