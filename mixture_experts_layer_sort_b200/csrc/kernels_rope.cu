@@ -23,8 +23,8 @@
 // 16 consecutive values (32 bytes in, 16 bytes of codes out) per lane, so that the
 // per-vector work (the max reduction, the scale, its reciprocal) is shared by 16 values
 // and a warp covers 512/D vectors per pass; the half-split partner of a value sits D/32
-// lanes away. The position and the lane's part of the table row are read once per
-// token, and two passes of vectors are in flight at once. The kernel moves 2D bytes in
+// lanes away. The position (one token ahead) and the lane's part of the table row are
+// read once per token, and up to four passes of vectors are in flight at once. The kernel moves 2D bytes in
 // and D + 4 bytes out per vector, plus 4 + 4D bytes per token: it is HBM-bound.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -56,18 +56,6 @@ struct RopeArgs {
 
 constexpr int kEPL = 16;   // values of a head vector per lane
 
-// 16 consecutive bf16 values (32 bytes) -> fp32
-__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[kEPL]) {
-  const uint4 u[2] = {__ldg(reinterpret_cast<const uint4*>(p)), __ldg(reinterpret_cast<const uint4*>(p) + 1)};
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(u);
-  #pragma unroll
-  for (int q = 0; q < kEPL / 2; ++q) {
-    const float2 f = __bfloat1622float2(h[q]);
-    v[2 * q] = f.x;
-    v[2 * q + 1] = f.y;
-  }
-}
-
 // n consecutive fp32 values (n a multiple of 4, 16-byte aligned)
 template <int n>
 __device__ __forceinline__ void load_f32(const float* p, float* v) {
@@ -81,12 +69,14 @@ __device__ __forceinline__ void load_f32(const float* p, float* v) {
   }
 }
 
+constexpr int kRopePasses = 4;   // passes of head vectors per warp in flight
+
 // D values per head vector, L = D / 16 lanes per vector (16 values each), 32 / L vectors
-// per pass of a warp; one warp per token: the position and the lane's part of the
-// token's cos/sin row are loaded once, then the token's heads two passes at a time,
-// all their loads issued before any value is used.
+// per pass of a warp; one warp per token: the position (loaded one token ahead) and the
+// lane's part of the token's cos/sin row are loaded once, then the token's heads up to
+// four passes at a time, all their loads issued before any value is used.
 template <int D>
-__global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) {
+__global__ void __launch_bounds__(kRopeThreads, 2) inv_rope_fp8_kernel(RopeArgs a) {
   constexpr int L = D / kEPL;          // lanes per head vector
   constexpr int HPW = 32 / L;          // head vectors per pass
   pdl_wait();
@@ -102,8 +92,10 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) 
   const bool upper = e0 >= D / 2;
   const int ang0 = a.interleaved ? e0 / 2 : (upper ? e0 - D / 2 : e0);
   const long long T = a.nvec / a.NH;
+  int pos_next = gwarp < T ? __ldg(a.positions + gwarp) : 0;
   for (long long t = gwarp; t < T; t += nwarps) {
-    const int pos = __ldg(a.positions + t);       // the same for the whole warp
+    const int pos = pos_next;                     // the same for the whole warp
+    if (t + nwarps < T) pos_next = __ldg(a.positions + t + nwarps);
     const bool valid = pos >= 0 && pos < a.max_pos;
     float c[kEPL], s[kEPL];                       // interleaved: the first 8 of each
     if (valid) {
@@ -116,37 +108,50 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(RopeArgs a) 
         load_f32<kEPL>(row + D / 2 + ang0, s);
       }
     }
-    for (int h0 = 0; h0 < a.NH; h0 += 2 * HPW) {
-      float x[2][kEPL];
+    for (int h0 = 0; h0 < a.NH; h0 += kRopePasses * HPW) {
+      // the raw bf16 values (two 16-byte vectors per pass) until each pass is used
+      uint4 xr[kRopePasses][2];
       #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kRopePasses; ++u) {
         const int h = h0 + u * HPW + hl;
         if (h < a.NH) {
-          load16(a.x + (t * a.NH + h) * D + e0, x[u]);
+          const uint4* p = reinterpret_cast<const uint4*>(a.x + (t * a.NH + h) * D + e0);
+          xr[u][0] = __ldg(p);
+          xr[u][1] = __ldg(p + 1);
         } else {
-          #pragma unroll
-          for (int q = 0; q < kEPL; ++q) x[u][q] = 0.f;
+          xr[u][0] = make_uint4(0u, 0u, 0u, 0u);
+          xr[u][1] = xr[u][0];
         }
       }
       #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kRopePasses; ++u) {
         if (h0 + u * HPW >= a.NH) break;          // warp-uniform
         const int h = h0 + u * HPW + hl;          // lanes past the last head compute zeros
+        float xv[kEPL];
+        {
+          const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(xr[u]);
+          #pragma unroll
+          for (int q = 0; q < kEPL / 2; ++q) {
+            const float2 f = __bfloat1622float2(hp[q]);
+            xv[2 * q] = f.x;
+            xv[2 * q + 1] = f.y;
+          }
+        }
         float y[kEPL];
         if (valid) {
           if (a.interleaved) {
             #pragma unroll
             for (int q = 0; q < kEPL / 2; ++q) {
-              const float pa = x[u][2 * q], pb = x[u][2 * q + 1];
+              const float pa = xv[2 * q], pb = xv[2 * q + 1];
               y[2 * q] = __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
               y[2 * q + 1] = __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]));
             }
           } else {
             #pragma unroll
             for (int q = 0; q < kEPL; ++q) {
-              const float other = __shfl_xor_sync(0xFFFFFFFFu, x[u][q], L / 2);
-              const float pa = upper ? other : x[u][q];
-              const float pb = upper ? x[u][q] : other;
+              const float other = __shfl_xor_sync(0xFFFFFFFFu, xv[q], L / 2);
+              const float pa = upper ? other : xv[q];
+              const float pb = upper ? xv[q] : other;
               y[q] = upper ? __fsub_rn(__fmul_rn(pb, c[q]), __fmul_rn(pa, s[q]))
                            : __fadd_rn(__fmul_rn(pa, c[q]), __fmul_rn(pb, s[q]));
             }

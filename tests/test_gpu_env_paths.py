@@ -4,10 +4,9 @@ select (each read once per process, so every setting runs in a child process):
   MOE_UNIFORM_SPLITS=1     one split-K factor per GEMM from the cost model instead of
                            the balanced unit schedule
   MOE_DISABLE_PDL=1        plain stream order instead of programmatic dependent launch
-  MOE_SMALL_BATCH=0        batches of up to 64 tokens take the full chain (align, gather,
-                           finalize) instead of the small-batch GEMMs
-  MOE_DISABLE_DIRECT_X=1   (with the full chain) small bf16 batches gather x instead of
-                           loading token rows
+  MOE_SMALL_BATCH=1        batches of up to 64 tokens take the small-batch GEMMs (no align,
+                           gather or finalize) instead of the full chain
+  MOE_DISABLE_DIRECT_X=1   small bf16 batches gather x instead of loading token rows
   MOE_MAX_STAGES1/2=2      the shallowest stage rings
 
 The shape (E=64, k=8, H=1024, I=1024) gives one to eight waves of tiles on a B200 at
@@ -45,9 +44,9 @@ print("PARITY_OK")
 SETTINGS = [
     {"MOE_UNIFORM_SPLITS": "1"},
     {"MOE_DISABLE_PDL": "1"},
-    {"MOE_SMALL_BATCH": "0"},
-    {"MOE_SMALL_BATCH": "0", "MOE_UNIFORM_SPLITS": "1"},
-    {"MOE_SMALL_BATCH": "0", "MOE_DISABLE_DIRECT_X": "1"},
+    {"MOE_DISABLE_DIRECT_X": "1"},
+    {"MOE_SMALL_BATCH": "1"},
+    {"MOE_SMALL_BATCH": "1", "MOE_UNIFORM_SPLITS": "1"},
     {"MOE_MAX_STAGES1": "2", "MOE_MAX_STAGES2": "2"},
 ]
 
