@@ -63,14 +63,16 @@ def parse_args():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default="decode",
                     choices=["tiny", "decode", "decode_fp8", "decode_e5m2", "large_decode", "prefill",
-                             "prefill_fp8", "prefill_m16384", "prefill_e48", "prefill_e48_fp8"])
+                             "prefill_fp8", "prefill_m16384", "prefill_e48", "prefill_e48_fp8", "inv_rope"],
+                    help="inv_rope: the inverse-RoPE + per-head FP8 kernel alone (--only-M picks one token count)")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="measure the headline workload only (skip decode FP8, large decode and prefill)")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--only-M", type=int, default=None, help="run a single batch size of the workload")
+    ap.add_argument("--only-M", type=int, default=None,
+                    help="run a single batch size of the workload (inv_rope: a single token count)")
     ap.add_argument("--fused-decode", action="store_true", help="single-launch decode path (bf16, M <= 64)")
     ap.add_argument("--warm-l2", action="store_true",
                     help="do not flush L2 between forwards (a labelled warm-cache figure, not the headline)")
@@ -291,6 +293,10 @@ def cpu_baseline_entry(wl, dtype, host_w, toks_np, budget_s, one_thread_Ms=(1, 4
 def reference_arm(args, ws, rank):
     """The CPU oracle as the reference arm: rank 0 times it, the others exit."""
     if rank != 0:
+        return 0
+    if args.workload == "inv_rope":
+        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the MoE layer; the "
+                          "inverse-RoPE kernel's CPU oracle is timed inside the default bench line"}))
         return 0
     from mixture_experts_layer_sort_b200 import synth
     wl, dtype = workload_spec(args.workload)
@@ -519,7 +525,7 @@ def measure_workload(name, layer, wl, dtype, Ms, toks, stream, flush, args, hbm_
 ROPE_SHAPE = {"NH": 16, "D": 128, "max_pos": 32768, "Ts": (1, 64, 4096, 16384)}
 
 
-def measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on):
+def measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on, Ts=None):
     """The inverse-RoPE + per-head FP8 quantisation kernel at several token counts (one
     kernel for all of them): device time per call with L2 flushed before each, and the
     achieved HBM bandwidth over its algorithmic bytes (2D bytes in, D codes + a 4-byte
@@ -534,7 +540,8 @@ def measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on):
     g = torch.Generator(device=dev).manual_seed(seed)
     steps = max(5, min(args.steps, 20))
     per_T = {}
-    for T in ROPE_SHAPE["Ts"]:
+    Ts = list(Ts or ROPE_SHAPE["Ts"])
+    for T in Ts:
         x = torch.randn((T, NH, D), generator=g, device=dev).to(torch.bfloat16)
         pos = torch.randint(0, max_pos, (T,), generator=g, device=dev, dtype=torch.int32)
         codes = torch.empty((T, NH, D), dtype=torch.uint8, device=dev)
@@ -565,7 +572,7 @@ def measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on):
         per_T[str(T)] = {"us": mean * 1e3, "us_p50": statistics.median(ms) * 1e3, "alg_MB": alg / 1e6,
                          "GBps": alg / (mean / 1e3) / 1e9, "frac_hbm": alg / (mean / 1e3) / 1e9 / hbm_gbs}
     entry = {"workload": f"inverse RoPE + per-head e4m3 quantisation, [T, {NH} heads, {D}] bf16, half-split "
-                         f"pairs, one launch per T in {list(ROPE_SHAPE['Ts'])}",
+                         f"pairs, one launch per T in {Ts}",
              "per_T": per_T, "bound": "hbm", "peak_GBps": hbm_gbs}
     if cpu_on:
         from oracle import rope_oracle as R
@@ -629,6 +636,24 @@ def extra_workloads(args, dev, stream, flush, dec_weights, seed, hbm_gbs, bf16_t
     return res
 
 
+def rope_only(args, ws, rank, local):
+    """The inverse-RoPE kernel on its own (every rank its own tokens; rank 0 prints)."""
+    import torch
+    dev = torch.device("cuda", local)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    hbm_gbs, _, peak_src = read_peaks()
+    res = measure_inv_rope(args, dev, stream, flush, args.seed + 1000 * rank, hbm_gbs, False,
+                           Ts=[args.only_M] if args.only_M else None)
+    barrier(ws)
+    if rank == 0:
+        print(json.dumps({"workload": "inv_rope", "n_gpus": ws, "peak_source": peak_src, **res}))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     ws, rank, local = dist_setup(args)
@@ -643,6 +668,8 @@ def main():
 
     from mixture_experts_layer_sort_b200 import MoELayer, synth
 
+    if args.workload == "inv_rope":
+        return rope_only(args, ws, rank, local)
     wl, dtype = workload_spec(args.workload)
     Ms = [args.only_M] if args.only_M else list(wl.Ms)
     dev = torch.device("cuda", local)
