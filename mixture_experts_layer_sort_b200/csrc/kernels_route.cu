@@ -22,96 +22,15 @@ namespace moe {
 namespace {
 
 constexpr int kRouteWarps = 8;
-constexpr int kPfMaxExperts = 512;
-constexpr long long kPfChunk = 64 << 10;   // bytes per bulk prefetch
-
-// A prefetch CTA of the router (small batches). The weights of a decode batch's
-// experts are the whole of its memory traffic, and every kernel boundary of the chain
-// (route -> align -> gate_up -> down) would otherwise stall that stream. So once the
-// routing is known, these CTAs ask L2 for the active experts' weight blocks; the GEMMs
-// that follow find them there, and HBM streams from the end of the routing on.
-// The CTA routes every token again (a warp per token, ids in shared memory), marks the
-// active experts, and spreads 64 KB bulk prefetches over the prefetch CTAs and their
-// threads: the first lg bytes of each expert's gate and up halves, then the first ld
-// bytes of its down block. When everything does not fit the budget, the down blocks
-// take it first (gate_up streams its own weights meanwhile) and gate_up the rest.
-template <int NPL>
-__device__ __forceinline__ void prefetch_weights(const RouteArgs& a, int c) {
-  __shared__ unsigned s_act[kPfMaxExperts / 32];
-  __shared__ int s_list[kPfMaxExperts];
-  __shared__ int s_ids[kRouteWarps][32];
-  __shared__ float s_w[kRouteWarps][32];
-  __shared__ int s_nact;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kPfMaxExperts / 32; i += blockDim.x) s_act[i] = 0u;
-  __syncthreads();
-  for (int t = warp; t < a.M; t += kRouteWarps) {
-    route_token<NPL>(a.logits + static_cast<size_t>(t) * a.E, a.E, a.k, lane, s_ids[warp], s_w[warp]);
-    __syncwarp();
-    if (lane < a.k) {
-      const int e = s_ids[warp][lane];
-      if (e >= 0 && e < a.E) atomicOr(&s_act[e >> 5], 1u << (e & 31));
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = (a.E + 31) / 32;
-    const unsigned m = lane < nw ? s_act[lane] : 0u;
-    const int cnt = __popc(m);
-    int incl = cnt;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pos = incl - cnt;
-    for (unsigned mm = m; mm != 0u; mm &= mm - 1u) s_list[pos++] = lane * 32 + __ffs(mm) - 1;
-    if (lane == 31) s_nact = incl;
-  }
-  __syncthreads();
-  const long long A = s_nact;
-  if (A == 0) return;
-  const long long half = a.w13_bytes / 2;
-  long long lg = half, ld = a.wd_bytes;
-  if (A * (a.w13_bytes + a.wd_bytes) > a.pf_bytes) {
-    ld = min(a.wd_bytes, a.pf_bytes / A) & ~127ll;
-    lg = min(half, (a.pf_bytes - A * ld) / (2 * A)) & ~127ll;
-  }
-  const long long ng = (lg + kPfChunk - 1) / kPfChunk;
-  const long long nd = (ld + kPfChunk - 1) / kPfChunk;
-  const long long items_g = A * 2 * ng;
-  const long long total = items_g + A * nd;
-  const long long stride = static_cast<long long>(a.pf_ctas) * blockDim.x;
-  for (long long i = c + static_cast<long long>(a.pf_ctas) * threadIdx.x; i < total; i += stride) {
-    const uint8_t* p;
-    long long len;
-    if (i < items_g) {
-      const long long ai = i / (2 * ng), r = i - ai * 2 * ng, hh = r / ng, ch = r - hh * ng;
-      p = a.w13 + s_list[ai] * a.w13_bytes + hh * half + ch * kPfChunk;
-      len = min(kPfChunk, lg - ch * kPfChunk);
-    } else {
-      const long long j = i - items_g, ai = j / nd, ch = j - ai * nd;
-      p = a.wd + s_list[ai] * a.wd_bytes + ch * kPfChunk;
-      len = min(kPfChunk, ld - ch * kPfChunk);
-    }
-    l2_prefetch_bulk(p, static_cast<uint32_t>(len));
-  }
-}
 
 // One warp per token (route_token); FP8 layers also fold the token's max |x| into
-// the per-tensor amax word. CTAs past the routing ones prefetch weights.
+// the per-tensor amax word.
 template <int NPL>
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
-  const int route_ctas = (a.M + kRouteWarps - 1) / kRouteWarps;
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
-  if (static_cast<int>(blockIdx.x) >= route_ctas) {
-    prefetch_weights<NPL>(a, static_cast<int>(blockIdx.x) - route_ctas);
-    return;
-  }
   if (t >= a.M) return;
   route_token<NPL>(a.logits + static_cast<size_t>(t) * a.E, a.E, a.k, lane, a.topk_ids + static_cast<size_t>(t) * a.k,
                    a.topk_w + static_cast<size_t>(t) * a.k);
@@ -319,7 +238,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
-  const int grid = (a.M + kRouteWarps - 1) / kRouteWarps + (a.pf_bytes > 0 ? a.pf_ctas : 0);
+  const int grid = (a.M + kRouteWarps - 1) / kRouteWarps;
   const dim3 g(grid), b(kRouteWarps * 32);
   if (a.E <= 32) return launch_kernel(route_kernel<1>, g, b, 0, s, a);
   if (a.E <= 64) return launch_kernel(route_kernel<2>, g, b, 0, s, a);

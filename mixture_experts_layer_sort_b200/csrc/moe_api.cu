@@ -383,18 +383,6 @@ bool direct_x_disabled() {
   return off;
 }
 
-// L2 prefetch budget of the router's prefetch CTAs, in bytes (MOE_L2_PREFETCH_MB; 0
-// turns the prefetch off). Batches of up to kPrefetchMaxTokens tokens use it.
-constexpr int kPrefetchMaxTokens = 64;
-long long l2_prefetch_bytes() {
-  static const long long b = [] {
-    const char* e = std::getenv("MOE_L2_PREFETCH_MB");
-    const long long mb = e ? std::atoll(e) : 80;
-    return mb > 0 ? mb << 20 : 0ll;
-  }();
-  return b;
-}
-
 // Whether new handles take the single-launch decode path for the batches it supports
 // (MOE_FUSED_DECODE=0 or 1 overrides the default).
 bool fused_decode_default() {
@@ -662,15 +650,6 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   ra.topk_ids = L->topk_ids;
   ra.topk_w = L->topk_w;
   ra.amax_x = fp8 ? L->amax : nullptr;
-  if (M <= kPrefetchMaxTokens && l2_prefetch_bytes() > 0) {
-    const long long el = fp8 ? 1 : 2;
-    ra.w13 = static_cast<const uint8_t*>(L->w13);
-    ra.wd = static_cast<const uint8_t*>(L->wd);
-    ra.w13_bytes = 2ll * L->I * L->H * el;
-    ra.wd_bytes = 1ll * L->H * L->I * el;
-    ra.pf_bytes = l2_prefetch_bytes();
-    ra.pf_ctas = L->num_sms;
-  }
   {
     KernelTimer kt(L, 0, st);
     MOE_CUDA(moe::launch_route(ra, st));

@@ -63,15 +63,6 @@ struct RouteArgs {
   int* topk_ids;           // [M, k]
   float* topk_w;           // [M, k]
   unsigned* amax_x;        // FP8 only (else nullptr): running max |x| as float bits
-  // L2 prefetch of the selected experts' weights (pf_bytes = 0: none). pf_ctas extra
-  // CTAs route every token again and issue bulk L2 prefetches of [0, len) of each
-  // active expert's blocks: w13 rows (gate and up halves) and wd rows, the down blocks
-  // taking the budget first when not everything fits.
-  const uint8_t* w13;      // [E] blocks of w13_bytes (gate half, then up half)
-  const uint8_t* wd;       // [E] blocks of wd_bytes
-  long long w13_bytes, wd_bytes;
-  long long pf_bytes;      // budget
-  int pf_ctas;
 };
 
 struct AlignArgs {

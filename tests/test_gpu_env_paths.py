@@ -8,8 +8,6 @@ select (each read once per process, so every setting runs in a child process):
                            gather or finalize) instead of the full chain
   MOE_DISABLE_DIRECT_X=1   small bf16 batches gather x instead of loading token rows
   MOE_MAX_STAGES1/2=2      the shallowest stage rings
-  MOE_L2_PREFETCH_MB=0     no L2 prefetch of the active experts' weights by the router
-  MOE_L2_PREFETCH_MB=4096  a budget that covers every expert (everything prefetched)
 
 The shape (E=64, k=8, H=1024, I=1024) gives one to eight waves of tiles on a B200 at
 M=64 (the balanced schedule's range) and fewer than one at M=1.
@@ -50,8 +48,6 @@ SETTINGS = [
     {"MOE_SMALL_BATCH": "1"},
     {"MOE_SMALL_BATCH": "1", "MOE_UNIFORM_SPLITS": "1"},
     {"MOE_MAX_STAGES1": "2", "MOE_MAX_STAGES2": "2"},
-    {"MOE_L2_PREFETCH_MB": "0"},
-    {"MOE_L2_PREFETCH_MB": "4096"},
 ]
 
 
