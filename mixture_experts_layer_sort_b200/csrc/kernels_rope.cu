@@ -185,11 +185,21 @@ __global__ void __launch_bounds__(kRopeThreads, 2) inv_rope_fp8_kernel(RopeArgs 
   }
 }
 
+// The grid is capped at the blocks that are resident at once (a grid-stride loop
+// over tokens), so that every warp runs several tokens with its position loads one
+// token ahead instead of blocks arriving in waves.
 template <int D>
 cudaError_t launch_rope(const RopeArgs& a, cudaStream_t s) {
+  static const int per_sm = [] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, inv_rope_fp8_kernel<D>, kRopeThreads, 0) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    return n;
+  }();
   const long long per_block = kRopeThreads / 32;   // tokens per block and round
   long long blocks = (a.nvec / a.NH + per_block - 1) / per_block;
-  const long long cap = 8ll * sm_count();
+  const long long cap = static_cast<long long>(per_sm) * sm_count();
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return launch_kernel(inv_rope_fp8_kernel<D>, dim3(static_cast<unsigned>(blocks)), dim3(kRopeThreads), 0, s, a);
