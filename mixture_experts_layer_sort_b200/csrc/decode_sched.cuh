@@ -20,22 +20,32 @@ constexpr int kSchedMaxPairs = 512;
 constexpr int kSchedMaxExperts = 512;
 constexpr int kSchedBalancedWaves = 8;  // as in the align kernel
 
-struct Sched {
+// Up to kMaxE experts; kMaxDone tokens finished by one down unit (at most a unit's
+// token rows).
+template <int kMaxE, int kMaxDone>
+struct SchedT {
+  static constexpr int kMaxExperts = kMaxE;
   int ids[kSchedMaxPairs];
   float w[kSchedMaxPairs];
-  int count[kSchedMaxExperts];
-  int off[kSchedMaxExperts + 1];       // compact offsets of each expert's pairs
-  int poff[kSchedMaxExperts + 1];      // padded offsets (rows of h)
-  int tmp[kSchedMaxExperts + 1];
-  int act[kSchedMaxExperts];           // active experts, ascending
-  int aidx[kSchedMaxExperts + 1];      // index of each expert among the active ones
-  unsigned mask[kSchedMaxExperts][2];  // tokens routed to each expert
+  int count[kMaxE];
+  int off[kMaxE + 1];                  // compact offsets of each expert's pairs
+  int poff[kMaxE + 1];                 // padded offsets (rows of h)
+  int act[kMaxE];                      // active experts, ascending
+  int aidx[kMaxE + 1];                 // index of each expert among the active ones
+  unsigned mask[kMaxE][2];             // tokens routed to each expert
   int pairs[kSchedMaxPairs];           // pair ids grouped by expert, ascending inside an expert
-  int done[256];                       // tokens completed by the current down unit
+  int done[kMaxDone];                  // tokens completed by the current down unit
   float red[8];                        // block reduction scratch
   int ndone;
   int nact, T1, S1, T2, S2, n_max, rows_used, flag;
 };
+
+// The single-launch decode kernel (the whole of shared memory is its own).
+using Sched = SchedT<kSchedMaxExperts, 256>;
+// The small-batch GEMMs, which share an SM with each other: up to 256 experts, and a
+// down unit's token rows are at most kSchedMaxTokens.
+constexpr int kSchedSmallMaxExperts = 256;
+using SchedSmall = SchedT<kSchedSmallMaxExperts, kSchedMaxTokens>;
 
 __host__ __device__ constexpr bool sched_supported(int M, int E, int k) {
   return M >= 1 && M <= kSchedMaxTokens && E <= kSchedMaxExperts && M * k <= kSchedMaxPairs;
@@ -43,8 +53,9 @@ __host__ __device__ constexpr bool sched_supported(int M, int E, int k) {
 
 // Tile t of a GEMM from the schedule: tile t = (active expert t / fb, row block t % fb);
 // every expert has a single token tile (n_e <= M <= 64).
+template <class S>
 struct SmemTileFn {
-  const Sched* s;
+  const S* s;
   int fb;
   __device__ __forceinline__ Tile operator()(int t) const {
     const int ai = t / fb;
@@ -58,7 +69,8 @@ struct SmemTileFn {
 };
 
 // Zero the counts and token masks (all threads; a barrier must follow before the build).
-__device__ __forceinline__ void sched_clear(Sched* s, int E, int tid, int nthreads) {
+template <class S>
+__device__ __forceinline__ void sched_clear(S* s, int E, int tid, int nthreads) {
   for (int e = tid; e < E; e += nthreads) {
     s->count[e] = 0;
     s->mask[e][0] = 0u;
@@ -71,7 +83,8 @@ __device__ __forceinline__ void sched_clear(Sched* s, int E, int tid, int nthrea
 // synchronises before reading the schedule. G = CTAs of the grid; fb1/fb2 tiles across
 // the output features and kb1/kb2 K blocks of gate_up/down; uniform = 1 forces one
 // split factor per GEMM.
-static __device__ void sched_build(Sched* s, int P, int E, int k, int fb1, int fb2, int kb1, int kb2, int G,
+template <class S>
+static __device__ void sched_build(S* s, int P, int E, int k, int fb1, int fb2, int kb1, int kb2, int G,
                             int ws1_rows_cap, int uniform, int tid, int nthreads) {
   const int warp = tid >> 5, lane = tid & 31;
   for (int p = tid; p < P; p += nthreads) {
@@ -90,9 +103,9 @@ static __device__ void sched_build(Sched* s, int P, int E, int k, int fb1, int f
   }
   __syncthreads();
   if (warp == 0) {
-    for (int e = lane; e < E; e += 32) s->tmp[e] = s->count[e] > 0 ? 1 : 0;
+    for (int e = lane; e < E; e += 32) s->aidx[e] = s->count[e] > 0 ? 1 : 0;
     __syncwarp();
-    warp_exclusive_scan(s->tmp, s->aidx, E, lane);
+    warp_exclusive_scan(s->aidx, s->aidx, E, lane);   // in place
     __syncwarp();
     for (int e = lane; e < E; e += 32)
       if (s->count[e] > 0) s->act[s->aidx[e]] = e;
@@ -146,7 +159,8 @@ static __device__ void sched_build(Sched* s, int P, int E, int k, int fb1, int f
 // Copies of the schedule for inspection and for the kernels that read the padded
 // permutation from global memory (the FP8 h quantiser): counts, padded offsets, the
 // padded pair list (pad = P) and the rows in use. One CTA calls it (all its threads).
-__device__ __forceinline__ void sched_publish(const Sched* s, int P, int E, int* counts, int* padded_offsets,
+template <class S>
+__device__ __forceinline__ void sched_publish(const S* s, int P, int E, int* counts, int* padded_offsets,
                                               int* padded_pairs, int* header, int tid, int nthreads) {
   for (int e = tid; e < E; e += nthreads) {
     counts[e] = s->count[e];

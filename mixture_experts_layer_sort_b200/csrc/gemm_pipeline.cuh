@@ -41,12 +41,17 @@ constexpr int kEpiThreads = 128;
 constexpr int kTokenTile = 256;   // widest token tile: the largest N of an M=128 MMA
 static_assert(kTokenTile == kTokenBlock, "the align kernel's token blocks are the GEMM token tiles");
 
-template <bool kFP8>
+// kSmem: dynamic shared memory of the kernel (default: the sm_100 opt-in maximum, one
+// CTA per SM); kTmem: TMEM columns it allocates (two accumulator buffers of kTmem / 2
+// columns). Two kernels whose sizes add up to at most one SM's shared memory and TMEM
+// can have CTAs resident on the same SM at once.
+template <bool kFP8, int kSmem = 232448, int kTmem = 512>
 struct Cfg {
   static constexpr int kATiles = 2;
   static constexpr int kABytes = kTileRows * kRowBytes;             // 16 KB per weight tile
-  static constexpr int kTmemCols = 512;                              // two buffers x two accumulators
-  static constexpr int kSmemBytes = 232448;                          // the sm_100 opt-in maximum
+  static constexpr int kTmemCols = kTmem;                            // two buffers x two accumulators
+  static constexpr int kBufCols = kTmem / 2;                         // columns of one buffer
+  static constexpr int kSmemBytes = kSmem;
   // [0, 1 KB): barriers and flags; [1 KB, 3 KB): two slots of the down epilogue's
   // per-column token row (int, 256 columns each); [3 KB, 5 KB): two slots of its
   // scaled routing weights (float); then the caller's extra bytes, then the ring
@@ -58,6 +63,7 @@ struct Cfg {
   static constexpr int kMmasPerBlock = kRowBytes / kMmaKBytes;
   static_assert(2 * kMaxStages * 8 + 40 + 4 + 16 <= kColTableOffset, "barrier area");
   static_assert(kColTableOffset + 2 * 2 * 256 * 4 <= kFixedBytes, "column tables");
+  static_assert(kTmem == 256 || kTmem == 512, "TMEM allocation");
 };
 
 struct Shared {
@@ -134,23 +140,28 @@ __device__ __forceinline__ void teardown(uint32_t tmem, int warp) {
 
 // Stage ring: a stage holds the two weight tiles plus n_max rows of activations
 // (n_max = widest token tile of the forward), so thin decode batches get a deeper
-// ring than prefill. Two TMEM buffers (columns 0 and 256) when a buffer's two
-// accumulators fit 256 columns, i.e. up to 128 tokens.
+// ring than prefill. Two TMEM buffers (columns 0 and kBufCols) when a buffer's two
+// accumulators fit kBufCols columns (up to 128 tokens with 512 columns, 64 with 256),
+// else one buffer of two accumulators kBufCols apart.
 struct Ring {
   int n_cap, stage_bytes, stages, nbuf;
-  uint32_t up_col;
+  uint32_t up_col, buf_col;
 };
 
 template <class C>
 __device__ __forceinline__ Ring make_ring(int n_max, int max_stages, int ring_bytes) {
   Ring r;
-  r.n_cap = n_max < 16 ? 16 : (n_max > kTokenTile ? kTokenTile : ((n_max + 15) & ~15));
+  // at most kTokenTile tokens, and two accumulators of n_cap columns in the allocation
+  // (a unit with more valid rows fails its bounds check and is reported, not run)
+  constexpr int kCap = kTokenTile < C::kTmemCols / 2 ? kTokenTile : C::kTmemCols / 2;
+  r.n_cap = n_max < 16 ? 16 : (n_max > kCap ? kCap : ((n_max + 15) & ~15));
   r.stage_bytes = (C::kATiles * C::kABytes + r.n_cap * kRowBytes + 1023) & ~1023;
   r.stages = ring_bytes / r.stage_bytes;
   if (r.stages > C::kMaxStages) r.stages = C::kMaxStages;
   if (max_stages >= 2 && r.stages > max_stages) r.stages = max_stages;
-  r.nbuf = r.n_cap <= 128 ? 2 : 1;
-  r.up_col = r.nbuf == 2 ? 128u : 256u;
+  r.nbuf = 2 * r.n_cap <= C::kBufCols ? 2 : 1;
+  r.up_col = r.nbuf == 2 ? C::kBufCols / 2 : C::kBufCols;
+  r.buf_col = C::kBufCols;
   return r;
 }
 
@@ -454,7 +465,7 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
     const uint32_t idesc = idesc_make(kFP8 ? static_cast<uint32_t>(a.f8) : 1u, 128u, n_pad);
     const int buf = rg.nbuf == 2 ? (ms.it & 1) : 0;
     const uint32_t acc_phase = rg.nbuf == 2 ? ((ms.it >> 1) & 1) : (ms.it & 1);
-    const uint32_t d_tmem = tmem + 256u * buf;
+    const uint32_t d_tmem = tmem + rg.buf_col * buf;
     ++ms.it;
     if (!mbar_wait_bounded(&sh.acc_empty[buf], acc_phase ^ 1u, abort_flag, wait_budget(a))) {
       report_error(a.err, kErrWaitAccEmpty);
@@ -559,7 +570,7 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
     }
     const int buf = rg.nbuf == 2 ? (es.iter & 1) : 0;
     const uint32_t acc_phase = rg.nbuf == 2 ? ((es.iter >> 1) & 1) : (es.iter & 1);
-    const uint32_t t_lane = t_lane0 + 256u * buf;
+    const uint32_t t_lane = t_lane0 + rg.buf_col * buf;
     ++es.iter;
     if (epi_tid == 0) *okf = mbar_wait_bounded(&sh.acc_full[buf], acc_phase, abort_flag, wait_budget(a)) ? 1 : 0;
     named_bar_sync(1, kEpiThreads);

@@ -362,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- both GEMMs
   const Ring rg = make_ring<C>(s->n_max, d.max_stages, sh.ring_bytes);
-  const UnitSchedule<SmemTileFn> src1(SmemTileFn{s, fb1}, s->T1, s->S1, kb1);
-  const UnitSchedule<SmemTileFn> src2(SmemTileFn{s, fb2}, s->T2, s->S2, kb2);
+  const UnitSchedule<SmemTileFn<Sched>> src1(SmemTileFn<Sched>{s, fb1}, s->T1, s->S1, kb1);
+  const UnitSchedule<SmemTileFn<Sched>> src2(SmemTileFn<Sched>{s, fb2}, s->T2, s->S2, kb2);
   GateUpHooks<kFP8> h1{&d, s, expert_ready, abort_flag};
   DownHooks<kFP8> h2{&d, s, expert_ready, token_cnt, fb1, k * fb2 * kb2, G, abort_flag};
 

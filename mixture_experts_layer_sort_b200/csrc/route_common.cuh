@@ -124,7 +124,8 @@ __device__ __forceinline__ int choose_splits_warp(int tiles, int kblocks, int sm
   return (tiles > 0 && best != ~0ull) ? static_cast<int>(pick) : 1;
 }
 
-// Exclusive scan of v[0..n) (n <= 32*chunk) by one warp; total written to v_out[n].
+// Exclusive scan of in[0..n) by one warp into out[0..n), the total into out[n]; out
+// may be in (each lane reads an element of its own chunk before writing it).
 __device__ __forceinline__ void warp_exclusive_scan(const int* in, int* out, int n, int lane) {
   const int chunk = (n + 31) / 32;
   const int lo = lane * chunk;
@@ -139,8 +140,9 @@ __device__ __forceinline__ void warp_exclusive_scan(const int* in, int* out, int
   }
   int run = incl - local;
   for (int i = lo; i < hi; ++i) {
+    const int v = in[i];
     out[i] = run;
-    run += in[i];
+    run += v;
   }
   if (lane == 31) out[n] = incl;
 }
