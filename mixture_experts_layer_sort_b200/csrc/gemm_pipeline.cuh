@@ -343,30 +343,6 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
     return true;
   };
   const int n_units = src.count();
-  const int et_all = a.w_expert_tiles > 0 ? static_cast<int>(a.w_expert_tiles) : a.w_rblocks * a.kblocks;
-  if (a.l2_prefetch > 0) {
-    // Ask L2 for this CTA's weight boxes beyond the first ring fill (up to l2_prefetch
-    // of them), spread over the warp's lanes, so that they stream from HBM while the
-    // ring's own loads and any dependency wait are pending; the ring's loads then find
-    // them in this SM's L2.
-    int seen = 0, n = 0;
-    for (int i = 0; i < n_units && n < a.l2_prefetch; ++i) {
-      const Unit un = src.unit(i, rg.n_cap);
-      if (!un.ok) continue;
-      const int rb0 = un.t.fblock * a.rb_step;
-      const int w1 = un.t.expert * et_all + rb0 * a.kblocks;
-      const int w2 = un.t.expert * et_all + (rb0 + a.second_rb) * a.kblocks;
-      const bool has2 = rb0 + a.second_rb < a.w_rblocks;   // (the loads read zeros past the end)
-      for (int kb = un.kb0; kb < un.kb1 && n < a.l2_prefetch; ++kb, ++seen) {
-        if (seen < rg.stages) continue;
-        if ((n & 31) == lane) {
-          tma_prefetch_l2_2d(tm_w, 0, (w1 + kb) * kTileRows);
-          if (has2) tma_prefetch_l2_2d(tm_w, 0, (w2 + kb) * kTileRows);
-        }
-        ++n;
-      }
-    }
-  }
   for (int i = 0; i < n_units && !ps.failed; ++i) {
     const Unit un = src.unit(i, rg.n_cap);
     if (!un.ok) continue;
@@ -374,8 +350,9 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
     // first tiled-weight block of the unit's two weight row blocks; a second block
     // past the end of the tensor reads zeros and is not stored by the epilogue
     const int rb0 = un.t.fblock * a.rb_step;
-    const int wtile = un.t.expert * et_all + rb0 * a.kblocks;
-    const int wtile2 = un.t.expert * et_all + (rb0 + a.second_rb) * a.kblocks;
+    const int et = a.w_expert_tiles > 0 ? static_cast<int>(a.w_expert_tiles) : a.w_rblocks * a.kblocks;
+    const int wtile = un.t.expert * et + rb0 * a.kblocks;
+    const int wtile2 = un.t.expert * et + (rb0 + a.second_rb) * a.kblocks;
     // activation rows of a stage: 16-row boxes, or (direct mode) the valid rows alone
     const int nrows = direct ? un.t.n_valid : nb16;
     const uint32_t tx = C::kATiles * C::kABytes + (direct ? un.t.n_valid : nb16 * 16) * kRowBytes;

@@ -383,16 +383,6 @@ bool direct_x_disabled() {
   return off;
 }
 
-// K blocks of weights past its first ring fill that a GEMM CTA of a decode batch (up to
-// 64 tokens) asks L2 for before its loads (MOE_GEMM_L2_PREFETCH; 0 = none).
-int gemm_l2_prefetch(int M) {
-  static const int n = [] {
-    const char* e = std::getenv("MOE_GEMM_L2_PREFETCH");
-    return e ? std::atoi(e) : 0;
-  }();
-  return M <= 64 ? n : 0;
-}
-
 // Whether new handles take the single-launch decode path for the batches it supports
 // (MOE_FUSED_DECODE=0 or 1 overrides the default).
 bool fused_decode_default() {
@@ -588,7 +578,6 @@ int forward_small(moe_layer* L, const void* x, const float* logits, int M, void*
   g.f8 = fp8_format(L);
   g.err = L->err;
   g.wait_budget = moe::wait_budget_cycles();
-  g.l2_prefetch = gemm_l2_prefetch(M);
 
   moe::SmallArgs s1 = sa;
   s1.g = g;
@@ -767,7 +756,6 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g.f8 = fp8_format(L);
   g.err = L->err;
   g.wait_budget = moe::wait_budget_cycles();
-  g.l2_prefetch = gemm_l2_prefetch(M);
 
   moe::GemmArgs g1 = g;
   g1.tiles = L->tiles1;

@@ -152,8 +152,6 @@ struct GemmArgs {
   int f8;                  // FP8 layers: code format of weights and activations (Fp8Format)
   int* err;
   long long wait_budget;   // SM cycles a pipeline wait may take (0: about a second)
-  int l2_prefetch;         // weight boxes past the first ring fill that the producer asks L2
-                           //   for before its loads start (0: none)
 };
 
 struct QuantHArgs {
