@@ -35,7 +35,7 @@ struct SchedT {
   unsigned mask[kMaxE][2];             // tokens routed to each expert
   int pairs[kSchedMaxPairs];           // pair ids grouped by expert, ascending inside an expert
   int done[kMaxDone];                  // tokens completed by the current down unit
-  float red[8];                        // block reduction scratch
+  float red[32];                       // block reduction scratch (one per warp)
   int ndone;
   int nact, T1, S1, T2, S2, n_max, rows_used, flag;
 };

@@ -23,7 +23,10 @@
 //
 // Roles: warp 0 = TMA producer (lane 0 owns the stage barriers and the weight loads,
 // the activation rows of a stage are spread over the lanes), warp 1 = TMEM owner and
-// MMA issuer, warps 2-5 = epilogue (TMEM lane quadrant = warp % 4). Units (a tile,
+// MMA issuer, warps 2-9 = epilogue: two warps per TMEM lane quadrant (warp % 4), which
+// take alternate 16-column chunks of the accumulators. With token tiles wider than 128
+// columns there is a single accumulator buffer, and the MMAs of the next tile wait
+// until the epilogue has read it: two warps per quadrant halve that wait. Units (a tile,
 // or one K range of a split tile) come from a unit source; dependencies of the
 // activation operand and completion signals come from hooks, so that one kernel can
 // run both GEMMs back to back.
@@ -36,8 +39,9 @@
 namespace moe {
 namespace pipe {
 
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;
+constexpr int kEpiWarps = kEpiThreads / 32;
 constexpr int kTokenTile = 256;   // widest token tile: the largest N of an M=128 MMA
 static_assert(kTokenTile == kTokenBlock, "the align kernel's token blocks are the GEMM token tiles");
 
@@ -268,7 +272,9 @@ struct GlobalTiles : UnitSchedule<GlobalTileFn> {
       : UnitSchedule<GlobalTileFn>(GlobalTileFn{tiles_}, T_, S_, K_) {}
 };
 
-__device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
+// silu(z) = z / (1 + e^-z) with the fast division (2 ulp): e^-z = inf for z < -88 gives
+// z * 0 = -0, the limit; the epilogue rounds the product to bf16 right after.
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.f + __expf(-z)); }
 
 // SM cycles a pipeline wait may take before it gives up (GemmArgs::wait_budget, 0 = the
 // default of about a second).
@@ -539,6 +545,7 @@ template <class C, bool kGateUp, bool kFP8, class Src, class Hooks>
 __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg, const Src& src, Hooks& hk,
                              EpiState& es, uint32_t tmem, volatile int* abort_flag, int warp, int lane) {
   const int q = warp & 3;                       // TMEM lane quadrant of this warp
+  const int half = (warp - 2) >> 2;             // its 16-column chunks: 2 m + half
   const int row = q * 32 + lane;                // weight row inside the tile
   const uint32_t t_lane0 = tmem + (static_cast<uint32_t>(q * 32) << 16);
   const int epi_tid = threadIdx.x - 64;
@@ -555,8 +562,8 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
       if (epi_tid == 0) report_error(a.err, kErrBadTile);
       continue;
     }
-    // One thread waits; the named barrier hands the outcome to the other 127, so
-    // that all of them leave together if the wait gives up. Flag and column-table
+    // One thread waits; the named barrier hands the outcome to the other epilogue
+    // threads, so that all of them leave together if the wait gives up. Flag and column-table
     // slots alternate per unit: no thread can be two units ahead of another.
     volatile int* okf = sh.flags + 2 + (es.iter & 1);
     int* s_tok = sh.col_tok + 256 * (es.iter & 1);
@@ -585,6 +592,15 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
     tc_fence_after();
     const int n_valid = un.t.n_valid;
     const int e = un.t.expert;
+    // this warp's chunks c = half, half + 2, ... < nchunks; the accumulator is released
+    // after the last of them is read (at once when there is none)
+    const int nchunks = (n_valid + 15) >> 4;
+    const int my_last = nchunks - 1 - ((nchunks - 1 - half) & 1);
+    if (my_last < 0) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+    }
 
     if constexpr (kGateUp) {
       const int col = un.t.fblock * kTileRows + row;
@@ -595,13 +611,14 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
       }
       const bool split = un.S > 1;
       const size_t ld_ws = static_cast<size_t>(2) * a.I;
-      for (int c0 = 0; c0 < n_valid; c0 += 16) {
+      for (int c = half; c < nchunks; c += 2) {
+        const int c0 = c * 16;
         float g[16], v[16];
         __syncwarp();
         tmem_ld16(t_lane + c0, g);
         tmem_ld16(t_lane + rg.up_col + c0, v);
         tmem_ld_wait();
-        if (c0 + 16 >= n_valid) {
+        if (c == my_last) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
@@ -638,8 +655,9 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
         if (sh.flags[1]) {
           wrote = true;
           __threadfence();
-          // 8 columns per batch: all 16 loads (L2, bypassing L1) are in flight together
-          for (int n0 = 0; n0 < n_valid; n0 += 8) {
+          // 8 columns per batch: all 16 loads (L2, bypassing L1) are in flight together;
+          // the two warps of a quadrant take alternate batches
+          for (int n0 = 8 * half; n0 < n_valid; n0 += 16) {
             float gs[8], us[8];
             #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -675,13 +693,14 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
       // to f*256 + 128 + row, when that block exists (H/128 odd: the last tile has one)
       const int col0 = un.t.fblock * 2 * kTileRows + row;
       const bool has2 = (un.t.fblock * 2 + 1) * kTileRows < a.H;
-      for (int c0 = 0; c0 < n_valid; c0 += 16) {
+      for (int c = half; c < nchunks; c += 2) {
+        const int c0 = c * 16;
         float y[16], y2[16];
         __syncwarp();
         tmem_ld16(t_lane + c0, y);
         tmem_ld16(t_lane + rg.up_col + c0, y2);
         tmem_ld_wait();
-        if (c0 + 16 >= n_valid) {
+        if (c == my_last) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
