@@ -40,12 +40,8 @@ struct SchedT {
   int nact, T1, S1, T2, S2, n_max, rows_used, flag;
 };
 
-// The single-launch decode kernel (the whole of shared memory is its own).
-using Sched = SchedT<kSchedMaxExperts, 256>;
-// The small-batch GEMMs, which share an SM with each other: up to 256 experts, and a
-// down unit's token rows are at most kSchedMaxTokens.
-constexpr int kSchedSmallMaxExperts = 256;
-using SchedSmall = SchedT<kSchedSmallMaxExperts, kSchedMaxTokens>;
+// The schedule of the single-launch decode kernel and of the small-batch GEMMs.
+using Sched = SchedT<kSchedMaxExperts, kSchedMaxTokens>;
 
 __host__ __device__ constexpr bool sched_supported(int M, int E, int k) {
   return M >= 1 && M <= kSchedMaxTokens && E <= kSchedMaxExperts && M * k <= kSchedMaxPairs;

@@ -23,10 +23,10 @@
 //
 // Roles: warp 0 = TMA producer (lane 0 owns the stage barriers and the weight loads,
 // the activation rows of a stage are spread over the lanes), warp 1 = TMEM owner and
-// MMA issuer, warps 2-9 = epilogue: two warps per TMEM lane quadrant (warp % 4), which
-// take alternate 16-column chunks of the accumulators. With token tiles wider than 128
-// columns there is a single accumulator buffer, and the MMAs of the next tile wait
-// until the epilogue has read it: two warps per quadrant halve that wait. Units (a tile,
+// MMA issuer, warps 2.. = epilogue: kEpiGroups warps per TMEM lane quadrant (warp % 4),
+// which take turns over the 16-column chunks of the accumulators. With token tiles wider
+// than 128 columns there is a single accumulator buffer, and the MMAs of the next tile
+// wait until the epilogue has read it: more warps per quadrant shorten that wait. Units (a tile,
 // or one K range of a split tile) come from a unit source; dependencies of the
 // activation operand and completion signals come from hooks, so that one kernel can
 // run both GEMMs back to back.
@@ -39,9 +39,12 @@
 namespace moe {
 namespace pipe {
 
-constexpr int kThreads = 320;
-constexpr int kEpiThreads = 256;
-constexpr int kEpiWarps = kEpiThreads / 32;
+// Epilogue warps per TMEM lane quadrant. Measured on one B200 at prefill size (E=256,
+// M=4096, one forward): 1 -> 4487 us, 2 -> 4280, 3 -> 4147, 4 -> 4223 (bf16); FP8
+// 2724 / 2491 / 2429 / 2422; decode unchanged.
+constexpr int kEpiGroups = 3;
+constexpr int kEpiThreads = 128 * kEpiGroups;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr int kTokenTile = 256;   // widest token tile: the largest N of an M=128 MMA
 static_assert(kTokenTile == kTokenBlock, "the align kernel's token blocks are the GEMM token tiles");
 
@@ -545,7 +548,7 @@ template <class C, bool kGateUp, bool kFP8, class Src, class Hooks>
 __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg, const Src& src, Hooks& hk,
                              EpiState& es, uint32_t tmem, volatile int* abort_flag, int warp, int lane) {
   const int q = warp & 3;                       // TMEM lane quadrant of this warp
-  const int half = (warp - 2) >> 2;             // its 16-column chunks: 2 m + half
+  const int grp = (warp - 2) >> 2;              // its 16-column chunks: grp + kEpiGroups * m
   const int row = q * 32 + lane;                // weight row inside the tile
   const uint32_t t_lane0 = tmem + (static_cast<uint32_t>(q * 32) << 16);
   const int epi_tid = threadIdx.x - 64;
@@ -592,10 +595,10 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
     tc_fence_after();
     const int n_valid = un.t.n_valid;
     const int e = un.t.expert;
-    // this warp's chunks c = half, half + 2, ... < nchunks; the accumulator is released
-    // after the last of them is read (at once when there is none)
+    // this warp's chunks c = grp, grp + kEpiGroups, ... < nchunks; the accumulator is
+    // released after the last of them is read (at once when there is none)
     const int nchunks = (n_valid + 15) >> 4;
-    const int my_last = nchunks - 1 - ((nchunks - 1 - half) & 1);
+    const int my_last = nchunks - 1 < grp ? -1 : grp + (nchunks - 1 - grp) / kEpiGroups * kEpiGroups;
     if (my_last < 0) {
       tc_fence_before();
       __syncwarp();
@@ -611,7 +614,7 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
       }
       const bool split = un.S > 1;
       const size_t ld_ws = static_cast<size_t>(2) * a.I;
-      for (int c = half; c < nchunks; c += 2) {
+      for (int c = grp; c < nchunks; c += kEpiGroups) {
         const int c0 = c * 16;
         float g[16], v[16];
         __syncwarp();
@@ -656,8 +659,8 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
           wrote = true;
           __threadfence();
           // 8 columns per batch: all 16 loads (L2, bypassing L1) are in flight together;
-          // the two warps of a quadrant take alternate batches
-          for (int n0 = 8 * half; n0 < n_valid; n0 += 16) {
+          // the warps of a quadrant take turns over the batches
+          for (int n0 = 8 * grp; n0 < n_valid; n0 += 8 * kEpiGroups) {
             float gs[8], us[8];
             #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -693,7 +696,7 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
       // to f*256 + 128 + row, when that block exists (H/128 odd: the last tile has one)
       const int col0 = un.t.fblock * 2 * kTileRows + row;
       const bool has2 = (un.t.fblock * 2 + 1) * kTileRows < a.H;
-      for (int c = half; c < nchunks; c += 2) {
+      for (int c = grp; c < nchunks; c += kEpiGroups) {
         const int c0 = c * 16;
         float y[16], y2[16];
         __syncwarp();

@@ -180,7 +180,6 @@ __global__ void __launch_bounds__(256) quant_x_kernel(QuantXArgs a) {
 // FP8: h (bf16) -> codes with s_h = amax(h)/F over the valid rows.
 __global__ void __launch_bounds__(256) quant_h_kernel(QuantHArgs a) {
   const int t = threadIdx.x % kRowThreads;
-  if (a.trigger_first) pdl_trigger();   // the next kernel may become resident before gate_up ends
   pdl_wait();
   pdl_trigger();
   const int used = a.header[kHdrRowsUsed];

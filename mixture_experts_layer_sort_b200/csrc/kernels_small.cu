@@ -17,11 +17,6 @@
 //   epilogue counts the K blocks added to each token and the CTA that adds a token's
 //   last one converts the token's fp32 row to bf16 and re-zeroes it: no finalize
 //   launch. Its last CTA records the FP8 scales of the forward and resets the amax words.
-// - the two GEMMs fit on one SM together (shared memory and TMEM split between them),
-//   so down's CTAs become resident while gate_up still streams its weights: down builds
-//   its schedule and loads its first weight stages then, and only its MMAs wait.
-#include <type_traits>
-
 #include "decode_sched.cuh"
 #include "fp8_format.cuh"
 #include "gemm_pipeline.cuh"
@@ -32,27 +27,10 @@ namespace {
 
 using namespace pipe;
 
-// Shared memory of the two GEMMs: together at most what one SM offers to two CTAs
-// (233472 bytes less 1 KB reserved per CTA). gate_up: 1 KB of alignment slack, the
-// fixed area, the schedule and three 34 KB stages (16-row token tiles) or two 40 KB
-// ones (64-row tiles); down: two stages of either. Each takes half of TMEM.
-constexpr int kSmallSmemGateUp = 128000;
-constexpr int kSmallSmemDown = 233472 - 2 * 1024 - kSmallSmemGateUp;
-template <bool kFP8>
-using CfgGateUp = Cfg<kFP8, kSmallSmemGateUp, 256>;
-template <bool kFP8>
-using CfgDown = Cfg<kFP8, kSmallSmemDown, 256>;
-static_assert(1024 + Cfg<false>::kFixedBytes + ((sizeof(SchedSmall) + 1023) / 1024) * 1024 + 3 * (34 * 1024) <=
-                  kSmallSmemGateUp,
-              "gate_up: three stages of 16-row tiles");
-static_assert(1024 + Cfg<false>::kFixedBytes + ((sizeof(SchedSmall) + 1023) / 1024) * 1024 + 2 * (40 * 1024) <=
-                  kSmallSmemDown,
-              "down: two stages of 64-row tiles");
-
 // gate_up: every activation row is a token row, ready once the kernel waited for its
 // predecessor (done before the schedule is built).
 struct SmallGateHooks {
-  const SchedSmall* s;
+  const Sched* s;
   int k;
   static constexpr bool kSignalTiles = false;
   static constexpr bool kTokenCompletion = false;
@@ -71,7 +49,7 @@ struct SmallGateHooks {
 // down: the activation rows (h or its codes) are written by the previous kernel: one
 // PDL wait; token rows are finished by whoever adds their last K block.
 struct SmallDownHooks {
-  SchedSmall* s;
+  Sched* s;
   float* acc;
   __nv_bfloat16* out;
   int* token_cnt;
@@ -136,10 +114,10 @@ template <bool kGateUp, bool kFP8>
 __global__ void __launch_bounds__(kThreads, 1)
     small_gemm_kernel(const __grid_constant__ SmallArgs a, const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_b) {
-  using C = std::conditional_t<kGateUp, CfgGateUp<kFP8>, CfgDown<kFP8>>;
+  using C = Cfg<kFP8>;
   extern __shared__ uint8_t smem_raw[];
-  const Shared sh = carve<C>(smem_raw, sizeof(SchedSmall));
-  SchedSmall* s = reinterpret_cast<SchedSmall*>(sh.extra);
+  const Shared sh = carve<C>(smem_raw, sizeof(Sched));
+  Sched* s = reinterpret_cast<Sched*>(sh.extra);
   volatile int* abort_flag = sh.flags;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -176,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_trigger();
   }
   const Ring rg = make_ring<C>(s->n_max, a.g.max_stages, sh.ring_bytes);
-  const UnitSchedule<SmemTileFn<SchedSmall>> src(SmemTileFn<SchedSmall>{s, kGateUp ? fb1 : fb2}, kGateUp ? s->T1 : s->T2,
+  const UnitSchedule<SmemTileFn<Sched>> src(SmemTileFn<Sched>{s, kGateUp ? fb1 : fb2}, kGateUp ? s->T1 : s->T2,
                                      kGateUp ? s->S1 : s->S2, kGateUp ? kb1 : kb2);
   SmallGateHooks hg{s, k};
   SmallDownHooks hd{s, a.g.acc, a.out, a.token_cnt, k, a.H, k * fb2 * kb2, warp != 0};
@@ -227,31 +205,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool kGateUp>
-constexpr int small_smem() {
-  return kGateUp ? kSmallSmemGateUp : kSmallSmemDown;
-}
-
 template <bool kGateUp, bool kFP8>
 cudaError_t launch_one(const SmallArgs& a, const CUtensorMap& w, const CUtensorMap& b, int grid, cudaStream_t s) {
   return launch_kernel(small_gemm_kernel<kGateUp, kFP8>, dim3(grid), dim3(kThreads),
-                       static_cast<size_t>(small_smem<kGateUp>()), s, a, w, b);
+                       static_cast<size_t>(Cfg<kFP8>::kSmemBytes), s, a, w, b);
 }
 
-// Both kernels ask for the largest shared-memory carve-out, so that an SM running one
-// of them has the room for a CTA of the other.
 template <bool kGateUp, bool kFP8>
 cudaError_t configure_one() {
-  cudaError_t e = cudaFuncSetAttribute(small_gemm_kernel<kGateUp, kFP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       small_smem<kGateUp>());
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(small_gemm_kernel<kGateUp, kFP8>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              cudaSharedmemCarveoutMaxShared);
+  return cudaFuncSetAttribute(small_gemm_kernel<kGateUp, kFP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<kFP8>::kSmemBytes);
 }
 
 }  // namespace
 
-bool small_supported(int M, int E, int k) { return sched_supported(M, E, k) && E <= kSchedSmallMaxExperts; }
+bool small_supported(int M, int E, int k) { return sched_supported(M, E, k) && E <= kSchedMaxExperts; }
 
 cudaError_t small_configure() {
   cudaError_t e;

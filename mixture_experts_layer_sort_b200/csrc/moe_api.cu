@@ -603,7 +603,6 @@ int forward_small(moe_layer* L, const void* x, const float* logits, int M, void*
     qa.I = L->I;
     qa.amax_h = L->amax + 1;
     qa.f8 = fp8_format(L);
-    qa.trigger_first = 1;
     KernelTimer kt(L, 4, st);
     MOE_CUDA(moe::launch_quant_h(qa, st));
     ++launches;

@@ -164,8 +164,6 @@ struct QuantHArgs {
   int f8;                  // FP8 code format (Fp8Format)
   const int* eflags;       // precision per expert (nullptr: none): only FP8 experts' rows
   const int* topk_ids;     // [P] (with eflags)
-  int trigger_first;       // 1: let the next kernel launch before waiting for gate_up
-                           //    (its own wait still covers this kernel's completion)
 };
 
 struct FinalizeArgs {
