@@ -31,6 +31,9 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
   const int lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
+  // max|h| starts at zero whatever path the previous forward took (gate_up, which folds
+  // into it, waits for this kernel to complete)
+  if (a.amax_h_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.amax_h_reset = 0u;
   if (t >= a.M) return;
   route_token<NPL>(a.logits + static_cast<size_t>(t) * a.E, a.E, a.k, lane, a.topk_ids + static_cast<size_t>(t) * a.k,
                    a.topk_w + static_cast<size_t>(t) * a.k);

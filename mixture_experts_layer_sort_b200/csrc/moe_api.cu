@@ -64,6 +64,7 @@ struct moe_layer {
   int* err = nullptr;
   int* sync = nullptr;          // single-launch decode: counters between its CTAs
   int* small_sync = nullptr;    // small batches: [M_cap] token K-block counts, then a CTA count
+  int4* gv_records = nullptr;   // thin batches: the plan's active experts [min(E, P_cap)]
   int* chunk_buf = nullptr;     // multi-block align: [2][chunks_cap][E] chunk counts and bases
   uint8_t* xq = nullptr;        // FP8 large batches: x quantised per token [M_cap, H]
   long long chunks_cap = 0;
@@ -92,6 +93,7 @@ struct moe_layer {
   // bookkeeping
   int last_M = 0, last_launches = 0;
   bool fused_decode = false;    // single-launch decode path for small batches
+  int gemv_max_m = 0;           // batches of up to this many tokens take the thin-batch path
   bool last_small = false;      // the last forward took the small-batch path (no gathered x)
   // per-kernel event timing
   bool profiling = false;
@@ -168,6 +170,7 @@ int configure_device(int dev) {
   MOE_CUDA(moe::align_configure());
   MOE_CUDA(moe::decode_configure());
   MOE_CUDA(moe::small_configure());
+  MOE_CUDA(moe::gemv_configure());
   if (dev < 64) g_configured |= 1ull << dev;
   return MOE_OK;
 }
@@ -245,6 +248,7 @@ int ensure_workspace(moe_layer* L, int M) {
   MOE_TRY(ws_alloc(L, &L->err, 4, true));
   MOE_TRY(ws_alloc(L, &L->sync, moe::decode_sync_words(L->E, cap) * 4, true));
   MOE_TRY(ws_alloc(L, &L->small_sync, (static_cast<size_t>(cap) + 8) * 4, true));
+  MOE_TRY(ws_alloc(L, &L->gv_records, moe::gemv_records_cap(L->E, P) * 16, false));
   if (is_fp8(L)) MOE_TRY(ws_alloc(L, &L->xq, static_cast<size_t>(cap) * L->H, false));
   L->chunks_cap = (P + moe::kAlignChunk - 1) / moe::kAlignChunk;
   MOE_TRY(ws_alloc(L, &L->chunk_buf, 2 * L->chunks_cap * L->E * 4, false));
@@ -393,6 +397,16 @@ bool fused_decode_default() {
   return on;
 }
 
+// K blocks per expert of the down weights that the thin-batch down kernel asks into L2
+// before it waits for gate_up (MOE_GEMV_PREFETCH_KB; default 0).
+int gemv_prefetch_kb() {
+  static const int v = [] {
+    const char* e = std::getenv("MOE_GEMV_PREFETCH_KB");
+    return e ? std::atoi(e) : 0;
+  }();
+  return v;
+}
+
 int decode_stage_cap() {
   static const int cap = [] {
     const char* e = std::getenv("MOE_MAX_STAGES_DECODE");
@@ -518,6 +532,7 @@ int forward_small(moe_layer* L, const void* x, const float* logits, int M, void*
   ra.topk_ids = L->topk_ids;
   ra.topk_w = L->topk_w;
   ra.amax_x = fp8 ? L->amax : nullptr;
+  ra.amax_h_reset = fp8 ? L->amax + 1 : nullptr;
   {
     KernelTimer kt(L, 0, st);
     MOE_CUDA(moe::launch_route(ra, st));
@@ -626,14 +641,92 @@ int forward_small(moe_layer* L, const void* x, const float* logits, int M, void*
   return MOE_OK;
 }
 
+// Largest batch that new handles send to the thin-batch path (kernels_gemv.cu):
+// MOE_GEMV_MAX_M overrides the built-in default. Measured on one B200 against the
+// tensor-core chain (decode layer E=128, H=2048, I=768): bf16 M=1 34.8 vs 43.1 us, M=4
+// 75.6 vs 75.8, M=16 211 vs 152; e4m3 M=1 37.0 vs 44.0, M=8 116 vs 80; the E=256,
+// H=7168 layer at M=1 148.7 vs 141.0 us. So: bf16 up to 4 tokens, FP8 up to 2, and
+// hidden sizes up to 4096.
+int gemv_max_default(int dtype, int H) {
+  static const int env = [] {
+    const char* e = std::getenv("MOE_GEMV_MAX_M");
+    return e ? std::atoi(e) : -1;
+  }();
+  if (env >= 0) return std::min(env, moe::kGemvMaxM);
+  if (dtype == MOE_DTYPE_MIXED_E4M3 || H > 4096) return 0;
+  return dtype == MOE_DTYPE_BF16 ? 4 : 2;
+}
+
+bool gemv_path(const moe_layer* L, int M) {
+  return M >= 1 && M <= L->gemv_max_m && !is_mixed(L) && moe::gemv_supported(M, L->E, L->k, L->H, L->I, L->num_sms);
+}
+
+// Thin batches: route + plan, gate_up and down as matrix-vector products on the CUDA
+// cores, three launches in all, `out` written by down.
+int forward_gemv(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
+  const bool fp8 = is_fp8(L);
+  moe::GemvArgs a{};
+  a.logits = logits;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.M = M;
+  a.E = L->E;
+  a.k = L->k;
+  a.H = L->H;
+  a.I = L->I;
+  a.topk_ids = L->topk_ids;
+  a.topk_w = L->topk_w;
+  a.counts = L->counts;
+  a.padded_offsets = L->poff;
+  a.padded_pairs = L->pairs;
+  a.header = L->header;
+  a.active = L->gv_records;
+  a.amax = L->amax;
+  a.xq = fp8 ? L->xq : nullptr;
+  a.last_scales = L->last_scales;
+  a.f8 = fp8_format(L);
+  a.w13 = static_cast<const uint8_t*>(L->w13);
+  a.wd = static_cast<const uint8_t*>(L->wd);
+  a.w_scales = L->wscales;
+  const int el = fp8 ? 1 : 2;
+  a.kb1 = L->H * el / moe::kRowBytes;
+  a.kb2 = L->I * el / moe::kRowBytes;
+  a.et1 = static_cast<long long>(2 * L->I / moe::kTileRows) * a.kb1;
+  a.et2 = static_cast<long long>(L->H / moe::kTileRows) * a.kb2;
+  a.h = L->h;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.prefetch_kb = gemv_prefetch_kb();
+  const int fmt = !fp8 ? 0 : (L->dtype == MOE_DTYPE_FP8_E5M2 ? 2 : 1);
+  moe::gemv_down_plan(a, L->num_sms);
+  {
+    KernelTimer kt(L, 0, st);
+    MOE_CUDA(moe::launch_gemv_plan(a, st));
+  }
+  {
+    KernelTimer kt(L, 3, st);
+    MOE_CUDA(moe::launch_gemv_gate_up(a, fmt, st));
+  }
+  {
+    KernelTimer kt(L, 5, st);
+    MOE_CUDA(moe::launch_gemv_down(a, fmt, st));
+  }
+  // FP8 x codes are token rows of xq: the debug copy of x_perm lays them out like the
+  // small-batch path's
+  L->last_small = fp8;
+  L->last_M = M;
+  L->last_launches = 3;
+  return MOE_OK;
+}
+
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
   L->last_small = false;
   if (is_mixed(L)) return forward_mixed(L, x, logits, M, out, st);
+  // the opt-in decode paths first, then the thin-batch path, else the chain
   if (L->fused_decode && M <= L->num_sms && moe::decode_supported(M, L->E, L->k))
     return forward_fused_decode(L, x, logits, M, out, st);
   if (small_batch_enabled() && moe::small_supported(M, L->E, L->k))
     return forward_small(L, x, logits, M, out, st);
+  if (gemv_path(L, M)) return forward_gemv(L, x, logits, M, out, st);
   const bool fp8 = is_fp8(L);
   const long long P = static_cast<long long>(M) * L->k;
   const int BN = moe::kTokenBlock;
@@ -650,6 +743,7 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   ra.topk_ids = L->topk_ids;
   ra.topk_w = L->topk_w;
   ra.amax_x = fp8 ? L->amax : nullptr;
+  ra.amax_h_reset = fp8 ? L->amax + 1 : nullptr;
   {
     KernelTimer kt(L, 0, st);
     MOE_CUDA(moe::launch_route(ra, st));
@@ -850,6 +944,7 @@ int forward_mixed(moe_layer* L, const void* x, const float* logits, int M, void*
   ra.topk_ids = L->topk_ids;
   ra.topk_w = L->topk_w;
   ra.amax_x = L->amax;
+  ra.amax_h_reset = L->amax + 1;
   {
     KernelTimer kt(L, 0, st);
     MOE_CUDA(moe::launch_route(ra, st));
@@ -1126,6 +1221,7 @@ int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
   L->device = dev;
   L->num_sms = prop.multiProcessorCount;
   L->fused_decode = fused_decode_default();
+  L->gemv_max_m = gemv_max_default(dtype, H);
   const size_t el = (dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_MIXED_E4M3) ? 2 : 1;
   if (cudaMalloc(&L->w13, static_cast<size_t>(E) * 2 * I * H * el) != cudaSuccess ||
       cudaMalloc(&L->wd, static_cast<size_t>(E) * H * I * el) != cudaSuccess ||
@@ -1411,6 +1507,13 @@ int moe_last_launch_count(moe_layer* L) { return L ? L->last_launches : 0; }
 int moe_set_fused_decode(moe_layer* L, int enable) {
   if (!L) return MOE_ERR_INVALID_ARG;
   L->fused_decode = enable != 0;
+  ++L->graph_gen;
+  return MOE_OK;
+}
+
+int moe_set_gemv_max_tokens(moe_layer* L, int max_tokens) {
+  if (!L || max_tokens > moe::kGemvMaxM) return MOE_ERR_INVALID_ARG;
+  L->gemv_max_m = max_tokens < 0 ? gemv_max_default(L->dtype, L->H) : max_tokens;
   ++L->graph_gen;
   return MOE_OK;
 }

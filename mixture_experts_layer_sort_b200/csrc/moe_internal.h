@@ -63,6 +63,7 @@ struct RouteArgs {
   int* topk_ids;           // [M, k]
   float* topk_w;           // [M, k]
   unsigned* amax_x;        // FP8 only (else nullptr): running max |x| as float bits
+  unsigned* amax_h_reset;  // when set: the max |h| word, zeroed before gate_up folds into it
 };
 
 struct AlignArgs {
@@ -282,6 +283,59 @@ cudaError_t launch_small_gate_up(const SmallArgs& a, const CUtensorMap& w, const
                                  cudaStream_t s);
 cudaError_t launch_small_down(const SmallArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int grid,
                               cudaStream_t s);
+
+// Thin batches (kernels_gemv.cu): when every expert holds only a few tokens, each
+// weight byte feeds one or two multiply-adds, far below the tensor cores' ridge, and
+// the layer is a set of matrix-vector products that the CUDA cores finish at HBM
+// speed. The forward is then route+plan -> gate_up -> down: no align, gather, split-K
+// or finalize step; down writes bf16 `out` directly.
+constexpr int kGemvMaxM = 16;        // largest batch of the path (token masks in the plan)
+inline long long gemv_records_cap(int E, long long P) { return P < E ? P : E; }
+constexpr int kHdrGemvActive = 7;    // header slot: number of active experts
+struct GemvArgs {
+  const float* logits;     // [M, E]
+  const __nv_bfloat16* x;  // [M, H]
+  int M, E, k, H, I;
+  int* topk_ids;           // [P]
+  float* topk_w;           // [P]
+  // plan written by the route kernel: the align kernel's padded groups (counts, padded
+  // offsets, padded pairs, rows used) and the active experts in ascending id order as
+  // {expert, tokens, first padded row, 0}, their number in header[kHdrGemvActive]
+  int* counts;
+  int* padded_offsets;
+  int* padded_pairs;
+  int* header;
+  int4* active;            // [min(E, P)] (gemv_records_cap)
+  unsigned* amax;          // FP8: [2] max|x| (stored by the route kernel), max|h| (atomic max)
+  uint8_t* xq;             // FP8: [M, H] codes of x (nullptr: bf16 layer)
+  float* last_scales;      // FP8: [2] s_x, s_h of the forward
+  int f8;                  // FP8 code format (Fp8Format)
+  // weights in the tiled layout (TileGeom below)
+  const uint8_t* w13;
+  const uint8_t* wd;
+  const float* w_scales;   // FP8: [E, 3]
+  long long et1, et2;      // stored tiles per expert slot
+  int kb1, kb2;            // 128-byte K blocks per row: H*b/128 (gate_up), I*b/128 (down)
+  __nv_bfloat16* h;        // [P, I] h rows by pair id
+  __nv_bfloat16* out;      // [M, H]
+  int prefetch_kb;         // down: K blocks per expert asked into L2 before the wait (0: none)
+  // down: each CTA takes a contiguous range of at most dn_units (token, 16 features)
+  // units, spanning at most dn_tokens tokens (the host sizes shared memory from both)
+  int dn_units, dn_tokens;
+  int grid;                // CTAs of gate_up and down (one per SM)
+};
+// The path serves 1 <= M <= kGemvMaxM when the per-CTA staging fits shared memory
+// (grid: one CTA per SM, `sms` of them).
+bool gemv_supported(int M, int E, int k, int H, int I, int sms);
+// Shared memory of the down kernel for a batch on `sms` SMs (fills a.grid, a.dn_units and
+// a.dn_tokens).
+size_t gemv_down_plan(GemvArgs& a, int sms);
+cudaError_t gemv_configure();
+// The three launches of the path (fmt: 0 bf16, 1 e4m3, 2 e5m2); gate_up and down run
+// one CTA per SM.
+cudaError_t launch_gemv_plan(const GemvArgs& a, cudaStream_t s);
+cudaError_t launch_gemv_gate_up(const GemvArgs& a, int fmt, cudaStream_t s);
+cudaError_t launch_gemv_down(const GemvArgs& a, int fmt, cudaStream_t s);
 
 // Weight preparation (load time, not on the forward path). Stored weights are
 // tiled: tile (e, rb, kb) = rows [rb*128, +128) x bytes [kb*128, +128) of expert e,

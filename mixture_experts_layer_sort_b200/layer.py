@@ -139,6 +139,10 @@ class MoELayer:
         """Single-launch decode path (bf16, M <= 64) instead of the kernel chain."""
         self._check("moe_set_fused_decode", self.lib.moe_set_fused_decode(self.handle, 1 if enable else 0))
 
+    def set_gemv_max_tokens(self, max_tokens: int):
+        """Largest batch run on the thin-batch (CUDA-core) path; 0 = never, -1 = default."""
+        self._check("moe_set_gemv_max_tokens", self.lib.moe_set_gemv_max_tokens(self.handle, int(max_tokens)))
+
     @property
     def last_launch_count(self) -> int:
         return self.lib.moe_last_launch_count(self.handle)

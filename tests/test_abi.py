@@ -81,6 +81,7 @@ def test_every_entry_point_rejects_a_null_handle(lib):
     assert lib.moe_forward_noalloc(None, None, None, 4, None, None) == -1
     assert lib.moe_load_weights_fp8(None, None, None, None, None, None) == -1
     assert lib.moe_set_fused_decode(None, 1) == -1
+    assert lib.moe_set_gemv_max_tokens(None, 1) == -1
     assert lib.moe_profile_enable(None, 1) == -1
     assert lib.moe_profile_read(None, None, None) == -1
     assert lib.moe_debug_routing(None, None, None, None, None, None, None, None) == -1

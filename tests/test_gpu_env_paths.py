@@ -8,6 +8,10 @@ select (each read once per process, so every setting runs in a child process):
                            gather or finalize) instead of the full chain
   MOE_DISABLE_DIRECT_X=1   small bf16 batches gather x instead of loading token rows
   MOE_MAX_STAGES1/2=2      the shallowest stage rings
+  MOE_GEMV_MAX_M=n         batches of up to n tokens take the thin-batch (CUDA-core) path
+                           (0: none; 16: FP8 layers too up to 16 tokens)
+  MOE_GEMV_PREFETCH_KB=4   the thin-batch down kernel asks L2 for its first weight blocks
+                           before it waits for gate_up
 
 The shape (E=64, k=8, H=1024, I=1024) gives one to eight waves of tiles on a B200 at
 M=64 (the balanced schedule's range) and fewer than one at M=1.
@@ -41,13 +45,18 @@ for dtype in ("bf16", "fp8"):
 print("PARITY_OK")
 """
 
+# MOE_GEMV_MAX_M=0 keeps the small batches on the tensor-core chain, whose alternatives
+# these are
 SETTINGS = [
-    {"MOE_UNIFORM_SPLITS": "1"},
+    {"MOE_UNIFORM_SPLITS": "1", "MOE_GEMV_MAX_M": "0"},
     {"MOE_DISABLE_PDL": "1"},
-    {"MOE_DISABLE_DIRECT_X": "1"},
+    {"MOE_DISABLE_PDL": "1", "MOE_GEMV_MAX_M": "0"},
+    {"MOE_DISABLE_DIRECT_X": "1", "MOE_GEMV_MAX_M": "0"},
     {"MOE_SMALL_BATCH": "1"},
     {"MOE_SMALL_BATCH": "1", "MOE_UNIFORM_SPLITS": "1"},
-    {"MOE_MAX_STAGES1": "2", "MOE_MAX_STAGES2": "2"},
+    {"MOE_MAX_STAGES1": "2", "MOE_MAX_STAGES2": "2", "MOE_GEMV_MAX_M": "0"},
+    {"MOE_GEMV_PREFETCH_KB": "4"},
+    {"MOE_GEMV_MAX_M": "16"},
 ]
 
 

@@ -61,6 +61,23 @@ def test_tiny_fp8(tiny_fp8, M):
     check_output(out, ref, "fp8")
 
 
+@pytest.mark.parametrize("M", [1, 3, 8, 16])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_tiny_chain_small_batches(tiny, tiny_fp8, dtype, M):
+    # the tensor-core chain at the sizes that the thin-batch path takes by default
+    c = tiny if dtype == "bf16" else tiny_fp8
+    c.layer.set_gemv_max_tokens(0)
+    try:
+        x, logits = tokens(c.E, c.H, M, seed=200 + M)
+        out = c.run(x, logits)
+        assert c.layer.last_launch_count >= 5
+        check_routing(c, logits, M)
+        ref, _ = oracle_full(c, x, logits, fp8=dtype == "fp8")
+        check_output(out, ref, dtype)
+    finally:
+        c.layer.set_gemv_max_tokens(-1)
+
+
 def test_fp8_weight_codes_bit_exact(tiny_fp8):
     g, u, d, sc = tiny_fp8.layer.debug_weights()
     for e in range(tiny_fp8.E):
