@@ -16,13 +16,13 @@
 //   down     one CTA per (token, 8 or 16 output features): the token's k experts'
 //            W_down rows times their h rows, weighted by the routing weights and
 //            summed in fp32, written to `out` as bf16 (no atomics, no finalize).
-// "Routing tokens to experts, moving data and combining expert outputs can add work
-// around the matrix multiplications"; fused kernels "combine routing, data movement and
-// expert calculations into fewer GPU operations" (toolboxkart.tech, "AWS SageMaker MoE
-// kernel optimizations H200", section "Why MoE inference needs specialized kernels").
-// The pages' thin-batch answer on Hopper is Swap-AB on the tensor cores (aib.vote, "AWS
-// SageMaker MoE kernel optimizations", second paragraph); the tensor-core chain keeps
-// it for wider batches, and this path replaces it where the product is a matrix-vector
+// The routing, the movement of tokens and the combination of the experts' outputs cost
+// work around the matrix products, and fusing them cuts the number of GPU operations
+// (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "Why MoE
+// inference needs specialized kernels").
+// On Hopper the thin-batch answer was Swap-AB on the tensor cores (aib.vote, "AWS
+// SageMaker MoE kernel optimizations", second paragraph); the tensor-core chain keeps it
+// for wider batches, and this path replaces it where the product is a matrix-vector
 // product.
 //
 // Every lane of a warp streams 16-byte pieces of the tiled weights (kernels_weights.cu:
@@ -223,10 +223,17 @@ __device__ __forceinline__ void weights8_f32(const uint4& u, int part, float (&f
 }
 
 // ------------------------------------------------------------------ streaming
-constexpr int kDepth = 8;
+// Each lane streams its own 16-byte pieces of the weights through a ring of kDepth
+// stages in shared memory with cp.async (L2 -> shared, no registers held while in
+// flight); a stage holds four pieces per lane, 2 KB per warp, and the ring runs across
+// unit boundaries. A lane reads back only what it copied itself, after
+// cp.async.wait_group: no barrier sits between the copy and the use. Two CTAs of 8 warps
+// per SM keep 16 x 8 KB = 128 KB of weights in flight per SM.
+constexpr int kDepth = 4;
+constexpr int kCtasPerSm = 2;   // two CTAs of 8 warps per SM: 16 warps to hide the dot products' latency
 constexpr int kStageWarp = 4 * 32 * 16;              // bytes of one stage of one warp
-constexpr int kRingWarp = kDepth * kStageWarp;       // 16 KB
-constexpr int kRingBytes = kGvWarps * kRingWarp;     // 128 KB per CTA
+constexpr int kRingWarp = kDepth * kStageWarp;       // 8 KB
+constexpr int kRingBytes = kGvWarps * kRingWarp;     // 64 KB per CTA
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, uint64_t pol) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(src),
@@ -255,7 +262,7 @@ constexpr int kGuMaxExperts = 16;   // experts one CTA's range may span (host-ch
 constexpr int kGuTokens = 4;        // tokens per pass: the register tile of a lane
 
 template <int kW>
-__global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_gate_up_kernel(GemvArgs a) {
   constexpr int kEPL = WTraits<kW>::kEPL, kKPB = WTraits<kW>::kKPB;
   constexpr int NT = kGuTokens;
   extern __shared__ __align__(128) uint8_t gv_smem[];
@@ -337,11 +344,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(GemvArgs a)
   __syncthreads();
   float sx = 1.f;
   if constexpr (kW != kWBf16) sx = fp8_scale_from_amax(__ldcg(a.amax), a.f8);
-  float acc[4][NT];
+  float acc[4][NT][2];   // two chains per (row, token): even and odd K elements
   #pragma unroll
   for (int i = 0; i < 4; ++i)
     #pragma unroll
-    for (int j = 0; j < NT; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = 0.f;
   int xo[NT];   // x row offsets (elements) of the current pass's tokens
   int c_ar = ar_first, c_g = g_first, c_pass = 0, c_kb = 0;   // stage being computed
   int n = 0, rec = 0;
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(GemvArgs a)
           #pragma unroll
           for (int i = 0; i < 4; ++i)
             #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[i][j] = fmaf(w[i][q], xv[q], acc[i][j]);
+            for (int q = 0; q < 8; ++q) acc[i][j][q & 1] = fmaf(w[i][q], xv[q], acc[i][j][q & 1]);
         }
       }
     }
@@ -388,11 +395,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(GemvArgs a)
       for (int i = 0; i < 4; ++i)
         #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          float v = acc[i][j];
+          float v = acc[i][j][0] + acc[i][j][1];
           v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
           v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
           v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-          acc[i][j] = v;
+          acc[i][j][0] = v;
         }
       if ((lane & 7) == 0) {
         float sg = 1.f, su = 1.f;
@@ -409,7 +416,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(GemvArgs a)
             __nv_bfloat16* hrow = a.h + static_cast<size_t>(s_pairs[rec * kGemvMaxM + NT * c_pass + j]) * a.I + f0 + q;
             #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-              const __nv_bfloat16 hb = __float2bfloat16_rn(silu_f(acc[hf][j] * sg) * (acc[2 + hf][j] * su));
+              const __nv_bfloat16 hb = __float2bfloat16_rn(silu_f(acc[hf][j][0] * sg) * (acc[2 + hf][j][0] * su));
               hrow[4 * hf] = hb;
               lmax = fmaxf(lmax, fabsf(__bfloat162float(hb)));
             }
@@ -419,7 +426,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(GemvArgs a)
       #pragma unroll
       for (int i = 0; i < 4; ++i)
         #pragma unroll
-        for (int j = 0; j < NT; ++j) acc[i][j] = 0.f;
+        for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = 0.f;
       if (++c_pass == (s_act[rec].y + NT - 1) / NT) {
         c_pass = 0;
         c_g += kGvWarps;
@@ -460,7 +467,7 @@ __device__ __forceinline__ void fp8_forward_done(const GemvArgs& a) {
 }
 
 template <int kW>
-__global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvArgs a) {
   constexpr int kEPL = WTraits<kW>::kEPL, kKPB = WTraits<kW>::kKPB;
   extern __shared__ __align__(128) uint8_t gv_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -556,7 +563,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(GemvArgs a) {
     }
   }
   __syncthreads();
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, y[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, y[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
   int ui = 0, jj = 0, kb = 0, t = t0, fg = u0 - t0 * fgroups;   // stage being computed
   const int kq = (lane & 7) * kEPL;
   #pragma unroll 1
@@ -578,7 +585,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(GemvArgs a) {
         float w[8];
         weights8_f32<kW>(wv[r], p8, w);
         #pragma unroll
-        for (int q = 0; q < 8; ++q) y[r] = fmaf(w[q], hv[q], y[r]);
+        for (int q = 0; q < 8; ++q) y[r][q & 1] = fmaf(w[q], hv[q], y[r][q & 1]);
       }
     }
     if (++kb == a.kb2) {
@@ -586,8 +593,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(GemvArgs a) {
       const float sc = s_sc[slot];
       #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        acc[r] = fmaf(sc, y[r], acc[r]);
-        y[r] = 0.f;
+        acc[r] = fmaf(sc, y[r][0] + y[r][1], acc[r]);
+        y[r][0] = y[r][1] = 0.f;
       }
       if (++jj == nj) {
         jj = 0;
@@ -657,6 +664,7 @@ cudaError_t configure_fmt() {
 
 bool gemv_supported(int M, int E, int k, int H, int I, int sms) {
   if (M < 1 || M > kGemvMaxM || k > 16 || E > 512 || sms < 1) return false;
+  sms *= kCtasPerSm;
   const long long groups = I / kGuRows;
   const long long U = std::min<long long>(E, static_cast<long long>(M) * k) * groups;
   const long long per_cta = (U + sms - 1) / sms;
@@ -667,6 +675,7 @@ bool gemv_supported(int M, int E, int k, int H, int I, int sms) {
 }
 
 size_t gemv_down_plan(GemvArgs& a, int sms) {
+  sms *= kCtasPerSm;
   a.grid = sms;
   down_shape(a.M, a.H, sms, a.dn_units, a.dn_tokens);
   return down_smem(a.dn_units, a.dn_tokens, a.k, a.I);

@@ -643,17 +643,16 @@ int forward_small(moe_layer* L, const void* x, const float* logits, int M, void*
 
 // Largest batch that new handles send to the thin-batch path (kernels_gemv.cu):
 // MOE_GEMV_MAX_M overrides the built-in default. Measured on one B200 against the
-// tensor-core chain (decode layer E=128, H=2048, I=768): bf16 M=1 34.8 vs 43.1 us, M=4
-// 75.6 vs 75.8, M=16 211 vs 152; e4m3 M=1 37.0 vs 44.0, M=8 116 vs 80; the E=256,
-// H=7168 layer at M=1 148.7 vs 141.0 us. So: bf16 up to 4 tokens, FP8 up to 2, and
-// hidden sizes up to 4096.
-int gemv_max_default(int dtype, int H) {
+// tensor-core chain, same box (decode layer E=128, H=2048, I=768): bf16 M=1 35.0 vs
+// 43.1 us, M=4 69.4 vs 75.6, M=16 203 vs 153; e4m3 M=1 36.8 vs 43.8, M=8 95.7 vs 79.5;
+// the E=256, H=7168 layer at M=1 135.1 vs 140.4. So: bf16 up to 4 tokens, FP8 up to 2.
+int gemv_max_default(int dtype, int) {
   static const int env = [] {
     const char* e = std::getenv("MOE_GEMV_MAX_M");
     return e ? std::atoi(e) : -1;
   }();
   if (env >= 0) return std::min(env, moe::kGemvMaxM);
-  if (dtype == MOE_DTYPE_MIXED_E4M3 || H > 4096) return 0;
+  if (dtype == MOE_DTYPE_MIXED_E4M3) return 0;
   return dtype == MOE_DTYPE_BF16 ? 4 : 2;
 }
 

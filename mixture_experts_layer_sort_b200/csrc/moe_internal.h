@@ -322,17 +322,17 @@ struct GemvArgs {
   // down: each CTA takes a contiguous range of at most dn_units (token, 16 features)
   // units, spanning at most dn_tokens tokens (the host sizes shared memory from both)
   int dn_units, dn_tokens;
-  int grid;                // CTAs of gate_up and down (one per SM)
+  int grid;                // CTAs of gate_up and down (two per SM)
 };
 // The path serves 1 <= M <= kGemvMaxM when the per-CTA staging fits shared memory
-// (grid: one CTA per SM, `sms` of them).
+// (grid: two CTAs per SM, `sms` SMs).
 bool gemv_supported(int M, int E, int k, int H, int I, int sms);
 // Shared memory of the down kernel for a batch on `sms` SMs (fills a.grid, a.dn_units and
 // a.dn_tokens).
 size_t gemv_down_plan(GemvArgs& a, int sms);
 cudaError_t gemv_configure();
 // The three launches of the path (fmt: 0 bf16, 1 e4m3, 2 e5m2); gate_up and down run
-// one CTA per SM.
+// two CTAs per SM.
 cudaError_t launch_gemv_plan(const GemvArgs& a, cudaStream_t s);
 cudaError_t launch_gemv_gate_up(const GemvArgs& a, int fmt, cudaStream_t s);
 cudaError_t launch_gemv_down(const GemvArgs& a, int fmt, cudaStream_t s);
