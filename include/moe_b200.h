@@ -231,21 +231,21 @@ MOE_API int moe_set_fused_decode(moe_layer* layer, int enable);
 
 /* Largest batch (tokens) that this handle runs on the thin-batch path, or 0 to send
  * every batch to the tensor-core kernel chain; a negative value restores the default
- * (4 tokens for bf16, 2 for FP8, 0 for MOE_DTYPE_MIXED_E4M3: where the path measured
- * faster than the chain; the environment variable MOE_GEMV_MAX_M sets the default of new
- * handles). At decode sizes an expert receives
- * one or two tokens, so each of its weight bytes feeds one or two multiply-adds: the
- * product is a matrix-vector product bound by streaming the weights, and a small batch
- * pays mostly for launches and synchronisation around that streaming (routing, data
- * movement and combining add work around the matrix products: toolboxkart.tech, "AWS
- * SageMaker MoE kernel optimizations H200",
- * section "Why MoE inference needs specialized kernels"). The thin-batch path runs
- * route + plan, gate_up and down on the CUDA cores (three launches, no split-K, `out`
- * written by down); results agree with the chain within the
- * tolerances of the layer.
- * Serves 1 <= M <= 16 with k <= 16 when the batch's activations fit one block's shared
- * memory next to a 128 KB weight ring (M*H*2 bytes of x; a token's k*I*2 bytes of h).
- * MOE_ERR_INVALID_ARG for a null handle or a value above 16. */
+ * (8 tokens, where the path measured faster than the chain; 0 for MOE_DTYPE_MIXED_E4M3;
+ * the environment variable MOE_GEMV_MAX_M sets the default of new handles). At decode
+ * sizes an expert receives one or two tokens, so each of its weight bytes feeds one or
+ * two multiply-adds: the product is a matrix-vector product bound by streaming the
+ * weights, and a small batch pays mostly for launches and synchronisation around that
+ * streaming (routing, data movement and combining add work around the matrix products:
+ * toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "Why MoE
+ * inference needs specialized kernels"). The thin-batch path runs route + plan, then
+ * gate_up and down as streams of warp-level tensor-core products (mma.sync on bf16
+ * values, or on the e4m3 / e5m2 codes themselves) fed by cp.async: three launches, no
+ * split-K, `out` written by down. Results agree with the chain within the tolerances of
+ * the layer. Serves 1 <= M <= 16 with k <= 16 when the batch's activations fit one
+ * block's shared memory next to a 64 KB weight ring (x: (M+1) rows of H values; h: a
+ * token's k rows of I values). MOE_ERR_INVALID_ARG for a null handle or a value above
+ * 16. */
 MOE_API int moe_set_gemv_max_tokens(moe_layer* layer, int max_tokens);
 
 /* Text of a status code (static storage). */

@@ -1,37 +1,37 @@
-// kernels_gemv.cu - the MoE layer for thin batches (up to 16 tokens) on the CUDA cores.
+// kernels_gemv.cu - the MoE layer for thin batches (up to 16 tokens).
 //
 // At decode sizes an expert receives one or two tokens: each weight byte then feeds one
 // or two multiply-adds, about 1 FLOP per byte, two orders of magnitude below the
 // tensor cores' ridge, and the time of the layer is the time to stream the active
-// experts' weights. What the tensor-core chain adds on top of that streaming is
-// latency: an align launch, a gather, split-K partial sums (a 128-row weight tile over
-// the whole reduction is more bytes than one SM should stream alone), and a finalize.
-// This path runs the same arithmetic as three launches:
+// experts' weights. What the tcgen05 chain adds on top of that streaming is latency: an
+// align launch, a gather, split-K partial sums (a 128-row weight tile over the whole
+// reduction is more bytes than one SM should stream alone), and a finalize. This path
+// runs the same arithmetic as three launches:
 //   plan     route every token (the top-k rule of route_common.cuh), group the pairs
 //            by expert (the align kernel's padded groups, kept for inspection) and
 //            list the active experts; FP8: amax(x), s_x and the x codes;
-//   gate_up  one CTA per (active expert, 8 intermediate features): 8 W_gate and 8 W_up
-//            rows times every token of the expert, h = silu(g) * u stored bf16 by
-//            pair; FP8: max|h| into the amax word;
-//   down     one CTA per (token, 8 or 16 output features): the token's k experts'
-//            W_down rows times their h rows, weighted by the routing weights and
-//            summed in fp32, written to `out` as bf16 (no atomics, no finalize).
+//   gate_up  units of (active expert, 8 intermediate features) spread over the warps of
+//            two CTAs per SM: 8 W_gate and 8 W_up rows times the expert's tokens, h =
+//            silu(g) * u stored bf16 by pair; FP8: max|h| into the amax word;
+//   down     units of (token, 16 output features): the token's k experts' W_down rows
+//            times their h rows, weighted by the routing weights and summed in fp32,
+//            written to `out` as bf16 (no atomics, no finalize).
 // The routing, the movement of tokens and the combination of the experts' outputs cost
 // work around the matrix products, and fusing them cuts the number of GPU operations
 // (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section "Why MoE
-// inference needs specialized kernels").
-// On Hopper the thin-batch answer was Swap-AB on the tensor cores (aib.vote, "AWS
-// SageMaker MoE kernel optimizations", second paragraph); the tensor-core chain keeps it
-// for wider batches, and this path replaces it where the product is a matrix-vector
-// product.
+// inference needs specialized kernels"). On Hopper the thin-batch answer was Swap-AB on
+// the tensor cores (aib.vote, "AWS SageMaker MoE kernel optimizations", second
+// paragraph); the tcgen05 chain keeps it for wider batches, and this path replaces it
+// where the product is a matrix-vector product.
 //
-// Every lane of a warp streams 16-byte pieces of the tiled weights (kernels_weights.cu:
-// a 128-row x 128-byte tile is 16 KB contiguous, rows in order), so one warp load
-// covers 4 consecutive 128-byte rows; the 8 lanes of a row split its 128 bytes and
-// meet in a shuffle reduction. Activations sit in shared memory as bf16 values (FP8
-// codes decode exactly into bf16), read once per K block and reused for every row the
-// lane holds. Products accumulate in fp32; FP8 scales are applied as in the
-// tensor-core epilogues (s_gate*s_x, s_up*s_x, routing weight * s_down * s_h).
+// The weight rows of a unit are the 16 rows (M) of warp-level tensor-core products
+// (mma.sync m16n8k16 on bf16, m16n8k32 on e4m3 / e5m2 codes): one instruction takes a
+// 16 x 32-byte slice of the weights, where a multiply-add per weight element would take
+// dozens, so a warp's instruction stream keeps up with the bytes it streams. The
+// tokens (up to 8) are the N of the product, and the activations (bf16 values or FP8
+// codes, exactly the operands of the tcgen05 chain's MMAs) sit in shared memory.
+// Products accumulate in fp32; FP8 scales are applied as in the chain's epilogues
+// (s_gate*s_x, s_up*s_x, routing weight * s_down * s_h).
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -57,13 +57,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p, int bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// Elements in one 16-byte piece of a weight row, and per 128-byte K block.
-template <int kW>
-struct WTraits {
-  static constexpr int kEPL = kW == kWBf16 ? 8 : 16;
-  static constexpr int kKPB = kEPL * 8;
-};
-
 // 8 bf16 values (16 bytes of shared memory) -> fp32.
 __device__ __forceinline__ void bf16x8_f32(const uint4& u, float* f) {
   const unsigned w[4] = {u.x, u.y, u.z, u.w};
@@ -72,25 +65,6 @@ __device__ __forceinline__ void bf16x8_f32(const uint4& u, float* f) {
     f[2 * q] = __uint_as_float(w[q] << 16);
     f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
   }
-}
-
-// 8 FP8 codes (8 bytes) -> their values as 8 bf16 (exact: every e4m3 and e5m2 value is a
-// bf16 value).
-__device__ __forceinline__ uint4 fp8x8_to_bf16(uint2 c, int f8) {
-  const unsigned w[2] = {c.x, c.y};
-  unsigned o[4];
-  #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const __nv_fp8x2_storage_t s = static_cast<__nv_fp8x2_storage_t>(w[q] >> (16 * hh));
-      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(s, f8 == kFp8E5M2 ? __NV_E5M2 : __NV_E4M3);
-      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&r));
-      const __nv_bfloat162 b = __floats2bfloat162_rn(v.x, v.y);
-      o[2 * q + hh] = *reinterpret_cast<const unsigned*>(&b);
-    }
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // 8 fp32 values -> 8 FP8 codes, v / s correctly rounded (ScaleDiv), RNE, saturating.
@@ -200,77 +174,96 @@ __global__ void __launch_bounds__(kPlanThreads, 1) gemv_plan_kernel(GemvArgs a) 
 }
 
 
-// 8 weights (half `part` of a 16-byte piece for FP8, the whole piece for bf16) -> fp32.
-template <int kW>
-__device__ __forceinline__ void weights8_f32(const uint4& u, int part, float (&f)[8]) {
-  if constexpr (kW == kWBf16) {
-    bf16x8_f32(u, f);
-  } else {
-    const unsigned lo = part == 0 ? u.x : u.z, hi = part == 0 ? u.y : u.w;
-    const unsigned w[2] = {lo, hi};
-    #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const __nv_fp8x2_storage_t c = static_cast<__nv_fp8x2_storage_t>(w[q] >> (16 * hh));
-        const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(c, kW == kWE5M2 ? __NV_E5M2 : __NV_E4M3);
-        const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&r));
-        f[4 * q + 2 * hh] = v.x;
-        f[4 * q + 2 * hh + 1] = v.y;
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------ streaming
-// Each lane streams its own 16-byte pieces of the weights through a ring of kDepth
-// stages in shared memory with cp.async (L2 -> shared, no registers held while in
-// flight); a stage holds four pieces per lane, 2 KB per warp, and the ring runs across
-// unit boundaries. A lane reads back only what it copied itself, after
-// cp.async.wait_group: no barrier sits between the copy and the use. Two CTAs of 8 warps
-// per SM keep 16 x 8 KB = 128 KB of weights in flight per SM.
+// Each warp streams its unit's weights through a ring of kDepth stages in shared memory
+// with cp.async (L2 -> shared, no registers held while in flight). A stage is one
+// 128-byte K block of the unit's 16 weight rows (2 KB); every lane copies four 16-byte
+// pieces of it, chunk c of row R landing at R*128 + ((c ^ (R & 7)) * 16), so that the
+// ldmatrix loads of the tensor-core fragments read eight rows of one chunk from eight
+// different bank groups. Per iteration a warp waits for its oldest stage, meets at a
+// warp barrier (its lanes' copies of that stage landed; their reads of the stage
+// refilled next are done), issues the next stage and multiplies. Two CTAs of 8 warps per
+// SM keep 16 x 6 KB of weights in flight per SM.
 constexpr int kDepth = 4;
-constexpr int kCtasPerSm = 2;   // two CTAs of 8 warps per SM: 16 warps to hide the dot products' latency
-constexpr int kStageWarp = 4 * 32 * 16;              // bytes of one stage of one warp
+constexpr int kCtasPerSm = 2;
+constexpr int kStageWarp = 16 * kRowBytes;           // bytes of one stage of one warp
 constexpr int kRingWarp = kDepth * kStageWarp;       // 8 KB
 constexpr int kRingBytes = kGvWarps * kRingWarp;     // 64 KB per CTA
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, uint64_t pol) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(src),
-               "l"(pol)
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(src), "l"(pol)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// the lane's piece i of ring slot d
-__device__ __forceinline__ uint8_t* ring_piece(uint8_t* ring_lane, int d, int i) {
-  return ring_lane + d * kStageWarp + i * 512;
+// Byte offset, inside a stage, of chunk c (16 bytes) of row R (128 bytes).
+__device__ __forceinline__ uint32_t swz(int R, int c) { return R * kRowBytes + ((c ^ (R & 7)) << 4); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
 }
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr) : "memory");
+}
+
+// d (16 x 8, fp32) += a (16 rows x one K step) * b (one K step x 8 columns): a K step is
+// 16 bf16 values, or 32 e4m3 / e5m2 codes, of every row (the product of two codes is
+// exact in fp32, as in the tensor-core chain's kind::f8f6f4).
+template <int kW>
+__device__ __forceinline__ void mma_step(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  if constexpr (kW == kWBf16)
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  else if constexpr (kW == kWE4M3)
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  else
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e5m2.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Activation rows in shared memory: bf16 values (bf16 layers) or FP8 codes, each row
+// padded by 16 bytes so that ldmatrix's eight rows fall into different bank groups.
+template <int kW>
+struct ActRows {
+  static constexpr int kEl = kW == kWBf16 ? 2 : 1;
+  __host__ __device__ static int stride(int len) { return len * kEl + 16; }   // bytes
+};
 
 // ------------------------------------------------------------------ gate_up
 // Units (a, g): active expert a, W_gate rows [8g, 8g + 8) and the W_up rows of the same
-// features, over the whole reduction, times the expert's tokens in passes of up to 4
-// (an expert with more tokens streams its rows once per pass). CTA c takes the
-// contiguous range [c*U/G, (c+1)*U/G) of the U = A*I/8 units (one or a few experts,
-// whose pairs it keeps in shared memory with every token row of x); warp w takes units
-// w, w + 8, ... of the range, K block after K block. In a K block lane l holds 16 bytes
-// of gate rows l/8 and l/8 + 4 and of the same up rows. Unit positions advance by 8
-// groups with a carry into the next expert (I/8 >= 16 groups per expert).
+// features (the 16 rows of one MMA: gate rows 0..7, up rows 8..15), over the whole
+// reduction, times the expert's tokens in passes of up to 8 (the MMA's N). CTA c takes
+// the contiguous range [c*U/G, (c+1)*U/G) of the U = A*I/8 units (one or a few experts,
+// whose pairs it keeps in shared memory with every token row of x: bf16, or FP8 codes);
+// warp w takes units w, w + 8, ... of the range, K block after K block. A lane's
+// accumulators hold gate and up of the same feature for two tokens, so SwiGLU needs no
+// exchange. Unit positions advance by 8 groups with a carry into the next expert (I/8 >=
+// 16 groups per expert).
 constexpr int kGuMaxExperts = 16;   // experts one CTA's range may span (host-checked)
-constexpr int kGuTokens = 4;        // tokens per pass: the register tile of a lane
+constexpr int kGuTokens = 8;        // tokens per pass: the N of one MMA
 
 template <int kW>
 __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_gate_up_kernel(GemvArgs a) {
-  constexpr int kEPL = WTraits<kW>::kEPL, kKPB = WTraits<kW>::kKPB;
   constexpr int NT = kGuTokens;
   extern __shared__ __align__(128) uint8_t gv_smem[];
   __shared__ int4 s_act[kGuMaxExperts];
   __shared__ int s_pairs[kGuMaxExperts * kGemvMaxM];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* ring = gv_smem + warp * kRingWarp + lane * 16;
-  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(gv_smem + kRingBytes);   // [M][H]
+  const uint32_t ring = smem_u32(gv_smem) + warp * kRingWarp;
+  uint8_t* xs = gv_smem + kRingBytes;                  // [M + 1][xstride]: token rows, a zero row
+  const int xstride = ActRows<kW>::stride(a.H);
   pdl_wait();
   pdl_trigger();
   // the plan was written by the previous kernel: read it from L2
@@ -300,6 +293,10 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_gate_up_kernel(Ge
       }
     }
   }
+  // this lane's four pieces of a stage: rows 4i + lane/8, chunk lane % 8
+  uint32_t dst[4];
+  #pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = swz(4 * i + (lane >> 3), lane & 7);
   int is_ar = ar_first, is_g = g_first, is_pass = 0, is_kb = 0;   // next stage to issue
   auto issue = [&](int s) {
     if (s < n_st) {
@@ -308,11 +305,11 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_gate_up_kernel(Ge
       const long long base = e * a.et1 + is_kb;
       const uint8_t* pg = a.w13 + ((base + static_cast<long long>(f0 >> 7) * a.kb1) * kTileRows + (f0 & 127)) * kRowBytes + lane * 16;
       const uint8_t* pu = a.w13 + ((base + static_cast<long long>((a.I + f0) >> 7) * a.kb1) * kTileRows + (f0 & 127)) * kRowBytes + lane * 16;
-      const int d = s % kDepth;
-      cp_async16(ring_piece(ring, d, 0), pg, pol);
-      cp_async16(ring_piece(ring, d, 1), pg + 512, pol);
-      cp_async16(ring_piece(ring, d, 2), pu, pol);
-      cp_async16(ring_piece(ring, d, 3), pu + 512, pol);
+      const uint32_t slot = ring + (s % kDepth) * kStageWarp;
+      cp_async16(slot + dst[0], pg, pol);
+      cp_async16(slot + dst[1], pg + 512, pol);
+      cp_async16(slot + dst[2], pu, pol);
+      cp_async16(slot + dst[3], pu + 512, pol);
       if (++is_kb == a.kb1) {
         is_kb = 0;
         if (++is_pass == (s_act[is_ar - a0].y + NT - 1) / NT) {
@@ -329,104 +326,73 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_gate_up_kernel(Ge
   };
   #pragma unroll 1
   for (int s = 0; s < kDepth - 1; ++s) issue(s);
-  // the range's pairs, and every token row of x (FP8: the values of its codes) as bf16
+  // the range's pairs, every token row of x (bf16, or its FP8 codes) and a zero row
   for (int i = tid; i < R * kGemvMaxM; i += kGvThreads) {
     const int r = i / kGemvMaxM, j = i - r * kGemvMaxM;
     if (j < s_act[r].y) s_pairs[i] = __ldcg(a.padded_pairs + s_act[r].z + j);
   }
-  const int vecs = a.H / 8;
-  for (int i = tid; i < a.M * vecs; i += kGvThreads) {
-    uint4 v;
-    if constexpr (kW == kWBf16) v = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
-    else v = fp8x8_to_bf16(__ldcg(reinterpret_cast<const uint2*>(a.xq) + i), a.f8);
-    reinterpret_cast<uint4*>(xs)[i] = v;
+  {
+    const int rowv = a.H * ActRows<kW>::kEl / 16;   // 16-byte vectors of a row
+    const uint4* src = kW == kWBf16 ? reinterpret_cast<const uint4*>(a.x) : reinterpret_cast<const uint4*>(a.xq);
+    for (int i = tid; i < (a.M + 1) * rowv; i += kGvThreads) {
+      const int m = i / rowv, v = i - m * rowv;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (m < a.M) val = kW == kWBf16 ? __ldg(src + i) : __ldcg(src + i);
+      *reinterpret_cast<uint4*>(xs + m * xstride + v * 16) = val;
+    }
   }
   __syncthreads();
   float sx = 1.f;
   if constexpr (kW != kWBf16) sx = fp8_scale_from_amax(__ldcg(a.amax), a.f8);
-  float acc[4][NT][2];   // two chains per (row, token): even and odd K elements
-  #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    #pragma unroll
-    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = 0.f;
-  int xo[NT];   // x row offsets (elements) of the current pass's tokens
+  const uint32_t xbase = smem_u32(xs);
+  const uint32_t zero_row = xbase + a.M * xstride;
+  const int a_row = lane & 15, a_hi = lane >> 4;        // A fragments: row, second chunk
+  const int b_tok = lane & 7, b_hi = (lane >> 3) & 1;   // B fragments: token, second chunk
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t brow = zero_row;   // this lane's token row of the current pass
   int c_ar = ar_first, c_g = g_first, c_pass = 0, c_kb = 0;   // stage being computed
   int n = 0, rec = 0;
   float lmax = 0.f;
-  const int kq = (lane & 7) * kEPL;   // the lane's first K element inside a K block
   #pragma unroll 1
   for (int s = 0; s < n_st; ++s) {
+    cp_async_wait<kDepth - 2>();
+    __syncwarp();
     issue(s + kDepth - 1);
-    cp_async_wait<kDepth - 1>();
     if (c_kb == 0) {   // a new pass: up to NT of the expert's tokens
       rec = c_ar - a0;
       n = s_act[rec].y - NT * c_pass;
       if (n > NT) n = NT;
-      #pragma unroll
-      for (int j = 0; j < NT; ++j) xo[j] = j < n ? (s_pairs[rec * kGemvMaxM + NT * c_pass + j] / a.k) * a.H : 0;
+      brow = b_tok < n ? xbase + (s_pairs[rec * kGemvMaxM + NT * c_pass + b_tok] / a.k) * xstride : zero_row;
     }
-    const int d = s % kDepth;
-    uint4 wv[4];
+    const uint32_t slot = ring + (s % kDepth) * kStageWarp;
     #pragma unroll
-    for (int i = 0; i < 4; ++i) wv[i] = *reinterpret_cast<const uint4*>(ring_piece(ring, d, i));
-    const int k0 = c_kb * kKPB + kq;
-    #pragma unroll
-    for (int part = 0; part < kEPL / 8; ++part) {
-      float w[4][8];
-      #pragma unroll
-      for (int i = 0; i < 4; ++i) weights8_f32<kW>(wv[i], part, w[i]);
-      #pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        if (j < n) {
-          float xv[8];
-          bf16x8_f32(*reinterpret_cast<const uint4*>(xs + xo[j] + k0 + 8 * part), xv);
-          #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[i][j][q & 1] = fmaf(w[i][q], xv[q], acc[i][j][q & 1]);
-        }
-      }
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t af[4], bf[2];
+      ldsm_x4(slot + swz(a_row, 2 * ks + a_hi), af);
+      ldsm_x2(brow + (c_kb * 8 + 2 * ks + b_hi) * 16, bf);
+      mma_step<kW>(d, af, bf);
     }
     if (++c_kb == a.kb1) {
-      // the pass is complete: the 8 lanes of each row meet, then lane 8q writes h of
-      // features f0 + q (gate piece 0, up piece 2) and f0 + q + 4 (pieces 1 and 3)
+      // the pass is complete: lane (g, t) holds gate and up of feature f0 + g for the
+      // pass's tokens 2t and 2t + 1
       c_kb = 0;
+      float sg = 1.f, su = 1.f;
+      if constexpr (kW != kWBf16) {
+        const int e = s_act[rec].x;
+        sg = __ldg(a.w_scales + e * 3 + 0) * sx;
+        su = __ldg(a.w_scales + e * 3 + 1) * sx;
+      }
+      const int g = lane >> 2, t2 = 2 * (lane & 3);
+      const int f = c_g * kGuRows + g;
       #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          float v = acc[i][j][0] + acc[i][j][1];
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-          acc[i][j][0] = v;
-        }
-      if ((lane & 7) == 0) {
-        float sg = 1.f, su = 1.f;
-        if constexpr (kW != kWBf16) {
-          const int e = s_act[rec].x;
-          sg = __ldg(a.w_scales + e * 3 + 0) * sx;
-          su = __ldg(a.w_scales + e * 3 + 1) * sx;
-        }
-        const int q = lane >> 3;
-        const int f0 = c_g * kGuRows;
-        #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if (j < n) {
-            __nv_bfloat16* hrow = a.h + static_cast<size_t>(s_pairs[rec * kGemvMaxM + NT * c_pass + j]) * a.I + f0 + q;
-            #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-              const __nv_bfloat16 hb = __float2bfloat16_rn(silu_f(acc[hf][j][0] * sg) * (acc[2 + hf][j][0] * su));
-              hrow[4 * hf] = hb;
-              lmax = fmaxf(lmax, fabsf(__bfloat162float(hb)));
-            }
-          }
+      for (int q = 0; q < 2; ++q) {
+        if (t2 + q < n) {
+          const __nv_bfloat16 hb = __float2bfloat16_rn(silu_f(d[q] * sg) * (d[2 + q] * su));
+          a.h[static_cast<size_t>(s_pairs[rec * kGemvMaxM + NT * c_pass + t2 + q]) * a.I + f] = hb;
+          lmax = fmaxf(lmax, fabsf(__bfloat162float(hb)));
         }
       }
-      #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        #pragma unroll
-        for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = 0.f;
+      d[0] = d[1] = d[2] = d[3] = 0.f;
       if (++c_pass == (s_act[rec].y + NT - 1) / NT) {
         c_pass = 0;
         c_g += kGvWarps;
@@ -446,17 +412,28 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_gate_up_kernel(Ge
 }
 
 // ------------------------------------------------------------------ down
+// Units (t, f): token t, output features [16f, 16f + 16) (the 16 rows of one MMA). CTA c
+// takes the contiguous range [c*U/G, (c+1)*U/G) of the U = M*H/16 units (a token or two,
+// whose routing and h rows it keeps in shared memory: bf16, or the codes of h under s_h
+// for FP8). Warp w takes the slots j = w, w + 8 (k <= 16) of every unit of the range: it
+// streams the 16 W_down rows of expert e_j over the whole reduction and multiplies them
+// by h of pair t*k + j (column 0 of the MMA; the other columns read a zero row). The
+// slot's sums, weighted by the routing weight (FP8: * s_down * s_h), meet in shared
+// memory when the range is done: out[t, f] in bf16, no atomics. The routing comes from
+// the route kernel, two launches back, so the first stages of weights stream in before
+// the wait for gate_up.
 constexpr int kDnRows = 16;
 
+// Byte offsets of the down kernel's shared memory regions (each 16-byte aligned).
 struct DownSmem {
   size_t part, e, sc, h, total;
-  __host__ __device__ DownSmem(int units, int tokens, int k, int I) {
+  __host__ __device__ DownSmem(int units, int tokens, int k, int hstride) {
     const size_t slots = (static_cast<size_t>(tokens) * k + 3) & ~size_t(3);
     part = kRingBytes;
     e = part + static_cast<size_t>(units) * kGvWarps * kDnRows * 4;
     sc = e + slots * 4;
     h = sc + slots * 4;
-    total = h + static_cast<size_t>(tokens) * k * I * 2;
+    total = h + (static_cast<size_t>(tokens) * k + 1) * hstride;   // + a zero row
   }
 };
 
@@ -468,7 +445,6 @@ __device__ __forceinline__ void fp8_forward_done(const GemvArgs& a) {
 
 template <int kW>
 __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvArgs a) {
-  constexpr int kEPL = WTraits<kW>::kEPL, kKPB = WTraits<kW>::kKPB;
   extern __shared__ __align__(128) uint8_t gv_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int k = a.k;
@@ -487,12 +463,13 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
   const int t0 = u0 / fgroups;
   const int T = (u1 - 1) / fgroups - t0 + 1;
   const int nu = u1 - u0;
-  uint8_t* ring = gv_smem + warp * kRingWarp + lane * 16;
-  const DownSmem L(a.dn_units, a.dn_tokens, k, a.I);
-  float* part = reinterpret_cast<float*>(gv_smem + L.part);
-  int* s_e = reinterpret_cast<int*>(gv_smem + L.e);
-  float* s_sc = reinterpret_cast<float*>(gv_smem + L.sc);
-  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(gv_smem + L.h);
+  const int hstride = ActRows<kW>::stride(a.I);
+  const uint32_t ring = smem_u32(gv_smem) + warp * kRingWarp;
+  const DownSmem L(a.dn_units, a.dn_tokens, k, hstride);
+  float* part = reinterpret_cast<float*>(gv_smem + L.part);    // [units][8 warps][16]
+  int* s_e = reinterpret_cast<int*>(gv_smem + L.e);            // [tokens * k]
+  float* s_sc = reinterpret_cast<float*>(gv_smem + L.sc);      // [tokens * k]
+  uint8_t* hs = gv_smem + L.h;                                 // [tokens * k + 1][hstride]
   for (int i = tid; i < T * k; i += kGvThreads) {
     s_e[i] = __ldcg(a.topk_ids + t0 * k + i);
     s_sc[i] = __ldcg(a.topk_w + t0 * k + i);
@@ -502,6 +479,9 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
   const uint64_t pol = l2_policy_evict_first();
   const int nj = warp < k ? (k - warp + kGvWarps - 1) / kGvWarps : 0;
   const int n_st = nu * nj * a.kb2;
+  uint32_t dst[4];
+  #pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = swz(4 * i + (lane >> 3), lane & 7);
   // next stage to issue: unit (token is_t, features is_f0), slot is_j, K block is_kb;
   // units advance by one feature group with a carry into the next token
   int is_t = t0, is_f0 = (u0 - t0 * fgroups) * kDnRows, is_j = 0, is_kb = 0;
@@ -509,9 +489,9 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
     if (s < n_st) {
       const long long e = s_e[(is_t - t0) * k + warp + kGvWarps * is_j];
       const uint8_t* p = a.wd + (((e * a.et2 + static_cast<long long>(is_f0 >> 7) * a.kb2 + is_kb) * kTileRows) + (is_f0 & 127)) * kRowBytes + lane * 16;
-      const int d = s % kDepth;
+      const uint32_t slot = ring + (s % kDepth) * kStageWarp;
       #pragma unroll
-      for (int i = 0; i < 4; ++i) cp_async16(ring_piece(ring, d, i), p + 512 * i, pol);
+      for (int i = 0; i < 4; ++i) cp_async16(slot + dst[i], p + 512 * i, pol);
       if (++is_kb == a.kb2) {
         is_kb = 0;
         if (++is_j == nj) {
@@ -529,6 +509,8 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
   #pragma unroll 1
   for (int s = 0; s < kDepth - 1; ++s) issue(s);
   if (a.prefetch_kb > 0) {
+    // L2 requests for the first K blocks of every (unit, slot) of the range, while gate_up
+    // may still be running
     const int pk = a.prefetch_kb < a.kb2 ? a.prefetch_kb : a.kb2;
     for (int i = tid; i < nu * k * pk; i += kGvThreads) {
       const int kb = i % pk, r = i / pk;
@@ -548,70 +530,68 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
     for (int i = tid; i < T * k; i += kGvThreads) s_sc[i] = s_sc[i] * (__ldg(a.w_scales + s_e[i] * 3 + 2) * s_h);
     if (c == 0 && tid == 0) fp8_forward_done(a);
   }
+  // h rows of the range's pairs (t0*k ...), written by gate_up: read from L2; FP8: their
+  // codes under s_h; then a zero row
   {
-    const int vecs = a.I / 8;
+    const int vecs = a.I / 8;   // 8 values per step
     const ScaleDiv dv(s_h);
     const uint4* h8 = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t0) * k * a.I);
     for (int i = tid; i < T * k * vecs; i += kGvThreads) {
-      uint4 v = __ldcg(h8 + i);
-      if constexpr (kW != kWBf16) {
+      const int r = i / vecs, v = i - r * vecs;
+      const uint4 x = __ldcg(h8 + i);
+      if constexpr (kW == kWBf16) {
+        *reinterpret_cast<uint4*>(hs + r * hstride + v * 16) = x;
+      } else {
         float f[8];
-        bf16x8_f32(v, f);
-        v = fp8x8_to_bf16(codes8(f, dv, a.f8), a.f8);
+        bf16x8_f32(x, f);
+        *reinterpret_cast<uint2*>(hs + r * hstride + v * 8) = codes8(f, dv, a.f8);
       }
-      reinterpret_cast<uint4*>(hs)[i] = v;
     }
+    for (int i = tid; i < hstride / 16; i += kGvThreads)
+      *reinterpret_cast<uint4*>(hs + T * k * hstride + i * 16) = make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, y[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-  int ui = 0, jj = 0, kb = 0, t = t0, fg = u0 - t0 * fgroups;   // stage being computed
-  const int kq = (lane & 7) * kEPL;
+  const uint32_t hbase = smem_u32(hs);
+  const uint32_t zero_row = hbase + T * k * hstride;
+  const int a_row = lane & 15, a_hi = lane >> 4;
+  const int b_hi = (lane >> 3) & 1;
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc0 = 0.f, acc1 = 0.f;   // lane (g, 0): features f0 + g and f0 + g + 8 of the unit
+  int ui = 0, jj = 0, kb = 0, t = t0;
+  int slot = 0;
+  uint32_t brow = zero_row;
   #pragma unroll 1
   for (int s = 0; s < n_st; ++s) {
+    cp_async_wait<kDepth - 2>();
+    __syncwarp();
     issue(s + kDepth - 1);
-    cp_async_wait<kDepth - 1>();
-    const int slot = (t - t0) * k + warp + kGvWarps * jj;
-    const int d = s % kDepth;
-    uint4 wv[4];
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) wv[i] = *reinterpret_cast<const uint4*>(ring_piece(ring, d, i));
-    const __nv_bfloat16* hrow = hs + static_cast<size_t>(slot) * a.I + kb * kKPB + kq;
-    #pragma unroll
-    for (int p8 = 0; p8 < kEPL / 8; ++p8) {
-      float hv[8];
-      bf16x8_f32(*reinterpret_cast<const uint4*>(hrow + 8 * p8), hv);
-      #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        float w[8];
-        weights8_f32<kW>(wv[r], p8, w);
-        #pragma unroll
-        for (int q = 0; q < 8; ++q) y[r][q & 1] = fmaf(w[q], hv[q], y[r][q & 1]);
-      }
+    if (kb == 0) {   // a new (unit, slot): column 0 is h of its pair
+      slot = (t - t0) * k + warp + kGvWarps * jj;
+      brow = (lane & 7) == 0 ? hbase + slot * hstride : zero_row;
     }
-    if (++kb == a.kb2) {
+    const uint32_t sl = ring + (s % kDepth) * kStageWarp;
+    #pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t af[4], bf[2];
+      ldsm_x4(sl + swz(a_row, 2 * ks + a_hi), af);
+      ldsm_x2(brow + (kb * 8 + 2 * ks + b_hi) * 16, bf);
+      mma_step<kW>(d, af, bf);
+    }
+    if (++kb == a.kb2) {   // the slot is complete: column 0, weighted
       kb = 0;
       const float sc = s_sc[slot];
-      #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        acc[r] = fmaf(sc, y[r][0] + y[r][1], acc[r]);
-        y[r][0] = y[r][1] = 0.f;
-      }
-      if (++jj == nj) {
+      acc0 = fmaf(sc, d[0], acc0);
+      acc1 = fmaf(sc, d[2], acc1);
+      d[0] = d[1] = d[2] = d[3] = 0.f;
+      if (++jj == nj) {   // the warp's last slot of the unit
         jj = 0;
-        #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          float v = acc[r];
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-          acc[r] = 0.f;
-          if ((lane & 7) == 0) part[(ui * kGvWarps + warp) * kDnRows + (lane >> 3) + 4 * r] = v;
+        if ((lane & 3) == 0) {
+          part[(ui * kGvWarps + warp) * kDnRows + (lane >> 2)] = acc0;
+          part[(ui * kGvWarps + warp) * kDnRows + (lane >> 2) + 8] = acc1;
         }
+        acc0 = acc1 = 0.f;
         ++ui;
-        if (++fg == fgroups) {
-          fg = 0;
-          ++t;
-        }
+        if ((u0 + ui) % fgroups == 0) ++t;
       }
     }
   }
@@ -623,13 +603,18 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
     #pragma unroll
     for (int w = 0; w < kGvWarps; ++w) sum += part[(uu * kGvWarps + w) * kDnRows + row];
     const int u = u0 + uu;
-    const int t = u / fgroups;
-    a.out[static_cast<size_t>(t) * a.H + (u - t * fgroups) * kDnRows + row] = __float2bfloat16_rn(sum);
+    const int tt = u / fgroups;
+    a.out[static_cast<size_t>(tt) * a.H + (u - tt * fgroups) * kDnRows + row] = __float2bfloat16_rn(sum);
   }
 }
 
-size_t gate_up_smem(int M, int H) { return kRingBytes + static_cast<size_t>(M) * H * 2; }
-size_t down_smem(int units, int tokens, int k, int I) { return DownSmem(units, tokens, k, I).total; }
+// Activation row stride in shared memory: the row plus 16 bytes (el: bytes per value).
+int act_stride(int len, int el) { return len * el + 16; }
+size_t gate_up_smem(int M, int H, int el) { return kRingBytes + static_cast<size_t>(M + 1) * act_stride(H, el); }
+size_t down_smem(int units, int tokens, int k, int I, int el) {
+  return DownSmem(units, tokens, k, act_stride(I, el)).total;
+}
+// dynamic shared memory of one CTA (two share an SM when both fit its 228 KB)
 constexpr size_t kGvSmemMax = 220 * 1024;
 
 void down_shape(int M, int H, int sms, int& units, int& tokens) {
@@ -642,13 +627,13 @@ void down_shape(int M, int H, int sms, int& units, int& tokens) {
 template <int kW>
 cudaError_t launch_gate_up_fmt(const GemvArgs& a, cudaStream_t s) {
   const dim3 grid(a.grid), block(kGvThreads);
-  return launch_kernel(gemv_gate_up_kernel<kW>, grid, block, gate_up_smem(a.M, a.H), s, a);
+  return launch_kernel(gemv_gate_up_kernel<kW>, grid, block, gate_up_smem(a.M, a.H, ActRows<kW>::kEl), s, a);
 }
 
 template <int kW>
 cudaError_t launch_down_fmt(const GemvArgs& a, cudaStream_t s) {
   const dim3 grid(a.grid), block(kGvThreads);
-  const size_t smem = down_smem(a.dn_units, a.dn_tokens, a.k, a.I);
+  const size_t smem = down_smem(a.dn_units, a.dn_tokens, a.k, a.I, ActRows<kW>::kEl);
   return launch_kernel(gemv_down_kernel<kW>, grid, block, smem, s, a);
 }
 
@@ -662,7 +647,8 @@ cudaError_t configure_fmt() {
 
 }  // namespace
 
-bool gemv_supported(int M, int E, int k, int H, int I, int sms) {
+bool gemv_supported(int M, int E, int k, int H, int I, int sms, bool fp8) {
+  const int el = fp8 ? 1 : 2;
   if (M < 1 || M > kGemvMaxM || k > 16 || E > 512 || sms < 1) return false;
   sms *= kCtasPerSm;
   const long long groups = I / kGuRows;
@@ -671,14 +657,14 @@ bool gemv_supported(int M, int E, int k, int H, int I, int sms) {
   if ((per_cta - 1) / groups + 2 > kGuMaxExperts) return false;
   int units, tokens;
   down_shape(M, H, sms, units, tokens);
-  return gate_up_smem(M, H) <= kGvSmemMax && down_smem(units, tokens, k, I) <= kGvSmemMax;
+  return gate_up_smem(M, H, el) <= kGvSmemMax && down_smem(units, tokens, k, I, el) <= kGvSmemMax;
 }
 
 size_t gemv_down_plan(GemvArgs& a, int sms) {
   sms *= kCtasPerSm;
   a.grid = sms;
   down_shape(a.M, a.H, sms, a.dn_units, a.dn_tokens);
-  return down_smem(a.dn_units, a.dn_tokens, a.k, a.I);
+  return down_smem(a.dn_units, a.dn_tokens, a.k, a.I, a.xq != nullptr ? 1 : 2);
 }
 
 cudaError_t gemv_configure() {

@@ -643,25 +643,24 @@ int forward_small(moe_layer* L, const void* x, const float* logits, int M, void*
 
 // Largest batch that new handles send to the thin-batch path (kernels_gemv.cu):
 // MOE_GEMV_MAX_M overrides the built-in default. Measured on one B200 against the
-// tensor-core chain, same box (decode layer E=128, H=2048, I=768): bf16 M=1 35.0 vs
-// 43.1 us, M=4 69.4 vs 75.6, M=16 203 vs 153; e4m3 M=1 36.8 vs 43.8, M=8 95.7 vs 79.5;
-// the E=256, H=7168 layer at M=1 135.1 vs 140.4. So: bf16 up to 4 tokens, FP8 up to 2.
+// tensor-core chain, same box (decode layer E=128, H=2048, I=768): bf16 M=1 33.1 vs
+// 43.1 us, M=4 63.7 vs 76.0, M=16 162 vs 152; e4m3 M=1 31.0 vs 44.7, M=8 67.9 vs 79.8;
+// the E=256, H=7168 layer at M=1 131.3 vs 140.2. So: up to 8 tokens.
 int gemv_max_default(int dtype, int) {
   static const int env = [] {
     const char* e = std::getenv("MOE_GEMV_MAX_M");
     return e ? std::atoi(e) : -1;
   }();
   if (env >= 0) return std::min(env, moe::kGemvMaxM);
-  if (dtype == MOE_DTYPE_MIXED_E4M3) return 0;
-  return dtype == MOE_DTYPE_BF16 ? 4 : 2;
+  return dtype == MOE_DTYPE_MIXED_E4M3 ? 0 : 8;
 }
 
 bool gemv_path(const moe_layer* L, int M) {
-  return M >= 1 && M <= L->gemv_max_m && !is_mixed(L) && moe::gemv_supported(M, L->E, L->k, L->H, L->I, L->num_sms);
+  return M >= 1 && M <= L->gemv_max_m && !is_mixed(L) && moe::gemv_supported(M, L->E, L->k, L->H, L->I, L->num_sms, is_fp8(L));
 }
 
-// Thin batches: route + plan, gate_up and down as matrix-vector products on the CUDA
-// cores, three launches in all, `out` written by down.
+// Thin batches: route + plan, then gate_up and down as streams of warp-level
+// tensor-core products, three launches in all, `out` written by down.
 int forward_gemv(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   const bool fp8 = is_fp8(L);
   moe::GemvArgs a{};

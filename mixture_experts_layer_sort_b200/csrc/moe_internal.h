@@ -326,7 +326,7 @@ struct GemvArgs {
 };
 // The path serves 1 <= M <= kGemvMaxM when the per-CTA staging fits shared memory
 // (grid: two CTAs per SM, `sms` SMs).
-bool gemv_supported(int M, int E, int k, int H, int I, int sms);
+bool gemv_supported(int M, int E, int k, int H, int I, int sms, bool fp8);
 // Shared memory of the down kernel for a batch on `sms` SMs (fills a.grid, a.dn_units and
 // a.dn_tokens).
 size_t gemv_down_plan(GemvArgs& a, int sms);

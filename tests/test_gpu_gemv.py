@@ -1,5 +1,6 @@
-"""GPU parity of the thin-batch path (kernels_gemv.cu): route + plan, gate_up and down
-as matrix-vector products on the CUDA cores, three launches, `out` written by down.
+"""GPU parity of the thin-batch path (kernels_gemv.cu): route + plan, then gate_up and
+down as streams of warp-level tensor-core products, three launches, `out` written by
+down.
 
 Against the oracle at the layer's tolerances, with the routing, the padded
 permutation, s_x and the FP8 x codes bit-exact, in bf16, e4m3 and e5m2; at the tiny,
@@ -123,8 +124,8 @@ def test_size_limits(dtype):
 
 
 def test_default_thresholds():
-    # bf16 handles take the path up to 4 tokens, FP8 handles up to 2
-    for dtype, top in (("bf16", 4), ("fp8", 2)):
+    # new handles take the path up to 8 tokens
+    for dtype, top in (("bf16", 8), ("fp8", 8)):
         c = Case(8, 2, 256, 512, dtype, w_std=0.02)
         c.cache = {}
         try:
