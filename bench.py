@@ -341,8 +341,9 @@ def reference_arm(args, ws, rank):
 
 # ----------------------------------------------------------------------------- main arm
 def traffic_from_profile(kernel_src_hash):
-    """Per-launch DRAM bytes of the gate_up GEMM from the committed ncu summary, or None
-    when the kernel source changed since the counters were taken."""
+    """Per-launch DRAM bytes of the gate_up kernel at each M of the decode sweep from the
+    committed ncu summary, or None when the kernel sources changed since the counters
+    were taken."""
     p = os.path.join(ROOT, "profiles", "gate_up_gemm_decode_traffic.txt")
     try:
         d = {}
@@ -360,7 +361,7 @@ def traffic_from_profile(kernel_src_hash):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for name in ("kernels_gemm.cu", "gemm_pipeline.cuh", "sm100.cuh", "moe_internal.h"):
+    for name in ("kernels_gemm.cu", "kernels_gemv.cu", "gemm_pipeline.cuh", "sm100.cuh", "moe_internal.h"):
         with open(os.path.join(ROOT, "mixture_experts_layer_sort_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -763,7 +764,8 @@ def main():
         "data": "synthetic",
         "config": bench_config(wl, Ms, ws, args.warm_l2),
         "launch": "CUDA graph replay per M" if run.graphs else "eager",
-        "roofline": {"bound": "hbm", "kernel": "gate_up grouped GEMM", "achieved": achieved, "peak": hbm_gbs,
+        "roofline": {"bound": "hbm",
+                     "kernel": "gate_up (the thin-batch tensor-core GEMV up to 8 tokens, the tcgen05 grouped GEMM above)", "achieved": achieved, "peak": hbm_gbs,
                      "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None, "traffic": traffic,
                      "peak_source": f"{peak_src} HBM copy bandwidth",
                      "alg_bytes_per_launch": gate_bytes / max(g_n, 1),
