@@ -183,12 +183,16 @@ __global__ void __launch_bounds__(kPlanThreads, 1) gemv_plan_kernel(GemvArgs a) 
 // different bank groups. Per iteration a warp waits for its oldest stage, meets at a
 // warp barrier (its lanes' copies of that stage landed; their reads of the stage
 // refilled next are done), issues the next stage and multiplies. Two CTAs of 8 warps per
-// SM keep 16 x 6 KB of weights in flight per SM.
-constexpr int kDepth = 4;
+// SM keep 16 x (kD - 1) x 2 KB of weights in flight per SM.
 constexpr int kCtasPerSm = 2;
 constexpr int kStageWarp = 16 * kRowBytes;           // bytes of one stage of one warp
-constexpr int kRingWarp = kDepth * kStageWarp;       // 8 KB
-constexpr int kRingBytes = kGvWarps * kRingWarp;     // 64 KB per CTA
+// ring depth kD (4..6 stages: 8-12 KB per warp, 64-96 KB per CTA), the deepest that lets
+// two CTAs share an SM next to the batch's activation rows
+template <int kD>
+struct Ring {
+  static constexpr int kWarp = kD * kStageWarp;
+  static constexpr int kBytes = kGvWarps * kWarp;
+};
 
 __device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* src, uint64_t pol) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(src), "l"(pol)
@@ -254,9 +258,11 @@ struct ActRows {
 constexpr int kGuMaxExperts = 16;   // experts one CTA's range may span (host-checked)
 constexpr int kGuTokens = 8;        // tokens per pass: the N of one MMA
 
-template <int kW>
+template <int kW, int kD>
 __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_gate_up_kernel(GemvArgs a) {
   constexpr int NT = kGuTokens;
+  constexpr int kDepth = kD;
+  constexpr int kRingWarp = Ring<kD>::kWarp, kRingBytes = Ring<kD>::kBytes;
   extern __shared__ __align__(128) uint8_t gv_smem[];
   __shared__ int4 s_act[kGuMaxExperts];
   __shared__ int s_pairs[kGuMaxExperts * kGemvMaxM];
@@ -427,9 +433,9 @@ constexpr int kDnRows = 16;
 // Byte offsets of the down kernel's shared memory regions (each 16-byte aligned).
 struct DownSmem {
   size_t part, e, sc, h, total;
-  __host__ __device__ DownSmem(int units, int tokens, int k, int hstride) {
+  __host__ __device__ DownSmem(int units, int tokens, int k, int hstride, int ring_bytes) {
     const size_t slots = (static_cast<size_t>(tokens) * k + 3) & ~size_t(3);
-    part = kRingBytes;
+    part = ring_bytes;
     e = part + static_cast<size_t>(units) * kGvWarps * kDnRows * 4;
     sc = e + slots * 4;
     h = sc + slots * 4;
@@ -443,8 +449,10 @@ __device__ __forceinline__ void fp8_forward_done(const GemvArgs& a) {
   a.amax[0] = 0u;
 }
 
-template <int kW>
+template <int kW, int kD>
 __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvArgs a) {
+  constexpr int kDepth = kD;
+  constexpr int kRingWarp = Ring<kD>::kWarp;
   extern __shared__ __align__(128) uint8_t gv_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int k = a.k;
@@ -465,7 +473,7 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
   const int nu = u1 - u0;
   const int hstride = ActRows<kW>::stride(a.I);
   const uint32_t ring = smem_u32(gv_smem) + warp * kRingWarp;
-  const DownSmem L(a.dn_units, a.dn_tokens, k, hstride);
+  const DownSmem L(a.dn_units, a.dn_tokens, k, hstride, Ring<kD>::kBytes);
   float* part = reinterpret_cast<float*>(gv_smem + L.part);    // [units][8 warps][16]
   int* s_e = reinterpret_cast<int*>(gv_smem + L.e);            // [tokens * k]
   float* s_sc = reinterpret_cast<float*>(gv_smem + L.sc);      // [tokens * k]
@@ -610,12 +618,25 @@ __global__ void __launch_bounds__(kGvThreads, kCtasPerSm) gemv_down_kernel(GemvA
 
 // Activation row stride in shared memory: the row plus 16 bytes (el: bytes per value).
 int act_stride(int len, int el) { return len * el + 16; }
-size_t gate_up_smem(int M, int H, int el) { return kRingBytes + static_cast<size_t>(M + 1) * act_stride(H, el); }
-size_t down_smem(int units, int tokens, int k, int I, int el) {
-  return DownSmem(units, tokens, k, act_stride(I, el)).total;
+size_t gate_up_smem(int M, int H, int el, int depth) {
+  return static_cast<size_t>(kGvWarps) * depth * kStageWarp + static_cast<size_t>(M + 1) * act_stride(H, el);
 }
-// dynamic shared memory of one CTA (two share an SM when both fit its 228 KB)
+size_t down_smem(int units, int tokens, int k, int I, int el, int depth) {
+  return DownSmem(units, tokens, k, act_stride(I, el), kGvWarps * depth * kStageWarp).total;
+}
+// dynamic shared memory of one CTA at most
 constexpr size_t kGvSmemMax = 220 * 1024;
+// dynamic shared memory of one CTA when two share an SM (228 KB per SM, 1 KB reserved per
+// CTA, the kernels' static arrays)
+constexpr size_t kTwoPerSm = 111 * 1024;
+
+// The deepest ring (4..6 stages) that keeps two CTAs per SM, given the smem of a depth.
+template <class F>
+int pick_depth(F smem_at) {
+  for (int d = 6; d > 4; --d)
+    if (smem_at(d) <= kTwoPerSm) return d;
+  return 4;
+}
 
 void down_shape(int M, int H, int sms, int& units, int& tokens) {
   const int fgroups = H / kDnRows;
@@ -627,22 +648,40 @@ void down_shape(int M, int H, int sms, int& units, int& tokens) {
 template <int kW>
 cudaError_t launch_gate_up_fmt(const GemvArgs& a, cudaStream_t s) {
   const dim3 grid(a.grid), block(kGvThreads);
-  return launch_kernel(gemv_gate_up_kernel<kW>, grid, block, gate_up_smem(a.M, a.H, ActRows<kW>::kEl), s, a);
+  const int el = ActRows<kW>::kEl;
+  const int d = pick_depth([&](int dd) { return gate_up_smem(a.M, a.H, el, dd); });
+  const size_t smem = gate_up_smem(a.M, a.H, el, d);
+  if (d == 6) return launch_kernel(gemv_gate_up_kernel<kW, 6>, grid, block, smem, s, a);
+  if (d == 5) return launch_kernel(gemv_gate_up_kernel<kW, 5>, grid, block, smem, s, a);
+  return launch_kernel(gemv_gate_up_kernel<kW, 4>, grid, block, smem, s, a);
 }
 
 template <int kW>
 cudaError_t launch_down_fmt(const GemvArgs& a, cudaStream_t s) {
   const dim3 grid(a.grid), block(kGvThreads);
-  const size_t smem = down_smem(a.dn_units, a.dn_tokens, a.k, a.I, ActRows<kW>::kEl);
-  return launch_kernel(gemv_down_kernel<kW>, grid, block, smem, s, a);
+  const int el = ActRows<kW>::kEl;
+  const int d = pick_depth([&](int dd) { return down_smem(a.dn_units, a.dn_tokens, a.k, a.I, el, dd); });
+  const size_t smem = down_smem(a.dn_units, a.dn_tokens, a.k, a.I, el, d);
+  if (d == 6) return launch_kernel(gemv_down_kernel<kW, 6>, grid, block, smem, s, a);
+  if (d == 5) return launch_kernel(gemv_down_kernel<kW, 5>, grid, block, smem, s, a);
+  return launch_kernel(gemv_down_kernel<kW, 4>, grid, block, smem, s, a);
+}
+
+template <int kW, int kD>
+cudaError_t configure_one() {
+  cudaError_t e;
+  const int mx = static_cast<int>(kGvSmemMax);
+  if ((e = cudaFuncSetAttribute(gemv_gate_up_kernel<kW, kD>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx)))
+    return e;
+  return cudaFuncSetAttribute(gemv_down_kernel<kW, kD>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
 }
 
 template <int kW>
 cudaError_t configure_fmt() {
   cudaError_t e;
-  const int mx = static_cast<int>(kGvSmemMax);
-  if ((e = cudaFuncSetAttribute(gemv_gate_up_kernel<kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx))) return e;
-  return cudaFuncSetAttribute(gemv_down_kernel<kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+  if ((e = configure_one<kW, 4>())) return e;
+  if ((e = configure_one<kW, 5>())) return e;
+  return configure_one<kW, 6>();
 }
 
 }  // namespace
@@ -657,14 +696,14 @@ bool gemv_supported(int M, int E, int k, int H, int I, int sms, bool fp8) {
   if ((per_cta - 1) / groups + 2 > kGuMaxExperts) return false;
   int units, tokens;
   down_shape(M, H, sms, units, tokens);
-  return gate_up_smem(M, H, el) <= kGvSmemMax && down_smem(units, tokens, k, I, el) <= kGvSmemMax;
+  return gate_up_smem(M, H, el, 4) <= kGvSmemMax && down_smem(units, tokens, k, I, el, 4) <= kGvSmemMax;
 }
 
 size_t gemv_down_plan(GemvArgs& a, int sms) {
   sms *= kCtasPerSm;
   a.grid = sms;
   down_shape(a.M, a.H, sms, a.dn_units, a.dn_tokens);
-  return down_smem(a.dn_units, a.dn_tokens, a.k, a.I, a.xq != nullptr ? 1 : 2);
+  return down_smem(a.dn_units, a.dn_tokens, a.k, a.I, a.xq != nullptr ? 1 : 2, 4);
 }
 
 cudaError_t gemv_configure() {
