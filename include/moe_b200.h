@@ -264,6 +264,14 @@ MOE_API int moe_get_device_error(moe_layer* layer, int* code);
 /* Number of kernels the last moe_forward launched (0 for M = 0). */
 MOE_API int moe_last_launch_count(moe_layer* layer);
 
+/* 1 when the last moe_forward ran its grouped GEMMs on CTA pairs (clusters of two
+ * CTAs issuing M = 256 tcgen05 MMAs, each CTA loading half of every token tile),
+ * else 0. No counterpart in the pages: an execution detail of this library, chosen
+ * per forward (wide token tiles: at least 96 tokens per expert on average, H a
+ * multiple of 512 and I of 256; MOE_PAIR_GEMM=0 / 1 in the environment forces it off /
+ * on where the shapes allow). 0 for a null handle. */
+MOE_API int moe_last_gemm_pairs(moe_layer* layer);
+
 /* Per-kernel timing. While enabled, every moe_forward records a CUDA event
  * before and after each kernel it launches, on the forward's stream. Kernel
  * slots: 0 route, 1 align, 2 gather, 3 gate_up GEMM, 4 h quantise (FP8 only),

@@ -29,6 +29,7 @@ SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_c_int]),
     "moe_get_device_error": (_c_int, [_c_void_p, ctypes.POINTER(ctypes.c_int)]),
     "moe_last_launch_count": (_c_int, [_c_void_p]),
+    "moe_last_gemm_pairs": (_c_int, [_c_void_p]),
     "moe_set_fused_decode": (_c_int, [_c_void_p, _c_int]),
     "moe_set_gemv_max_tokens": (_c_int, [_c_void_p, _c_int]),
     "moe_profile_enable": (_c_int, [_c_void_p, _c_int]),

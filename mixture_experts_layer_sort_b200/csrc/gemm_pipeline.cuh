@@ -52,8 +52,12 @@ static_assert(kTokenTile == kTokenBlock, "the align kernel's token blocks are th
 // CTA per SM); kTmem: TMEM columns it allocates (two accumulator buffers of kTmem / 2
 // columns). Two kernels whose sizes add up to at most one SM's shared memory and TMEM
 // can have CTAs resident on the same SM at once.
-template <bool kFP8, int kSmem = 232448, int kTmem = 512>
+// kPair: the tiles of a unit are split over a CTA pair (a cluster of two) that runs
+// M = 256 MMAs: each CTA holds its own two weight tiles and half of the activation rows,
+// the pair's first CTA issues the MMAs, and each CTA's TMEM receives its own rows.
+template <bool kFP8, int kSmem = 232448, int kTmem = 512, bool kPair_ = false>
 struct Cfg {
+  static constexpr bool kPair = kPair_;
   static constexpr int kATiles = 2;
   static constexpr int kABytes = kTileRows * kRowBytes;             // 16 KB per weight tile
   static constexpr int kTmemCols = kTmem;                            // two buffers x two accumulators
@@ -112,24 +116,32 @@ __device__ __forceinline__ Shared carve(uint8_t* raw, int extra_bytes) {
 template <class C>
 __device__ __forceinline__ uint32_t prologue(const Shared& s, int warp) {
   if (threadIdx.x == 0) {
+    // pair: the first CTA's full barriers count both CTAs' bytes (the second CTA's are
+    // unused); every CTA's empty barriers take the first CTA's commits
     for (int i = 0; i < C::kMaxStages; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s.acc_full[b], 1);
-      mbar_init(&s.acc_empty[b], kEpiThreads / 32);
+      mbar_init(&s.acc_empty[b], (C::kPair ? 2 : 1) * (kEpiThreads / 32));
     }
     mbar_init(s.drain, 1);
     for (int i = 0; i < 4; ++i) s.flags[i] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(s.tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (C::kPair) {
+      tmem_alloc_pair(s.tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s.tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (C::kPair) cluster_sync();   // both CTAs' barriers exist before either signals the other
+  else __syncthreads();
   tc_fence_after();
   return *s.tmem_slot;
 }
@@ -137,11 +149,13 @@ __device__ __forceinline__ uint32_t prologue(const Shared& s, int warp) {
 template <class C>
 __device__ __forceinline__ void teardown(uint32_t tmem, int warp) {
   tc_fence_before();
-  __syncthreads();
+  if constexpr (C::kPair) cluster_sync();   // neither CTA leaves while the other may still signal it
+  else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, C::kTmemCols);
+    if constexpr (C::kPair) tmem_dealloc_pair(tmem, C::kTmemCols);
+    else tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -161,8 +175,10 @@ __device__ __forceinline__ Ring make_ring(int n_max, int max_stages, int ring_by
   // at most kTokenTile tokens, and two accumulators of n_cap columns in the allocation
   // (a unit with more valid rows fails its bounds check and is reported, not run)
   constexpr int kCap = kTokenTile < C::kTmemCols / 2 ? kTokenTile : C::kTmemCols / 2;
-  r.n_cap = n_max < 16 ? 16 : (n_max > kCap ? kCap : ((n_max + 15) & ~15));
-  r.stage_bytes = (C::kATiles * C::kABytes + r.n_cap * kRowBytes + 1023) & ~1023;
+  // a pair's N is a multiple of 32, so that each CTA holds whole 16-row boxes of it
+  constexpr int kGran = C::kPair ? 32 : 16;
+  r.n_cap = n_max < kGran ? kGran : (n_max > kCap ? kCap : ((n_max + kGran - 1) & ~(kGran - 1)));
+  r.stage_bytes = (C::kATiles * C::kABytes + (C::kPair ? r.n_cap / 2 : r.n_cap) * kRowBytes + 1023) & ~1023;
   r.stages = ring_bytes / r.stage_bytes;
   if (r.stages > C::kMaxStages) r.stages = C::kMaxStages;
   if (max_stages >= 2 && r.stages > max_stages) r.stages = max_stages;
@@ -202,7 +218,7 @@ struct GlobalTileFn {
   __device__ __forceinline__ Tile operator()(int t) const { return tiles[t]; }
 };
 
-// The units of CTA blockIdx.x (of gridDim.x) over T tiles given by a tile function
+// The units of worker w (of nw: CTAs, or CTA pairs) over T tiles given by a tile function
 // (a list in global memory, or a schedule held in shared memory); count() of them,
 // unit(i) in the order every role of the CTA walks them. Two ways of dealing them
 // out, chosen by S:
@@ -217,6 +233,7 @@ template <class TileFn>
 struct UnitSchedule {
   TileFn tiles;
   int T, S, K;
+  int w, nw;               // this worker (a CTA, or a CTA pair) and the number of workers
   int bal_tiles;           // tiles [0, bal_tiles) form the balanced region
   int g_bal;               // CTAs that share it (each with a non-empty range)
   int bal_total;           // its K blocks
@@ -225,12 +242,14 @@ struct UnitSchedule {
 
   // The balanced region holds fewer than two waves of tiles of at most 256 K blocks,
   // so c * bal_total stays far below 2^31 for any grid of up to a few hundred CTAs.
-  __device__ __forceinline__ UnitSchedule(TileFn tiles_, int T_, int S_, int K_)
-      : tiles(tiles_), T(T_), S(S_), K(K_), bal_tiles(0), g_bal(0), bal_total(0), x0(0), x1(0), n_bal(0),
-        n_whole(0) {
+  __device__ __forceinline__ UnitSchedule(TileFn tiles_, int T_, int S_, int K_, bool pair = false)
+      : tiles(tiles_), T(T_), S(S_), K(K_),
+        w(pair ? static_cast<int>(blockIdx.x) >> 1 : static_cast<int>(blockIdx.x)),
+        nw(pair ? static_cast<int>(gridDim.x) >> 1 : static_cast<int>(gridDim.x)), bal_tiles(0), g_bal(0),
+        bal_total(0), x0(0), x1(0), n_bal(0), n_whole(0) {
     if (S != 0 || T <= 0 || K <= 0) return;
-    const int G = static_cast<int>(gridDim.x);
-    const int c = static_cast<int>(blockIdx.x);
+    const int G = nw;
+    const int c = w;
     const int waves = T / G, rem = T - waves * G;
     bal_tiles = rem == 0 ? 0 : (waves == 0 ? T : rem + G);
     bal_total = bal_tiles * K;
@@ -247,12 +266,12 @@ struct UnitSchedule {
   __device__ __forceinline__ int owner(int x) const { return ((x + 1) * g_bal - 1) / bal_total; }
   __device__ __forceinline__ int count() const {
     if (S == 0) return n_bal + n_whole;
-    const int n = T * S, c = static_cast<int>(blockIdx.x);
-    return c < n ? (n - 1 - c) / static_cast<int>(gridDim.x) + 1 : 0;
+    const int n = T * S, c = w;
+    return c < n ? (n - 1 - c) / nw + 1 : 0;
   }
   __device__ __forceinline__ Unit unit(int i, int n_cap) const {
     if (S != 0) {
-      const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+      const int u = w + i * nw;
       const int t = u / S;
       return make_unit(tiles(t), t, u - t * S, S, K, n_cap);
     }
@@ -265,14 +284,14 @@ struct UnitSchedule {
       const int sharers = owner(first + K - 1) - owner(first) + 1;
       return make_unit_range(tiles(t), t, kb0, kb1, sharers, n_cap);
     }
-    const int t = bal_tiles + static_cast<int>(blockIdx.x) + (i - n_bal) * static_cast<int>(gridDim.x);
+    const int t = bal_tiles + w + (i - n_bal) * nw;
     return make_unit_range(tiles(t), t, 0, K, 1, n_cap);
   }
 };
 
 struct GlobalTiles : UnitSchedule<GlobalTileFn> {
-  __device__ __forceinline__ GlobalTiles(const Tile* tiles_, int T_, int S_, int K_)
-      : UnitSchedule<GlobalTileFn>(GlobalTileFn{tiles_}, T_, S_, K_) {}
+  __device__ __forceinline__ GlobalTiles(const Tile* tiles_, int T_, int S_, int K_, bool pair = false)
+      : UnitSchedule<GlobalTileFn>(GlobalTileFn{tiles_}, T_, S_, K_, pair) {}
 };
 
 // silu(z) = z / (1 + e^-z) with the fast division (2 ulp): e^-z = inf for z < -88 gives
@@ -320,7 +339,11 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
   // columns of pad rows are never stored)
   auto load_b = [&](int stg, int kc, int row_start, int nb) {
     uint8_t* bdst = sh.ring + stg * rg.stage_bytes + C::kATiles * C::kABytes;
-    if (!direct) {
+    if constexpr (C::kPair) {
+      const uint32_t bar = mapa_shared(smem_u32(&sh.full[stg]), 0);
+      for (int j = lane; j < nb; j += 32)
+        tma_load_2d_pair(bdst + j * 16 * kRowBytes, tm_b, bar, kc, row_start + 16 * j, pol_b);
+    } else if (!direct) {
       for (int j = lane; j < nb; j += 32)
         tma_load_2d(bdst + j * 16 * kRowBytes, tm_b, &sh.full[stg], kc, row_start + 16 * j, pol_b);
     } else {
@@ -351,14 +374,19 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
     npend -= i;
     return true;
   };
+  // pair: this CTA's weight row blocks sit pair_rb blocks after the first CTA's, and it
+  // holds activation rows [N/2, N) of the unit (the first CTA rows [0, N/2))
+  const int rank = C::kPair ? static_cast<int>(cluster_ctarank()) : 0;
   const int n_units = src.count();
   for (int i = 0; i < n_units && !ps.failed; ++i) {
     const Unit un = src.unit(i, rg.n_cap);
     if (!un.ok) continue;
-    const int nb16 = (un.t.n_valid + 15) >> 4;
+    const int half = ((un.t.n_valid + 31) & ~31) >> 1;
+    const int nb16 = C::kPair ? half >> 4 : (un.t.n_valid + 15) >> 4;
+    const int row0 = un.t.row_start + rank * half;
     // first tiled-weight block of the unit's two weight row blocks; a second block
     // past the end of the tensor reads zeros and is not stored by the epilogue
-    const int rb0 = un.t.fblock * a.rb_step;
+    const int rb0 = un.t.fblock * a.rb_step + rank * a.pair_rb;
     const int et = a.w_expert_tiles > 0 ? static_cast<int>(a.w_expert_tiles) : a.w_rblocks * a.kblocks;
     const int wtile = un.t.expert * et + rb0 * a.kblocks;
     const int wtile2 = un.t.expert * et + (rb0 + a.second_rb) * a.kblocks;
@@ -373,6 +401,13 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
         if (!ok) {
           report_error(a.err, kErrWaitEmpty);
           *abort_flag = 1;
+        } else if constexpr (C::kPair) {
+          // both CTAs' loads count on the first CTA's barrier, which expects both halves
+          uint8_t* st = sh.ring + ps.stage * rg.stage_bytes;
+          const uint32_t bar = mapa_shared(smem_u32(&sh.full[ps.stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&sh.full[ps.stage], 2 * tx);
+          tma_load_2d_pair(st, tm_w, bar, 0, (wtile + kb) * kTileRows, pol_w);
+          tma_load_2d_pair(st + C::kABytes, tm_w, bar, 0, (wtile2 + kb) * kTileRows, pol_w);
         } else {
           uint8_t* st = sh.ring + ps.stage * rg.stage_bytes;
           mbar_arrive_expect_tx(&sh.full[ps.stage], tx);
@@ -399,11 +434,11 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
       const int kc = kb * C::kKPerBlock;
       if (!ps.failed && npend > 0 && !drain(false)) ps.failed = true;
       if (!ps.failed && npend == 0 && hk.ready(dep)) {
-        load_b(ps.stage, kc, un.t.row_start, nrows);
+        load_b(ps.stage, kc, row0, nrows);
       } else if (!ps.failed) {
         pend_stage[npend] = ps.stage;
         pend_kc[npend] = kc;
-        pend_row[npend] = un.t.row_start;
+        pend_row[npend] = row0;
         pend_nb[npend] = nrows;
         pend_dep[npend] = dep;
         if (++npend == rg.stages && !drain(true)) ps.failed = true;
@@ -438,10 +473,36 @@ __device__ void run_producer(const GemmArgs& a, const CUtensorMap* tm_w, const C
   }
 }
 
+// Pair: wait until the MMAs have released every stage this CTA filled, so that no
+// arrival of the other CTA's commits is still on its way when the CTA leaves.
+template <class C>
+__device__ void producer_tail(const Shared& sh, const Ring& rg, const ProducerState& ps, int lane) {
+  if (ps.failed || lane != 0) return;
+  int zero = 0;
+  int st = ps.stage;
+  uint32_t ph = ps.phase;
+  for (int i = 0; i < rg.stages; ++i) {
+    mbar_wait_bounded(&sh.empty[st], ph ^ 1u, &zero, 1ll << 26);
+    if (++st == rg.stages) {
+      st = 0;
+      ph ^= 1u;
+    }
+  }
+}
+
 // After a failure: let the copies already in flight land before shared memory goes away.
 template <class C>
 __device__ void producer_quiesce(const Shared& sh, const Ring& rg, const ProducerState& ps, int lane) {
   if (!ps.failed || lane != 0) return;
+  if constexpr (C::kPair) {
+    if (cluster_ctarank() != 0) {
+      // its loads count on the other CTA's barriers: give them time to land instead
+      const long long t0 = clock64();
+      while (clock64() - t0 < (1ll << 17)) {
+      }
+      return;
+    }
+  }
   int zero = 0;
   int st = ps.stage, ph = static_cast<int>(ps.phase);
   const int pending = ps.issued < rg.stages ? ps.issued : rg.stages;
@@ -469,14 +530,15 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
   for (int i = 0; i < n_units && !ms.failed; ++i) {
     const Unit un = src.unit(i, rg.n_cap);
     if (!un.ok) continue;
-    const uint32_t n_pad = static_cast<uint32_t>((un.t.n_valid + 15) & ~15);
+    const uint32_t n_pad = C::kPair ? static_cast<uint32_t>((un.t.n_valid + 31) & ~31)
+                                    : static_cast<uint32_t>((un.t.n_valid + 15) & ~15);
     // operand format: bf16 = 1 under kind::f16; the FP8 format code under kind::f8f6f4
-    const uint32_t idesc = idesc_make(kFP8 ? static_cast<uint32_t>(a.f8) : 1u, 128u, n_pad);
+    const uint32_t idesc = idesc_make(kFP8 ? static_cast<uint32_t>(a.f8) : 1u, C::kPair ? 256u : 128u, n_pad);
     const int buf = rg.nbuf == 2 ? (ms.it & 1) : 0;
     const uint32_t acc_phase = rg.nbuf == 2 ? ((ms.it >> 1) & 1) : (ms.it & 1);
     const uint32_t d_tmem = tmem + rg.buf_col * buf;
     ++ms.it;
-    if (!mbar_wait_bounded(&sh.acc_empty[buf], acc_phase ^ 1u, abort_flag, wait_budget(a))) {
+    if (!mbar_wait_bounded(&sh.acc_empty[buf], acc_phase ^ 1u, abort_flag, wait_budget(a), C::kPair)) {
       report_error(a.err, kErrWaitAccEmpty);
       *abort_flag = 1;
       ms.failed = true;
@@ -500,7 +562,13 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
         const uint64_t bd = sdesc_k_sw128(b0 + koff);
         const uint64_t ad0 = sdesc_k_sw128(a0 + koff);
         const uint64_t ad1 = sdesc_k_sw128(a0 + C::kABytes + koff);
-        if constexpr (kFP8) {
+        if constexpr (C::kPair && kFP8) {
+          mma_f8_pair(d_tmem, ad0, bd, idesc, accum);
+          mma_f8_pair(d_tmem + rg.up_col, ad1, bd, idesc, accum);
+        } else if constexpr (C::kPair) {
+          mma_bf16_pair(d_tmem, ad0, bd, idesc, accum);
+          mma_bf16_pair(d_tmem + rg.up_col, ad1, bd, idesc, accum);
+        } else if constexpr (kFP8) {
           mma_f8(d_tmem, ad0, bd, idesc, accum);
           mma_f8(d_tmem + rg.up_col, ad1, bd, idesc, accum);
         } else {
@@ -508,24 +576,30 @@ __device__ void run_mma(const GemmArgs& a, const Shared& sh, const Ring& rg, con
           mma_bf16(d_tmem + rg.up_col, ad1, bd, idesc, accum);
         }
       }
-      mma_commit(&sh.empty[ms.stage]);   // frees the stage once these MMAs have read it
+      // frees the stage (in both CTAs of a pair) once these MMAs have read it
+      if constexpr (C::kPair) mma_commit_pair(&sh.empty[ms.stage]);
+      else mma_commit(&sh.empty[ms.stage]);
       if (++ms.stage == rg.stages) {
         ms.stage = 0;
         ms.phase ^= 1u;
       }
     }
     if (ms.failed) break;
-    mma_commit(&sh.acc_full[buf]);       // accumulator complete
+    // accumulator complete (in both CTAs of a pair)
+    if constexpr (C::kPair) mma_commit_pair(&sh.acc_full[buf]);
+    else mma_commit(&sh.acc_full[buf]);
   }
 }
 
 // After the MMA thread gave up: make every MMA it issued complete (they write TMEM and
 // arrive on stage barriers) before the CTA frees TMEM and leaves. tcgen05.commit
 // tracks all earlier MMAs of the thread; the wait is bounded as well.
+template <class C>
 __device__ __forceinline__ void mma_drain(const Shared& sh, const MmaState& ms) {
   if (!ms.failed) return;
   int zero = 0;
-  mma_commit(sh.drain);
+  if constexpr (C::kPair) mma_commit_pair(sh.drain);
+  else mma_commit(sh.drain);
   mbar_wait_bounded(sh.drain, 0u, &zero, 1ll << 26);
 }
 
@@ -552,6 +626,13 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
   const int row = q * 32 + lane;                // weight row inside the tile
   const uint32_t t_lane0 = tmem + (static_cast<uint32_t>(q * 32) << 16);
   const int epi_tid = threadIdx.x - 64;
+  // pair: this CTA's rows are the weight row blocks pair_rb after the first CTA's, and
+  // both CTAs' epilogues release an accumulator on the first CTA's barrier
+  const int rank = C::kPair ? static_cast<int>(cluster_ctarank()) : 0;
+  auto release_acc = [&](int b) {
+    if constexpr (C::kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&sh.acc_empty[b]), 0));
+    else mbar_arrive(&sh.acc_empty[b]);
+  };
   float sx = 1.f, sh_scale = 1.f;
   if constexpr (kFP8) {
     // written by other CTAs (or kernels): read from L2, not a possibly stale L1 line
@@ -602,11 +683,11 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
     if (my_last < 0) {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+      if (lane == 0) release_acc(buf);
     }
 
     if constexpr (kGateUp) {
-      const int col = un.t.fblock * kTileRows + row;
+      const int col = (un.t.fblock * a.rb_step + rank * a.pair_rb) * kTileRows + row;
       float sg = 1.f, su = 1.f;
       if constexpr (kFP8) {
         sg = __ldg(a.w_scales + e * 3 + 0) * sx;
@@ -624,7 +705,7 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
         if (c == my_last) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+          if (lane == 0) release_acc(buf);
         }
         #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -649,9 +730,10 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
         __threadfence();
         named_bar_sync(1, kEpiThreads);
         if (epi_tid == 0) {
-          const int old = atomicAdd(a.tile_counters + un.tile, 1);
+          const int ctr = C::kPair ? 2 * un.tile + rank : un.tile;   // a pair's CTAs finish their own rows
+          const int old = atomicAdd(a.tile_counters + ctr, 1);
           const int last = (old == un.S - 1) ? 1 : 0;
-          if (last) a.tile_counters[un.tile] = 0;
+          if (last) a.tile_counters[ctr] = 0;
           sh.flags[1] = last;
         }
         named_bar_sync(1, kEpiThreads);
@@ -692,10 +774,11 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
         if (wrote) hk.tile_done(un, epi_tid, es.lmax);
       }
     } else {
-      // rows of the first weight block go to features f*256 + row, the second block's
-      // to f*256 + 128 + row, when that block exists (H/128 odd: the last tile has one)
-      const int col0 = un.t.fblock * 2 * kTileRows + row;
-      const bool has2 = (un.t.fblock * 2 + 1) * kTileRows < a.H;
+      // rows of the first weight block go to features rb*128 + row, the second block's
+      // to (rb + 1)*128 + row, when that block exists (H/128 odd: the last tile has one)
+      const int rb = un.t.fblock * a.rb_step + rank * a.pair_rb;
+      const int col0 = rb * kTileRows + row;
+      const bool has2 = (rb + 1) * kTileRows < a.H;
       for (int c = grp; c < nchunks; c += kEpiGroups) {
         const int c0 = c * 16;
         float y[16], y2[16];
@@ -706,7 +789,7 @@ __device__ void run_epilogue(const GemmArgs& a, const Shared& sh, const Ring& rg
         if (c == my_last) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+          if (lane == 0) release_acc(buf);
         }
         #pragma unroll
         for (int j = 0; j < 16; ++j)

@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       MmaState ms;
       run_mma<C, kFP8>(d.g1, sh, rg, src1, ms, tmem, abort_flag);
       if (!ms.failed) run_mma<C, kFP8>(d.g2, sh, rg, src2, ms, tmem, abort_flag);
-      mma_drain(sh, ms);
+      mma_drain<C>(sh, ms);
     }
   } else {
     const int epi_tid = tid - 64;

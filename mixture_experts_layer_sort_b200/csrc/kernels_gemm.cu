@@ -46,11 +46,11 @@ struct PdlHooks {
   __device__ __forceinline__ void down_done(const Unit&, const int*, int) {}
 };
 
-template <bool kGateUp, bool kFP8>
+template <bool kGateUp, bool kFP8, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs a, const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_b) {
-  using C = Cfg<kFP8>;
+  using C = Cfg<kFP8, 232448, 512, kPair>;
   extern __shared__ uint8_t smem_raw[];
   const Shared sh = carve<C>(smem_raw, 0);
   volatile int* abort_flag = sh.flags;
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const Ring rg = make_ring<C>(a.header[kHdrMaxRows], a.max_stages, sh.ring_bytes);
   const int t_off = a.hdr_tile_offset > 0 ? a.header[a.hdr_tile_offset] : 0;
-  const GlobalTiles src(a.tiles + t_off, a.header[a.hdr_tiles], a.header[a.hdr_splits], a.kblocks);
+  const GlobalTiles src(a.tiles + t_off, a.header[a.hdr_tiles], a.header[a.hdr_splits], a.kblocks, kPair);
   // Everyone but the producer warp waits for the previous kernel here. Otherwise the
   // tile list comes from the align kernel, at least two launches back, and is
   // complete already (see pdl_wait in sm100.cuh).
@@ -83,11 +83,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     ProducerState ps;
     run_producer<C>(a, &tm_w, &tm_b, sh, rg, src, hk, ps, abort_flag, lane);
     producer_quiesce<C>(sh, rg, ps, lane);
+    if constexpr (kPair) producer_tail<C>(sh, rg, ps, lane);
   } else if (warp == 1) {
     if (lane == 0) {
-      MmaState ms;
-      run_mma<C, kFP8>(a, sh, rg, src, ms, tmem, abort_flag);
-      mma_drain(sh, ms);
+      // pair: the first CTA issues the MMAs of both
+      if (!kPair || cluster_ctarank() == 0) {
+        MmaState ms;
+        run_mma<C, kFP8>(a, sh, rg, src, ms, tmem, abort_flag);
+        mma_drain<C>(sh, ms);
+      }
     }
   } else {
     EpiState es;
@@ -98,14 +102,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool kGateUp, bool kFP8>
-cudaError_t launch_one(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int grid, cudaStream_t s) {
-  return launch_kernel(grouped_gemm_kernel<kGateUp, kFP8>, dim3(grid), dim3(kThreads),
-                       static_cast<size_t>(Cfg<kFP8>::kSmemBytes), s, a, w, b);
+cudaError_t launch_one(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& b, int grid, cudaStream_t s,
+                       bool pair) {
+  if (!pair)
+    return launch_kernel(grouped_gemm_kernel<kGateUp, kFP8, false>, dim3(grid), dim3(kThreads),
+                         static_cast<size_t>(Cfg<kFP8>::kSmemBytes), s, a, w, b);
+  // clusters of two CTAs, with programmatic dependent launch as for every kernel of the chain
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid & ~1);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg<kFP8>::kSmemBytes);
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kGateUp, kFP8, true>, a, w, b);
 }
 
 template <bool kGateUp, bool kFP8>
 cudaError_t configure_one() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kFP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kFP8, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<kFP8>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kFP8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               Cfg<kFP8>::kSmemBytes);
 }
 
@@ -119,14 +144,36 @@ cudaError_t gemm_configure() {
   return configure_one<false, true>();
 }
 
+int gemm_pair_clusters() {
+  // the bf16 and FP8 kernels take the same resources (one CTA per SM: all of its shared
+  // memory and TMEM); a pair needs two such SMs of one GPC
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg<false>::kSmemBytes);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true, false, true>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
 cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8, int grid,
-                         cudaStream_t s) {
-  return fp8 ? launch_one<true, true>(a, w, x, grid, s) : launch_one<true, false>(a, w, x, grid, s);
+                         cudaStream_t s, bool pair) {
+  return fp8 ? launch_one<true, true>(a, w, x, grid, s, pair) : launch_one<true, false>(a, w, x, grid, s, pair);
 }
 
 cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int grid,
-                         cudaStream_t s) {
-  return fp8 ? launch_one<false, true>(a, w, h, grid, s) : launch_one<false, false>(a, w, h, grid, s);
+                         cudaStream_t s, bool pair) {
+  return fp8 ? launch_one<false, true>(a, w, h, grid, s, pair) : launch_one<false, false>(a, w, h, grid, s, pair);
 }
 
 }  // namespace moe

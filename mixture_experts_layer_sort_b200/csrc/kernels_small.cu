@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       MmaState ms;
       run_mma<C, kFP8>(a.g, sh, rg, src, ms, tmem, abort_flag);
-      mma_drain(sh, ms);
+      mma_drain<C>(sh, ms);
     }
   } else {
     EpiState es;

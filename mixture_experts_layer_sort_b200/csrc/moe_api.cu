@@ -34,6 +34,7 @@ using moe::Tile;
 
 struct moe_layer {
   int E = 0, k = 0, H = 0, I = 0, dtype = 0, device = 0, num_sms = 0;
+  int pair_clusters = 0;        // CTA pairs of the grouped GEMMs resident at once
   bool loaded = false;
   // weights (library owned)
   void* w13 = nullptr;          // [E, 2I, H] gate rows then up rows of each expert (bf16 or e4m3)
@@ -95,6 +96,7 @@ struct moe_layer {
   bool fused_decode = false;    // single-launch decode path for small batches
   int gemv_max_m = 0;           // batches of up to this many tokens take the thin-batch path
   bool last_small = false;      // the last forward took the small-batch path (no gathered x)
+  bool last_pair = false;       // the last forward's grouped GEMMs ran on CTA pairs
   // per-kernel event timing
   bool profiling = false;
   struct Timed {
@@ -377,6 +379,18 @@ int drain_profile(moe_layer* L) {
   }
   L->pending.clear();
   return MOE_OK;
+}
+
+// Whether the chain's grouped GEMMs run on CTA pairs (M = 256 MMAs, each CTA loading half
+// of a token tile): for wide token tiles (at least 96 tokens per expert on average), where
+// the bytes each SM pulls per weight byte bound the GEMMs. MOE_PAIR_GEMM=0 never, =1
+// whenever the shapes allow (read at every forward).
+bool pair_gemm(const moe_layer* L, long long P, bool direct) {
+  if (direct || L->H % 512 != 0 || L->I % 256 != 0 || L->pair_clusters < 1) return false;
+  const char* e = std::getenv("MOE_PAIR_GEMM");
+  if (e && e[0] == '0') return false;
+  if (e && e[0] == '1') return true;
+  return P >= 96ll * L->E;
 }
 
 bool direct_x_disabled() {
@@ -718,6 +732,7 @@ int forward_gemv(moe_layer* L, const void* x, const float* logits, int M, void* 
 int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* out, cudaStream_t st) {
   MOE_TRY(ensure_workspace(L, M));
   L->last_small = false;
+  L->last_pair = false;
   if (is_mixed(L)) return forward_mixed(L, x, logits, M, out, st);
   // the opt-in decode paths first, then the thin-batch path, else the chain
   if (L->fused_decode && M <= L->num_sms && moe::decode_supported(M, L->E, L->k))
@@ -748,18 +763,27 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   }
   ++launches;
 
+  // The smallest bf16 batches (P <= 16) skip the gather: gate_up reads each token's x row
+  // itself with 1-row TMA boxes. Measured: faster at M=1, slower from M=4 on (16-row
+  // boxes of gathered rows stream better than 128-byte row reads).
+  const bool direct = !fp8 && P <= 16 && !direct_x_disabled();
+  // CTA pairs: a tile covers two CTAs' weight row blocks (gate_up 2 x 128 features, down
+  // 4 x 128), and the pairs are the workers the split-K rule counts
+  const bool pair = pair_gemm(L, P, direct);
+
   moe::AlignArgs aa{};
   aa.topk_ids = L->topk_ids;
   aa.P = static_cast<int>(P);
   aa.E = L->E;
   aa.k = L->k;
   aa.BN = BN;
-  aa.fblocks1 = L->I / moe::kTileRows;
-  aa.fblocks2 = (L->H / moe::kTileRows + 1) / 2;
+  aa.fblocks1 = L->I / (pair ? 2 * moe::kTileRows : moe::kTileRows);
+  aa.fblocks2 = pair ? L->H / (4 * moe::kTileRows) : (L->H / moe::kTileRows + 1) / 2;
   const int kper = fp8 ? 128 : 64;
   aa.kblocks1 = L->H / kper;
   aa.kblocks2 = L->I / kper;
-  aa.num_sms = L->num_sms;
+  aa.num_sms = pair ? L->pair_clusters : L->num_sms;
+  const int gemm_grid = pair ? 2 * L->pair_clusters : L->num_sms;
   aa.ws1_rows_cap = static_cast<int>(L->ws1_rows_cap);
   aa.acc_slabs = acc_slabs(M, L->H, aa.fblocks2);
   aa.uniform_splits = moe::uniform_splits() ? 1 : 0;
@@ -804,10 +828,6 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
     ++launches;
   }
 
-  // The smallest bf16 batches (P <= 16) skip the gather: gate_up reads each token's x row
-  // itself with 1-row TMA boxes. Measured: faster at M=1, slower from M=4 on (16-row
-  // boxes of gathered rows stream better than 128-byte row reads).
-  const bool direct = !fp8 && P <= 16 && !direct_x_disabled();
   CUtensorMap tm_xd{};
   if (direct) MOE_TRY(encode_map(&tm_xd, x, false, L->H, M, 1));
 
@@ -854,15 +874,17 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g1.hdr_splits = moe::kHdrSplits1;
   g1.kblocks = aa.kblocks1;
   g1.w_rblocks = 2 * L->I / moe::kTileRows;
-  g1.rb_step = 1;
+  g1.rb_step = pair ? 2 : 1;
+  g1.pair_rb = pair ? 1 : 0;
   g1.second_rb = L->I / moe::kTileRows;
   g1.max_stages = moe::gemm_max_stages(true);
   g1.wait_first = direct ? 1 : 0;
   g1.direct_pairs = direct ? L->pairs : nullptr;
   {
     KernelTimer kt(L, 3, st);
-    MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, direct ? tm_xd : L->tm_x, fp8, L->num_sms, st));
+    MOE_CUDA(moe::launch_gemm1(g1, L->tm_w13, direct ? tm_xd : L->tm_x, fp8, gemm_grid, st, pair));
   }
+  L->last_pair = pair;
   ++launches;
 
   if (fp8) {
@@ -889,12 +911,13 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g2.hdr_splits = moe::kHdrSplits2;
   g2.kblocks = aa.kblocks2;
   g2.w_rblocks = L->H / moe::kTileRows;
-  g2.rb_step = 2;
+  g2.rb_step = pair ? 4 : 2;
+  g2.pair_rb = pair ? 2 : 0;
   g2.second_rb = 1;
   g2.max_stages = moe::gemm_max_stages(false);
   {
     KernelTimer kt(L, 5, st);
-    MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, L->num_sms, st));
+    MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, gemm_grid, st, pair));
   }
   ++launches;
 
@@ -1218,6 +1241,7 @@ int moe_create(int E, int topk, int H, int I, int dtype, moe_layer** out) {
   L->dtype = dtype;
   L->device = dev;
   L->num_sms = prop.multiProcessorCount;
+  L->pair_clusters = std::min(moe::gemm_pair_clusters(), L->num_sms / 2);
   L->fused_decode = fused_decode_default();
   L->gemv_max_m = gemv_max_default(dtype, H);
   const size_t el = (dtype == MOE_DTYPE_BF16 || dtype == MOE_DTYPE_MIXED_E4M3) ? 2 : 1;
@@ -1501,6 +1525,8 @@ int moe_get_device_error(moe_layer* L, int* code) {
 }
 
 int moe_last_launch_count(moe_layer* L) { return L ? L->last_launches : 0; }
+
+int moe_last_gemm_pairs(moe_layer* L) { return (L && L->last_pair) ? 1 : 0; }
 
 int moe_set_fused_decode(moe_layer* L, int enable) {
   if (!L) return MOE_ERR_INVALID_ARG;

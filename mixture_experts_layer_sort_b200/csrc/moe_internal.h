@@ -133,6 +133,8 @@ struct GemmArgs {
   int hdr_tile_offset;     // header slot holding the index of this GEMM's first tile (0: none)
   int rb_step;             // tile row block f covers weight row blocks f*rb_step and
   int second_rb;           //   f*rb_step + second_rb (gate_up: 1 and I/128; down: 2 and 1)
+  int pair_rb;             // CTA-pair kernels: the second CTA's row blocks are pair_rb further
+                           //   (gate_up: rb_step 2, pair_rb 1; down: rb_step 4, pair_rb 2)
   // gate_up epilogue
   __nv_bfloat16* h;        // [rows_cap, I]
   int I;
@@ -219,14 +221,19 @@ constexpr int kAlignChunk = 1024;   // pairs per block of the multi-block align 
 cudaError_t launch_align_count(const AlignArgs& a, cudaStream_t s);
 cudaError_t launch_align_scatter(const AlignArgs& a, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s);
+// pair: clusters of two CTAs running M = 256 MMAs (grid even; a.rb_step / a.pair_rb and the
+// align kernel's tile lists set up for pairs)
 cudaError_t launch_gemm1(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& x, bool fp8, int grid,
-                         cudaStream_t s);
+                         cudaStream_t s, bool pair = false);
 cudaError_t launch_gemm2(const GemmArgs& a, const CUtensorMap& w, const CUtensorMap& h, bool fp8, int grid,
-                         cudaStream_t s);
+                         cudaStream_t s, bool pair = false);
 cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s);
 cudaError_t launch_quant_x(const QuantXArgs& a, cudaStream_t s);
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
 cudaError_t gemm_configure();    // opt-in dynamic shared memory sizes (current device)
+// CTA pairs of the grouped GEMMs that can be resident at once on the current device (0:
+// none): the pair kernels' grid is twice this, so that every pair runs in one wave.
+int gemm_pair_clusters();
 cudaError_t align_configure();
 
 // Single-launch decode path (kernels_decode.cu): the whole layer for M <= 64 tokens

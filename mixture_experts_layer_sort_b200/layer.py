@@ -140,12 +140,17 @@ class MoELayer:
         self._check("moe_set_fused_decode", self.lib.moe_set_fused_decode(self.handle, 1 if enable else 0))
 
     def set_gemv_max_tokens(self, max_tokens: int):
-        """Largest batch run on the thin-batch (CUDA-core) path; 0 = never, -1 = default."""
+        """Largest batch run on the thin-batch path (warp-level tensor-core products); 0 = never, -1 = default."""
         self._check("moe_set_gemv_max_tokens", self.lib.moe_set_gemv_max_tokens(self.handle, int(max_tokens)))
 
     @property
     def last_launch_count(self) -> int:
         return self.lib.moe_last_launch_count(self.handle)
+
+    @property
+    def last_gemm_pairs(self) -> bool:
+        """Whether the last forward's grouped GEMMs ran on CTA pairs."""
+        return self.lib.moe_last_gemm_pairs(self.handle) == 1
 
     KERNEL_SLOTS = ("route", "align", "gather", "gate_up", "quant_h", "down", "finalize")
 

@@ -73,6 +73,7 @@ def test_null_handles_are_rejected(lib):
     assert lib.moe_reserve(None, 4, None) == -1
     assert lib.moe_get_device_error(None, None) == -1
     assert lib.moe_last_launch_count(None) == 0
+    assert lib.moe_last_gemm_pairs(None) == 0
 
 
 def test_every_entry_point_rejects_a_null_handle(lib):
