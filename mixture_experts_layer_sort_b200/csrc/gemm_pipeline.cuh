@@ -48,14 +48,18 @@ constexpr int kThreads = 64 + kEpiThreads;
 constexpr int kTokenTile = 256;   // widest token tile: the largest N of an M=128 MMA
 static_assert(kTokenTile == kTokenBlock, "the align kernel's token blocks are the GEMM token tiles");
 
-// kSmem: dynamic shared memory of the kernel (default: the sm_100 opt-in maximum, one
-// CTA per SM); kTmem: TMEM columns it allocates (two accumulator buffers of kTmem / 2
-// columns). Two kernels whose sizes add up to at most one SM's shared memory and TMEM
-// can have CTAs resident on the same SM at once.
+// kSmem: dynamic shared memory of the kernel (default 224 KB, one CTA per SM: 3 KB under
+// the sm_100 opt-in maximum, so that a CTA of a one-row kernel launched next to it, a
+// gather or h quantisation with its own 1 KB reserve, can share the SM and the GEMM's
+// first weight loads overlap it under programmatic dependent launch); kTmem: TMEM
+// columns it allocates (two accumulator buffers of kTmem / 2 columns). Two kernels whose
+// sizes add up to at most one SM's shared memory and TMEM can have CTAs resident on the
+// same SM at once.
 // kPair: the tiles of a unit are split over a CTA pair (a cluster of two) that runs
 // M = 256 MMAs: each CTA holds its own two weight tiles and half of the activation rows,
 // the pair's first CTA issues the MMAs, and each CTA's TMEM receives its own rows.
-template <bool kFP8, int kSmem = 232448, int kTmem = 512, bool kPair_ = false>
+constexpr int kGemmSmem = 229376;
+template <bool kFP8, int kSmem = kGemmSmem, int kTmem = 512, bool kPair_ = false>
 struct Cfg {
   static constexpr bool kPair = kPair_;
   static constexpr int kATiles = 2;

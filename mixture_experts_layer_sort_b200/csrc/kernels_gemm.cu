@@ -50,7 +50,7 @@ template <bool kGateUp, bool kFP8, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs a, const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_b) {
-  using C = Cfg<kFP8, 232448, 512, kPair>;
+  using C = Cfg<kFP8, kGemmSmem, 512, kPair>;
   extern __shared__ uint8_t smem_raw[];
   const Shared sh = carve<C>(smem_raw, 0);
   volatile int* abort_flag = sh.flags;

@@ -117,8 +117,9 @@ __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, void* __
 // stride over the rows (the grid is capped at a few blocks per SM), so that a
 // thread's stores of one row overlap its loads of the next. With `xq` set (large FP8
 // batches) the token rows are already quantised and the rows are byte copies.
+// (at most 85 registers: a CTA fits next to a grouped-GEMM CTA on one SM)
 template <bool kFP8>
-__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
+__global__ void __launch_bounds__(256, 3) gather_kernel(GatherArgs a) {
   const int t = threadIdx.x % kRowThreads;
   pdl_wait();
   pdl_trigger();
@@ -240,6 +241,22 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
 
 }  // namespace
 
+// The one-row kernels ask for the largest shared-memory carveout, as the grouped GEMMs
+// need it: an SM then never has to change its L1 / shared split between the two, and a
+// GEMM CTA can start next to one of theirs.
+cudaError_t route_configure() {
+  const int c = cudaSharedmemCarveoutMaxShared;
+  const cudaFuncAttribute at = cudaFuncAttributePreferredSharedMemoryCarveout;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(route_kernel<1>, at, c)) || (e = cudaFuncSetAttribute(route_kernel<2>, at, c)) ||
+      (e = cudaFuncSetAttribute(route_kernel<4>, at, c)) || (e = cudaFuncSetAttribute(route_kernel<8>, at, c)) ||
+      (e = cudaFuncSetAttribute(route_kernel<16>, at, c)) || (e = cudaFuncSetAttribute(gather_kernel<false>, at, c)) ||
+      (e = cudaFuncSetAttribute(gather_kernel<true>, at, c)) || (e = cudaFuncSetAttribute(quant_x_kernel, at, c)) ||
+      (e = cudaFuncSetAttribute(quant_h_kernel, at, c)))
+    return e;
+  return cudaFuncSetAttribute(finalize_kernel, at, c);
+}
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   const int grid = (a.M + kRouteWarps - 1) / kRouteWarps;
   const dim3 g(grid), b(kRouteWarps * 32);
@@ -253,7 +270,10 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
 // Row kernels: one block per two rows, or (capped) at most 8 blocks per SM striding
 // over the rows. Measured at prefill size on one box: the bf16 gather (14 KB
 // row copies) is faster uncapped (127 vs 141 us), the FP8 row kernels (quantising,
-// or copying 1-byte rows) capped (x: 116 vs 150 us, h: 68 vs 81 us).
+// or copying 1-byte rows) capped (x: 116 vs 150 us, h: 68 vs 81 us). At decode sizes
+// (at most 8192 padded rows) the gather and the h quantisation run one block per SM, so
+// that the grouped GEMM launched after them finds room for its CTAs at once (decode bf16
+// M = 16 / 64 and e4m3 M = 32 / 64 1.4-2.5 us faster).
 int row_grid(int rows, bool capped) {
   const int g = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
   const int cap = 8 * sm_count();
@@ -263,7 +283,8 @@ int row_grid(int rows, bool capped) {
 cudaError_t launch_gather(const GatherArgs& a, bool fp8, cudaStream_t s) {
   if (a.eflags != nullptr)
     return launch_kernel(gather_mixed_kernel, dim3(row_grid(a.rows_bound, true)), dim3(256), 0, s, a);
-  const int grid = row_grid(a.rows_bound, fp8);
+  int grid = row_grid(a.rows_bound, fp8);
+  if (a.rows_bound <= 8192 && grid > sm_count()) grid = sm_count();
   if (fp8) return launch_kernel(gather_kernel<true>, dim3(grid), dim3(256), 0, s, a);
   return launch_kernel(gather_kernel<false>, dim3(grid), dim3(256), 0, s, a);
 }
@@ -273,7 +294,8 @@ cudaError_t launch_quant_x(const QuantXArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_quant_h(const QuantHArgs& a, cudaStream_t s) {
-  const int grid = row_grid(a.rows_bound, true);
+  int grid = row_grid(a.rows_bound, true);
+  if (a.rows_bound <= 8192 && grid > sm_count()) grid = sm_count();
   return launch_kernel(quant_h_kernel, dim3(grid), dim3(256), 0, s, a);
 }
 

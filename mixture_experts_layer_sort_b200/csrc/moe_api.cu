@@ -170,6 +170,7 @@ int configure_device(int dev) {
   if (dev < 64 && (g_configured >> dev) & 1ull) return MOE_OK;
   MOE_CUDA(moe::gemm_configure());
   MOE_CUDA(moe::align_configure());
+  MOE_CUDA(moe::route_configure());
   MOE_CUDA(moe::decode_configure());
   MOE_CUDA(moe::small_configure());
   MOE_CUDA(moe::gemv_configure());

@@ -235,6 +235,7 @@ cudaError_t gemm_configure();    // opt-in dynamic shared memory sizes (current 
 // none): the pair kernels' grid is twice this, so that every pair runs in one wave.
 int gemm_pair_clusters();
 cudaError_t align_configure();
+cudaError_t route_configure();   // shared-memory carveout of the one-row kernels
 
 // Single-launch decode path (kernels_decode.cu): the whole layer for M <= 64 tokens
 // (bf16 or FP8) in one cooperative persistent kernel.
