@@ -18,11 +18,15 @@ namespace {
 using namespace pipe;
 
 // The activation operand depends on the previous kernel of the stream: one PDL wait.
+// Down with the combine folded in: token rows are finished by whoever adds their last
+// K block (done / ndone: a shared-memory list of the rows a unit completed).
 struct PdlHooks {
   bool waited;
   const GemmArgs* a;
+  int* done;
+  int* ndone;
   static constexpr bool kSignalTiles = false;
-  static constexpr bool kTokenCompletion = false;
+  static constexpr bool kTokenCompletion = true;
   __device__ __forceinline__ int dep(const Unit&) const { return 0; }
   __device__ __forceinline__ bool ready(int) const { return waited; }
   __device__ __forceinline__ bool wait(int) {
@@ -43,7 +47,42 @@ struct PdlHooks {
     return __ldcg(a->direct_pairs + un.t.row_start + j) / a->k;
   }
   __device__ __forceinline__ void tile_done(const Unit&, int, float) {}
-  __device__ __forceinline__ void down_done(const Unit&, const int*, int) {}
+  __device__ __forceinline__ void down_done(const Unit& un, const int* s_tok, int epi_tid) {
+    if (a->token_cnt == nullptr) return;
+    __threadfence();                        // this unit's adds happen before the counts move
+    named_bar_sync(1, kEpiThreads);
+    if (epi_tid == 0) *ndone = 0;
+    named_bar_sync(1, kEpiThreads);
+    const int add = un.kb1 - un.kb0;
+    const int need = a->token_need;
+    for (int j = epi_tid; j < un.t.n_valid; j += kEpiThreads) {
+      const int t = s_tok[j];
+      if (atomicAdd(a->token_cnt + t, add) == need - add) done[atomicAdd(ndone, 1)] = t;
+    }
+    named_bar_sync(1, kEpiThreads);
+    const int nd = *ndone;
+    if (nd > 0) {
+      __threadfence();
+      const int H = a->H;
+      for (int i = 0; i < nd; ++i) {
+        const int t = done[i];
+        float4* acc4 = reinterpret_cast<float4*>(a->acc + static_cast<size_t>(t) * H);
+        uint2* out4 = reinterpret_cast<uint2*>(a->out + static_cast<size_t>(t) * H);
+        for (int c = epi_tid; c < H / 4; c += kEpiThreads) {
+          const float4 v = __ldcg(acc4 + c);
+          __stcg(acc4 + c, make_float4(0.f, 0.f, 0.f, 0.f));
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+          uint2 o;
+          o.x = *reinterpret_cast<const unsigned*>(&lo);
+          o.y = *reinterpret_cast<const unsigned*>(&hi);
+          out4[c] = o;
+        }
+        if (epi_tid == 0) a->token_cnt[t] = 0;
+      }
+    }
+    named_bar_sync(1, kEpiThreads);         // the list is reused by the next unit
+  }
 };
 
 template <bool kGateUp, bool kFP8, bool kPair>
@@ -52,7 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_b) {
   using C = Cfg<kFP8, kGemmSmem, 512, kPair>;
   extern __shared__ uint8_t smem_raw[];
-  const Shared sh = carve<C>(smem_raw, 0);
+  // down: 1 KB + 4 bytes for the list of token rows a unit completes
+  const Shared sh = carve<C>(smem_raw, kGateUp ? 0 : 2048);
   volatile int* abort_flag = sh.flags;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -77,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();
     pdl_trigger();
   }
-  PdlHooks hk{a.wait_first != 0, &a};
+  PdlHooks hk{a.wait_first != 0, &a, reinterpret_cast<int*>(sh.extra), reinterpret_cast<int*>(sh.extra) + 256};
 
   if (warp == 0) {
     ProducerState ps;
@@ -97,6 +137,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     EpiState es;
     run_epilogue<C, kGateUp, kFP8>(a, sh, rg, src, hk, es, tmem, abort_flag, warp, lane);
     if constexpr (kGateUp && kFP8) publish_amax(a.amax_h, es.lmax, lane);
+  }
+  if constexpr (!kGateUp) {
+    if (a.token_cnt != nullptr) {
+      // the last CTA: FP8 scales of the forward, amax words cleared for the next one
+      __syncthreads();
+      if (threadIdx.x == 64) {
+        __threadfence();
+        if (atomicAdd(a.cta_done, 1) == static_cast<int>(gridDim.x) - 1) {
+          __threadfence();
+          if constexpr (kFP8) {
+            a.last_scales[0] = fp8_scale_from_amax(__ldcg(a.amax), a.f8);
+            a.last_scales[1] = fp8_scale_from_amax(__ldcg(a.amax + 1), a.f8);
+            a.amax[0] = 0u;
+            a.amax[1] = 0u;
+          }
+          *a.cta_done = 0;
+        }
+      }
+    }
   }
   teardown<C>(tmem, warp);
 }

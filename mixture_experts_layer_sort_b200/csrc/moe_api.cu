@@ -394,6 +394,17 @@ bool pair_gemm(const moe_layer* L, long long P, bool direct) {
   return P >= 96ll * L->E;
 }
 
+// Whether the chain's down GEMM finishes each token row itself (the epilogue that adds
+// its last K block writes `out`) instead of a finalize launch: MOE_FOLD_FINALIZE=1 (read
+// at every forward). Off by default: measured on one B200, the per-unit fence and counts
+// cost more than the launch they save (decode bf16 M=64 214.7 -> 224.9 us, e4m3 M=32
+// 122.6 -> 135.0, prefill bf16 3998 -> 6263: with one TMEM buffer the MMAs wait for the
+// longer epilogue).
+bool fold_finalize() {
+  const char* e = std::getenv("MOE_FOLD_FINALIZE");
+  return e && e[0] == '1';
+}
+
 bool direct_x_disabled() {
   static const bool off = [] {
     const char* e = std::getenv("MOE_DISABLE_DIRECT_X");
@@ -916,24 +927,38 @@ int forward_impl(moe_layer* L, const void* x, const float* logits, int M, void* 
   g2.pair_rb = pair ? 2 : 0;
   g2.second_rb = 1;
   g2.max_stages = moe::gemm_max_stages(false);
+  // the combine: token rows finished inside the down GEMM (counts of the K blocks each
+  // token receives: k experts x tiles across H x K blocks, once per CTA of a pair), or a
+  // finalize launch
+  const bool fold = fold_finalize();
+  if (fold) {
+    g2.token_cnt = L->small_sync;
+    g2.cta_done = L->small_sync + L->M_cap;
+    g2.token_need = L->k * aa.fblocks2 * aa.kblocks2 * (pair ? 2 : 1);
+    g2.out = static_cast<__nv_bfloat16*>(out);
+    g2.amax = fp8 ? L->amax : nullptr;
+    g2.last_scales = fp8 ? L->last_scales : nullptr;
+  }
   {
     KernelTimer kt(L, 5, st);
     MOE_CUDA(moe::launch_gemm2(g2, L->tm_wd, L->tm_h, fp8, gemm_grid, st, pair));
   }
   ++launches;
 
-  moe::FinalizeArgs fa{};
-  fa.acc = L->acc;
-  fa.out = static_cast<__nv_bfloat16*>(out);
-  fa.n = static_cast<long long>(M) * L->H;
-  fa.amax = fp8 ? L->amax : nullptr;
-  fa.last_scales = fp8 ? L->last_scales : nullptr;
-  fa.f8 = fp8_format(L);
-  {
-    KernelTimer kt(L, 6, st);
-    MOE_CUDA(moe::launch_finalize(fa, st));
+  if (!fold) {
+    moe::FinalizeArgs fa{};
+    fa.acc = L->acc;
+    fa.out = static_cast<__nv_bfloat16*>(out);
+    fa.n = static_cast<long long>(M) * L->H;
+    fa.amax = fp8 ? L->amax : nullptr;
+    fa.last_scales = fp8 ? L->last_scales : nullptr;
+    fa.f8 = fp8_format(L);
+    {
+      KernelTimer kt(L, 6, st);
+      MOE_CUDA(moe::launch_finalize(fa, st));
+    }
+    ++launches;
   }
-  ++launches;
 
   L->last_M = M;
   L->last_launches = launches;

@@ -149,6 +149,15 @@ struct GemmArgs {
   const int* padded_pairs;
   const float* topk_w;
   int k, P;
+  // down with the combine folded in (token_cnt set): the epilogue that adds a token's last
+  // K block turns its row of `acc` into `out` (and clears it); the last CTA to finish
+  // writes the FP8 scales of the forward and clears the amax words. No finalize launch.
+  int* token_cnt;          // [M] K blocks added per token (zero between forwards)
+  int token_need;          // K blocks a token receives in all (k x tiles across H x K blocks)
+  int* cta_done;           // CTAs finished (zero between forwards)
+  __nv_bfloat16* out;      // [M, H]
+  unsigned* amax;          // FP8: [2] the forward's amax words (cleared at the end)
+  float* last_scales;      // FP8: [2] s_x, s_h of the forward
   int max_stages;          // upper bound of the stage ring depth (<= the kernel's own maximum)
   int wait_first;          // 1: the previous kernel wrote the tile list (wait before reading it)
   const int* direct_pairs; // gate_up only: B rows are x rows of token pairs[row]/k (x map box = 1 row)
