@@ -4,8 +4,9 @@
 //
 // Orientation: every tile is "swap-AB". The expert's weight rows fill the MMA's
 // M = 128 slot and the expert's few tokens are the N dimension (16..256), i.e. the
-// kernel computes D^T = W * X^T instead of X * W^T. (A B)^T = B^T A^T changes no
-// arithmetic (kongchang.com, "MoE Kernel Engineering Optimization Practices on
+// kernel computes D^T = W * X^T instead of X * W^T (M = 256 over a CTA pair, kPair
+// below, each CTA holding 128 of the rows and half of the tokens). (A B)^T = B^T A^T
+// changes no arithmetic (kongchang.com, "MoE Kernel Engineering Optimization Practices on
 // Amazon SageMaker AI", section "Swap-AB: Making WGMMA Run at Full Utilization");
 // it keeps the tensor-core rows busy when decode gives an expert a handful of
 // tokens (toolboxkart.tech, "AWS SageMaker MoE kernel optimizations H200", section

@@ -9,6 +9,14 @@
 // every CTA streams the same weight bytes. With programmatic dependent launch, the
 // weight loads of the first stages go out before the kernel waits for its
 // predecessor; only the activation loads wait.
+//
+// For wide token tiles (prefill) the same kernels run on CTA pairs: clusters of two
+// CTAs, the pair being the worker of the schedule. A pair's tile covers twice the weight
+// rows (gate_up: 2 x 128 features; down: 4 x 128 output rows); each CTA loads its own
+// two weight tiles and half of the token tile, and the first CTA issues M = 256 MMAs
+// (tcgen05 cta_group::2) that read both CTAs' shared memory and write each CTA's rows into
+// its own TMEM. Per weight byte an SM then pulls half the activation bytes, which is what
+// bounds these GEMMs once tiles are 128-256 tokens wide.
 #include "gemm_pipeline.cuh"
 
 namespace moe {
