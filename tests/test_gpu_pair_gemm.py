@@ -103,3 +103,18 @@ def test_auto_choice_prefill_shape(dtype, monkeypatch):
         check(c, 64, 991, False)
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_balanced_schedule_on_pairs(dtype, monkeypatch):
+    # 64 experts x ~96 tokens: 256 gate_up and 128 down pair tiles, between one and eight
+    # waves of the 74 pairs, so both GEMMs take the balanced schedule (tiles cut between
+    # pairs at K-block boundaries, split-K fix-ups counted per CTA of a pair)
+    monkeypatch.delenv("MOE_PAIR_GEMM", raising=False)
+    c = Case(64, 8, 1024, 1024, dtype, w_std=0.02)
+    c.cache = {}
+    c.layer.set_gemv_max_tokens(0)
+    try:
+        check(c, 768, 995, True)
+    finally:
+        c.close()
