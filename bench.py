@@ -3,10 +3,15 @@
 
 Headline workload (N=1): the decode layer E=128 experts, top-8, H=2048, I=768,
 bf16 weights (1.2 GB), at the four decode batch sizes M = 1, 4, 16, 64. One
-step = one forward at each of the four M (85 tokens); the L2 cache (126 MB) is
-flushed before every forward by writing a 252 MB buffer, outside the timed
-events. Each forward is replayed from a CUDA graph captured once per M (the
-forward is a fixed launch chain with no host synchronisation).
+step = one forward at each of the four M (85 tokens). No forward finds its
+weights in the L2 cache (126 MB): consecutive forwards use different weight
+sets (identically shaped layers with their own seeded weights, as the MoE layers
+of successive transformer blocks), enough of them that at least 252 MB of other
+weights stream through L2 between two forwards on one set (`--l2 flush` instead
+writes a 252 MB buffer before every forward, outside the timed events; the
+dirty lines it leaves are written back during the timed forward). Each forward
+is replayed from a CUDA graph captured once per (M, weight set) (the forward is
+a fixed launch chain with no host synchronisation).
 
 The same line carries, under "workloads", the other shapes the metric names,
 each measured the same way: decode FP8 e4m3 (M = 1, 8, 32, 64, from the same
@@ -53,6 +58,8 @@ NOMINAL_HBM_GBS = 8000.0          # the "~8 TB/s" the layer's target is stated a
 NOMINAL_BF16_TFLOPS = 2250.0      # B200 datasheet dense bf16 (FP8: twice)
 DECODE_TARGET = 0.70              # decode shapes: fraction of the HBM roofline
 L2_FLUSH_BYTES = 252 << 20
+L2_BYTES = 126 << 20
+MAX_WEIGHT_SETS = 16
 
 
 def parse_args():
@@ -74,9 +81,15 @@ def parse_args():
     ap.add_argument("--only-M", type=int, default=None,
                     help="run a single batch size of the workload (inv_rope: a single token count)")
     ap.add_argument("--fused-decode", action="store_true", help="single-launch decode path (bf16, M <= 64)")
+    ap.add_argument("--l2", default="rotate", choices=["rotate", "flush", "warm"],
+                    help="rotate: consecutive forwards on different weight sets (inputs larger than L2); "
+                         "flush: a 252 MB write before every forward; warm: one set, no flush")
     ap.add_argument("--warm-l2", action="store_true",
-                    help="do not flush L2 between forwards (a labelled warm-cache figure, not the headline)")
-    return ap.parse_args()
+                    help="same as --l2 warm (a labelled warm-cache figure, not the headline)")
+    a = ap.parse_args()
+    if a.warm_l2:
+        a.l2 = "warm"
+    return a
 
 
 def workload_spec(name):
@@ -127,13 +140,36 @@ def alg_flops_layer(wl, M):
     return 6 * M * wl.k * wl.H * wl.I
 
 
-def bench_config(wl, Ms, ws, warm_l2):
+def l2_plan(wl, dtype, mode):
+    """How the forwards of a workload are kept from finding their weights in L2:
+    ("rotate", R, text): consecutive forwards use R different weight sets, R chosen so
+    that at least 2 x L2 of other weights stream through between two forwards on one set
+    (a forward streams at least the weights of k experts); ("flush", 1, text) when that
+    needs more than MAX_WEIGHT_SETS sets or is not asked for; ("warm", 1, text)."""
+    if mode == "warm":
+        return "warm", 1, "warm: one weight set, not flushed between forwards"
+    per_expert = 3 * wl.H * wl.I * weight_bytes(dtype)
+    fewest = min(wl.k, wl.E) * per_expert
+    R = -(-2 * L2_BYTES // fewest) + 1
+    if mode == "rotate" and R <= MAX_WEIGHT_SETS:
+        return "rotate", R, (f"inputs larger than L2: consecutive forwards on different weight sets ({R} sets, "
+                             f"{R * wl.E * per_expert / 1e9:.1f} GB in all; at least {(R - 1) * fewest / 2**20:.0f} "
+                             f"MB of other weights stream through the 126 MB L2 between two forwards on one set), "
+                             f"no flush")
+    return "flush", 1, "flushed (252 MB write) before every forward, outside the timed events"
+
+
+def set_seed(seed, r):
+    """Weight seed of set r (set 0 is the workload's own seed)."""
+    return seed if r == 0 else seed + 7919 * r
+
+
+def bench_config(wl, Ms, ws, l2_text):
     """The workload description both arms print (the reference arm prints the same dict)."""
     return {"workload": wl.description + f", one step = one forward at each M in {list(Ms)}",
             "E": wl.E, "topk": wl.k, "H": wl.H, "I": wl.I, "Ms": list(Ms), "global_batch": sum(Ms) * ws,
             "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-            "l2": ("warm: not flushed between forwards" if warm_l2 else
-                   "flushed (252 MB write) before every forward, outside the timed events")}
+            "l2": l2_text}
 
 
 def cpu_model():
@@ -329,7 +365,7 @@ def reference_arm(args, ws, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": bench_config(wl, Ms, args.gpus, getattr(args, "warm_l2", False)),
+        "config": bench_config(wl, Ms, args.gpus, l2_plan(wl, dtype, getattr(args, "l2", "rotate"))[2]),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
                          "sample": f"full sweep M={Ms} ({tokens} tokens) per step"},
@@ -368,53 +404,69 @@ def kernel_source_hash():
 
 
 class Runner:
-    """Times one layer on one workload: graph replay per M with an L2 flush before every
-    forward (outside the events), then an eager pass, then a pass with the library's
-    per-kernel CUDA events (on the forward's stream)."""
+    """Times one workload on one or more identically shaped layers (weight sets): graph
+    replay per (M, set), consecutive forwards on consecutive sets (or, with a flush buffer,
+    a 252 MB write before every forward, outside the events), then an eager pass, then a
+    pass with the library's per-kernel CUDA events (on the forward's stream)."""
 
-    def __init__(self, layer, wl, dtype, Ms, toks, stream, flush, use_graph):
+    def __init__(self, layers, wl, dtype, Ms, toks, stream, flush, use_graph):
         import torch
         self.torch = torch
-        self.layer, self.wl, self.dtype, self.Ms, self.toks = layer, wl, dtype, list(Ms), toks
+        self.layers, self.wl, self.dtype, self.Ms, self.toks = list(layers), wl, dtype, list(Ms), toks
         self.stream, self.flush = stream, flush
+        self.fi = 0   # forwards issued so far: forward i runs on set i % R
         dev = toks[self.Ms[0]][0].device
         self.outs = {M: torch.empty((M, wl.H), dtype=torch.bfloat16, device=dev) for M in self.Ms}
-        layer.reserve(max(self.Ms))
+        for lay in self.layers:
+            lay.reserve(max(self.Ms))
         self.A, self.launches = {}, {}
+        layer = self.layers[0]
         with torch.cuda.stream(stream):
             for M in self.Ms:
+                # the routing depends on the logits only: every set activates the same experts
                 layer.forward(*toks[M], out=self.outs[M])
                 self.A[M] = int(torch.count_nonzero(layer.debug_routing(M)["counts"]).item())
                 layer.forward(*toks[M], out=self.outs[M])
                 self.launches[M] = layer.last_launch_count
+                for lay in self.layers[1:]:
+                    lay.forward(*toks[M], out=self.outs[M])
         torch.cuda.synchronize()
         self.graphs = {}
         if use_graph:
             for M in self.Ms:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    layer.forward(*toks[M], out=self.outs[M])
-                self.graphs[M] = g
+                for r, lay in enumerate(self.layers):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        lay.forward(*toks[M], out=self.outs[M])
+                    self.graphs[(M, r)] = g
             torch.cuda.synchronize()
 
-    def forward(self, M):
+    def _next(self):
+        """Set of the next forward; flushes L2 first in flush mode."""
+        r = self.fi % len(self.layers)
+        self.fi += 1
+        if self.flush is not None:
+            self.flush.zero_()
+        return r
+
+    def forward(self, M, r):
         if self.graphs:
-            self.graphs[M].replay()
+            self.graphs[(M, r)].replay()
         else:
-            self.layer.forward(*self.toks[M], out=self.outs[M])
+            self.layers[r].forward(*self.toks[M], out=self.outs[M])
 
     def step(self, events=None):
         for i, M in enumerate(self.Ms):
-            self.flush.zero_()
+            r = self._next()
             if events is not None:
                 events[i][0].record(self.stream)
-            self.forward(M)
+            self.forward(M, r)
             if events is not None:
                 events[i][1].record(self.stream)
 
     def warm(self, n):
         with self.torch.cuda.stream(self.stream):
-            for _ in range(n):
+            for _ in range(max(n, len(self.layers))):
                 self.step()
         self.torch.cuda.synchronize()
 
@@ -439,30 +491,35 @@ class Runner:
         with torch.cuda.stream(self.stream):
             for _ in range(reps):
                 for M in self.Ms:
-                    self.flush.zero_()
+                    r = self._next()
                     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     e0.record(self.stream)
-                    self.layer.forward(*self.toks[M], out=self.outs[M])
+                    self.layers[r].forward(*self.toks[M], out=self.outs[M])
                     e1.record(self.stream)
                     got[M].append((e0, e1))
         torch.cuda.synchronize()
         return {M: statistics.median(a.elapsed_time(b) for a, b in v) for M, v in got.items()}
 
     def kernel_profile(self, reps):
-        """{kernel: (ms, launches)} over `reps` eager steps, and the gate_up / down
-        algorithmic weight bytes those launches moved."""
+        """{kernel: (ms, launches)} over `reps` eager steps (summed over the sets), and the
+        gate_up / down algorithmic weight bytes those launches moved."""
         wl, bw = self.wl, weight_bytes(self.dtype)
-        self.layer.profile_enable(True)
+        for lay in self.layers:
+            lay.profile_enable(True)
         gate_bytes = down_bytes = 0.0
         with self.torch.cuda.stream(self.stream):
             for _ in range(reps):
                 for M in self.Ms:
-                    self.flush.zero_()
-                    self.layer.forward(*self.toks[M], out=self.outs[M])
+                    r = self._next()
+                    self.layers[r].forward(*self.toks[M], out=self.outs[M])
                     gate_bytes += self.A[M] * 2 * wl.H * wl.I * bw
                     down_bytes += self.A[M] * wl.H * wl.I * bw
-        prof = self.layer.profile_read()
-        self.layer.profile_enable(False)
+        prof = {}
+        for lay in self.layers:
+            for k, (ms, n) in lay.profile_read().items():
+                a, b = prof.get(k, (0.0, 0))
+                prof[k] = (a + ms, b + n)
+            lay.profile_enable(False)
         return prof, gate_bytes, down_bytes
 
     def close(self):
@@ -492,9 +549,37 @@ def per_M_summary(wl, dtype, Ms, per_M_ms, eager, A, launches, hbm_gbs, bf16_tf)
     return out
 
 
-def measure_workload(name, layer, wl, dtype, Ms, toks, stream, flush, args, hbm_gbs, bf16_tf):
-    """One workload entry of the bench line (an extra workload next to the headline)."""
-    r = Runner(layer, wl, dtype, Ms, toks, stream, flush, use_graph=not args.no_graph)
+def make_layer_sets(wl, dtypes, R, seed, dev, first=None, keep_first=False, fused_decode=False):
+    """R weight sets of a workload's shape: for each set r, one layer per dtype in `dtypes`,
+    all loaded from set r's bf16 weights (drawn with set_seed(seed, r); set 0's tensors may
+    be passed in as `first`). Returns {dtype: [layer of set 0, ...]} and, with keep_first,
+    set 0's bf16 tensors."""
+    import torch
+    from mixture_experts_layer_sort_b200 import MoELayer, synth
+    out = {d: [] for d in dtypes}
+    w0 = None
+    for r in range(R):
+        w = first if (r == 0 and first is not None) else \
+            synth.make_weights(wl.E, wl.H, wl.I, wl.w_std, seed=set_seed(seed, r), device=dev)
+        for d in dtypes:
+            lay = MoELayer(wl.E, wl.k, wl.H, wl.I, d)
+            lay.load_weights(*w)
+            if fused_decode:
+                lay.set_fused_decode(True)
+            out[d].append(lay)
+        if r == 0 and keep_first:
+            w0 = w
+        del w
+    torch.cuda.empty_cache()
+    return out, w0
+
+
+def measure_workload(name, layers, wl, dtype, Ms, toks, stream, args, hbm_gbs, bf16_tf, flush_buf):
+    """One workload entry of the bench line (an extra workload next to the headline), on
+    `layers` (one per weight set; in flush mode the first alone, with flush_buf)."""
+    mode, R, l2_text = l2_plan(wl, dtype, args.l2)
+    flush = flush_buf if mode == "flush" else None
+    r = Runner(layers[:R], wl, dtype, Ms, toks, stream, flush, use_graph=not args.no_graph)
     r.warm(max(3, args.warmup))
     steps = max(5, min(args.steps, 20))
     per_M_ms, _ = r.timed(steps)
@@ -513,6 +598,7 @@ def measure_workload(name, layer, wl, dtype, Ms, toks, stream, flush, args, hbm_
     dom = max(("gate_up", "down"), key=lambda k: prof[k][0])
     summary = per_M_summary(wl, dtype, Ms, per_M_ms, eager, r.A, r.launches, hbm_gbs, bf16_tf)
     entry = {"workload": wl.description + f", one step = one forward at each M in {list(Ms)}",
+             "l2": l2_text,
              "dtype": dtype_name(dtype), "Ms": list(Ms), "steps": steps, "ms_per_step": ms,
              "tokens_per_s": sum(Ms) / (ms / 1e3), "per_M": summary,
              "dominant_gemm": dict(kernel=dom, **gemm[dom]), "gemm_event_GBps": gemm,
@@ -594,18 +680,19 @@ def measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on, Ts=None):
 
 
 def extra_workloads(args, dev, stream, flush, dec_weights, seed, hbm_gbs, bf16_tf, cpu_on):
-    """Decode FP8 (from the decode weights), large decode and prefill bf16 + FP8 (from one
-    E=256 bf16 weight set), each measured like the headline."""
+    """Decode FP8 (from the decode weight sets), large decode and prefill bf16 + FP8 (from
+    the E=256 bf16 weight sets), each measured like the headline."""
     import torch
-    from mixture_experts_layer_sort_b200 import MoELayer, synth
+    from mixture_experts_layer_sort_b200 import synth
     res = {}
     wl = synth.WORKLOADS["decode_fp8"]
-    lay = MoELayer(wl.E, wl.k, wl.H, wl.I, "fp8")
-    lay.load_weights(*dec_weights)
+    R = l2_plan(wl, "fp8", args.l2)[1]
+    sets, _ = make_layer_sets(wl, ("fp8",), R, args.seed, dev, first=dec_weights)
     toks = {M: synth.make_tokens(wl.E, wl.H, M, seed=seed, device=dev) for M in wl.Ms}
-    res["decode_fp8"] = measure_workload("decode_fp8", lay, wl, "fp8", wl.Ms, toks, stream, flush, args,
-                                         hbm_gbs, bf16_tf)
-    lay.close()
+    res["decode_fp8"] = measure_workload("decode_fp8", sets["fp8"], wl, "fp8", wl.Ms, toks, stream, args,
+                                         hbm_gbs, bf16_tf, flush)
+    for lay in sets["fp8"]:
+        lay.close()
     if cpu_on:
         host_w = [synth.bf16_to_f32_numpy(w) for w in dec_weights]
         tnp = {M: (toks[M][0].float().cpu().numpy(), toks[M][1].cpu().numpy()) for M in wl.Ms}
@@ -614,24 +701,22 @@ def extra_workloads(args, dev, stream, flush, dec_weights, seed, hbm_gbs, bf16_t
     del toks
 
     wl4, wl5 = synth.WORKLOADS["large_decode"], synth.WORKLOADS["prefill"]
-    wg, wu, wd = synth.make_weights(wl4.E, wl4.H, wl4.I, wl4.w_std, seed=args.seed, device=dev)
-    big = MoELayer(wl4.E, wl4.k, wl4.H, wl4.I, "bf16")
-    big.load_weights(wg, wu, wd)
-    big8 = MoELayer(wl5.E, wl5.k, wl5.H, wl5.I, "fp8")
-    big8.load_weights(wg, wu, wd)
-    del wg, wu, wd
-    torch.cuda.empty_cache()
+    R = max(l2_plan(wl4, "bf16", args.l2)[1], l2_plan(wl5, "bf16", args.l2)[1], l2_plan(wl5, "fp8", args.l2)[1])
+    sets, _ = make_layer_sets(wl4, ("bf16", "fp8"), R, args.seed, dev)
     toks = {M: synth.make_tokens(wl4.E, wl4.H, M, seed=seed, device=dev, zipf_s=wl4.zipf_s) for M in wl4.Ms}
-    res["large_decode"] = measure_workload("large_decode", big, wl4, "bf16", wl4.Ms, toks, stream, flush, args,
-                                           hbm_gbs, bf16_tf)
+    res["large_decode"] = measure_workload("large_decode", sets["bf16"], wl4, "bf16", wl4.Ms, toks, stream, args,
+                                           hbm_gbs, bf16_tf, flush)
     del toks
     toks = {M: synth.make_tokens(wl5.E, wl5.H, M, seed=seed, device=dev) for M in wl5.Ms}
-    res["prefill"] = measure_workload("prefill", big, wl5, "bf16", wl5.Ms, toks, stream, flush, args,
-                                      hbm_gbs, bf16_tf)
-    big.close()
-    res["prefill_fp8"] = measure_workload("prefill_fp8", big8, wl5, "fp8", wl5.Ms, toks, stream, flush, args,
-                                          hbm_gbs, bf16_tf)
-    big8.close()
+    res["prefill"] = measure_workload("prefill", sets["bf16"], wl5, "bf16", wl5.Ms, toks, stream, args,
+                                      hbm_gbs, bf16_tf, flush)
+    for lay in sets["bf16"]:
+        lay.close()
+    res["prefill_fp8"] = measure_workload("prefill_fp8", sets["fp8"], wl5, "fp8", wl5.Ms, toks, stream, args,
+                                          hbm_gbs, bf16_tf, flush)
+    for lay in sets["fp8"]:
+        lay.close()
+    del sets, toks
     torch.cuda.empty_cache()
     res["inv_rope_fp8"] = measure_inv_rope(args, dev, stream, flush, seed, hbm_gbs, cpu_on)
     return res
@@ -667,7 +752,7 @@ def main():
 
     import torch
 
-    from mixture_experts_layer_sort_b200 import MoELayer, synth
+    from mixture_experts_layer_sort_b200 import synth
 
     if args.workload == "inv_rope":
         return rope_only(args, ws, rank, local)
@@ -675,18 +760,20 @@ def main():
     Ms = [args.only_M] if args.only_M else list(wl.Ms)
     dev = torch.device("cuda", local)
     seed = args.seed + 1000 * rank
-    wg, wu, wd = synth.make_weights(wl.E, wl.H, wl.I, wl.w_std, seed=args.seed, device=dev)
-    layer = MoELayer(wl.E, wl.k, wl.H, wl.I, dtype)
-    layer.load_weights(wg, wu, wd)
-    if args.fused_decode:
-        layer.set_fused_decode(True)
+    l2_mode, n_sets, l2_text = l2_plan(wl, dtype, args.l2)
+    sets, w0 = make_layer_sets(wl, (dtype,), n_sets, args.seed, dev, keep_first=True,
+                               fused_decode=args.fused_decode)
+    layers = sets[dtype]
+    wg, wu, wd = w0
     toks = {M: synth.make_tokens(wl.E, wl.H, M, seed=seed, device=dev, zipf_s=wl.zipf_s) for M in Ms}
-    flush = torch.empty(L2_FLUSH_BYTES if not args.warm_l2 else 0, dtype=torch.uint8, device=dev)
+    # the flush buffer: the flush mode's 252 MB write, and the inverse-RoPE measurement
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
     tokens_per_step = sum(Ms)
     hbm_gbs, bf16_tf, peak_src = read_peaks()
 
-    run = Runner(layer, wl, dtype, Ms, toks, stream, flush, use_graph=not args.no_graph)
+    run = Runner(layers, wl, dtype, Ms, toks, stream, flush if l2_mode == "flush" else None,
+                 use_graph=not args.no_graph)
     run.warm(args.warmup)
 
     # ---------------------------------------------------------------- timed region
@@ -724,17 +811,21 @@ def main():
                     torch.empty((M, wl.H), dtype=torch.bfloat16).pin_memory()) for M in Ms}
         h2d = sum(M * wl.H * 2 + M * wl.E * 4 for M in Ms)
         d2h = sum(M * wl.H * 2 for M in Ms)
-        for _ in range(2):
+        for lay in layers:
             for M in Ms:
-                layer.forward_host(*host[M], stream=stream)
+                lay.forward_host(*host[M], stream=stream)
         e_times = []
+        fi = 0
         for s in range(args.steps):
             tot = 0.0
             for M in Ms:
-                flush.zero_()
+                lay = layers[fi % len(layers)]   # the same rotation over the weight sets
+                fi += 1
+                if l2_mode == "flush":
+                    flush.zero_()
                 torch.cuda.synchronize()
                 a = time.perf_counter()
-                layer.forward_host(*host[M], stream=stream)
+                lay.forward_host(*host[M], stream=stream)
                 tot += time.perf_counter() - a
             e_times.append(tot)
         e_sec = max_over_ranks(statistics.mean(e_times), ws)
@@ -762,7 +853,7 @@ def main():
         "vs_baseline": None,
         "dtype": dtype_name(dtype),
         "data": "synthetic",
-        "config": bench_config(wl, Ms, ws, args.warm_l2),
+        "config": bench_config(wl, Ms, ws, l2_text),
         "launch": "CUDA graph replay per M" if run.graphs else "eager",
         "roofline": {"bound": "hbm",
                      "kernel": "gate_up (the thin-batch tensor-core GEMV up to 8 tokens, the tcgen05 grouped GEMM above)", "achieved": achieved, "peak": hbm_gbs,
@@ -790,7 +881,8 @@ def main():
     if rank == 0:
         print(json.dumps(line))
     run.close()
-    layer.close()
+    for lay in layers:
+        lay.close()
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -70,4 +70,26 @@ def test_reference_arm_prints_one_line(capsys):
     # the same workload description as the main arm, so both lines name one config
     from mixture_experts_layer_sort_b200 import synth
     wl = synth.WORKLOADS["tiny"]
-    assert line["config"] == bench.bench_config(wl, list(wl.Ms), 1, False)
+    assert line["config"] == bench.bench_config(wl, list(wl.Ms), 1, bench.l2_plan(wl, "bf16", "rotate")[2])
+
+
+def test_l2_plan_weight_sets():
+    """The rotation keeps at least 2 x L2 of other weights between two forwards on one
+    set: the decode layer needs 5 bf16 sets (M = 1 streams 8 experts, 75.5 MB) and 8 e4m3
+    sets; the E=256 layer 2; the tiny layer would need hundreds and is flushed instead."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_sort_b200 import synth
+    W = synth.WORKLOADS
+    assert bench.l2_plan(W["decode"], "bf16", "rotate")[:2] == ("rotate", 5)
+    assert bench.l2_plan(W["decode_fp8"], "fp8", "rotate")[:2] == ("rotate", 8)
+    assert bench.l2_plan(W["large_decode"], "bf16", "rotate")[:2] == ("rotate", 2)
+    assert bench.l2_plan(W["prefill"], "fp8", "rotate")[:2] == ("rotate", 2)
+    assert bench.l2_plan(W["tiny"], "bf16", "rotate")[:2] == ("flush", 1)
+    assert bench.l2_plan(W["decode"], "bf16", "flush")[:2] == ("flush", 1)
+    assert bench.l2_plan(W["decode"], "bf16", "warm")[:2] == ("warm", 1)
+    for name, dt in (("decode", "bf16"), ("decode_fp8", "fp8"), ("large_decode", "bf16"), ("prefill", "fp8")):
+        wl = W[name]
+        mode, R, _ = bench.l2_plan(wl, dt, "rotate")
+        fewest = wl.k * 3 * wl.H * wl.I * bench.weight_bytes(dt)
+        assert (R - 1) * fewest >= 2 * bench.L2_BYTES and (R - 2) * fewest < 2 * bench.L2_BYTES
