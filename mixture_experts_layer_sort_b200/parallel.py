@@ -40,10 +40,17 @@ class TensorParallelMoE:
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor | None = None, stream=None):
         """This rank's partial output, then the all-reduce that sums the ranks' partials
-        (in place in `out`, on the current stream)."""
+        (in place in `out`). Both run on `stream` (a torch.cuda.Stream or a raw
+        cudaStream_t handle), or on the current stream when it is None, so the collective
+        is ordered after the forward that writes `out`."""
         out = self.layer.forward(x, logits, out=out, stream=stream)
         if self.world > 1:
-            dist.all_reduce(out, op=dist.ReduceOp.SUM, group=self.group)
+            if stream is None:
+                dist.all_reduce(out, op=dist.ReduceOp.SUM, group=self.group)
+            else:
+                s = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(stream)
+                with torch.cuda.stream(s):
+                    dist.all_reduce(out, op=dist.ReduceOp.SUM, group=self.group)
         return out
 
     __call__ = forward

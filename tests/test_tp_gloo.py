@@ -93,3 +93,40 @@ def test_shard_sizes_must_be_multiples_of_128():
         TensorParallelMoE(8, 2, 256, 768, rank=0, world=8, layer=object())   # 96 per rank
     tp = TensorParallelMoE(8, 2, 256, 1024, rank=3, world=8, layer=object())
     assert tp.I_full == 1024 and tp.rank == 3
+
+
+def test_all_reduce_runs_on_the_forward_stream(monkeypatch):
+    """With an explicit stream the all-reduce is issued inside that stream's context, so
+    it is ordered after the forward that wrote `out` (the CUDA stream objects are
+    replaced by recorders: no GPU is needed)."""
+    sys.path.insert(0, ROOT)
+    import contextlib
+    import torch
+    from mixture_experts_layer_sort_b200 import parallel
+    events = []
+
+    class FakeStream:
+        def __init__(self, handle):
+            self.handle = handle
+
+    @contextlib.contextmanager
+    def fake_stream_ctx(s):
+        events.append(("enter", s.handle))
+        yield
+        events.append(("exit", s.handle))
+
+    class Layer:
+        def forward(self, x, logits, out=None, stream=None):
+            events.append(("forward", stream))
+            return out
+
+    monkeypatch.setattr(torch.cuda, "ExternalStream", FakeStream)
+    monkeypatch.setattr(torch.cuda, "stream", fake_stream_ctx)
+    monkeypatch.setattr(parallel.dist, "all_reduce", lambda t, op=None, group=None: events.append(("all_reduce",)))
+    tp = parallel.TensorParallelMoE(8, 2, 256, 1024, rank=0, world=2, layer=Layer())
+    out = torch.zeros(2, 4)
+    tp.forward(None, None, out=out, stream=0x1234)
+    assert events == [("forward", 0x1234), ("enter", 0x1234), ("all_reduce",), ("exit", 0x1234)]
+    events.clear()
+    tp.forward(None, None, out=out)                   # no stream: the current one, no context switch
+    assert events == [("forward", None), ("all_reduce",)]
