@@ -54,6 +54,24 @@ class MoELayer:
         if code != 0:
             raise MoEError(fn, code)
 
+    def _check_tokens(self, fn, x, logits, out, on_gpu: bool):
+        """The library takes raw pointers and trusts their sizes: reject tensors whose
+        shape, dtype, layout or device would make it read or write outside them."""
+        bad = []
+        M = x.shape[0] if x.dim() == 2 else -1
+        if x.dim() != 2 or x.shape[1] != self.H or x.dtype != torch.bfloat16 or not x.is_contiguous():
+            bad.append(f"x must be a contiguous bf16 [M, {self.H}] tensor (got {x.dtype} {tuple(x.shape)})")
+        if tuple(logits.shape) != (M, self.E) or logits.dtype != torch.float32 or not logits.is_contiguous():
+            bad.append(f"logits must be a contiguous fp32 [{M}, {self.E}] tensor (got {logits.dtype} "
+                       f"{tuple(logits.shape)})")
+        if tuple(out.shape) != (M, self.H) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+            bad.append(f"out must be a contiguous bf16 [{M}, {self.H}] tensor (got {out.dtype} {tuple(out.shape)})")
+        for name, t in (("x", x), ("logits", logits), ("out", out)):
+            if t.is_cuda != on_gpu:
+                bad.append(f"{name} must be in {'device' if on_gpu else 'host'} memory")
+        if bad:
+            raise ValueError(f"{fn}: " + "; ".join(bad))
+
     @property
     def is_fp8(self) -> bool:
         return self.dtype in (FP8, FP8_E5M2)
@@ -113,6 +131,7 @@ class MoELayer:
         M = x.shape[0]
         if out is None:
             out = torch.empty((M, self.H), dtype=torch.bfloat16, device=x.device)
+        self._check_tokens("moe_forward", x, logits, out, on_gpu=True)
         self._check("moe_forward", self.lib.moe_forward(
             self.handle, _ptr(x), _ptr(logits), M, _ptr(out), _stream(stream)))
         return out
@@ -122,6 +141,7 @@ class MoELayer:
     def forward_noalloc(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor, stream=None):
         """moe_forward_noalloc: the same forward with all per-call scratch taken from the
         library's fixed 32 MiB device array (no allocation inside the call)."""
+        self._check_tokens("moe_forward_noalloc", x, logits, out, on_gpu=True)
         self._check("moe_forward_noalloc", self.lib.moe_forward_noalloc(
             self.handle, _ptr(x), _ptr(logits), x.shape[0], _ptr(out), _stream(stream)))
         return out
@@ -131,6 +151,7 @@ class MoELayer:
 
     def forward_host(self, x_cpu: torch.Tensor, logits_cpu: torch.Tensor, out_cpu: torch.Tensor, stream=None):
         M = x_cpu.shape[0]
+        self._check_tokens("moe_forward_host", x_cpu, logits_cpu, out_cpu, on_gpu=False)
         self._check("moe_forward_host", self.lib.moe_forward_host(
             self.handle, _ptr(x_cpu), _ptr(logits_cpu), M, _ptr(out_cpu), _stream(stream)))
         return out_cpu
