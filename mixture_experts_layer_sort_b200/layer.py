@@ -238,11 +238,28 @@ def inv_rope_fp8_quant(x: torch.Tensor, positions: torch.Tensor, cos_sin: torch.
     """moe_inv_rope_fp8_quant: x [T, NH, D] bf16, positions [T] int32, cos_sin [max_pos, D]
     fp32 (device) -> (codes [T, NH, D] uint8, scales [T, NH] fp32)."""
     lib = load_library()
+    if x.dim() != 3 or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError(f"moe_inv_rope_fp8_quant: x must be a contiguous bf16 [T, NH, D] tensor "
+                         f"(got {x.dtype} {tuple(x.shape)})")
     T, NH, D = x.shape
     if codes is None:
         codes = torch.empty((T, NH, D), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((T, NH), dtype=torch.float32, device=x.device)
+    bad = []
+    if tuple(positions.shape) != (T,) or positions.dtype != torch.int32 or not positions.is_contiguous():
+        bad.append(f"positions must be a contiguous int32 [{T}] tensor")
+    if cos_sin.dim() != 2 or cos_sin.shape[1] != D or cos_sin.dtype != torch.float32 or not cos_sin.is_contiguous():
+        bad.append(f"cos_sin must be a contiguous fp32 [max_pos, {D}] tensor")
+    if tuple(codes.shape) != (T, NH, D) or codes.dtype != torch.uint8 or not codes.is_contiguous():
+        bad.append(f"codes must be a contiguous uint8 [{T}, {NH}, {D}] tensor")
+    if tuple(scales.shape) != (T, NH) or scales.dtype != torch.float32 or not scales.is_contiguous():
+        bad.append(f"scales must be a contiguous fp32 [{T}, {NH}] tensor")
+    for name, t in (("x", x), ("positions", positions), ("cos_sin", cos_sin), ("codes", codes), ("scales", scales)):
+        if not t.is_cuda:
+            bad.append(f"{name} must be in device memory")
+    if bad:
+        raise ValueError("moe_inv_rope_fp8_quant: " + "; ".join(bad))
     rc = lib.moe_inv_rope_fp8_quant(_ptr(x), _ptr(positions), _ptr(cos_sin), cos_sin.shape[0], T, NH, D,
                                     1 if interleaved else 0, _DTYPES[fmt], _ptr(codes), _ptr(scales),
                                     _stream(stream))

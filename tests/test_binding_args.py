@@ -75,3 +75,18 @@ def test_device_entry_points_reject_host_tensors():
     with pytest.raises(ValueError, match="device memory"):
         lay.forward_noalloc(x, logits, out)
     assert lay.lib.calls == []
+
+
+def test_inv_rope_rejects_malformed_tensors():
+    from mixture_experts_layer_sort_b200.layer import inv_rope_fp8_quant
+    x = torch.zeros((4, 2, 128), dtype=torch.bfloat16)
+    pos = torch.zeros(4, dtype=torch.int32)
+    tab = torch.zeros((16, 128), dtype=torch.float32)
+    with pytest.raises(ValueError, match="x must be"):
+        inv_rope_fp8_quant(x.float(), pos, tab)
+    with pytest.raises(ValueError, match="positions must be"):
+        inv_rope_fp8_quant(x, pos.long(), tab)
+    with pytest.raises(ValueError, match="cos_sin must be"):
+        inv_rope_fp8_quant(x, pos, torch.zeros((16, 64), dtype=torch.float32))
+    with pytest.raises(ValueError, match="device memory"):    # well formed, but on the host
+        inv_rope_fp8_quant(x, pos, tab)
