@@ -54,6 +54,16 @@ class MoELayer:
         if code != 0:
             raise MoEError(fn, code)
 
+    def _check_weights(self, fn, tensors, I_rows: int, dtype):
+        """W_gate [E, I_rows, H], W_up [E, I_rows, H], W_down [E, H, I_rows], contiguous, of
+        `dtype`, in device memory (the load kernels read them through raw pointers)."""
+        shapes = ((self.E, I_rows, self.H), (self.E, I_rows, self.H), (self.E, self.H, I_rows))
+        for name, t, shape in zip(("w_gate", "w_up", "w_down"), tensors, shapes):
+            if (not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != dtype or tuple(t.shape) != shape
+                    or not t.is_contiguous()):
+                got = f"{t.dtype} {tuple(t.shape)} on {t.device}" if isinstance(t, torch.Tensor) else type(t).__name__
+                raise ValueError(f"{fn}: {name} must be a contiguous {dtype} {list(shape)} device tensor (got {got})")
+
     def _check_tokens(self, fn, x, logits, out, on_gpu: bool):
         """The library takes raw pointers and trusts their sizes: reject tensors whose
         shape, dtype, layout or device would make it read or write outside them."""
@@ -90,9 +100,7 @@ class MoELayer:
     # ------------------------------------------------------------------ weights
     def load_weights(self, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, stream=None):
         """bf16 device tensors W_gate [E,I,H], W_up [E,I,H], W_down [E,H,I]."""
-        for t, shape in ((w_gate, (self.E, self.I, self.H)), (w_up, (self.E, self.I, self.H)),
-                         (w_down, (self.E, self.H, self.I))):
-            assert t.is_cuda and t.dtype == torch.bfloat16 and tuple(t.shape) == shape and t.is_contiguous()
+        self._check_weights("moe_load_weights", (w_gate, w_up, w_down), self.I, torch.bfloat16)
         self._check("moe_load_weights", self.lib.moe_load_weights(
             self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), _stream(stream)))
 
@@ -100,8 +108,10 @@ class MoELayer:
                            stream=None):
         """A "mixed" layer: bf16 device tensors as for load_weights, and expert_fp8 [E]
         booleans (host) choosing e4m3 (True) or bf16 (False) per expert."""
+        self._check_weights("moe_load_weights_mixed", (w_gate, w_up, w_down), self.I, torch.bfloat16)
         flags = torch.as_tensor([1 if f else 0 for f in expert_fp8], dtype=torch.uint8)
-        assert flags.numel() == self.E
+        if flags.numel() != self.E:
+            raise ValueError(f"moe_load_weights_mixed: expert_fp8 must hold {self.E} flags (got {flags.numel()})")
         self._check("moe_load_weights_mixed", self.lib.moe_load_weights_mixed(
             self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), flags.data_ptr(), _stream(stream)))
 
@@ -111,15 +121,16 @@ class MoELayer:
         device tensors W_gate [E,I_full,H], W_up [E,I_full,H], W_down [E,H,I_full]
         (I_full = I * num_shards); the slicing happens in the library's load kernels."""
         I_full = self.I * num_shards
-        for t, shape in ((w_gate, (self.E, I_full, self.H)), (w_up, (self.E, I_full, self.H)),
-                         (w_down, (self.E, self.H, I_full))):
-            assert t.is_cuda and t.dtype == torch.bfloat16 and tuple(t.shape) == shape and t.is_contiguous()
+        self._check_weights("moe_load_weights_shard", (w_gate, w_up, w_down), I_full, torch.bfloat16)
         self._check("moe_load_weights_shard", self.lib.moe_load_weights_shard(
             self.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), I_full, shard, num_shards, _stream(stream)))
 
     def load_weights_fp8(self, q_gate, q_up, q_down, scales, stream=None):
         """uint8 e4m3 codes (device) and scales [E,3] fp32 (host)."""
+        self._check_weights("moe_load_weights_fp8", (q_gate, q_up, q_down), self.I, torch.uint8)
         sc = torch.as_tensor(scales, dtype=torch.float32).contiguous().cpu()
+        if tuple(sc.shape) != (self.E, 3):
+            raise ValueError(f"moe_load_weights_fp8: scales must be [{self.E}, 3] (got {tuple(sc.shape)})")
         self._check("moe_load_weights_fp8", self.lib.moe_load_weights_fp8(
             self.handle, _ptr(q_gate), _ptr(q_up), _ptr(q_down), sc.data_ptr(), _stream(stream)))
 

@@ -90,3 +90,18 @@ def test_inv_rope_rejects_malformed_tensors():
         inv_rope_fp8_quant(x, pos, torch.zeros((16, 64), dtype=torch.float32))
     with pytest.raises(ValueError, match="device memory"):    # well formed, but on the host
         inv_rope_fp8_quant(x, pos, tab)
+
+
+def test_weight_loads_reject_malformed_tensors():
+    lay = _layer()
+    E, H, I = 8, 256, 512
+    host = [torch.zeros(s, dtype=torch.bfloat16) for s in ((E, I, H), (E, I, H), (E, H, I))]
+    with pytest.raises(ValueError, match="w_gate must be"):          # host memory
+        lay.load_weights(*host)
+    with pytest.raises(ValueError, match="w_gate must be"):
+        lay.load_weights_mixed(*host, [True] * E)
+    with pytest.raises(ValueError, match="w_gate must be"):          # the full tensors of 2 shards
+        lay.load_weights_shard(*host, 0, 2)
+    with pytest.raises(ValueError, match="w_gate must be"):          # codes are uint8
+        lay.load_weights_fp8(*host, torch.ones(E, 3))
+    assert lay.lib.calls == []
