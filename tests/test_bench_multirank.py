@@ -93,3 +93,22 @@ def test_l2_plan_weight_sets():
         mode, R, _ = bench.l2_plan(wl, dt, "rotate")
         fewest = wl.k * 3 * wl.H * wl.I * bench.weight_bytes(dt)
         assert (R - 1) * fewest >= 2 * bench.L2_BYTES and (R - 2) * fewest < 2 * bench.L2_BYTES
+
+
+def test_roofline_numerators_by_hand():
+    """The bytes and FLOPs the roofline fractions divide by, worked out by hand for the
+    decode layer (E=128, k=8, H=2048, I=768) and the prefill layer (E=256, H=7168,
+    I=2048): each active expert streams W_gate, W_up and W_down once (3*H*I weights),
+    plus x in, out back, the logits and (FP8) the scale table; 2*M*k*3*H*I FLOPs."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_sort_b200 import synth
+    dec, pre = synth.WORKLOADS["decode"], synth.WORKLOADS["prefill"]
+    # M = 1 activates k = 8 experts: 8 * 3 * 2048 * 768 * 2 B + 2048*2*2 (x, out) + 128*4 (logits)
+    assert bench.alg_bytes_layer(dec, "bf16", 1, 8) == 75497472 + 8192 + 512
+    # e4m3: one byte per weight, plus 128 experts x 3 fp32 scales
+    assert bench.alg_bytes_layer(dec, "fp8", 1, 8) == 37748736 + 8192 + 512 + 1536
+    # prefill, every expert active: 256 * 3 * 7168 * 2048 * 2 B = 22.5 GB of weights
+    assert bench.alg_bytes_layer(pre, "bf16", 4096, 256) == 22548578304 + 4096 * 7168 * 4 + 4096 * 256 * 4
+    assert bench.alg_flops_layer(dec, 1) == 2 * 8 * 3 * 2048 * 768
+    assert bench.alg_flops_layer(pre, 4096) == 2 * 4096 * 8 * 3 * 7168 * 2048
